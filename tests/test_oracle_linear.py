@@ -1,0 +1,355 @@
+"""Pins for the oracle's linear-layer functions (CPU only).
+
+The checks reduce the oracle's layer functions to things fixed outside it:
+the page facts in tests/golden/page_facts.json, special cases that collapse
+to a textbook routine (pure vector-wise int8, a plain fp matmul), numpy's
+integer and fp64 matmul on tiny inputs, closed forms, and torch's own casts
+for the dequant rule weight.to(bf16) * weight_scale.
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "page_facts.json")
+with open(GOLDEN) as _f:
+    FACTS = json.load(_f)
+THR = FACTS["outlier_threshold"]["value"]
+
+
+def bits_to_f64(bits, dt):
+    return oracle.bits_to_torch(np.ascontiguousarray(bits), dt).double().numpy()
+
+
+def rand_x(M, K, seed, dtype=torch.bfloat16, clip=None):
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn((M, K), generator=g)
+    if clip is not None:
+        x = x.clamp(-clip, clip)
+    return x.to(dtype)
+
+
+def rand_w(N, K, seed, dtype=torch.bfloat16):
+    g = torch.Generator().manual_seed(seed + 17)
+    return (torch.randn((N, K), generator=g) * 0.02).to(dtype)
+
+
+# --------------------------------------------------------- outlier set ----
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+def test_threshold_boundary(dtype):
+    assert THR == 6.0
+    K = 64
+    x = torch.zeros((4, K), dtype=torch.float32)
+    # the next representable value above 6.0 in this dtype
+    nxt = torch.tensor([THR], dtype=dtype)
+    nxt = (nxt.view(torch.int16) + 1).view(dtype).item()
+    x[0, 3] = THR            # exactly at the threshold: not an outlier (strict >)
+    x[1, 5] = nxt            # just above: outlier
+    x[2, 7] = -nxt           # just below -6: outlier (absolute value)
+    x[3, 9] = -THR           # exactly -6: not an outlier
+    x[0, 11] = 5.99
+    X = x.to(dtype)
+    assert nxt > THR
+    r = oracle.int8_outlier_prep(X, THR)
+    assert r["O"].tolist() == [5, 7]
+    assert r["count"] == 2
+    # the outlier columns carry zero codes and are copied exactly into X_O
+    assert np.all(r["Xq"][:, [5, 7]] == 0)
+    xo = bits_to_f64(r["X_O"], r["dt"])
+    assert xo[1, 0] == nxt and xo[2, 1] == -nxt and xo[0, 0] == 0.0
+
+
+def test_outlier_test_spans_all_tokens():
+    # A column is an outlier when ANY token of the call exceeds the
+    # threshold; its small values in other tokens are excluded too.
+    X = rand_x(16, 128, 1, clip=2.0).float()
+    X[7, 40] = 7.5
+    X = X.to(torch.bfloat16)
+    r = oracle.int8_outlier_prep(X, THR)
+    assert r["O"].tolist() == [40]
+    xf = X.float().numpy()
+    keep = np.ones(128, bool)
+    keep[40] = False
+    expect_absmax = np.abs(xf[:, keep]).max(axis=1).astype(np.float32)
+    assert np.array_equal(r["s_x"], expect_absmax / np.float32(127.0))
+
+
+def test_threshold_disabled_values():
+    X = rand_x(8, 64, 2)
+    X[0, 0] = 100.0
+    for thr in (0.0, -1.0, float("inf")):
+        r = oracle.int8_outlier_prep(X, thr)
+        assert r["count"] == 0
+
+
+# ---------------------------------------- special cases of LLM.int8 ------
+
+def vectorwise_int8_reference(X, Wq, s_w):
+    """Plain vector-wise int8 written with torch/numpy primitives (no outliers)."""
+    x = X.float()
+    absmax = x.abs().amax(dim=1)
+    s_x = absmax / torch.tensor(127.0)
+    inv = torch.tensor(1.0) / s_x
+    t = x * inv[:, None]
+    q = torch.where(x == 0, torch.zeros_like(t), torch.round(t).clamp(-127, 127)).to(torch.int64)
+    C = q.numpy() @ Wq.astype(np.int64).T
+    Y = C.astype(np.float64) * s_x.double().numpy()[:, None] * s_w.astype(np.float64)[None, :]
+    return q.numpy().astype(np.int8), s_x.numpy(), C, Y
+
+
+@pytest.mark.parametrize("how", ["clipped", "threshold_inf", "threshold_zero"])
+def test_no_outliers_equals_pure_vectorwise_int8(how):
+    M, K, N = 24, 160, 40
+    if how == "clipped":
+        X, thr = rand_x(M, K, 3, clip=THR), THR
+    else:
+        X = rand_x(M, K, 3)
+        X[2, 9] = 50.0
+        thr = float("inf") if how == "threshold_inf" else 0.0
+    W = rand_w(N, K, 3)
+    Wq, s_w = oracle.quantize_weight(W, "int8_row")
+    q_ref, s_ref, C_ref, Y_ref = vectorwise_int8_reference(X, Wq, s_w)
+    p = oracle.int8_outlier_prep(X, thr)
+    assert p["count"] == 0
+    assert np.array_equal(p["Xq"], q_ref)
+    assert np.array_equal(p["s_x"], s_ref)
+    r = oracle.int8_outlier_forward(X, Wq, s_w, thr)
+    assert np.array_equal(r["C"].astype(np.int64), C_ref)
+    np.testing.assert_allclose(r["Y64"], Y_ref, rtol=1e-12, atol=1e-12)
+
+
+def test_all_outliers_equals_plain_fp_matmul():
+    M, K, N = 12, 96, 20
+    X = rand_x(M, K, 4).float()
+    X[M - 1, :] = 8.0                         # every column exceeds the threshold somewhere
+    X = X.to(torch.bfloat16)
+    W = rand_w(N, K, 4)
+    Wq, s_w = oracle.quantize_weight(W, "int8_row")
+    p = oracle.int8_outlier_prep(X, THR)
+    assert p["count"] == K and np.all(p["Xq"] == 0)
+    r = oracle.int8_outlier_forward(X, Wq, s_w, THR)
+    assert np.all(r["C"] == 0)
+    # dequant rule weight.to(bf16) * weight_scale, through torch's own ops
+    W_deq = (torch.from_numpy(Wq).float() * torch.from_numpy(s_w)[:, None]).to(torch.bfloat16)
+    Y_ref = X.double().numpy() @ W_deq.double().numpy().T
+    np.testing.assert_allclose(r["Y64"], Y_ref, rtol=1e-12, atol=1e-12)
+
+
+def test_outlier_weights_follow_dequant_rule():
+    W = rand_w(32, 64, 5)
+    Wq, s_w = oracle.quantize_weight(W, "int8_row")
+    O = np.array([0, 3, 63], np.int32)
+    for dtype, dt in ((torch.bfloat16, oracle.BF16), (torch.float16, oracle.F16)):
+        got = oracle.outlier_weights(Wq, s_w, O, dt)
+        ref = (torch.from_numpy(Wq[:, O]).float() * torch.from_numpy(s_w)[:, None]).to(dtype)
+        assert np.array_equal(got, ref.view(torch.int16).numpy().view(np.uint16))
+
+
+def test_mixed_decomposition_matches_split_sum():
+    # Y = int8 part + fp part, each checked against numpy on its own.
+    M, K, N = 20, 128, 24
+    X = rand_x(M, K, 6).float()
+    X[3, 10] = -9.0
+    X[15, 100] = 12.0
+    X = X.to(torch.float16)
+    W = rand_w(N, K, 6, torch.float16)
+    bias = (torch.arange(N, dtype=torch.float32) / 7).to(torch.float16)
+    Wq, s_w = oracle.quantize_weight(W, "int8_row")
+    p = oracle.int8_outlier_prep(X, THR)
+    assert p["O"].tolist() == [10, 100]
+    r = oracle.int8_outlier_forward(X, Wq, s_w, THR, bias=bias)
+    C = p["Xq"].astype(np.int64) @ Wq.astype(np.int64).T
+    assert np.array_equal(r["C"].astype(np.int64), C)
+    W_deq = (torch.from_numpy(Wq[:, p["O"]]).float() * torch.from_numpy(s_w)[:, None]).to(torch.float16)
+    F = X.double().numpy()[:, p["O"]] @ W_deq.double().numpy().T
+    Y = C * p["s_x"].astype(np.float64)[:, None] * s_w.astype(np.float64)[None, :] + F + bias.double().numpy()
+    np.testing.assert_allclose(r["Y64"], Y, rtol=1e-12, atol=1e-12)
+    # the rounded output is the fp16 rounding of Y64 (torch's cast from exact fp32 values)
+    yb = torch.from_numpy(r["Y64"]).to(torch.float16).view(torch.int16).numpy().view(np.uint16)
+    mism = np.nonzero(yb != r["Y"])[0]
+    # torch casts fp64 -> fp16 through fp32; a double rounding may differ by one ulp
+    assert mism.size <= 2
+
+
+def test_brute_force_tiny_int32():
+    # every code pattern of a 2x2x2 block at extreme values, and random
+    # tiny shapes, against numpy's int64 matmul
+    rng = np.random.default_rng(7)
+    for M, N, K in [(1, 1, 16), (2, 3, 32), (4, 4, 48), (3, 2, 16)]:
+        for trial in range(4):
+            X = torch.from_numpy(rng.uniform(-5.9, 5.9, (M, K)).astype(np.float32)).to(torch.bfloat16)
+            W = torch.from_numpy(rng.normal(0, 0.02, (N, K)).astype(np.float32)).to(torch.bfloat16)
+            Wq, s_w = oracle.quantize_weight(W, "int8_row")
+            p = oracle.int8_outlier_prep(X, THR)
+            r = oracle.int8_outlier_forward(X, Wq, s_w, THR)
+            assert np.array_equal(r["C"].astype(np.int64),
+                                  p["Xq"].astype(np.int64) @ Wq.astype(np.int64).T)
+    # all sign patterns of +-absmax rows: codes are exactly +-127
+    for pattern in range(16):
+        signs = np.array([1 if (pattern >> b) & 1 else -1 for b in range(4)], np.float32)
+        X = torch.from_numpy(np.tile(signs, (2, 4)) * 3.0).to(torch.bfloat16)     # [2,16]
+        W = torch.from_numpy(np.tile(signs[::-1].copy(), (3, 4)) * 0.5).to(torch.bfloat16)
+        Wq, s_w = oracle.quantize_weight(W, "int8_row")
+        p = oracle.int8_outlier_prep(X, THR)
+        assert set(np.unique(np.abs(p["Xq"]))) == {127}
+        r = oracle.int8_outlier_forward(X, Wq, s_w, THR)
+        assert np.array_equal(r["C"].astype(np.int64), p["Xq"].astype(np.int64) @ Wq.astype(np.int64).T)
+
+
+def test_int32_bound_at_largest_k():
+    # K = 12288 with every code at 127: C = 12288 * 127^2 = 198,193,152 < 2^31
+    K = 12288
+    X = torch.ones((1, K), dtype=torch.bfloat16)
+    W = torch.full((2, K), 0.25, dtype=torch.bfloat16)
+    W[1] = -0.25
+    Wq, s_w = oracle.quantize_weight(W, "int8_row")
+    r = oracle.int8_outlier_forward(X, Wq, s_w, THR)
+    assert r["C"].tolist() == [[198193152, -198193152]]
+    assert 198193152 < 2 ** 31
+
+
+def test_massive_activation_goes_to_fp_path():
+    f = FACTS["massive_activation_text_encoder"]
+    wl = workloads.get_workload("te_fp8_dynamic_mlp")
+    lin = workloads.Linear("t", 16, 4096, 8)
+    X, W, _ = workloads.make_linear(wl, lin)
+    assert X[0, f["channel"]].item() == 12992.0 and X[5, f["channel"]].item() == 9024.0
+    p = oracle.int8_outlier_prep(X, THR)
+    assert f["channel"] in p["O"].tolist()
+    # the massive value does not enter the int8 row scale
+    assert p["s_x"][0] < np.float32(THR) / np.float32(127.0) * np.float32(1.0001)
+
+
+# ------------------------------------------------------------------ FP8 ---
+
+def decode_e4m3_torch(codes):
+    return torch.from_numpy(np.ascontiguousarray(codes)).view(torch.float8_e4m3fn).double().numpy()
+
+
+def test_fp8_static_acc_exact_and_scaled():
+    M, K, N = 16, 128, 24
+    X = rand_x(M, K, 8)
+    W = rand_w(N, K, 8)
+    Wq, ws = oracle.quantize_weight(W, "fp8_tensor")
+    assert ws[0] == np.float32(np.abs(W.float().numpy()).max()) / np.float32(448.0)
+    x_scale = oracle.absmax_scale(rand_x(M, K, 9), 448.0)
+    r = oracle.fp8_forward(X, Wq, ws, x_scale=x_scale)
+    a = decode_e4m3_torch(r["Xq"])
+    b = decode_e4m3_torch(Wq)
+    acc = a @ b.T
+    assert np.array_equal(r["acc"], acc)                    # exact in fp64
+    np.testing.assert_allclose(r["Y64"], acc * float(x_scale) * float(ws[0]), rtol=1e-15)
+    # activations above input_scale*448 saturate to +-448
+    inv = np.float32(1.0) / np.float32(x_scale)
+    big = X.float().numpy() * inv > 464
+    assert np.all(r["Xq"][big] == 0x7E)
+
+
+def test_fp8_codes_vs_torch_cast():
+    X = rand_x(32, 64, 10)
+    s = oracle.absmax_scale(X, 448.0)
+    codes = oracle.fp8_static_prep(X, s)
+    inv = torch.tensor(1.0, dtype=torch.float32) / torch.tensor(s, dtype=torch.float32)
+    ref = (X.float() * inv).clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(codes, ref)
+
+
+def test_fp8_dynamic_scales_and_channel_dequant():
+    M, K, N = 8, 256, 16
+    X = rand_x(M, K, 11).float()
+    X[0, 2] = 12992.0                               # massive value: row scale = 29 exactly
+    X = X.to(torch.bfloat16)
+    W = rand_w(N, K, 11)
+    Wq, sb = oracle.quantize_weight(W, "fp8_channel")
+    assert sb.dtype == np.uint16 and sb.shape == (N,)  # bf16 [out, 1]
+    # weight.to(bf16) * weight_scale recovers W to within e4m3's relative step (2^-4 half-ulp)
+    w_scale = torch.from_numpy(sb.view(np.int16)).view(torch.bfloat16)[:, None]
+    deq = (torch.from_numpy(Wq).view(torch.float8_e4m3fn).to(torch.bfloat16) * w_scale).float()
+    wf = W.float()
+    rowmax = wf.abs().amax(1, keepdim=True)
+    assert torch.all((deq - wf).abs() <= rowmax * 2.0 ** -4 * 1.02 + 1e-30)
+    r = oracle.fp8_forward(X, Wq, sb, x_scale=None)
+    assert r["s_x"][0] == 29.0
+    a = decode_e4m3_torch(r["Xq"])
+    acc = a @ decode_e4m3_torch(Wq).T
+    assert np.array_equal(r["acc"], acc)
+    sw = w_scale.double().numpy().reshape(-1)
+    np.testing.assert_allclose(r["Y64"], acc * r["s_x"].astype(np.float64)[:, None] * sw[None, :],
+                               rtol=1e-15)
+
+
+# ---------------------------------------------------------------- W4A8 ---
+
+def unpack_int4(packed, K):
+    lo = (packed & 0x0F).astype(np.int16)
+    hi = (packed >> 4).astype(np.int16)
+    q = np.empty((packed.shape[0], K), np.int16)
+    q[:, 0::2] = np.where(lo >= 8, lo - 16, lo)
+    q[:, 1::2] = np.where(hi >= 8, hi - 16, hi)
+    return q
+
+
+def test_int4_pack_layout_and_range():
+    W = rand_w(8, 256, 12)
+    q, s = oracle.quantize_weight(W, "int4_g128")
+    assert q.shape == (8, 128) and s.shape == (8, 2)
+    u = unpack_int4(q, 256)
+    assert u.min() >= -7 and u.max() <= 7
+    for j in range(8):
+        for k in (0, 1, 2, 127, 128, 255):
+            assert oracle.lib().orc_int4_unpack(q.ctypes.data, 256, j, k) == u[j, k]
+    # scale = group absmax / 7
+    wf = W.float().numpy().reshape(8, 2, 128)
+    assert np.array_equal(s, np.abs(wf).max(axis=2).astype(np.float32) / np.float32(7.0))
+
+
+def test_w4a8_equal_group_scales_reduce_to_per_channel():
+    M, K, N, G = 6, 384, 10, 128
+    X = rand_x(M, K, 13)
+    g = torch.Generator().manual_seed(14)
+    W = torch.randn((N, K), generator=g) * 0.02
+    W.view(N, K // G, G)[:, :, 0] = 0.1           # identical absmax in every group -> equal scales
+    W = W.to(torch.bfloat16)
+    q, s = oracle.quantize_weight(W, "int4_g128")
+    assert np.all(s == s[:, :1])
+    r = oracle.w4a8_forward(X, q, s, group=G, want_cg=True)
+    u = unpack_int4(q, K).astype(np.int64)
+    C = r["Xq"].astype(np.int64) @ u.T
+    assert np.array_equal(r["Cg"].sum(axis=2).astype(np.int64), C)
+    for gi in range(K // G):
+        sl = slice(gi * G, (gi + 1) * G)
+        assert np.array_equal(r["Cg"][:, :, gi].astype(np.int64),
+                              r["Xq"][:, sl].astype(np.int64) @ u[:, sl].T)
+    Y = C * r["s_x"].astype(np.float64)[:, None] * s[:, 0].astype(np.float64)[None, :]
+    np.testing.assert_allclose(r["Y64"], Y, rtol=1e-12)
+    # its activation codes are the pure vector-wise int8 codes
+    p = oracle.int8_outlier_prep(X, 0.0)
+    assert np.array_equal(p["Xq"], r["Xq"]) and np.array_equal(p["s_x"], r["s_x"])
+
+
+def test_rows_subset_matches_full():
+    wl = workloads.get_workload("tiny_int8")
+    X, W, bias = workloads.make_linear(wl, wl.linears[0])
+    Wq, s_w = oracle.quantize_weight(W, "int8_row")
+    full = oracle.int8_outlier_forward(X, Wq, s_w, THR, bias=bias)
+    rows = [0, 5, 63, 17]
+    sub = oracle.int8_outlier_forward(X, Wq, s_w, THR, bias=bias, rows=rows)
+    assert np.array_equal(sub["C"], full["C"][rows])
+    assert np.array_equal(sub["Y64"], full["Y64"][rows])
+
+
+def test_zero_rows_and_degenerate_scales():
+    X = rand_x(4, 64, 15).float()
+    X[1] = 0.0
+    X = X.to(torch.bfloat16)
+    p = oracle.int8_outlier_prep(X, THR)
+    assert p["s_x"][1] == 0.0 and np.all(p["Xq"][1] == 0)
+    assert np.all(np.isfinite(p["s_x"])) and np.all(p["s_x"][[0, 2, 3]] > 0)
+    xq, sx = oracle.fp8_dynamic_prep(X)
+    assert sx[1] == 0.0 and np.all(xq[1] == 0)
