@@ -1,0 +1,192 @@
+/*
+ * qlin.h -- C ABI of libqlin.so: one quantized linear layer, Y = X W^T, on
+ * NVIDIA B200 (sm_100a), in the four weight/activation formats the
+ * Qwen-Image-2.1 model-card pages use:
+ *
+ *   - LLM.int8 mixed-precision decomposition (ixim/Image21-INT8, section
+ *     "Quantization": bitsandbytes LLM.int8, outlier threshold 6.0, outlier
+ *     handling in floating point) with vector-wise int8: per-token absmax/127
+ *     activation scales, per-output-channel absmax/127 weight scales, int32
+ *     accumulation, dequant by the outer product of the two scale vectors;
+ *   - FP8 E4M3 W8A8 with static per-tensor fp32 weight_scale and input_scale
+ *     (Darkstar-Qwen-Image-2.1-Base-ModelOpt-FP8, section "Precision map");
+ *   - FP8 E4M3 weights with one bf16 scale per output channel, shape [out,1],
+ *     and dynamic per-token FP8 activations (Qwen-Image-2.1-Text-Encoder-FP8,
+ *     section "Format"; dequant rule weight.to(bf16) * weight_scale);
+ *   - int4 per-group weights with int8 activations and fp32 scales
+ *     (Qwen-Image-fni8, section "Format"), group 128 along K.
+ *
+ * Conventions shared by every entry point:
+ *   - Shapes: X is [M,K] row-major, W is [N,K] row-major (K contiguous), Y is
+ *     [M,N] row-major. M = tokens, K = in-features, N = out-features.
+ *   - Every data pointer is a DEVICE pointer unless its comment says "host".
+ *     The caller owns all memory. The library allocates and frees no device
+ *     memory and never synchronises the stream inside a forward: all work is
+ *     enqueued on `stream` (a cudaStream_t passed as void*; NULL = the legacy
+ *     default stream).
+ *   - Alignment: every device pointer must be 16-byte aligned; K must be a
+ *     positive multiple of 16 (of 128 for the int4 format) and at most 32768.
+ *     M and N are arbitrary (M = 0 or N = 0 is a no-op that returns QLIN_OK).
+ *   - Scratch: entry points that need scratch take `workspace` (device) and
+ *     `ws_bytes`; qlin_workspace_bytes() gives the size. A workspace may be
+ *     reused by calls that are ordered on one stream, not by calls that may
+ *     overlap.
+ *   - dtype of X, bias and Y: QLIN_F16 or QLIN_BF16 (all three the same).
+ *     bias is nullable ([N]).
+ *   - Errors: every call returns a qlin_status; nothing crosses the ABI as an
+ *     exception. Argument errors are detected on the host before anything is
+ *     enqueued. A device-side wait that runs out of time (QLIN_ERR_TIMEOUT)
+ *     is recorded in a device status word that qlin_get_device_status()
+ *     reads. qlin_last_error_string() describes the last error of the
+ *     calling thread.
+ *   - Thread safety: calls from several host threads are safe; the error
+ *     string is thread-local.
+ */
+#ifndef QLIN_H
+#define QLIN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define QLIN_API __attribute__((visibility("default")))
+#else
+#define QLIN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum qlin_status {
+    QLIN_OK = 0,
+    QLIN_ERR_INVALID_ARG = 1,   /* null pointer, negative size, bad enum            */
+    QLIN_ERR_UNSUPPORTED = 2,   /* shape / device outside what the kernels support  */
+    QLIN_ERR_ALIGNMENT = 3,     /* pointer not 16-byte aligned, K not a multiple    */
+    QLIN_ERR_WORKSPACE = 4,     /* workspace missing or smaller than required       */
+    QLIN_ERR_CUDA = 5,          /* a CUDA runtime call or a launch failed           */
+    QLIN_ERR_TIMEOUT = 6        /* a bounded device-side wait ran out of time       */
+} qlin_status;
+
+typedef enum qlin_dtype { QLIN_F16 = 0, QLIN_BF16 = 1 } qlin_dtype;
+
+/* Weight formats (offline quantisation, qlin_quantize_weight). */
+typedef enum qlin_wmode {
+    QLIN_W_INT8_ROW = 0,     /* Wq int8 [N,K];  w_scale fp32 [N]   = absmax_k|W[j,k]| / 127          */
+    QLIN_W_FP8_TENSOR = 1,   /* Wq e4m3 [N,K];  w_scale fp32 [1]   = absmax|W| / 448                 */
+    QLIN_W_FP8_CHANNEL = 2,  /* Wq e4m3 [N,K];  w_scale bf16 [N,1] = bf16(absmax_k|W[j,k]| / 448)    */
+    QLIN_W_INT4_G128 = 3     /* Wq uint8 [N,K/2] (k even: low nibble, k odd: high nibble, two's
+                                complement, codes in [-7,7]); w_scale fp32 [N,K/128] = absmax/7      */
+} qlin_wmode;
+
+/* Operations whose scratch size qlin_workspace_bytes() reports. */
+typedef enum qlin_op {
+    QLIN_OP_INT8_OUTLIER = 0,   /* qlin_int8_outlier_forward                        */
+    QLIN_OP_FP8 = 1,            /* qlin_fp8_forward                                 */
+    QLIN_OP_W4A8 = 2,           /* qlin_w4a8_forward                                */
+    QLIN_OP_QUANTIZE_WEIGHT = 3,/* qlin_quantize_weight and qlin_calibrate_input_scale */
+    QLIN_OP_INT8_PREP = 4       /* qlin_int8_prep                                   */
+} qlin_op;
+
+/* Bytes of device scratch `op` needs for an [M,K] x [N,K]^T problem (0 when
+ * none is needed). Host-only, never fails; returns 0 for invalid sizes. */
+QLIN_API size_t qlin_workspace_bytes(qlin_op op, int64_t M, int64_t N, int64_t K);
+
+/* Offline weight quantisation (not part of the timed forward).
+ * W: [N,K] in `wdt`. Wq / w_scale: layouts listed with qlin_wmode. Codes are
+ * round-half-even (int8/int4, clamped to +-127 / +-7) or round-to-nearest-even
+ * saturating E4M3 (max 448), computed as code(w * (1/s)) with every step in
+ * IEEE fp32. workspace: qlin_workspace_bytes(QLIN_OP_QUANTIZE_WEIGHT, 0, N, K)
+ * bytes (only QLIN_W_FP8_TENSOR uses it). */
+QLIN_API qlin_status qlin_quantize_weight(const void *W, qlin_dtype wdt, int64_t N, int64_t K,
+                                 qlin_wmode mode, void *Wq, void *w_scale,
+                                 void *workspace, size_t ws_bytes, void *stream);
+
+/* Max calibration of a static FP8 input scale (Darkstar ModelOpt-FP8 page,
+ * "Provenance": calibration with the max algorithm):
+ * *x_scale (device fp32) = absmax(X) / 448 over a calibration batch X [M,K].
+ * workspace: qlin_workspace_bytes(QLIN_OP_QUANTIZE_WEIGHT, M, 0, K) bytes. */
+QLIN_API qlin_status qlin_calibrate_input_scale(const void *X, qlin_dtype xdt, int64_t M, int64_t K,
+                                       float *x_scale, void *workspace, size_t ws_bytes,
+                                       void *stream);
+
+/* LLM.int8 forward (ixim/Image21-INT8, "Quantization"):
+ *   O       = { k : |X[i,k]| > threshold for some token i of this call }
+ *   s_x[i]  = max_{k not in O} |X[i,k]| / 127;  Xq = rne(X / s_x), 0 on O
+ *   C       = Xq Wq^T (int8 x int8 -> int32, tcgen05 kind::i8)
+ *   F       = X[:,O] W_O^T, W_O = dtype(fp32(Wq[:,O]) * w_scale)  (the
+ *             floating-point outlier part, dequant rule weight.to(dtype)*scale)
+ *   Y       = dtype(C * s_x[i] * w_scale[j] + F + bias[j]).
+ * threshold <= 0 or +inf turns the decomposition off (pure vector-wise int8).
+ * Wq int8 [N,K], w_scale fp32 [N] from qlin_quantize_weight(QLIN_W_INT8_ROW).
+ * Y [M,N] in xdt. workspace: qlin_workspace_bytes(QLIN_OP_INT8_OUTLIER, M, N, K).
+ * The number of outlier columns stays on the device (no host sync). */
+QLIN_API qlin_status qlin_int8_outlier_forward(const void *X, qlin_dtype xdt, int64_t M, int64_t K,
+                                      const int8_t *Wq, const float *w_scale, int64_t N,
+                                      float threshold, const void *bias, void *Y,
+                                      void *workspace, size_t ws_bytes, void *stream);
+
+/* FP8 E4M3 W8A8 forward.
+ *   wmode QLIN_W_FP8_TENSOR: w_scale -> fp32 scalar (ModelOpt-FP8 page,
+ *     "Precision map"); wmode QLIN_W_FP8_CHANNEL: w_scale -> bf16 [N]
+ *     (Text-Encoder-FP8 page, "Format").
+ *   x_scale -> fp32 scalar: static per-tensor input scale, Xq = e4m3(X / x_scale);
+ *   x_scale == NULL: dynamic per-token scales s_x[i] = absmax_i / 448.
+ *   acc = sum_k dec(Xq) dec(Wq) (fp32 accumulate, tcgen05 kind::f8f6f4),
+ *   Y = dtype(acc * s_x * s_w + bias).
+ * workspace: qlin_workspace_bytes(QLIN_OP_FP8, M, N, K). */
+QLIN_API qlin_status qlin_fp8_forward(const void *X, qlin_dtype xdt, int64_t M, int64_t K,
+                             const uint8_t *Wq, const void *w_scale, qlin_wmode wmode,
+                             int64_t N, const float *x_scale, const void *bias, void *Y,
+                             void *workspace, size_t ws_bytes, void *stream);
+
+/* ---------------- parity exports: the same kernels, intermediates written out ------ */
+
+/* LLM.int8 activation prep alone. Outputs: Xq int8 [M,K]; s_x fp32 [M];
+ * flags uint32 [ceil(K/32)] (bit k%32 of word k/32 set iff column k is an
+ * outlier); O int32 [K] (ascending outlier columns, first *count valid);
+ * count int32 [1]; X_O [M, ostride] in xdt (X[:,O], zero-padded to a multiple
+ * of 8 columns; ostride >= round_up(K,8), a multiple of 8).
+ * workspace: qlin_workspace_bytes(QLIN_OP_INT8_PREP, M, 0, K). */
+QLIN_API qlin_status qlin_int8_prep(const void *X, qlin_dtype xdt, int64_t M, int64_t K, float threshold,
+                           int8_t *Xq, float *s_x, uint32_t *flags, int32_t *O, int32_t *count,
+                           void *X_O, int64_t ostride, void *workspace, size_t ws_bytes,
+                           void *stream);
+
+/* Outlier weight columns: W_O[j,o] = dtype(fp32(Wq[j,O[o]]) * w_scale[j]) for
+ * o < *count, zero up to the next multiple of 8; W_O is [N, ostride] in dt. */
+QLIN_API qlin_status qlin_outlier_weights(const int8_t *Wq, const float *w_scale, int64_t N, int64_t K,
+                                 const int32_t *O, const int32_t *count, qlin_dtype dt,
+                                 void *W_O, int64_t ostride, void *stream);
+
+/* Raw int8 GEMM: C[M,N] int32 = Xq[M,K] Wq[N,K]^T, exact (|C| <= K*127^2). */
+QLIN_API qlin_status qlin_int8_gemm_i32(const int8_t *Xq, const int8_t *Wq, int64_t M, int64_t N,
+                               int64_t K, int32_t *C, void *stream);
+
+/* FP8 activation prep alone: Xq e4m3 [M,K]; s_x fp32 [M] (dynamic mode,
+ * x_scale == NULL; ignored and may be NULL in static mode). */
+QLIN_API qlin_status qlin_fp8_prep(const void *X, qlin_dtype xdt, int64_t M, int64_t K,
+                          const float *x_scale, uint8_t *Xq, float *s_x, void *stream);
+
+/* ---------------- status ------------------------------------------------------------ */
+
+/* Reads (and with reset != 0 clears) the device status word of the current
+ * device into *status (host pointer): QLIN_OK, or QLIN_ERR_TIMEOUT if a
+ * kernel gave up on a bounded wait. Synchronises the device. */
+QLIN_API qlin_status qlin_get_device_status(int32_t *status, int reset);
+
+/* Sets the limit of every bounded device-side wait, in nanoseconds (default
+ * 2e9). Synchronous; call it outside stream capture. */
+QLIN_API qlin_status qlin_set_wait_timeout_ns(uint64_t ns);
+
+/* Message for the last error returned on the calling thread ("" if none). */
+QLIN_API const char *qlin_last_error_string(void);
+
+/* ABI version of this header (major * 100 + minor). */
+QLIN_API int qlin_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QLIN_H */

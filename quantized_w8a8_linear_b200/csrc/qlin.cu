@@ -1,0 +1,555 @@
+// qlin.cu -- the C ABI declared in include/qlin.h (single translation unit:
+// the kernels of prep.cuh and gemm.cuh are instantiated and launched here).
+//
+// Host side of every entry point: validate arguments, carve the caller's
+// workspace, build the TMA tensor maps, and enqueue kernels on the caller's
+// stream. No device memory is allocated or freed and no stream is
+// synchronised inside a forward.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/qlin.h"
+#include "common.cuh"
+#include "gemm.cuh"
+#include "prep.cuh"
+
+using namespace qlin;
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+qlin_status fail(qlin_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+qlin_status ok() {
+  g_err[0] = '\0';
+  return QLIN_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
+
+constexpr int64_t kMaxK = 32768;
+
+qlin_status check_cuda(cudaError_t e, const char* what) {
+  if (e != cudaSuccess) return fail(QLIN_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return QLIN_OK;
+}
+
+// ---- per-device facts (SM count, sm_100 check), cached ------------------
+struct DeviceInfo {
+  int sms = 0;
+  bool sm100 = false;
+  bool gemm_attr_set[64] = {};
+};
+std::mutex g_dev_mu;
+DeviceInfo g_dev[16];
+
+qlin_status device_info(DeviceInfo** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 16) return fail(QLIN_ERR_CUDA, "cudaGetDevice failed");
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (d.sms == 0) {
+    cudaDeviceProp prop;
+    qlin_status s = check_cuda(cudaGetDeviceProperties(&prop, dev), "cudaGetDeviceProperties");
+    if (s != QLIN_OK) return s;
+    d.sms = prop.multiProcessorCount;
+    d.sm100 = (prop.major == 10 && prop.minor == 0);
+  }
+  if (!d.sm100) return fail(QLIN_ERR_UNSUPPORTED, "libqlin needs an sm_100 (B200) device");
+  *out = &d;
+  return QLIN_OK;
+}
+
+// ---- TMA descriptors -----------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+qlin_status get_encode(PFN_cuTensorMapEncodeTiled_v12000* fn) {
+  std::call_once(g_encode_once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  if (!g_encode) return fail(QLIN_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  *fn = g_encode;
+  return QLIN_OK;
+}
+
+// 8-bit row-major [rows, K] matrix, box of box_rows x 128 bytes, 128B swizzle.
+qlin_status make_tmap_k128(CUtensorMap* m, const void* base, int64_t rows, int64_t K, int box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc;
+  qlin_status s = get_encode(&enc);
+  if (s != QLIN_OK) return s;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(K)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(GEMM_BK), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(QLIN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return QLIN_OK;
+}
+
+// ---- GEMM launch ------------------------------------------------------------
+constexpr int kBN = 256;
+constexpr int kStages = 4;
+
+template <int KIND, int EPI, typename TOut>
+qlin_status launch_gemm(const void* A, const void* B, const EpiParams& ep, cudaStream_t st, int attr_slot) {
+  DeviceInfo* d;
+  qlin_status s = device_info(&d);
+  if (s != QLIN_OK) return s;
+  CUtensorMap ta, tb;
+  if ((s = make_tmap_k128(&ta, A, ep.M, ep.K, GEMM_BM)) != QLIN_OK) return s;
+  if ((s = make_tmap_k128(&tb, B, ep.N, ep.K, kBN)) != QLIN_OK) return s;
+  auto kern = k_gemm<KIND, EPI, TOut, kBN, kStages>;
+  constexpr int smem = GemmSmem<kBN, kStages>::TOTAL;
+  if (!d->gemm_attr_set[attr_slot]) {
+    s = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
+                   "cudaFuncSetAttribute");
+    if (s != QLIN_OK) return s;
+    d->gemm_attr_set[attr_slot] = true;
+  }
+  const int64_t tiles = ((ep.M + GEMM_BM - 1) / GEMM_BM) * ((ep.N + kBN - 1) / kBN);
+  const int grid = static_cast<int>(tiles < d->sms ? tiles : d->sms);
+  kern<<<grid, GEMM_THREADS, smem, st>>>(ta, tb, ep);
+  return check_cuda(cudaGetLastError(), "k_gemm launch");
+}
+
+// ---- row quantiser dispatch (V = 16-byte vectors per thread) ------------------
+template <typename T, int CODE, bool SBF16, bool OUTL>
+qlin_status launch_rowquant(const void* X, int64_t rows, int64_t K, uint8_t* Q, float* s32, uint16_t* sbf,
+                            const uint32_t* flags, const int32_t* wpre, const int32_t* count, uint16_t* X_O,
+                            int64_t ostride, cudaStream_t st) {
+  if (rows == 0) return QLIN_OK;
+  const int64_t per = (K / 8 + PREP_THREADS - 1) / PREP_THREADS;
+  const T* x = static_cast<const T*>(X);
+  const dim3 grid(static_cast<unsigned>(rows));
+#define QLIN_RQ(VV)                                                                                           \
+  k_rowquant<T, VV, CODE, SBF16, OUTL><<<grid, PREP_THREADS, 0, st>>>(x, K, Q, s32, sbf, flags, wpre, count, \
+                                                                      X_O, ostride)
+  if (per <= 1) QLIN_RQ(1);
+  else if (per <= 2) QLIN_RQ(2);
+  else if (per <= 4) QLIN_RQ(4);
+  else if (per <= 8) QLIN_RQ(8);
+  else if (per <= 12) QLIN_RQ(12);
+  else if (per <= 16) QLIN_RQ(16);
+  else if (per <= 24) QLIN_RQ(24);
+  else QLIN_RQ(32);
+#undef QLIN_RQ
+  return check_cuda(cudaGetLastError(), "k_rowquant launch");
+}
+
+// ---- LLM.int8 workspace layout -----------------------------------------------
+struct Int8Ws {
+  uint32_t* done;     // [1]  compaction counter
+  int32_t* count;     // [1]
+  uint32_t* flags;    // [NW]
+  int32_t* wpre;      // [NW]
+  int32_t* O;         // [K]
+  float* s_x;         // [M]
+  int8_t* Xq;         // [M,K]
+  uint16_t* X_O;      // [M,ostride]
+  uint16_t* W_O;      // [N,ostride]
+  int64_t ostride;
+  size_t memset_bytes;  // zeroed each call: done, count, flags
+  size_t total;
+};
+
+Int8Ws int8_layout(void* base, int64_t M, int64_t N, int64_t K, bool with_gemm_parts) {
+  Int8Ws w{};
+  uint8_t* p = static_cast<uint8_t*>(base);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    uint8_t* r = p ? p + off : nullptr;
+    off = static_cast<size_t>(round_up(static_cast<int64_t>(off + bytes), 256));
+    return r;
+  };
+  const int64_t NW = (K + 31) / 32;
+  uint8_t* hdr = take(16 + 4 * NW);
+  w.done = reinterpret_cast<uint32_t*>(hdr);
+  w.count = reinterpret_cast<int32_t*>(hdr ? hdr + 4 : nullptr);
+  w.flags = reinterpret_cast<uint32_t*>(hdr ? hdr + 16 : nullptr);
+  w.memset_bytes = static_cast<size_t>(16 + 4 * NW);
+  w.wpre = reinterpret_cast<int32_t*>(take(4 * NW));
+  w.O = reinterpret_cast<int32_t*>(take(4 * K));
+  w.ostride = round_up(K, 8);
+  if (with_gemm_parts) {
+    w.s_x = reinterpret_cast<float*>(take(4 * M));
+    w.Xq = reinterpret_cast<int8_t*>(take(static_cast<size_t>(M * K)));
+    w.X_O = reinterpret_cast<uint16_t*>(take(static_cast<size_t>(2 * M * w.ostride)));
+    w.W_O = reinterpret_cast<uint16_t*>(take(static_cast<size_t>(2 * N * w.ostride)));
+  }
+  w.total = off;
+  return w;
+}
+
+bool decomposition_on(float thr) { return thr > 0.0f && !std::isinf(thr); }
+
+template <typename T>
+qlin_status int8_prep_impl(const void* X, int64_t M, int64_t K, float thr, const Int8Ws& w, int8_t* Xq, float* s_x,
+                           uint16_t* X_O, int64_t ostride, cudaStream_t st) {
+  qlin_status s = check_cuda(cudaMemsetAsync(w.done, 0, w.memset_bytes, st), "cudaMemsetAsync");
+  if (s != QLIN_OK) return s;
+  if (decomposition_on(thr) && M > 0) {
+    const int rpb = 32;
+    const dim3 grid(static_cast<unsigned>((K / 8 + PREP_THREADS - 1) / PREP_THREADS),
+                    static_cast<unsigned>((M + rpb - 1) / rpb));
+    k_outlier_flags<T><<<grid, PREP_THREADS, 0, st>>>(static_cast<const T*>(X), M, K, thr, rpb, w.flags, w.wpre,
+                                                      w.O, w.count, w.done);
+    if ((s = check_cuda(cudaGetLastError(), "k_outlier_flags launch")) != QLIN_OK) return s;
+    return launch_rowquant<T, 0, false, true>(X, M, K, reinterpret_cast<uint8_t*>(Xq), s_x, nullptr, w.flags,
+                                              w.wpre, w.count, X_O, ostride, st);
+  }
+  return launch_rowquant<T, 0, false, false>(X, M, K, reinterpret_cast<uint8_t*>(Xq), s_x, nullptr, nullptr,
+                                             nullptr, nullptr, nullptr, 0, st);
+}
+
+qlin_status check_common(const void* X, qlin_dtype dt, int64_t M, int64_t K, int64_t N) {
+  if (dt != QLIN_F16 && dt != QLIN_BF16) return fail(QLIN_ERR_INVALID_ARG, "dtype must be QLIN_F16 or QLIN_BF16");
+  if (M < 0 || N < 0 || K < 0) return fail(QLIN_ERR_INVALID_ARG, "negative size");
+  if (K == 0 || K % 16 != 0) return fail(QLIN_ERR_ALIGNMENT, "K must be a positive multiple of 16 (got %lld)",
+                                         static_cast<long long>(K));
+  if (K > kMaxK) return fail(QLIN_ERR_UNSUPPORTED, "K = %lld exceeds %lld", static_cast<long long>(K),
+                             static_cast<long long>(kMaxK));
+  if (X == nullptr && M > 0) return fail(QLIN_ERR_INVALID_ARG, "X is NULL");
+  if (!aligned16(X)) return fail(QLIN_ERR_ALIGNMENT, "X is not 16-byte aligned");
+  return QLIN_OK;
+}
+
+#define QLIN_TRY(...)                  \
+  do {                                 \
+    qlin_status _s = (__VA_ARGS__);    \
+    if (_s != QLIN_OK) return _s;      \
+  } while (0)
+
+#define QLIN_REQ_PTR(p, name)                                                          \
+  do {                                                                                 \
+    if ((p) == nullptr) return fail(QLIN_ERR_INVALID_ARG, "%s is NULL", name);         \
+    if (!aligned16(p)) return fail(QLIN_ERR_ALIGNMENT, "%s is not 16-byte aligned", name); \
+  } while (0)
+
+}  // namespace
+
+// =============================================================================
+// C ABI
+// =============================================================================
+extern "C" {
+
+int qlin_version(void) { return 100; }
+
+const char* qlin_last_error_string(void) { return g_err; }
+
+size_t qlin_workspace_bytes(qlin_op op, int64_t M, int64_t N, int64_t K) {
+  if (M < 0 || N < 0 || K <= 0) return 0;
+  switch (op) {
+    case QLIN_OP_INT8_OUTLIER:
+      return int8_layout(nullptr, M, N, K, true).total;
+    case QLIN_OP_INT8_PREP:
+      return int8_layout(nullptr, M, N, K, false).total;
+    case QLIN_OP_FP8:
+      return static_cast<size_t>(round_up(M * K, 256) + round_up(4 * M, 256));
+    case QLIN_OP_QUANTIZE_WEIGHT:
+      return 256;
+    default:
+      return 0;
+  }
+}
+
+qlin_status qlin_get_device_status(int32_t* status, int reset) {
+  if (!status) return fail(QLIN_ERR_INVALID_ARG, "status is NULL");
+  QLIN_TRY(check_cuda(cudaDeviceSynchronize(), "cudaDeviceSynchronize"));
+  int v = 0;
+  QLIN_TRY(check_cuda(cudaMemcpyFromSymbol(&v, qlin::g_status, sizeof(int)), "cudaMemcpyFromSymbol"));
+  *status = v;
+  if (reset) {
+    const int z = 0;
+    QLIN_TRY(check_cuda(cudaMemcpyToSymbol(qlin::g_status, &z, sizeof(int)), "cudaMemcpyToSymbol"));
+  }
+  return ok();
+}
+
+qlin_status qlin_set_wait_timeout_ns(uint64_t ns) {
+  const unsigned long long v = ns;
+  QLIN_TRY(check_cuda(cudaMemcpyToSymbol(qlin::g_wait_timeout_ns, &v, sizeof(v)), "cudaMemcpyToSymbol"));
+  return ok();
+}
+
+qlin_status qlin_quantize_weight(const void* W, qlin_dtype wdt, int64_t N, int64_t K, qlin_wmode mode, void* Wq,
+                                 void* w_scale, void* workspace, size_t ws_bytes, void* stream) {
+  QLIN_TRY(check_common(W, wdt, N, K, 0));
+  if (mode == QLIN_W_INT4_G128 && K % 128 != 0) return fail(QLIN_ERR_ALIGNMENT, "int4 format needs K % 128 == 0");
+  if (N == 0) return ok();
+  QLIN_REQ_PTR(Wq, "Wq");
+  QLIN_REQ_PTR(w_scale, "w_scale");
+  DeviceInfo* d;
+  QLIN_TRY(device_info(&d));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool bf = (wdt == QLIN_BF16);
+  const int64_t nvec = N * K / 8;
+  switch (mode) {
+    case QLIN_W_INT8_ROW:
+      QLIN_TRY(bf ? launch_rowquant<__nv_bfloat16, 0, false, false>(W, N, K, static_cast<uint8_t*>(Wq),
+                                                                     static_cast<float*>(w_scale), nullptr, nullptr,
+                                                                     nullptr, nullptr, nullptr, 0, st)
+                  : launch_rowquant<__half, 0, false, false>(W, N, K, static_cast<uint8_t*>(Wq),
+                                                             static_cast<float*>(w_scale), nullptr, nullptr, nullptr,
+                                                             nullptr, nullptr, 0, st));
+      return ok();
+    case QLIN_W_FP8_CHANNEL:
+      QLIN_TRY(bf ? launch_rowquant<__nv_bfloat16, 1, true, false>(W, N, K, static_cast<uint8_t*>(Wq), nullptr,
+                                                                    static_cast<uint16_t*>(w_scale), nullptr,
+                                                                    nullptr, nullptr, nullptr, 0, st)
+                  : launch_rowquant<__half, 1, true, false>(W, N, K, static_cast<uint8_t*>(Wq), nullptr,
+                                                            static_cast<uint16_t*>(w_scale), nullptr, nullptr,
+                                                            nullptr, nullptr, 0, st));
+      return ok();
+    case QLIN_W_FP8_TENSOR: {
+      if (workspace == nullptr || ws_bytes < qlin_workspace_bytes(QLIN_OP_QUANTIZE_WEIGHT, 0, N, K))
+        return fail(QLIN_ERR_WORKSPACE, "workspace too small");
+      QLIN_REQ_PTR(workspace, "workspace");
+      uint32_t* amax = static_cast<uint32_t*>(workspace);
+      QLIN_TRY(check_cuda(cudaMemsetAsync(amax, 0, 4, st), "cudaMemsetAsync"));
+      const int grid = d->sms * 4;
+      if (bf) {
+        k_absmax<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(W), nvec, amax);
+        k_fp8_tensor_quant<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(W), nvec, amax,
+                                                                static_cast<uint8_t*>(Wq),
+                                                                static_cast<float*>(w_scale));
+      } else {
+        k_absmax<__half><<<grid, 256, 0, st>>>(static_cast<const __half*>(W), nvec, amax);
+        k_fp8_tensor_quant<__half><<<grid, 256, 0, st>>>(static_cast<const __half*>(W), nvec, amax,
+                                                         static_cast<uint8_t*>(Wq), static_cast<float*>(w_scale));
+      }
+      QLIN_TRY(check_cuda(cudaGetLastError(), "fp8 tensor quant launch"));
+      return ok();
+    }
+    case QLIN_W_INT4_G128: {
+      const int64_t warps = N * (K / 128);
+      const int64_t blocks = (warps * 32 + 255) / 256;
+      if (bf)
+        k_int4_group_quant<__nv_bfloat16><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+            static_cast<const __nv_bfloat16*>(W), N, K, static_cast<uint8_t*>(Wq), static_cast<float*>(w_scale));
+      else
+        k_int4_group_quant<__half><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+            static_cast<const __half*>(W), N, K, static_cast<uint8_t*>(Wq), static_cast<float*>(w_scale));
+      QLIN_TRY(check_cuda(cudaGetLastError(), "int4 quant launch"));
+      return ok();
+    }
+    default:
+      return fail(QLIN_ERR_INVALID_ARG, "unknown weight mode %d", static_cast<int>(mode));
+  }
+}
+
+qlin_status qlin_calibrate_input_scale(const void* X, qlin_dtype xdt, int64_t M, int64_t K, float* x_scale,
+                                       void* workspace, size_t ws_bytes, void* stream) {
+  QLIN_TRY(check_common(X, xdt, M, K, 0));
+  QLIN_REQ_PTR(x_scale, "x_scale");
+  if (workspace == nullptr || ws_bytes < qlin_workspace_bytes(QLIN_OP_QUANTIZE_WEIGHT, M, 0, K))
+    return fail(QLIN_ERR_WORKSPACE, "workspace too small");
+  QLIN_REQ_PTR(workspace, "workspace");
+  DeviceInfo* d;
+  QLIN_TRY(device_info(&d));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t* amax = static_cast<uint32_t*>(workspace);
+  QLIN_TRY(check_cuda(cudaMemsetAsync(amax, 0, 4, st), "cudaMemsetAsync"));
+  const int64_t nvec = M * K / 8;
+  if (nvec > 0) {
+    if (xdt == QLIN_BF16)
+      k_absmax<__nv_bfloat16><<<d->sms * 4, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(X), nvec, amax);
+    else
+      k_absmax<__half><<<d->sms * 4, 256, 0, st>>>(static_cast<const __half*>(X), nvec, amax);
+  }
+  k_scale_from_absmax<<<1, 1, 0, st>>>(amax, 448.0f, x_scale);
+  QLIN_TRY(check_cuda(cudaGetLastError(), "calibration launch"));
+  return ok();
+}
+
+qlin_status qlin_int8_prep(const void* X, qlin_dtype xdt, int64_t M, int64_t K, float threshold, int8_t* Xq,
+                           float* s_x, uint32_t* flags, int32_t* O, int32_t* count, void* X_O, int64_t ostride,
+                           void* workspace, size_t ws_bytes, void* stream) {
+  QLIN_TRY(check_common(X, xdt, M, K, 0));
+  QLIN_REQ_PTR(Xq, "Xq");
+  QLIN_REQ_PTR(s_x, "s_x");
+  QLIN_REQ_PTR(flags, "flags");
+  QLIN_REQ_PTR(O, "O");
+  QLIN_REQ_PTR(count, "count");
+  QLIN_REQ_PTR(X_O, "X_O");
+  if (ostride < round_up(K, 8) || ostride % 8 != 0)
+    return fail(QLIN_ERR_INVALID_ARG, "ostride must be a multiple of 8 and >= round_up(K, 8)");
+  if (workspace == nullptr || ws_bytes < qlin_workspace_bytes(QLIN_OP_INT8_PREP, M, 0, K))
+    return fail(QLIN_ERR_WORKSPACE, "workspace too small");
+  QLIN_REQ_PTR(workspace, "workspace");
+  DeviceInfo* d;
+  QLIN_TRY(device_info(&d));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Int8Ws w = int8_layout(workspace, M, 0, K, false);
+  QLIN_TRY(xdt == QLIN_BF16
+               ? int8_prep_impl<__nv_bfloat16>(X, M, K, threshold, w, Xq, s_x, static_cast<uint16_t*>(X_O), ostride,
+                                               st)
+               : int8_prep_impl<__half>(X, M, K, threshold, w, Xq, s_x, static_cast<uint16_t*>(X_O), ostride, st));
+  const int64_t NW = (K + 31) / 32;
+  QLIN_TRY(check_cuda(cudaMemcpyAsync(flags, w.flags, 4 * NW, cudaMemcpyDeviceToDevice, st), "copy flags"));
+  QLIN_TRY(check_cuda(cudaMemcpyAsync(count, w.count, 4, cudaMemcpyDeviceToDevice, st), "copy count"));
+  QLIN_TRY(check_cuda(cudaMemcpyAsync(O, w.O, 4 * K, cudaMemcpyDeviceToDevice, st), "copy O"));
+  return ok();
+}
+
+qlin_status qlin_outlier_weights(const int8_t* Wq, const float* w_scale, int64_t N, int64_t K, const int32_t* O,
+                                 const int32_t* count, qlin_dtype dt, void* W_O, int64_t ostride, void* stream) {
+  if (dt != QLIN_F16 && dt != QLIN_BF16) return fail(QLIN_ERR_INVALID_ARG, "bad dtype");
+  if (N < 0 || K <= 0) return fail(QLIN_ERR_INVALID_ARG, "bad sizes");
+  if (N == 0) return ok();
+  QLIN_REQ_PTR(Wq, "Wq");
+  QLIN_REQ_PTR(w_scale, "w_scale");
+  QLIN_REQ_PTR(O, "O");
+  QLIN_REQ_PTR(count, "count");
+  QLIN_REQ_PTR(W_O, "W_O");
+  if (ostride < round_up(K, 8) || ostride % 8 != 0) return fail(QLIN_ERR_INVALID_ARG, "bad ostride");
+  DeviceInfo* d;
+  QLIN_TRY(device_info(&d));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (dt == QLIN_BF16)
+    k_gather_wo<__nv_bfloat16><<<d->sms * 4, 256, 0, st>>>(Wq, w_scale, N, K, O, count,
+                                                           static_cast<uint16_t*>(W_O), ostride);
+  else
+    k_gather_wo<__half><<<d->sms * 4, 256, 0, st>>>(Wq, w_scale, N, K, O, count, static_cast<uint16_t*>(W_O),
+                                                    ostride);
+  QLIN_TRY(check_cuda(cudaGetLastError(), "k_gather_wo launch"));
+  return ok();
+}
+
+qlin_status qlin_int8_gemm_i32(const int8_t* Xq, const int8_t* Wq, int64_t M, int64_t N, int64_t K, int32_t* C,
+                               void* stream) {
+  if (M < 0 || N < 0) return fail(QLIN_ERR_INVALID_ARG, "negative size");
+  if (K <= 0 || K % 16 != 0) return fail(QLIN_ERR_ALIGNMENT, "K must be a positive multiple of 16");
+  if (K > kMaxK) return fail(QLIN_ERR_UNSUPPORTED, "K too large");
+  if (M == 0 || N == 0) return ok();
+  QLIN_REQ_PTR(Xq, "Xq");
+  QLIN_REQ_PTR(Wq, "Wq");
+  QLIN_REQ_PTR(C, "C");
+  EpiParams ep{};
+  ep.M = M; ep.N = N; ep.K = K; ep.Y = C;
+  QLIN_TRY((launch_gemm<0, EPI_I32, __nv_bfloat16>(Xq, Wq, ep, static_cast<cudaStream_t>(stream), 0)));
+  return ok();
+}
+
+qlin_status qlin_int8_outlier_forward(const void* X, qlin_dtype xdt, int64_t M, int64_t K, const int8_t* Wq,
+                                      const float* w_scale, int64_t N, float threshold, const void* bias, void* Y,
+                                      void* workspace, size_t ws_bytes, void* stream) {
+  QLIN_TRY(check_common(X, xdt, M, K, N));
+  if (M == 0 || N == 0) return ok();
+  QLIN_REQ_PTR(Wq, "Wq");
+  QLIN_REQ_PTR(w_scale, "w_scale");
+  QLIN_REQ_PTR(Y, "Y");
+  if (bias != nullptr && !aligned16(bias)) return fail(QLIN_ERR_ALIGNMENT, "bias is not 16-byte aligned");
+  if (workspace == nullptr || ws_bytes < qlin_workspace_bytes(QLIN_OP_INT8_OUTLIER, M, N, K))
+    return fail(QLIN_ERR_WORKSPACE, "workspace too small (need %zu bytes)",
+                qlin_workspace_bytes(QLIN_OP_INT8_OUTLIER, M, N, K));
+  QLIN_REQ_PTR(workspace, "workspace");
+  DeviceInfo* d;
+  QLIN_TRY(device_info(&d));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Int8Ws w = int8_layout(workspace, M, N, K, true);
+  const bool bf = (xdt == QLIN_BF16);
+  QLIN_TRY(bf ? int8_prep_impl<__nv_bfloat16>(X, M, K, threshold, w, w.Xq, w.s_x, w.X_O, w.ostride, st)
+              : int8_prep_impl<__half>(X, M, K, threshold, w, w.Xq, w.s_x, w.X_O, w.ostride, st));
+  if (decomposition_on(threshold)) {
+    if (bf)
+      k_gather_wo<__nv_bfloat16><<<d->sms * 4, 256, 0, st>>>(Wq, w_scale, N, K, w.O, w.count, w.W_O, w.ostride);
+    else
+      k_gather_wo<__half><<<d->sms * 4, 256, 0, st>>>(Wq, w_scale, N, K, w.O, w.count, w.W_O, w.ostride);
+    QLIN_TRY(check_cuda(cudaGetLastError(), "k_gather_wo launch"));
+  }
+  EpiParams ep{};
+  ep.M = M; ep.N = N; ep.K = K; ep.Y = Y;
+  ep.s_x = w.s_x; ep.s_w = w_scale; ep.bias = static_cast<const uint16_t*>(bias);
+  ep.count = w.count; ep.X_O = w.X_O; ep.W_O = w.W_O; ep.ostride = w.ostride;
+  if (bf) QLIN_TRY((launch_gemm<0, EPI_INT8_OUTLIER, __nv_bfloat16>(w.Xq, Wq, ep, st, 1)));
+  else QLIN_TRY((launch_gemm<0, EPI_INT8_OUTLIER, __half>(w.Xq, Wq, ep, st, 2)));
+  return ok();
+}
+
+qlin_status qlin_fp8_prep(const void* X, qlin_dtype xdt, int64_t M, int64_t K, const float* x_scale, uint8_t* Xq,
+                          float* s_x, void* stream) {
+  QLIN_TRY(check_common(X, xdt, M, K, 0));
+  if (M == 0) return ok();
+  QLIN_REQ_PTR(Xq, "Xq");
+  DeviceInfo* d;
+  QLIN_TRY(device_info(&d));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool bf = (xdt == QLIN_BF16);
+  if (x_scale != nullptr) {
+    QLIN_REQ_PTR(x_scale, "x_scale");
+    const int64_t nvec = M * K / 8;
+    if (bf) k_fp8_static<__nv_bfloat16><<<d->sms * 8, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(X), nvec,
+                                                                    x_scale, Xq);
+    else k_fp8_static<__half><<<d->sms * 8, 256, 0, st>>>(static_cast<const __half*>(X), nvec, x_scale, Xq);
+    return check_cuda(cudaGetLastError(), "k_fp8_static launch") == QLIN_OK ? ok() : QLIN_ERR_CUDA;
+  }
+  QLIN_REQ_PTR(s_x, "s_x");
+  QLIN_TRY(bf ? launch_rowquant<__nv_bfloat16, 1, false, false>(X, M, K, Xq, s_x, nullptr, nullptr, nullptr, nullptr,
+                                                                 nullptr, 0, st)
+              : launch_rowquant<__half, 1, false, false>(X, M, K, Xq, s_x, nullptr, nullptr, nullptr, nullptr,
+                                                         nullptr, 0, st));
+  return ok();
+}
+
+qlin_status qlin_fp8_forward(const void* X, qlin_dtype xdt, int64_t M, int64_t K, const uint8_t* Wq,
+                             const void* w_scale, qlin_wmode wmode, int64_t N, const float* x_scale, const void* bias,
+                             void* Y, void* workspace, size_t ws_bytes, void* stream) {
+  QLIN_TRY(check_common(X, xdt, M, K, N));
+  if (wmode != QLIN_W_FP8_TENSOR && wmode != QLIN_W_FP8_CHANNEL)
+    return fail(QLIN_ERR_INVALID_ARG, "wmode must be QLIN_W_FP8_TENSOR or QLIN_W_FP8_CHANNEL");
+  if (M == 0 || N == 0) return ok();
+  QLIN_REQ_PTR(Wq, "Wq");
+  QLIN_REQ_PTR(w_scale, "w_scale");
+  QLIN_REQ_PTR(Y, "Y");
+  if (bias != nullptr && !aligned16(bias)) return fail(QLIN_ERR_ALIGNMENT, "bias is not 16-byte aligned");
+  if (workspace == nullptr || ws_bytes < qlin_workspace_bytes(QLIN_OP_FP8, M, N, K))
+    return fail(QLIN_ERR_WORKSPACE, "workspace too small");
+  QLIN_REQ_PTR(workspace, "workspace");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* Xq = static_cast<uint8_t*>(workspace);
+  float* s_x = reinterpret_cast<float*>(Xq + round_up(M * K, 256));
+  if (wmode == QLIN_W_FP8_TENSOR && x_scale == nullptr)
+    return fail(QLIN_ERR_UNSUPPORTED, "per-tensor weight scales need a static x_scale");
+  if (wmode == QLIN_W_FP8_CHANNEL && x_scale != nullptr)
+    return fail(QLIN_ERR_UNSUPPORTED, "per-channel weight scales go with dynamic per-token activations (x_scale NULL)");
+  QLIN_TRY(qlin_fp8_prep(X, xdt, M, K, x_scale, Xq, s_x, stream));
+  EpiParams ep{};
+  ep.M = M; ep.N = N; ep.K = K; ep.Y = Y;
+  ep.bias = static_cast<const uint16_t*>(bias);
+  const bool bf = (xdt == QLIN_BF16);
+  if (wmode == QLIN_W_FP8_TENSOR) {
+    ep.x_scale = x_scale;
+    ep.w_scale = static_cast<const float*>(w_scale);
+    if (bf) QLIN_TRY((launch_gemm<1, EPI_FP8_TENSOR, __nv_bfloat16>(Xq, Wq, ep, st, 3)));
+    else QLIN_TRY((launch_gemm<1, EPI_FP8_TENSOR, __half>(Xq, Wq, ep, st, 4)));
+  } else {
+    ep.s_x = s_x;
+    ep.s_w_bf16 = static_cast<const uint16_t*>(w_scale);
+    if (bf) QLIN_TRY((launch_gemm<1, EPI_FP8_ROWCOL, __nv_bfloat16>(Xq, Wq, ep, st, 5)));
+    else QLIN_TRY((launch_gemm<1, EPI_FP8_ROWCOL, __half>(Xq, Wq, ep, st, 6)));
+  }
+  return ok();
+}
+
+}  // extern "C"
