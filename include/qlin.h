@@ -126,12 +126,30 @@ QLIN_API qlin_status qlin_int8_outlier_forward(const void *X, qlin_dtype xdt, in
                                       float threshold, const void *bias, void *Y,
                                       void *workspace, size_t ws_bytes, void *stream);
 
+/* The two stages of qlin_int8_outlier_forward, for callers that schedule
+ * (or time) them separately; the forward is exactly prepare then gemm on the
+ * same stream and workspace.
+ *   prepare: outlier detection, activation codes/scales, X_O and W_O
+ *            (HBM-bound kernels), all written into `workspace`;
+ *   gemm:    the tcgen05 int8 GEMM with the fused dequant + outlier + bias
+ *            epilogue, reading what prepare left in `workspace`. */
+QLIN_API qlin_status qlin_int8_outlier_prepare(const void *X, qlin_dtype xdt, int64_t M, int64_t K,
+                                      const int8_t *Wq, const float *w_scale, int64_t N,
+                                      float threshold, void *workspace, size_t ws_bytes,
+                                      void *stream);
+QLIN_API qlin_status qlin_int8_outlier_gemm(qlin_dtype xdt, int64_t M, int64_t K, const int8_t *Wq,
+                                   const float *w_scale, int64_t N, const void *bias, void *Y,
+                                   void *workspace, size_t ws_bytes, void *stream);
+
 /* FP8 E4M3 W8A8 forward.
  *   wmode QLIN_W_FP8_TENSOR: w_scale -> fp32 scalar (ModelOpt-FP8 page,
  *     "Precision map"); wmode QLIN_W_FP8_CHANNEL: w_scale -> bf16 [N]
  *     (Text-Encoder-FP8 page, "Format").
- *   x_scale -> fp32 scalar: static per-tensor input scale, Xq = e4m3(X / x_scale);
- *   x_scale == NULL: dynamic per-token scales s_x[i] = absmax_i / 448.
+ *   x_scale -> fp32 scalar: static per-tensor input scale, Xq = e4m3(X / x_scale)
+ *     (required with QLIN_W_FP8_TENSOR);
+ *   x_scale == NULL: dynamic per-token scales s_x[i] = absmax_i / 448
+ *     (required with QLIN_W_FP8_CHANNEL). Other pairings return
+ *     QLIN_ERR_UNSUPPORTED: the pages pair the scales this way.
  *   acc = sum_k dec(Xq) dec(Wq) (fp32 accumulate, tcgen05 kind::f8f6f4),
  *   Y = dtype(acc * s_x * s_w + bias).
  * workspace: qlin_workspace_bytes(QLIN_OP_FP8, M, N, K). */
@@ -139,6 +157,13 @@ QLIN_API qlin_status qlin_fp8_forward(const void *X, qlin_dtype xdt, int64_t M, 
                              const uint8_t *Wq, const void *w_scale, qlin_wmode wmode,
                              int64_t N, const float *x_scale, const void *bias, void *Y,
                              void *workspace, size_t ws_bytes, void *stream);
+
+/* The GEMM stage of qlin_fp8_forward: Xq e4m3 [M,K] and (dynamic mode) s_x
+ * fp32 [M] as qlin_fp8_prep wrote them. Same wmode / x_scale rules. */
+QLIN_API qlin_status qlin_fp8_gemm(qlin_dtype xdt, int64_t M, int64_t K, const uint8_t *Xq,
+                          const float *s_x, const uint8_t *Wq, const void *w_scale,
+                          qlin_wmode wmode, int64_t N, const float *x_scale, const void *bias,
+                          void *Y, void *stream);
 
 /* ---------------- parity exports: the same kernels, intermediates written out ------ */
 

@@ -52,6 +52,9 @@ def _load() -> ctypes.CDLL:
         "qlin_calibrate_input_scale": (st, [P, i32, i64, i64, P, P, sz, P]),
         "qlin_int8_outlier_forward": (st, [P, i32, i64, i64, P, P, i64, f32, P, P, P, sz, P]),
         "qlin_fp8_forward": (st, [P, i32, i64, i64, P, P, i32, i64, P, P, P, P, sz, P]),
+        "qlin_int8_outlier_prepare": (st, [P, i32, i64, i64, P, P, i64, f32, P, sz, P]),
+        "qlin_int8_outlier_gemm": (st, [i32, i64, i64, P, P, i64, P, P, P, sz, P]),
+        "qlin_fp8_gemm": (st, [i32, i64, i64, P, P, P, P, i32, i64, P, P, P, P]),
         "qlin_int8_prep": (st, [P, i32, i64, i64, f32, P, P, P, P, P, P, i64, P, sz, P]),
         "qlin_outlier_weights": (st, [P, P, i64, i64, P, P, i32, P, i64, P]),
         "qlin_int8_gemm_i32": (st, [P, P, i64, i64, i64, P, P]),
@@ -180,6 +183,39 @@ def qlin_int8_outlier_forward(X: torch.Tensor, Wq: torch.Tensor, w_scale: torch.
         ws = workspace(QLIN_OP_INT8_OUTLIER, M, N, K, X.device)
     _check(lib.qlin_int8_outlier_forward(_ptr(X), _dt(X), M, K, _ptr(Wq), _ptr(w_scale), N, float(threshold),
                                          _ptr(bias), _ptr(Y), _ptr(ws), ws.numel(), _stream(X.device)))
+    return Y
+
+
+def qlin_int8_outlier_prepare(X: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tensor, threshold: float,
+                              ws: torch.Tensor) -> None:
+    """Stage 1 of the LLM.int8 forward: outlier set, codes, scales, X_O, W_O into `ws`."""
+    M, K = X.shape
+    N = Wq.shape[0]
+    _check(lib.qlin_int8_outlier_prepare(_ptr(X), _dt(X), M, K, _ptr(Wq), _ptr(w_scale), N, float(threshold),
+                                         _ptr(ws), ws.numel(), _stream(X.device)))
+
+
+def qlin_int8_outlier_gemm(dtype: torch.dtype, M: int, K: int, Wq: torch.Tensor, w_scale: torch.Tensor,
+                           Y: torch.Tensor, ws: torch.Tensor, bias: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Stage 2 of the LLM.int8 forward: tcgen05 GEMM + fused epilogue, reading `ws`."""
+    N = Wq.shape[0]
+    dt = QLIN_BF16 if dtype == torch.bfloat16 else QLIN_F16
+    _check(lib.qlin_int8_outlier_gemm(dt, M, K, _ptr(Wq), _ptr(w_scale), N, _ptr(bias), _ptr(Y), _ptr(ws),
+                                      ws.numel(), _stream(Wq.device)))
+    return Y
+
+
+def qlin_fp8_gemm(Xq: torch.Tensor, s_x: Optional[torch.Tensor], Wq: torch.Tensor, w_scale: torch.Tensor,
+                  wmode: int, dtype: torch.dtype, x_scale: Optional[torch.Tensor] = None,
+                  bias: Optional[torch.Tensor] = None, Y: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """GEMM stage of the FP8 forward on codes from qlin_fp8_prep."""
+    M, K = Xq.shape
+    N = Wq.shape[0]
+    if Y is None:
+        Y = torch.empty((M, N), dtype=dtype, device=Xq.device)
+    dt = QLIN_BF16 if dtype == torch.bfloat16 else QLIN_F16
+    _check(lib.qlin_fp8_gemm(dt, M, K, _ptr(Xq), _ptr(s_x), _ptr(Wq), _ptr(w_scale), wmode, N, _ptr(x_scale),
+                             _ptr(bias), _ptr(Y), _stream(Xq.device)))
     return Y
 
 

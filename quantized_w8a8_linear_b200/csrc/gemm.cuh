@@ -50,111 +50,154 @@ struct GemmSmem {
   static constexpr int A_BYTES = GEMM_BM * GEMM_BK;
   static constexpr int B_BYTES = BN * GEMM_BK;
   static constexpr int TILE_BYTES = STAGES * (A_BYTES + B_BYTES);
-  static constexpr int BAR_BYTES = 8 * (2 * STAGES + 4 + 1) + 16;
-  static constexpr int TOTAL = 1024 + TILE_BYTES + BAR_BYTES;   // 1024: alignment slack
+  static constexpr int EPI_BYTES = static_cast<int>(sizeof(float) * 2 * BN + sizeof(uint32_t) * 16 * BN);
+  static constexpr int BAR_BYTES = 8 * (2 * STAGES + 4 + 2) + 16;
+  static constexpr int TOTAL = 1024 + TILE_BYTES + EPI_BYTES + BAR_BYTES;   // 1024: alignment slack
 };
 
-// 32 consecutive fp32 column values starting at n0 (0 past N).
-__device__ __forceinline__ void load_cols_f32(const float* p, int64_t n0, int64_t N, bool full, float (&o)[32]) {
-  if (full) {
-    const float4* q = reinterpret_cast<const float4*>(p + n0);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float4 v = __ldg(q + i);
-      o[4 * i] = v.x; o[4 * i + 1] = v.y; o[4 * i + 2] = v.z; o[4 * i + 3] = v.w;
+// Per-tile epilogue data staged in shared memory by the epilogue warps:
+// column scales, bias, and (LLM.int8) the tile's slice of the dequantised
+// outlier weight columns, up to 32 outliers as packed 16-bit pairs. All
+// lanes of a warp read the same word (a broadcast), so there are no bank
+// conflicts.
+template <int BN>
+struct EpiStage {
+  float sw[BN];
+  float bias[BN];
+  uint32_t wo[BN][16];
+};
+
+// Barrier among the epilogue threads, on an mbarrier (arrival count = the
+// epilogue thread count) so that the wait is bounded like every other wait.
+__device__ __forceinline__ bool epi_bar(uint64_t* bar, uint32_t& phase, volatile int* abort_flag) {
+  mbar_arrive(bar);
+  const bool ok = mbar_wait(bar, phase, abort_flag);
+  phase ^= 1u;
+  return ok;
+}
+
+template <typename TOut, int EPI, int BN>
+__device__ __forceinline__ void epi_stage(const EpiParams& p, EpiStage<BN>& es, int64_t n_base, int et, int cn,
+                                          int cnt) {
+  for (int j = et; j < BN; j += 32 * GEMM_EPI_WARPS) {
+    const int64_t n = n_base + j;
+    float sw = 0.0f, b = 0.0f;
+    if (n < p.N) {
+      if constexpr (EPI == EPI_INT8_OUTLIER) sw = __ldg(p.s_w + n);
+      if constexpr (EPI == EPI_FP8_ROWCOL) sw = to_f<__nv_bfloat16>(__ldg(p.s_w_bf16 + n));
+      if (p.bias != nullptr) b = to_f<TOut>(__ldg(p.bias + n));
     }
-  } else {
-#pragma unroll
-    for (int j = 0; j < 32; ++j) o[j] = (n0 + j < N) ? __ldg(p + n0 + j) : 0.0f;
+    es.sw[j] = sw;
+    es.bias[j] = b;
+  }
+  if (cn > 0) {
+    const int nq = cn / 8;   // 16-byte quads of 8 outlier values per column
+    for (int idx = et; idx < BN * nq; idx += 32 * GEMM_EPI_WARPS) {
+      const int j = idx / nq, qd = idx - j * nq;
+      const int64_t n = n_base + j;
+      uint4 v = make_uint4(0u, 0u, 0u, 0u);
+      if (n < p.N && qd * 8 < cnt) v = __ldg(reinterpret_cast<const uint4*>(p.W_O + n * p.ostride + qd * 8));
+      *reinterpret_cast<uint4*>(&es.wo[j][qd * 4]) = v;
+    }
   }
 }
 
-// 32 consecutive 16-bit column values (as float) starting at n0 (0 past N).
-template <typename T>
-__device__ __forceinline__ void load_cols_h(const uint16_t* p, int64_t n0, int64_t N, bool full, float (&o)[32]) {
-  if (full) {
-    const uint4* q = reinterpret_cast<const uint4*>(p + n0);
+template <typename TOut>
+__device__ __forceinline__ void store_chunk(const EpiParams& p, const float (&acc)[32], int64_t row, int64_t n0) {
+  const int64_t N = p.N;
+  uint16_t* y = reinterpret_cast<uint16_t*>(p.Y) + row * N + n0;
+  if (n0 + 32 <= N && (N & 7) == 0) {
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      uint16_t h[8];
-      unpack8(__ldg(q + i), h);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) o[8 * i + e] = to_f<T>(h[e]);
+      uint4 v;
+      v.x = pack2<TOut>(acc[8 * i + 0], acc[8 * i + 1]);
+      v.y = pack2<TOut>(acc[8 * i + 2], acc[8 * i + 3]);
+      v.z = pack2<TOut>(acc[8 * i + 4], acc[8 * i + 5]);
+      v.w = pack2<TOut>(acc[8 * i + 6], acc[8 * i + 7]);
+      reinterpret_cast<uint4*>(y)[i] = v;
     }
   } else {
 #pragma unroll
-    for (int j = 0; j < 32; ++j) o[j] = (n0 + j < N) ? to_f<T>(__ldg(p + n0 + j)) : 0.0f;
+    for (int j = 0; j < 32; ++j)
+      if (n0 + j < N) y[j] = from_f<TOut>(acc[j]);
   }
 }
 
-template <typename TOut, int EPI>
-__device__ __forceinline__ void epilogue_chunk(const EpiParams& p, const uint32_t (&r)[32], int64_t row,
-                                               int64_t n0, float sx, float alpha, int cnt) {
-  const int64_t N = p.N;
-  const bool full = (n0 + 32 <= N);
-  if constexpr (EPI == EPI_I32) {
-    int32_t* y = reinterpret_cast<int32_t*>(p.Y) + row * N + n0;
-    if (full && (N & 3) == 0) {
+// One accumulator tile, one thread per row: TMEM -> registers in chunks of
+// 32 columns, then y = acc * scales (+ outlier part) + bias -> Y.
+// CN: outlier columns handled from shared memory (0, 8, 16 or 32; a bucket
+// >= the count, zero-padded); CN < 0: more than 32 outliers, the weight
+// columns are read from global memory (correct for any count, not fast).
+template <typename TOut, int EPI, int BN, int CN>
+__device__ __forceinline__ void epi_tile(const EpiParams& p, const EpiStage<BN>& es, uint32_t t_row, int64_t row,
+                                         bool row_ok, int64_t n_base, float sx, float alpha, int cnt) {
+  constexpr int NX = CN > 0 ? CN : 1;
+  float xo[NX];
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
-        reinterpret_cast<int4*>(y)[i] = make_int4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
-    } else {
+  for (int i = 0; i < NX; ++i) xo[i] = 0.0f;
+  if constexpr (CN > 0) {
 #pragma unroll
-      for (int j = 0; j < 32; ++j)
-        if (n0 + j < N) y[j] = static_cast<int32_t>(r[j]);
+    for (int qd = 0; qd < CN / 8; ++qd) {
+      if (row_ok && qd * 8 < cnt) {
+        uint16_t h[8];
+        unpack8(*reinterpret_cast<const uint4*>(p.X_O + row * p.ostride + qd * 8), h);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) xo[qd * 8 + e] = to_f<TOut>(h[e]);
+      }
     }
-  } else {
-    float acc[32];
-    float cs[32];
-    if constexpr (EPI == EPI_INT8_OUTLIER) {
-      load_cols_f32(p.s_w, n0, N, full, cs);
+  }
+#pragma unroll 1
+  for (int c = 0; c < BN / 32; ++c) {
+    uint32_t r[32];
+    __syncwarp();
+    tmem_ld32(t_row + static_cast<uint32_t>(c * 32), r);
+    tmem_ld_wait();
+    const int64_t n0 = n_base + c * 32;
+    if (row_ok && n0 < p.N) {
+      if constexpr (EPI == EPI_I32) {
+        int32_t* y = reinterpret_cast<int32_t*>(p.Y) + row * p.N + n0;
+        if (n0 + 32 <= p.N && (p.N & 3) == 0) {
 #pragma unroll
-      for (int j = 0; j < 32; ++j) acc[j] = static_cast<float>(static_cast<int32_t>(r[j])) * (sx * cs[j]);
-      // floating-point outlier part: F[row, n] = sum_o X_O[row, o] * W_O[n, o]
-      for (int o0 = 0; o0 < cnt; o0 += 8) {
-        uint16_t xh[8];
-        unpack8(*reinterpret_cast<const uint4*>(p.X_O + row * p.ostride + o0), xh);
-        float xo[8];
+          for (int i = 0; i < 8; ++i)
+            reinterpret_cast<int4*>(y)[i] = make_int4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
+        } else {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) xo[e] = to_f<TOut>(xh[e]);
+          for (int j = 0; j < 32; ++j)
+            if (n0 + j < p.N) y[j] = static_cast<int32_t>(r[j]);
+        }
+      } else {
+        float acc[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-          if (full || n0 + j < N) {
-            uint16_t wh[8];
-            unpack8(__ldg(reinterpret_cast<const uint4*>(p.W_O + (n0 + j) * p.ostride + o0)), wh);
+          const int jj = c * 32 + j;
+          float a;
+          if constexpr (EPI == EPI_INT8_OUTLIER) a = static_cast<float>(static_cast<int32_t>(r[j])) * (sx * es.sw[jj]);
+          else if constexpr (EPI == EPI_FP8_TENSOR) a = __uint_as_float(r[j]) * alpha;
+          else a = __uint_as_float(r[j]) * (sx * es.sw[jj]);
+          if constexpr (CN > 0) {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) acc[j] = fmaf(xo[e], to_f<TOut>(wh[e]), acc[j]);
+            for (int qd = 0; qd < CN / 8; ++qd) {
+              uint16_t h[8];
+              unpack8(*reinterpret_cast<const uint4*>(&es.wo[jj][qd * 4]), h);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) a = fmaf(xo[qd * 8 + e], to_f<TOut>(h[e]), a);
+            }
           }
+          if constexpr (CN < 0) {
+            for (int o0 = 0; o0 < cnt; o0 += 8) {
+              uint16_t xh[8], wh[8];
+              unpack8(*reinterpret_cast<const uint4*>(p.X_O + row * p.ostride + o0), xh);
+              if (n0 + j < p.N) {
+                unpack8(__ldg(reinterpret_cast<const uint4*>(p.W_O + (n0 + j) * p.ostride + o0)), wh);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) a = fmaf(to_f<TOut>(xh[e]), to_f<TOut>(wh[e]), a);
+              }
+            }
+          }
+          acc[j] = a + es.bias[jj];
         }
+        store_chunk<TOut>(p, acc, row, n0);
       }
-    } else if constexpr (EPI == EPI_FP8_TENSOR) {
-#pragma unroll
-      for (int j = 0; j < 32; ++j) acc[j] = __uint_as_float(r[j]) * alpha;
-    } else {  // EPI_FP8_ROWCOL
-      load_cols_h<__nv_bfloat16>(p.s_w_bf16, n0, N, full, cs);
-#pragma unroll
-      for (int j = 0; j < 32; ++j) acc[j] = __uint_as_float(r[j]) * (sx * cs[j]);
-    }
-    if (p.bias != nullptr) {
-      load_cols_h<TOut>(p.bias, n0, N, full, cs);
-#pragma unroll
-      for (int j = 0; j < 32; ++j) acc[j] += cs[j];
-    }
-    uint16_t* y = reinterpret_cast<uint16_t*>(p.Y) + row * N + n0;
-    if (full && (N & 7) == 0) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        uint4 v;
-        v.x = pack2<TOut>(acc[8 * i + 0], acc[8 * i + 1]);
-        v.y = pack2<TOut>(acc[8 * i + 2], acc[8 * i + 3]);
-        v.z = pack2<TOut>(acc[8 * i + 4], acc[8 * i + 5]);
-        v.w = pack2<TOut>(acc[8 * i + 6], acc[8 * i + 7]);
-        reinterpret_cast<uint4*>(y)[i] = v;
-      }
-    } else {
-#pragma unroll
-      for (int j = 0; j < 32; ++j)
-        if (n0 + j < N) y[j] = from_f<TOut>(acc[j]);
     }
   }
 }
@@ -167,12 +210,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * L::A_BYTES;
-  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + L::TILE_BYTES);
+  EpiStage<BN>& es = *reinterpret_cast<EpiStage<BN>*>(smem + L::TILE_BYTES);
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + L::TILE_BYTES + L::EPI_BYTES);
   uint64_t* empty_bar = full_bar + STAGES;
   uint64_t* tfull_bar = empty_bar + STAGES;     // [2]
   uint64_t* tempty_bar = tfull_bar + 2;         // [2]
   uint64_t* drain_bar = tempty_bar + 2;         // [1]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain_bar + 1);
+  uint64_t* epi_mbar = drain_bar + 1;           // [1]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(epi_mbar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -193,6 +238,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       mbar_init(&tempty_bar[b], GEMM_EPI_WARPS);
     }
     mbar_init(drain_bar, 1);
+    mbar_init(epi_mbar, 32 * GEMM_EPI_WARPS);
     *abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -276,14 +322,24 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   } else {
     // ---------------- epilogue ----------------
     const int q = warp & 3;   // TMEM lane quarter this warp may access
+    const int et = threadIdx.x - 64;
     int cnt = 0;
     float alpha = 0.0f;
     if constexpr (EPI == EPI_INT8_OUTLIER) cnt = *p.count;
     if constexpr (EPI == EPI_FP8_TENSOR) alpha = __ldg(p.x_scale) * __ldg(p.w_scale);
+    const int cn = cnt == 0 ? 0 : cnt <= 8 ? 8 : cnt <= 16 ? 16 : cnt <= 32 ? 32 : -1;
     int acc = 0;
     uint32_t acc_phase = 0;
+    uint32_t bar_phase = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
       const int mb = tile % num_m, nb = tile / num_m;
+      const int64_t n_base = static_cast<int64_t>(nb) * BN;
+      if constexpr (EPI != EPI_I32) {
+        // the previous tile's readers are done with the staging area
+        if (!epi_bar(epi_mbar, bar_phase, abort_flag)) break;
+        epi_stage<TOut, EPI, BN>(p, es, n_base, et, cn, cnt);
+        if (!epi_bar(epi_mbar, bar_phase, abort_flag)) break;
+      }
       if (!mbar_wait(&tfull_bar[acc], acc_phase, abort_flag)) break;
       tc_fence_after();
       const int64_t row = static_cast<int64_t>(mb) * GEMM_BM + q * 32 + lane;
@@ -291,13 +347,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       float sx = 0.0f;
       if constexpr (EPI == EPI_INT8_OUTLIER || EPI == EPI_FP8_ROWCOL) sx = row_ok ? __ldg(p.s_x + row) : 0.0f;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
-#pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(t_row + static_cast<uint32_t>(c * 32), r);
-        tmem_ld_wait();
-        const int64_t n0 = static_cast<int64_t>(nb) * BN + c * 32;
-        if (row_ok && n0 < N) epilogue_chunk<TOut, EPI>(p, r, row, n0, sx, alpha, cnt);
+      if constexpr (EPI == EPI_INT8_OUTLIER) {
+        if (cn == 0) epi_tile<TOut, EPI, BN, 0>(p, es, t_row, row, row_ok, n_base, sx, alpha, cnt);
+        else if (cn == 8) epi_tile<TOut, EPI, BN, 8>(p, es, t_row, row, row_ok, n_base, sx, alpha, cnt);
+        else if (cn == 16) epi_tile<TOut, EPI, BN, 16>(p, es, t_row, row, row_ok, n_base, sx, alpha, cnt);
+        else if (cn == 32) epi_tile<TOut, EPI, BN, 32>(p, es, t_row, row, row_ok, n_base, sx, alpha, cnt);
+        else epi_tile<TOut, EPI, BN, -1>(p, es, t_row, row, row_ok, n_base, sx, alpha, cnt);
+      } else {
+        epi_tile<TOut, EPI, BN, 0>(p, es, t_row, row, row_ok, n_base, sx, alpha, cnt);
       }
       tc_fence_before();
       __syncwarp();

@@ -1,12 +1,10 @@
 // prep.cuh -- HBM-bound kernels around the GEMM:
-//   * k_outlier_flags: LLM.int8 outlier-column detection (any |x| > threshold
-//     in the column, over every token of the call) into a bitmap, with the
-//     last CTA compacting the bitmap into the ascending outlier list O, the
-//     outlier count and per-word prefix counts;
-//   * k_rowquant: per-row absmax (optionally excluding outlier columns),
-//     scale, and int8 or E4M3 codes, plus the exact copy of the outlier
-//     columns into X_O; it also quantises weights row by row;
-//   * k_gather_wo: dequantised outlier weight columns
+//   * k_prep_rows: per-row absmax, scale and int8 or E4M3 codes (activations
+//     and weights); for LLM.int8 activations the same cooperative launch also
+//     detects the outlier columns (any |x| > threshold in the column, over
+//     every token of the call), excludes them from the row absmax, copies
+//     them exactly into X_O and writes the outlier weight columns W_O;
+//   * k_gather_wo: dequantised outlier weight columns (standalone)
 //     W_O[j,o] = dtype(fp32(Wq[j,O[o]]) * s_w[j]) (the weight.to(dtype) *
 //     weight_scale rule of the Text-Encoder-FP8 page, "Format");
 //   * k_fp8_static: per-tensor static E4M3 activation codes;
@@ -16,41 +14,381 @@
 // Rows are read as 16-byte vectors of 8 elements (K % 8 == 0), coalesced
 // across the threads of a CTA.
 #pragma once
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace qlin {
 
 constexpr int PREP_THREADS = 128;
 
-// 8 flags (bit e set iff |x_e| > thr) for one 16-byte vector of 8 elements.
+// Running per-column maximum of |x| on raw 16-bit patterns: for finite fp16
+// or bf16 values, clearing the sign bit gives a pattern whose unsigned order
+// is the order of |x|, so two columns are handled per 32-bit max.
+__device__ __forceinline__ uint32_t umax16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// Running max of |x| over packed 16-bit pairs: the magnitude of the result is
+// the larger magnitude (its sign bit is meaningless and cleared at the end).
 template <typename T>
-__device__ __forceinline__ uint32_t outlier_bits8(const uint4& u, float thr) {
+__device__ __forceinline__ uint32_t absmax2(uint32_t m, uint32_t x);
+template <>
+__device__ __forceinline__ uint32_t absmax2<__nv_bfloat16>(uint32_t m, uint32_t x) {
+  uint32_t d;
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(m), "r"(x));
+  return d;
+}
+template <>
+__device__ __forceinline__ uint32_t absmax2<__half>(uint32_t m, uint32_t x) {
+  uint32_t d;
+  asm("max.xorsign.abs.f16x2 %0, %1, %2;" : "=r"(d) : "r"(m), "r"(x));
+  return d;
+}
+
+// Packed fp32 multiply (two IEEE round-to-nearest products per instruction).
+__device__ __forceinline__ unsigned long long mul_f32x2(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ unsigned long long pair_f32(uint32_t lo, uint32_t hi) {
+  return static_cast<unsigned long long>(lo) | (static_cast<unsigned long long>(hi) << 32);
+}
+
+__device__ __forceinline__ void colmax_accum(uint4& m, const uint4& u) {
+  m.x = umax16x2(m.x, u.x & 0x7FFF7FFFu);
+  m.y = umax16x2(m.y, u.y & 0x7FFF7FFFu);
+  m.z = umax16x2(m.z, u.z & 0x7FFF7FFFu);
+  m.w = umax16x2(m.w, u.w & 0x7FFF7FFFu);
+}
+
+// Outlier weight column value W_O[j,o] = dtype(fp32(Wq[j,O[o]]) * s_w[j]) for
+// o < count, 0 for count <= o < pad (the weight.to(dtype) * weight_scale rule).
+template <typename T>
+__device__ __forceinline__ void gather_wo_elem(const int8_t* __restrict__ Wq, const float* __restrict__ s_w,
+                                               int64_t K, const int32_t* __restrict__ O, int cnt, int pad,
+                                               uint16_t* __restrict__ W_O, int64_t ostride, int64_t t) {
+  const int64_t j = t / pad;
+  const int o = static_cast<int>(t - j * pad);
+  float val = 0.0f;
+  if (o < cnt) val = __fmul_rn(static_cast<float>(Wq[j * K + __ldg(O + o)]), __ldg(s_w + j));
+  W_O[j * ostride + o] = from_f<T>(val);
+}
+
+// Optional work folded into the row quantiser's launch: the outlier weight
+// columns W_O (N rows), grid-stride over N * pad.
+struct WoGather {
+  const int8_t* Wq;
+  const float* s_w;
+  int64_t N;
+  const int32_t* O;
+  uint16_t* W_O;
+};
+
+// Round-half-even of an fp32 value in (-2^22, 2^22) to an integer, read from
+// the low byte of t + 1.5 * 2^23: the add rounds to nearest even, and within
+// [2^23, 2^24) the float spacing is 1, so the low byte is the two's-complement
+// low byte of rne(t).
+__device__ __forceinline__ uint32_t rne_low_byte(float t) { return __float_as_uint(__fadd_rn(t, 12582912.0f)); }
+
+// 8 int8 codes of one vector, no outlier in it, normal scale (so |t| < 127.5
+// and no clamp is needed): code = rne(x * inv), one fp32 multiply (two
+// elements per instruction) and one fp32 add. The add is a scalar __fadd_rn on
+// purpose: a packed multiply followed by a packed add was measured to be
+// contracted into one fused multiply-add, which rounds ties differently.
+template <typename T>
+__device__ __forceinline__ uint2 quant8_int8_fast(const uint4& u, float inv) {
+  const unsigned long long inv2 = pair_f32(__float_as_uint(inv), __float_as_uint(inv));
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+  uint32_t f[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint32_t lo, hi;
+    if constexpr (std::is_same<T, __nv_bfloat16>::value) {
+      lo = w[i] << 16;
+      hi = w[i] & 0xFFFF0000u;
+    } else {
+      lo = __float_as_uint(to_f<T>(static_cast<uint16_t>(w[i] & 0xFFFFu)));
+      hi = __float_as_uint(to_f<T>(static_cast<uint16_t>(w[i] >> 16)));
+    }
+    const unsigned long long t = mul_f32x2(pair_f32(lo, hi), inv2);
+    f[2 * i] = rne_low_byte(__uint_as_float(static_cast<uint32_t>(t)));
+    f[2 * i + 1] = rne_low_byte(__uint_as_float(static_cast<uint32_t>(t >> 32)));
+  }
+  const uint32_t lo = __byte_perm(__byte_perm(f[0], f[1], 0x0040), __byte_perm(f[2], f[3], 0x0040), 0x5410);
+  const uint32_t hi = __byte_perm(__byte_perm(f[4], f[5], 0x0040), __byte_perm(f[6], f[7], 0x0040), 0x5410);
+  return make_uint2(lo, hi);
+}
+
+// Mask that keeps the non-outlier 16-bit lanes of word i (elements 2i, 2i+1)
+// of a vector whose outlier flags are the 8 bits of om.
+__device__ __forceinline__ uint32_t keep_mask(uint32_t om, int i) {
+  return (((om >> (2 * i)) & 1u) ? 0u : 0x0000FFFFu) | (((om >> (2 * i + 1)) & 1u) ? 0u : 0xFFFF0000u);
+}
+
+// ---------------------------------------------------------------------------
+// Row quantiser (persistent; a "row unit" of RW warps handles one row at a
+// time; each thread copies its own V 16-byte vectors of the unit's next
+// PF_DEPTH - 1 rows into private shared-memory slots with cp.async, so those
+// rows are in flight while the current one is quantised).
+//
+// CODE 0: int8 (QMAX 127), CODE 1: E4M3 (QMAX 448). SCALE_BF16: the stored
+// scale is bf16(absmax / QMAX) and the codes use that rounded value (the
+// [out,1] bf16 weight scales of the Text-Encoder-FP8 page).
+//
+// OUTL (LLM.int8 activations) reads X from HBM once, in one cooperative
+// launch:
+//   pass 1   every row is quantised with the absmax over its entries with
+//            |x| <= thr (entries above the threshold get code 0 and set their
+//            column's bit in the outlier bitmap). Because a column outside
+//            the outlier set O holds no entry above the threshold, this absmax
+//            equals the exact one (over k not in O) unless the maximum sits in
+//            a column of O; the raw absmax pattern is kept per row;
+//   barrier  bounded grid-wide barrier (flags and the counter are zeroed by
+//            the host before the launch; all CTAs are co-resident);
+//   compact  every CTA scans the bitmap into shared memory (per-word prefix
+//            counts); CTA 0 writes the ascending list O and the count;
+//   fix-up   per row, one warp reads the row's values in the O columns:
+//            copies them to X_O (zero-padded to a multiple of 8), sets their
+//            codes to 0, and if the largest of them that is <= thr reaches
+//            the kept absmax, requantises the whole row with the exact absmax;
+//   W_O      the dequantised outlier weight columns (wo.N > 0).
+// ---------------------------------------------------------------------------
+constexpr int RQ_THREADS = 256;
+constexpr int RQ_WARPS = RQ_THREADS / 32;
+constexpr int PF_DEPTH = 2;   // row slots per thread (current row + 1 in flight)
+
+struct PrepArgs {
+  int64_t M, K;
+  float thr;
+  uint32_t thr_bits;   // largest 16-bit |x| pattern with value <= thr
+  int rw;              // warps per row unit (1, 2, 4 or 8)
+  uint8_t* Q;
+  float* s_f32;
+  uint16_t* s_bf16;
+  uint16_t* amax_bits; // [M] pass-1 absmax pattern (OUTL)
+  uint32_t* flags;     // [NW] outlier bitmap (zero on entry for OUTL)
+  int32_t* O;          // [K]  ascending outlier columns (written by CTA 0)
+  int32_t* count;      // [1]
+  uint32_t* sync;      // grid barrier counter (zero on entry for OUTL)
+  uint16_t* X_O;
+  int64_t ostride;
+  WoGather wo;
+};
+
+// The (o+1)-th outlier column, from the shared bitmap and its word prefixes.
+__device__ __forceinline__ int outlier_col(const uint32_t* sflags, const int32_t* swpre, int NW, int o) {
+  int lo = 0, hi = NW - 1;   // largest w with swpre[w] <= o
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (swpre[mid] <= o) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo * 32 + static_cast<int>(__fns(sflags[lo], 0, o - swpre[lo] + 1));
+}
+
+template <typename T, int CODE>
+__device__ __forceinline__ uint2 quant_vec(const uint4& v, uint32_t om, float inv, bool fast, bool zero) {
+  if constexpr (CODE == 0) {
+    if (fast && om == 0u) return quant8_int8_fast<T>(v, inv);
+    uint16_t h[8];
+    unpack8(v, h);
+    uint32_t lo = 0, hi = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int q = (zero || ((om >> e) & 1u)) ? 0 : q_int(to_f<T>(h[e]), inv, 127);
+      const uint32_t b = static_cast<uint32_t>(q) & 0xFFu;
+      if (e < 4) lo |= b << (8 * e);
+      else hi |= b << (8 * (e - 4));
+    }
+    return make_uint2(lo, hi);
+  } else {
+    uint16_t h[8];
+    unpack8(v, h);
+    float t[8];
+    if (fast) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) t[e] = __fmul_rn(to_f<T>(h[e]), inv);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) t[e] = q_e4m3_in(to_f<T>(h[e]), inv);
+    }
+    uint2 out;
+    out.x = e4m3x2(t[0], t[1]) | (e4m3x2(t[2], t[3]) << 16);
+    out.y = e4m3x2(t[4], t[5]) | (e4m3x2(t[6], t[7]) << 16);
+    if (zero) out = make_uint2(0u, 0u);
+    return out;
+  }
+}
+
+// 8 flags: bit e set iff the 16-bit |x| pattern of element e exceeds tb.
+__device__ __forceinline__ uint32_t above_bits(const uint4& v, uint32_t tb) {
   uint16_t h[8];
-  unpack8(u, h);
+  unpack8(v, h);
   uint32_t m = 0;
 #pragma unroll
-  for (int e = 0; e < 8; ++e) m |= (fabsf(to_f<T>(h[e])) > thr ? 1u : 0u) << e;
+  for (int e = 0; e < 8; ++e) m |= ((h[e] & 0x7FFFu) > tb ? 1u : 0u) << e;
   return m;
 }
 
-// Compaction of the outlier bitmap by one CTA of PREP_THREADS threads:
-// wpre[w] = number of set bits in words [0, w); O lists the set columns in
-// ascending order; *count = total. NW <= 8 * PREP_THREADS.
-__device__ void compact_flags(const uint32_t* flags, int NW, int32_t* wpre, int32_t* O, int32_t* count) {
-  __shared__ int warp_tot[PREP_THREADS / 32];
-  const int tid = threadIdx.x;
-  const int per = (NW + PREP_THREADS - 1) / PREP_THREADS;   // <= 8
-  const int w0 = tid * per;
-  uint32_t words[8];
-  int local = 0;
+// Running packed |x| max of one vector into m2 (16-bit pairs).
+template <typename T>
+__device__ __forceinline__ uint32_t vec_absmax2(uint32_t m2, const uint4& x) {
+  return absmax2<T>(absmax2<T>(m2, x.x), absmax2<T>(absmax2<T>(x.y, x.z), x.w));
+}
+
+// Largest |x| pattern held in a packed pair accumulator.
+__device__ __forceinline__ uint32_t pair_max_bits(uint32_t m2) {
+  return max(m2 & 0x7FFFu, (m2 >> 16) & 0x7FFFu);
+}
+
+template <typename T, int V, int CODE, bool SCALE_BF16, bool OUTL>
+__global__ void __launch_bounds__(RQ_THREADS, 3) k_prep_rows(const T* __restrict__ X, const PrepArgs a) {
+  extern __shared__ uint32_t psm[];   // OUTL: sflags[NW], swpre[NW]
+  __shared__ uint32_t red[2][RQ_WARPS];
+  const int64_t M = a.M, K = a.K;
+  const int KV = static_cast<int>(K / 8);
+  const int NW = static_cast<int>((K + 31) / 32);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int rw = a.rw;
+  const int units = RQ_WARPS / rw;
+  const int unit = warp / rw;
+  const int ut = tid - unit * rw * 32;   // thread index inside the unit
+  const int UT = rw * 32;
+  uint32_t* sflags = psm;
+  int32_t* swpre = reinterpret_cast<int32_t*>(psm + NW);
+  constexpr float QMAX = CODE == 0 ? 127.0f : 448.0f;
+
+  // max over the unit (warp redux, then the unit's warps through shared
+  // memory, double-buffered so one named barrier per reduction suffices)
+  int rpar = 0;
+  auto unit_max = [&](uint32_t v) -> uint32_t {
+    v = __reduce_max_sync(0xffffffffu, v);
+    if (rw == 1) return v;
+    if (lane == 0) red[rpar][warp] = v;
+    asm volatile("bar.sync %0, %1;" ::"r"(1 + unit), "r"(UT) : "memory");
+    uint32_t m = 0;
+    for (int i = 0; i < rw; ++i) m = max(m, red[rpar][unit * rw + i]);
+    rpar ^= 1;
+    return m;
+  };
+
+  // ---------------- pass 1: rows of this unit, PF_DEPTH - 1 rows in flight ----------------
+  // staging: [PF_DEPTH][V][RQ_THREADS] 16-byte vectors, each thread only
+  // touches its own column, so cp.async.wait_group alone orders it
+  uint4* stage = reinterpret_cast<uint4*>(psm + ((OUTL ? 2 * NW : 0) + 3) / 4 * 4);
+  const int64_t first = static_cast<int64_t>(blockIdx.x) * units + unit;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * units;
+  auto issue = [&](int64_t r, int slot) {
+    const uint4* xr = reinterpret_cast<const uint4*>(X + (r < M ? r : 0) * K);
 #pragma unroll
-  for (int u = 0; u < 8; ++u) {
-    const int w = w0 + u;
-    words[u] = (u < per && w < NW) ? __ldcg(flags + w) : 0u;
-    local += __popc(words[u]);
+    for (int u = 0; u < V; ++u) {
+      const int idx = ut + u * UT;
+      cp_async16(&stage[(slot * V + u) * RQ_THREADS + tid], xr + idx, r < M && idx < KV);
+    }
+    cp_async_commit();
+  };
+#pragma unroll
+  for (int d = 0; d < PF_DEPTH - 1; ++d) issue(first + d * stride, d);
+  int slot = 0;
+  for (int64_t row = first; row < M; row += stride) {
+    issue(row + (PF_DEPTH - 1) * stride, (slot + PF_DEPTH - 1) % PF_DEPTH);
+    cp_async_wait<PF_DEPTH - 1>();   // this thread's copies of `row` have landed
+    uint4 cur[V];
+#pragma unroll
+    for (int u = 0; u < V; ++u) {
+      const int idx = ut + u * UT;
+      cur[u] = idx < KV ? stage[(slot * V + u) * RQ_THREADS + tid] : make_uint4(0u, 0u, 0u, 0u);
+    }
+    slot = (slot + 1) % PF_DEPTH;
+    uint32_t m2 = 0;
+#pragma unroll
+    for (int u = 0; u < V; ++u) m2 = vec_absmax2<T>(m2, cur[u]);
+    uint32_t mb = unit_max(pair_max_bits(m2));
+    uint32_t om[V];
+#pragma unroll
+    for (int u = 0; u < V; ++u) om[u] = 0u;
+    if (OUTL && mb > a.thr_bits) {
+      // some entry of this row exceeds the threshold: flag its column and
+      // leave it out of the absmax
+      uint32_t mm = 0;
+#pragma unroll
+      for (int u = 0; u < V; ++u) {
+        const int idx = ut + u * UT;
+        if (idx < KV) {
+          om[u] = above_bits(cur[u], a.thr_bits);
+          if (om[u]) atomicOr(a.flags + (idx >> 2), om[u] << ((idx & 3) * 8));
+        }
+        uint4 x = cur[u];
+        x.x &= keep_mask(om[u], 0);
+        x.y &= keep_mask(om[u], 1);
+        x.z &= keep_mask(om[u], 2);
+        x.w &= keep_mask(om[u], 3);
+        mm = vec_absmax2<T>(mm, x);
+      }
+      mb = unit_max(pair_max_bits(mm));
+    }
+    float s = to_f<T>(static_cast<uint16_t>(mb)) / QMAX;
+    if constexpr (SCALE_BF16) {
+      const uint16_t sb = __bfloat16_as_ushort(__float2bfloat16_rn(s));
+      s = __uint_as_float(static_cast<uint32_t>(sb) << 16);
+      if (ut == 0) a.s_bf16[row] = sb;
+    } else {
+      if (ut == 0) a.s_f32[row] = s;
+    }
+    if constexpr (OUTL) {
+      if (ut == 0) a.amax_bits[row] = static_cast<uint16_t>(mb);
+    }
+    const float inv = 1.0f / s;
+    const bool zero = (s == 0.0f);
+    // a normal scale keeps |x * inv| below QMAX + 1/2 for every entry in the absmax
+    const bool fast = s >= 1.17549435e-38f;
+    uint2* qr = reinterpret_cast<uint2*>(a.Q + row * K);
+#pragma unroll
+    for (int u = 0; u < V; ++u) {
+      const int idx = ut + u * UT;
+      if (idx < KV) qr[idx] = quant_vec<T, CODE>(cur[u], om[u], inv, fast, zero);
+    }
   }
-  // exclusive scan of `local` over the CTA
-  const int lane = tid & 31, warp = tid >> 5;
+  cp_async_wait<0>();
+  if constexpr (!OUTL) return;
+
+  // ---------------- grid barrier (bounded) ----------------
+  __shared__ int bar_ok;
+  __syncthreads();
+  if (tid == 0) {
+    __threadfence();
+    atomicAdd(a.sync, 1u);
+    int ok = 1;
+    const uint64_t t0 = globaltimer();
+    while (*reinterpret_cast<volatile uint32_t*>(a.sync) < gridDim.x) {
+      if (globaltimer() - t0 > g_wait_timeout_ns) {
+        atomicExch(&g_status, 6 /* QLIN_ERR_TIMEOUT */);
+        ok = 0;
+        break;
+      }
+    }
+    __threadfence();
+    bar_ok = ok;
+  }
+  __syncthreads();
+  if (!bar_ok) return;
+
+  // ---------------- compaction of the bitmap into shared memory ----------------
+  __shared__ int warp_tot[RQ_WARPS];
+  const int per = (NW + RQ_THREADS - 1) / RQ_THREADS;   // <= 4 (K <= 32768)
+  int local = 0;
+  for (int u = 0; u < per; ++u) {
+    const int w = tid * per + u;
+    if (w < NW) {
+      const uint32_t word = __ldcg(a.flags + w);
+      sflags[w] = word;
+      local += __popc(word);
+    }
+  }
   int incl = local;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -59,169 +397,91 @@ __device__ void compact_flags(const uint32_t* flags, int NW, int32_t* wpre, int3
   }
   if (lane == 31) warp_tot[warp] = incl;
   __syncthreads();
-  int base = 0;
-  for (int i = 0; i < warp; ++i) base += warp_tot[i];
+  int base = 0, cnt = 0;
+  for (int i = 0; i < RQ_WARPS; ++i) {
+    if (i < warp) base += warp_tot[i];
+    cnt += warp_tot[i];
+  }
   int run = base + incl - local;
-#pragma unroll
-  for (int u = 0; u < 8; ++u) {
-    const int w = w0 + u;
-    if (u < per && w < NW) {
-      wpre[w] = run;
-      uint32_t bits = words[u];
-      while (bits) {
-        const int b = __ffs(bits) - 1;
-        O[run++] = w * 32 + b;
-        bits &= bits - 1;
-      }
-    }
-  }
-  if (tid == PREP_THREADS - 1) *count = run;
-}
-
-// grid: (ceil(KV / PREP_THREADS), ceil(M / rows_per_block)); KV = K / 8.
-// flags and *done must be zero on entry.
-template <typename T>
-__global__ void __launch_bounds__(PREP_THREADS) k_outlier_flags(const T* __restrict__ X, int64_t M, int64_t K,
-                                                              float thr, int rows_per_block, uint32_t* flags,
-                                                              int32_t* wpre, int32_t* O, int32_t* count,
-                                                              uint32_t* done) {
-  const int64_t KV = K / 8;
-  const int64_t v = static_cast<int64_t>(blockIdx.x) * PREP_THREADS + threadIdx.x;
-  const int64_t r0 = static_cast<int64_t>(blockIdx.y) * rows_per_block;
-  const int64_t r1 = min(M, r0 + rows_per_block);
-  uint32_t mask = 0;
-  if (v < KV) {
-    const uint4* p = reinterpret_cast<const uint4*>(X + r0 * K) + v;
-    int64_t r = r0;
-    for (; r + 4 <= r1; r += 4) {
-      const uint4 a = ld_nc_v4(p), b = ld_nc_v4(p + KV), c = ld_nc_v4(p + 2 * KV), d = ld_nc_v4(p + 3 * KV);
-      mask |= outlier_bits8<T>(a, thr) | outlier_bits8<T>(b, thr) | outlier_bits8<T>(c, thr) |
-              outlier_bits8<T>(d, thr);
-      p += 4 * KV;
-    }
-    for (; r < r1; ++r, p += KV) mask |= outlier_bits8<T>(ld_nc_v4(p), thr);
-  }
-  // four consecutive threads hold the 32 columns of one bitmap word
-  uint32_t w = mask << ((v & 3) * 8);
-  w |= __shfl_xor_sync(0xffffffffu, w, 1);
-  w |= __shfl_xor_sync(0xffffffffu, w, 2);
-  if ((v & 3) == 0 && v < KV && w != 0u) atomicOr(flags + (v >> 2), w);
-
-  // the last CTA to finish compacts the bitmap
-  __shared__ int is_last;
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) is_last = (atomicAdd(done, 1u) == gridDim.x * gridDim.y - 1);
-  __syncthreads();
-  if (!is_last) return;
-  __threadfence();
-  compact_flags(flags, static_cast<int>((K + 31) / 32), wpre, O, count);
-}
-
-// One CTA per row. CODE 0: int8 (QMAX 127), CODE 1: E4M3 (QMAX 448).
-// SCALE_BF16: the stored scale is bf16(absmax / QMAX) and the codes use that
-// rounded value (the [out,1] bf16 weight scales of the Text-Encoder-FP8 page).
-// OUTL: columns flagged in `flags` are excluded from the absmax, get code 0,
-// and are copied exactly into X_O[row, o] (o = rank of the column in O), the
-// row zero-padded to a multiple of 8 outlier columns.
-template <typename T, int V, int CODE, bool SCALE_BF16, bool OUTL>
-__global__ void __launch_bounds__(PREP_THREADS) k_rowquant(const T* __restrict__ X, int64_t K, uint8_t* __restrict__ Q,
-                                                         float* __restrict__ s_f32, uint16_t* __restrict__ s_bf16,
-                                                         const uint32_t* __restrict__ flags,
-                                                         const int32_t* __restrict__ wpre,
-                                                         const int32_t* __restrict__ count_ptr,
-                                                         uint16_t* __restrict__ X_O, int64_t ostride) {
-  __shared__ float red[PREP_THREADS / 32];
-  const int64_t row = blockIdx.x;
-  const int64_t KV = K / 8;
-  const uint4* xr = reinterpret_cast<const uint4*>(X + row * K);
-  uint4 vals[V];
-  uint32_t om[V];
-  float amax = 0.0f;
-#pragma unroll
-  for (int u = 0; u < V; ++u) {
-    const int64_t idx = threadIdx.x + static_cast<int64_t>(u) * PREP_THREADS;
-    om[u] = 0u;
-    if (idx < KV) {
-      vals[u] = ld_nc_v4(xr + idx);
-      if constexpr (OUTL) om[u] = (__ldg(flags + (idx >> 2)) >> ((idx & 3) * 8)) & 0xFFu;
-      uint16_t h[8];
-      unpack8(vals[u], h);
-#pragma unroll
-      for (int e = 0; e < 8; ++e)
-        if (!((om[u] >> e) & 1u)) amax = fmaxf(amax, fabsf(to_f<T>(h[e])));
-    } else {
-      vals[u] = make_uint4(0, 0, 0, 0);
-    }
-  }
-  amax = warp_max(amax);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
-  __syncthreads();
-  amax = red[0];
-#pragma unroll
-  for (int w = 1; w < PREP_THREADS / 32; ++w) amax = fmaxf(amax, red[w]);
-
-  constexpr float QMAX = CODE == 0 ? 127.0f : 448.0f;
-  float s = amax / QMAX;
-  if constexpr (SCALE_BF16) {
-    const uint16_t sb = __bfloat16_as_ushort(__float2bfloat16_rn(s));
-    s = __uint_as_float(static_cast<uint32_t>(sb) << 16);
-    if (threadIdx.x == 0) s_bf16[row] = sb;
-  } else {
-    if (threadIdx.x == 0) s_f32[row] = s;
-  }
-  const float inv = 1.0f / s;
-  const bool zero = (s == 0.0f);
-
-#pragma unroll
-  for (int u = 0; u < V; ++u) {
-    const int64_t idx = threadIdx.x + static_cast<int64_t>(u) * PREP_THREADS;
-    if (idx < KV) {
-      uint16_t h[8];
-      unpack8(vals[u], h);
-      uint32_t lo = 0, hi = 0;
-      if constexpr (CODE == 0) {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int q = (zero || ((om[u] >> e) & 1u)) ? 0 : q_int(to_f<T>(h[e]), inv, 127);
-          const uint32_t b = static_cast<uint32_t>(q) & 0xFFu;
-          if (e < 4) lo |= b << (8 * e);
-          else hi |= b << (8 * (e - 4));
-        }
-      } else {
-        float t[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) t[e] = q_e4m3_in(to_f<T>(h[e]), inv);
-        lo = e4m3x2(t[0], t[1]) | (e4m3x2(t[2], t[3]) << 16);
-        hi = e4m3x2(t[4], t[5]) | (e4m3x2(t[6], t[7]) << 16);
-        if (zero) lo = hi = 0u;
-      }
-      *reinterpret_cast<uint2*>(Q + row * K + idx * 8) = make_uint2(lo, hi);
-      if constexpr (OUTL) {
-        if (om[u]) {
-          const uint32_t word = __ldg(flags + (idx >> 2));
-          const int base = __ldg(wpre + (idx >> 2));
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            if ((om[u] >> e) & 1u) {
-              const int bit = static_cast<int>((idx & 3) * 8) + e;
-              const int o = base + __popc(word & ((1u << bit) - 1u));
-              X_O[row * ostride + o] = h[e];
-            }
-          }
+  for (int u = 0; u < per; ++u) {
+    const int w = tid * per + u;
+    if (w < NW) {
+      swpre[w] = run;
+      if (blockIdx.x == 0) {
+        uint32_t bits = sflags[w];
+        int o = run;
+        while (bits) {
+          a.O[o++] = w * 32 + (__ffs(bits) - 1);
+          bits &= bits - 1;
         }
       }
+      run += __popc(sflags[w]);
     }
   }
-  if constexpr (OUTL) {
-    const int cnt = __ldg(count_ptr);
-    const int pad = (cnt + 7) & ~7;
-    for (int o = cnt + threadIdx.x; o < pad; o += PREP_THREADS) X_O[row * ostride + o] = 0;
+  if (blockIdx.x == 0 && tid == 0) *a.count = cnt;
+  __syncthreads();
+  if (cnt == 0) return;
+  const int pad = (cnt + 7) & ~7;
+
+  // ---------------- fix-up: one warp per row ----------------
+  for (int64_t row = static_cast<int64_t>(blockIdx.x) * RQ_WARPS + warp; row < M;
+       row += static_cast<int64_t>(gridDim.x) * RQ_WARPS) {
+    const T* xr = X + row * K;
+    uint32_t mo = 0;   // largest |x| pattern <= threshold among the outlier columns
+    for (int o = lane; o < pad; o += 32) {
+      uint16_t h = 0;
+      if (o < cnt) {
+        const int k = outlier_col(sflags, swpre, NW, o);
+        h = reinterpret_cast<const uint16_t*>(xr)[k];
+        a.Q[row * K + k] = 0;
+        const uint32_t ah = h & 0x7FFFu;
+        if (ah <= a.thr_bits) mo = max(mo, ah);
+      }
+      a.X_O[row * a.ostride + o] = h;
+    }
+    mo = __reduce_max_sync(0xffffffffu, mo);
+    const uint32_t mb = __ldcg(a.amax_bits + row);
+    if (mo >= mb) {
+      // the pass-1 absmax may sit in an outlier column: requantise exactly
+      uint32_t m = 0;
+      for (int64_t idx = lane; idx < KV; idx += 32) {
+        uint4 x = ld_nc_v4(reinterpret_cast<const uint4*>(xr) + idx);
+        const uint32_t omv = (sflags[idx >> 2] >> ((idx & 3) * 8)) & 0xFFu;
+        x.x &= keep_mask(omv, 0);
+        x.y &= keep_mask(omv, 1);
+        x.z &= keep_mask(omv, 2);
+        x.w &= keep_mask(omv, 3);
+        m = vec_absmax2<T>(m, x);
+      }
+      m = __reduce_max_sync(0xffffffffu, pair_max_bits(m));
+      const float s = to_f<T>(static_cast<uint16_t>(m)) / QMAX;
+      if (lane == 0) a.s_f32[row] = s;
+      const float inv = 1.0f / s;
+      const bool zero = (s == 0.0f), fast = s >= 1.17549435e-38f;
+      for (int64_t idx = lane; idx < KV; idx += 32) {
+        const uint4 x = ld_nc_v4(reinterpret_cast<const uint4*>(xr) + idx);
+        const uint32_t omv = (sflags[idx >> 2] >> ((idx & 3) * 8)) & 0xFFu;
+        *reinterpret_cast<uint2*>(a.Q + row * K + idx * 8) = quant_vec<T, CODE>(x, omv, inv, fast, zero);
+      }
+    }
+  }
+
+  // ---------------- outlier weight columns ----------------
+  if (a.wo.N > 0) {
+    const int64_t total = a.wo.N * pad;
+    for (int64_t t = static_cast<int64_t>(blockIdx.x) * RQ_THREADS + tid; t < total;
+         t += static_cast<int64_t>(gridDim.x) * RQ_THREADS) {
+      const int64_t j = t / pad;
+      const int o = static_cast<int>(t - j * pad);
+      float val = 0.0f;
+      if (o < cnt)
+        val = __fmul_rn(static_cast<float>(a.wo.Wq[j * K + outlier_col(sflags, swpre, NW, o)]), __ldg(a.wo.s_w + j));
+      a.wo.W_O[j * a.ostride + o] = from_f<T>(val);
+    }
   }
 }
 
-// W_O[j,o] = dtype(fp32(Wq[j,O[o]]) * s_w[j]) for o < count, 0 up to the
-// next multiple of 8. Grid-stride over N * pad.
+// Standalone outlier weight gather (grid-stride over N * pad).
 template <typename T>
 __global__ void __launch_bounds__(256) k_gather_wo(const int8_t* __restrict__ Wq, const float* __restrict__ s_w,
                                                  int64_t N, int64_t K, const int32_t* __restrict__ O,
@@ -232,13 +492,8 @@ __global__ void __launch_bounds__(256) k_gather_wo(const int8_t* __restrict__ Wq
   const int pad = (cnt + 7) & ~7;
   const int64_t total = N * pad;
   for (int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < total;
-       t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t j = t / pad;
-    const int o = static_cast<int>(t - j * pad);
-    float val = 0.0f;
-    if (o < cnt) val = __fmul_rn(static_cast<float>(Wq[j * K + __ldg(O + o)]), __ldg(s_w + j));
-    W_O[j * ostride + o] = from_f<T>(val);
-  }
+       t += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    gather_wo_elem<T>(Wq, s_w, K, O, cnt, pad, W_O, ostride, t);
 }
 
 // Static per-tensor E4M3 codes: Xq = e4m3(x * (1 / *x_scale)); all-zero

@@ -12,6 +12,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 
 #include "../../include/qlin.h"
 #include "common.cuh"
@@ -133,43 +134,104 @@ qlin_status launch_gemm(const void* A, const void* B, const EpiParams& ep, cudaS
   return check_cuda(cudaGetLastError(), "k_gemm launch");
 }
 
-// ---- row quantiser dispatch (V = 16-byte vectors per thread) ------------------
+// ---- row quantiser dispatch ---------------------------------------------------
+template <typename T, int V, int CODE, bool SBF16, bool OUTL>
+qlin_status launch_prep_v(const void* X, const PrepArgs& a, int sms, cudaStream_t st) {
+  auto kern = k_prep_rows<T, V, CODE, SBF16, OUTL>;
+  const int NW = static_cast<int>((a.K + 31) / 32);
+  const size_t smem = ((OUTL ? static_cast<size_t>(8 * NW) : 0) + 15) / 16 * 16 +
+                      static_cast<size_t>(PF_DEPTH) * V * RQ_THREADS * 16;
+  static bool attr_set[16] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 16 && !attr_set[dev]) {
+    qlin_status s0 = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024),
+                                "cudaFuncSetAttribute");
+    if (s0 != QLIN_OK) return s0;
+    attr_set[dev] = true;
+  }
+  int per_sm = 0;
+  qlin_status s = check_cuda(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, RQ_THREADS, smem),
+                             "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+  if (s != QLIN_OK) return s;
+  if (per_sm < 1) return fail(QLIN_ERR_UNSUPPORTED, "row quantiser does not fit on an SM");
+  const int units = RQ_WARPS / a.rw;
+  const int64_t want = (a.M + units - 1) / units;
+  const int64_t cap = static_cast<int64_t>(per_sm) * sms;
+  const unsigned grid = static_cast<unsigned>(want < cap ? want : cap);
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(RQ_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;   // the grid barrier needs every CTA resident
+  attr[0].val.cooperative = OUTL ? 1 : 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return check_cuda(cudaLaunchKernelEx(&cfg, kern, static_cast<const T*>(X), a), "k_prep_rows launch");
+}
+
 template <typename T, int CODE, bool SBF16, bool OUTL>
+qlin_status launch_prep(const void* X, PrepArgs a, cudaStream_t st) {
+  if (a.M == 0) return QLIN_OK;
+  DeviceInfo* d;
+  qlin_status s = device_info(&d);
+  if (s != QLIN_OK) return s;
+  const int64_t KV = a.K / 8;
+  int rw = 1;   // warps per row: the smallest power of two giving <= 6 vectors per lane
+  while (rw < 8 && (KV + 32 * rw - 1) / (32 * rw) > 6) rw *= 2;
+  a.rw = rw;
+  const int64_t per = (KV + 32 * rw - 1) / (32 * rw);
+  if (per <= 2) return launch_prep_v<T, 2, CODE, SBF16, OUTL>(X, a, d->sms, st);
+  if (per <= 4) return launch_prep_v<T, 4, CODE, SBF16, OUTL>(X, a, d->sms, st);
+  if (per <= 6) return launch_prep_v<T, 6, CODE, SBF16, OUTL>(X, a, d->sms, st);
+  if (per <= 8) return launch_prep_v<T, 8, CODE, SBF16, OUTL>(X, a, d->sms, st);
+  return launch_prep_v<T, 16, CODE, SBF16, OUTL>(X, a, d->sms, st);
+}
+
+// Largest 16-bit |x| pattern (of T) whose value is <= thr (thr > 0 finite):
+// |x| > thr exactly when the pattern of |x| exceeds it.
+template <typename T>
+uint32_t threshold_bits(float thr) {
+  auto val = [](uint32_t p) {
+    if constexpr (std::is_same<T, __nv_bfloat16>::value) return __bfloat162float(__ushort_as_bfloat16(static_cast<unsigned short>(p)));
+    else return __half2float(__ushort_as_half(static_cast<unsigned short>(p)));
+  };
+  const uint32_t top = std::is_same<T, __nv_bfloat16>::value ? 0x7F7Fu : 0x7BFFu;   // largest finite
+  if (val(top) <= thr) return top;
+  uint32_t lo = 0, hi = top;   // val(lo) <= thr < val(hi)
+  while (hi - lo > 1) {
+    const uint32_t mid = (lo + hi) / 2;
+    if (val(mid) <= thr) lo = mid;
+    else hi = mid;
+  }
+  return lo;
+}
+
+// Row quantiser without outlier handling (weights, FP8 dynamic activations,
+// int8 activations with the decomposition off).
+template <typename T, int CODE, bool SBF16>
 qlin_status launch_rowquant(const void* X, int64_t rows, int64_t K, uint8_t* Q, float* s32, uint16_t* sbf,
-                            const uint32_t* flags, const int32_t* wpre, const int32_t* count, uint16_t* X_O,
-                            int64_t ostride, cudaStream_t st) {
-  if (rows == 0) return QLIN_OK;
-  const int64_t per = (K / 8 + PREP_THREADS - 1) / PREP_THREADS;
-  const T* x = static_cast<const T*>(X);
-  const dim3 grid(static_cast<unsigned>(rows));
-#define QLIN_RQ(VV)                                                                                           \
-  k_rowquant<T, VV, CODE, SBF16, OUTL><<<grid, PREP_THREADS, 0, st>>>(x, K, Q, s32, sbf, flags, wpre, count, \
-                                                                      X_O, ostride)
-  if (per <= 1) QLIN_RQ(1);
-  else if (per <= 2) QLIN_RQ(2);
-  else if (per <= 4) QLIN_RQ(4);
-  else if (per <= 8) QLIN_RQ(8);
-  else if (per <= 12) QLIN_RQ(12);
-  else if (per <= 16) QLIN_RQ(16);
-  else if (per <= 24) QLIN_RQ(24);
-  else QLIN_RQ(32);
-#undef QLIN_RQ
-  return check_cuda(cudaGetLastError(), "k_rowquant launch");
+                            cudaStream_t st) {
+  PrepArgs a{};
+  a.M = rows; a.K = K; a.Q = Q; a.s_f32 = s32; a.s_bf16 = sbf;
+  return launch_prep<T, CODE, SBF16, false>(X, a, st);
 }
 
 // ---- LLM.int8 workspace layout -----------------------------------------------
 struct Int8Ws {
-  uint32_t* done;     // [1]  compaction counter
+  uint32_t* sync;     // [1]  grid barrier counter of the prep kernel
   int32_t* count;     // [1]
   uint32_t* flags;    // [NW]
-  int32_t* wpre;      // [NW]
   int32_t* O;         // [K]
   float* s_x;         // [M]
+  uint16_t* amax;     // [M] pass-1 absmax patterns of the prep kernel
   int8_t* Xq;         // [M,K]
   uint16_t* X_O;      // [M,ostride]
   uint16_t* W_O;      // [N,ostride]
   int64_t ostride;
-  size_t memset_bytes;  // zeroed each call: done, count, flags
+  size_t memset_bytes;  // zeroed each call: sync, count, flags
   size_t total;
 };
 
@@ -184,13 +246,13 @@ Int8Ws int8_layout(void* base, int64_t M, int64_t N, int64_t K, bool with_gemm_p
   };
   const int64_t NW = (K + 31) / 32;
   uint8_t* hdr = take(16 + 4 * NW);
-  w.done = reinterpret_cast<uint32_t*>(hdr);
+  w.sync = reinterpret_cast<uint32_t*>(hdr);
   w.count = reinterpret_cast<int32_t*>(hdr ? hdr + 4 : nullptr);
   w.flags = reinterpret_cast<uint32_t*>(hdr ? hdr + 16 : nullptr);
   w.memset_bytes = static_cast<size_t>(16 + 4 * NW);
-  w.wpre = reinterpret_cast<int32_t*>(take(4 * NW));
   w.O = reinterpret_cast<int32_t*>(take(4 * K));
   w.ostride = round_up(K, 8);
+  w.amax = reinterpret_cast<uint16_t*>(take(2 * M));
   if (with_gemm_parts) {
     w.s_x = reinterpret_cast<float*>(take(4 * M));
     w.Xq = reinterpret_cast<int8_t*>(take(static_cast<size_t>(M * K)));
@@ -205,21 +267,19 @@ bool decomposition_on(float thr) { return thr > 0.0f && !std::isinf(thr); }
 
 template <typename T>
 qlin_status int8_prep_impl(const void* X, int64_t M, int64_t K, float thr, const Int8Ws& w, int8_t* Xq, float* s_x,
-                           uint16_t* X_O, int64_t ostride, cudaStream_t st) {
-  qlin_status s = check_cuda(cudaMemsetAsync(w.done, 0, w.memset_bytes, st), "cudaMemsetAsync");
+                           uint16_t* X_O, int64_t ostride, cudaStream_t st,
+                           WoGather wo = WoGather{nullptr, nullptr, 0, nullptr, nullptr}) {
+  qlin_status s = check_cuda(cudaMemsetAsync(w.sync, 0, w.memset_bytes, st), "cudaMemsetAsync");
   if (s != QLIN_OK) return s;
-  if (decomposition_on(thr) && M > 0) {
-    const int rpb = 32;
-    const dim3 grid(static_cast<unsigned>((K / 8 + PREP_THREADS - 1) / PREP_THREADS),
-                    static_cast<unsigned>((M + rpb - 1) / rpb));
-    k_outlier_flags<T><<<grid, PREP_THREADS, 0, st>>>(static_cast<const T*>(X), M, K, thr, rpb, w.flags, w.wpre,
-                                                      w.O, w.count, w.done);
-    if ((s = check_cuda(cudaGetLastError(), "k_outlier_flags launch")) != QLIN_OK) return s;
-    return launch_rowquant<T, 0, false, true>(X, M, K, reinterpret_cast<uint8_t*>(Xq), s_x, nullptr, w.flags,
-                                              w.wpre, w.count, X_O, ostride, st);
+  if (M == 0) return QLIN_OK;
+  if (decomposition_on(thr)) {
+    PrepArgs a{};
+    a.M = M; a.K = K; a.thr = thr; a.thr_bits = threshold_bits<T>(thr);
+    a.Q = reinterpret_cast<uint8_t*>(Xq); a.s_f32 = s_x; a.amax_bits = w.amax;
+    a.flags = w.flags; a.O = w.O; a.count = w.count; a.sync = w.sync; a.X_O = X_O; a.ostride = ostride; a.wo = wo;
+    return launch_prep<T, 0, false, true>(X, a, st);
   }
-  return launch_rowquant<T, 0, false, false>(X, M, K, reinterpret_cast<uint8_t*>(Xq), s_x, nullptr, nullptr,
-                                             nullptr, nullptr, nullptr, 0, st);
+  return launch_rowquant<T, 0, false>(X, M, K, reinterpret_cast<uint8_t*>(Xq), s_x, nullptr, st);
 }
 
 qlin_status check_common(const void* X, qlin_dtype dt, int64_t M, int64_t K, int64_t N) {
@@ -306,20 +366,16 @@ qlin_status qlin_quantize_weight(const void* W, qlin_dtype wdt, int64_t N, int64
   const int64_t nvec = N * K / 8;
   switch (mode) {
     case QLIN_W_INT8_ROW:
-      QLIN_TRY(bf ? launch_rowquant<__nv_bfloat16, 0, false, false>(W, N, K, static_cast<uint8_t*>(Wq),
-                                                                     static_cast<float*>(w_scale), nullptr, nullptr,
-                                                                     nullptr, nullptr, nullptr, 0, st)
-                  : launch_rowquant<__half, 0, false, false>(W, N, K, static_cast<uint8_t*>(Wq),
-                                                             static_cast<float*>(w_scale), nullptr, nullptr, nullptr,
-                                                             nullptr, nullptr, 0, st));
+      QLIN_TRY(bf ? launch_rowquant<__nv_bfloat16, 0, false>(W, N, K, static_cast<uint8_t*>(Wq),
+                                                              static_cast<float*>(w_scale), nullptr, st)
+                  : launch_rowquant<__half, 0, false>(W, N, K, static_cast<uint8_t*>(Wq), static_cast<float*>(w_scale),
+                                                      nullptr, st));
       return ok();
     case QLIN_W_FP8_CHANNEL:
-      QLIN_TRY(bf ? launch_rowquant<__nv_bfloat16, 1, true, false>(W, N, K, static_cast<uint8_t*>(Wq), nullptr,
-                                                                    static_cast<uint16_t*>(w_scale), nullptr,
-                                                                    nullptr, nullptr, nullptr, 0, st)
-                  : launch_rowquant<__half, 1, true, false>(W, N, K, static_cast<uint8_t*>(Wq), nullptr,
-                                                            static_cast<uint16_t*>(w_scale), nullptr, nullptr,
-                                                            nullptr, nullptr, 0, st));
+      QLIN_TRY(bf ? launch_rowquant<__nv_bfloat16, 1, true>(W, N, K, static_cast<uint8_t*>(Wq), nullptr,
+                                                             static_cast<uint16_t*>(w_scale), st)
+                  : launch_rowquant<__half, 1, true>(W, N, K, static_cast<uint8_t*>(Wq), nullptr,
+                                                     static_cast<uint16_t*>(w_scale), st));
       return ok();
     case QLIN_W_FP8_TENSOR: {
       if (workspace == nullptr || ws_bytes < qlin_workspace_bytes(QLIN_OP_QUANTIZE_WEIGHT, 0, N, K))
@@ -451,15 +507,13 @@ qlin_status qlin_int8_gemm_i32(const int8_t* Xq, const int8_t* Wq, int64_t M, in
   return ok();
 }
 
-qlin_status qlin_int8_outlier_forward(const void* X, qlin_dtype xdt, int64_t M, int64_t K, const int8_t* Wq,
-                                      const float* w_scale, int64_t N, float threshold, const void* bias, void* Y,
-                                      void* workspace, size_t ws_bytes, void* stream) {
+qlin_status qlin_int8_outlier_prepare(const void* X, qlin_dtype xdt, int64_t M, int64_t K, const int8_t* Wq,
+                                      const float* w_scale, int64_t N, float threshold, void* workspace,
+                                      size_t ws_bytes, void* stream) {
   QLIN_TRY(check_common(X, xdt, M, K, N));
   if (M == 0 || N == 0) return ok();
   QLIN_REQ_PTR(Wq, "Wq");
   QLIN_REQ_PTR(w_scale, "w_scale");
-  QLIN_REQ_PTR(Y, "Y");
-  if (bias != nullptr && !aligned16(bias)) return fail(QLIN_ERR_ALIGNMENT, "bias is not 16-byte aligned");
   if (workspace == nullptr || ws_bytes < qlin_workspace_bytes(QLIN_OP_INT8_OUTLIER, M, N, K))
     return fail(QLIN_ERR_WORKSPACE, "workspace too small (need %zu bytes)",
                 qlin_workspace_bytes(QLIN_OP_INT8_OUTLIER, M, N, K));
@@ -469,22 +523,48 @@ qlin_status qlin_int8_outlier_forward(const void* X, qlin_dtype xdt, int64_t M, 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   Int8Ws w = int8_layout(workspace, M, N, K, true);
   const bool bf = (xdt == QLIN_BF16);
-  QLIN_TRY(bf ? int8_prep_impl<__nv_bfloat16>(X, M, K, threshold, w, w.Xq, w.s_x, w.X_O, w.ostride, st)
-              : int8_prep_impl<__half>(X, M, K, threshold, w, w.Xq, w.s_x, w.X_O, w.ostride, st));
-  if (decomposition_on(threshold)) {
-    if (bf)
-      k_gather_wo<__nv_bfloat16><<<d->sms * 4, 256, 0, st>>>(Wq, w_scale, N, K, w.O, w.count, w.W_O, w.ostride);
-    else
-      k_gather_wo<__half><<<d->sms * 4, 256, 0, st>>>(Wq, w_scale, N, K, w.O, w.count, w.W_O, w.ostride);
-    QLIN_TRY(check_cuda(cudaGetLastError(), "k_gather_wo launch"));
-  }
+  const WoGather wo{Wq, w_scale, N, w.O, w.W_O};
+  QLIN_TRY(bf ? int8_prep_impl<__nv_bfloat16>(X, M, K, threshold, w, w.Xq, w.s_x, w.X_O, w.ostride, st, wo)
+              : int8_prep_impl<__half>(X, M, K, threshold, w, w.Xq, w.s_x, w.X_O, w.ostride, st, wo));
+  (void)d;
+  return ok();
+}
+
+qlin_status qlin_int8_outlier_gemm(qlin_dtype xdt, int64_t M, int64_t K, const int8_t* Wq, const float* w_scale,
+                                   int64_t N, const void* bias, void* Y, void* workspace, size_t ws_bytes,
+                                   void* stream) {
+  if (xdt != QLIN_F16 && xdt != QLIN_BF16) return fail(QLIN_ERR_INVALID_ARG, "bad dtype");
+  if (M < 0 || N < 0) return fail(QLIN_ERR_INVALID_ARG, "negative size");
+  if (K <= 0 || K % 16 != 0) return fail(QLIN_ERR_ALIGNMENT, "K must be a positive multiple of 16");
+  if (K > kMaxK) return fail(QLIN_ERR_UNSUPPORTED, "K too large");
+  if (M == 0 || N == 0) return ok();
+  QLIN_REQ_PTR(Wq, "Wq");
+  QLIN_REQ_PTR(w_scale, "w_scale");
+  QLIN_REQ_PTR(Y, "Y");
+  if (bias != nullptr && !aligned16(bias)) return fail(QLIN_ERR_ALIGNMENT, "bias is not 16-byte aligned");
+  if (workspace == nullptr || ws_bytes < qlin_workspace_bytes(QLIN_OP_INT8_OUTLIER, M, N, K))
+    return fail(QLIN_ERR_WORKSPACE, "workspace too small");
+  QLIN_REQ_PTR(workspace, "workspace");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Int8Ws w = int8_layout(workspace, M, N, K, true);
   EpiParams ep{};
   ep.M = M; ep.N = N; ep.K = K; ep.Y = Y;
   ep.s_x = w.s_x; ep.s_w = w_scale; ep.bias = static_cast<const uint16_t*>(bias);
   ep.count = w.count; ep.X_O = w.X_O; ep.W_O = w.W_O; ep.ostride = w.ostride;
-  if (bf) QLIN_TRY((launch_gemm<0, EPI_INT8_OUTLIER, __nv_bfloat16>(w.Xq, Wq, ep, st, 1)));
+  if (xdt == QLIN_BF16) QLIN_TRY((launch_gemm<0, EPI_INT8_OUTLIER, __nv_bfloat16>(w.Xq, Wq, ep, st, 1)));
   else QLIN_TRY((launch_gemm<0, EPI_INT8_OUTLIER, __half>(w.Xq, Wq, ep, st, 2)));
   return ok();
+}
+
+qlin_status qlin_int8_outlier_forward(const void* X, qlin_dtype xdt, int64_t M, int64_t K, const int8_t* Wq,
+                                      const float* w_scale, int64_t N, float threshold, const void* bias, void* Y,
+                                      void* workspace, size_t ws_bytes, void* stream) {
+  QLIN_TRY(check_common(X, xdt, M, K, N));
+  if (M == 0 || N == 0) return ok();
+  QLIN_REQ_PTR(Y, "Y");
+  if (bias != nullptr && !aligned16(bias)) return fail(QLIN_ERR_ALIGNMENT, "bias is not 16-byte aligned");
+  QLIN_TRY(qlin_int8_outlier_prepare(X, xdt, M, K, Wq, w_scale, N, threshold, workspace, ws_bytes, stream));
+  return qlin_int8_outlier_gemm(xdt, M, K, Wq, w_scale, N, bias, Y, workspace, ws_bytes, stream);
 }
 
 qlin_status qlin_fp8_prep(const void* X, qlin_dtype xdt, int64_t M, int64_t K, const float* x_scale, uint8_t* Xq,
@@ -505,10 +585,47 @@ qlin_status qlin_fp8_prep(const void* X, qlin_dtype xdt, int64_t M, int64_t K, c
     return check_cuda(cudaGetLastError(), "k_fp8_static launch") == QLIN_OK ? ok() : QLIN_ERR_CUDA;
   }
   QLIN_REQ_PTR(s_x, "s_x");
-  QLIN_TRY(bf ? launch_rowquant<__nv_bfloat16, 1, false, false>(X, M, K, Xq, s_x, nullptr, nullptr, nullptr, nullptr,
-                                                                 nullptr, 0, st)
-              : launch_rowquant<__half, 1, false, false>(X, M, K, Xq, s_x, nullptr, nullptr, nullptr, nullptr,
-                                                         nullptr, 0, st));
+  QLIN_TRY(bf ? launch_rowquant<__nv_bfloat16, 1, false>(X, M, K, Xq, s_x, nullptr, st)
+              : launch_rowquant<__half, 1, false>(X, M, K, Xq, s_x, nullptr, st));
+  return ok();
+}
+
+qlin_status qlin_fp8_gemm(qlin_dtype xdt, int64_t M, int64_t K, const uint8_t* Xq, const float* s_x,
+                          const uint8_t* Wq, const void* w_scale, qlin_wmode wmode, int64_t N, const float* x_scale,
+                          const void* bias, void* Y, void* stream) {
+  if (xdt != QLIN_F16 && xdt != QLIN_BF16) return fail(QLIN_ERR_INVALID_ARG, "bad dtype");
+  if (wmode != QLIN_W_FP8_TENSOR && wmode != QLIN_W_FP8_CHANNEL)
+    return fail(QLIN_ERR_INVALID_ARG, "wmode must be QLIN_W_FP8_TENSOR or QLIN_W_FP8_CHANNEL");
+  if (M < 0 || N < 0) return fail(QLIN_ERR_INVALID_ARG, "negative size");
+  if (K <= 0 || K % 16 != 0) return fail(QLIN_ERR_ALIGNMENT, "K must be a positive multiple of 16");
+  if (K > kMaxK) return fail(QLIN_ERR_UNSUPPORTED, "K too large");
+  if (M == 0 || N == 0) return ok();
+  QLIN_REQ_PTR(Xq, "Xq");
+  QLIN_REQ_PTR(Wq, "Wq");
+  QLIN_REQ_PTR(w_scale, "w_scale");
+  QLIN_REQ_PTR(Y, "Y");
+  if (bias != nullptr && !aligned16(bias)) return fail(QLIN_ERR_ALIGNMENT, "bias is not 16-byte aligned");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  EpiParams ep{};
+  ep.M = M; ep.N = N; ep.K = K; ep.Y = Y;
+  ep.bias = static_cast<const uint16_t*>(bias);
+  const bool bf = (xdt == QLIN_BF16);
+  if (wmode == QLIN_W_FP8_TENSOR) {
+    if (x_scale == nullptr) return fail(QLIN_ERR_UNSUPPORTED, "per-tensor weight scales need a static x_scale");
+    QLIN_REQ_PTR(x_scale, "x_scale");
+    ep.x_scale = x_scale;
+    ep.w_scale = static_cast<const float*>(w_scale);
+    if (bf) QLIN_TRY((launch_gemm<1, EPI_FP8_TENSOR, __nv_bfloat16>(Xq, Wq, ep, st, 3)));
+    else QLIN_TRY((launch_gemm<1, EPI_FP8_TENSOR, __half>(Xq, Wq, ep, st, 4)));
+  } else {
+    if (x_scale != nullptr)
+      return fail(QLIN_ERR_UNSUPPORTED, "per-channel weight scales go with dynamic per-token activations");
+    QLIN_REQ_PTR(s_x, "s_x");
+    ep.s_x = s_x;
+    ep.s_w_bf16 = static_cast<const uint16_t*>(w_scale);
+    if (bf) QLIN_TRY((launch_gemm<1, EPI_FP8_ROWCOL, __nv_bfloat16>(Xq, Wq, ep, st, 5)));
+    else QLIN_TRY((launch_gemm<1, EPI_FP8_ROWCOL, __half>(Xq, Wq, ep, st, 6)));
+  }
   return ok();
 }
 
@@ -518,38 +635,18 @@ qlin_status qlin_fp8_forward(const void* X, qlin_dtype xdt, int64_t M, int64_t K
   QLIN_TRY(check_common(X, xdt, M, K, N));
   if (wmode != QLIN_W_FP8_TENSOR && wmode != QLIN_W_FP8_CHANNEL)
     return fail(QLIN_ERR_INVALID_ARG, "wmode must be QLIN_W_FP8_TENSOR or QLIN_W_FP8_CHANNEL");
-  if (M == 0 || N == 0) return ok();
-  QLIN_REQ_PTR(Wq, "Wq");
-  QLIN_REQ_PTR(w_scale, "w_scale");
-  QLIN_REQ_PTR(Y, "Y");
-  if (bias != nullptr && !aligned16(bias)) return fail(QLIN_ERR_ALIGNMENT, "bias is not 16-byte aligned");
-  if (workspace == nullptr || ws_bytes < qlin_workspace_bytes(QLIN_OP_FP8, M, N, K))
-    return fail(QLIN_ERR_WORKSPACE, "workspace too small");
-  QLIN_REQ_PTR(workspace, "workspace");
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  uint8_t* Xq = static_cast<uint8_t*>(workspace);
-  float* s_x = reinterpret_cast<float*>(Xq + round_up(M * K, 256));
   if (wmode == QLIN_W_FP8_TENSOR && x_scale == nullptr)
     return fail(QLIN_ERR_UNSUPPORTED, "per-tensor weight scales need a static x_scale");
   if (wmode == QLIN_W_FP8_CHANNEL && x_scale != nullptr)
     return fail(QLIN_ERR_UNSUPPORTED, "per-channel weight scales go with dynamic per-token activations (x_scale NULL)");
+  if (M == 0 || N == 0) return ok();
+  if (workspace == nullptr || ws_bytes < qlin_workspace_bytes(QLIN_OP_FP8, M, N, K))
+    return fail(QLIN_ERR_WORKSPACE, "workspace too small");
+  QLIN_REQ_PTR(workspace, "workspace");
+  uint8_t* Xq = static_cast<uint8_t*>(workspace);
+  float* s_x = reinterpret_cast<float*>(Xq + round_up(M * K, 256));
   QLIN_TRY(qlin_fp8_prep(X, xdt, M, K, x_scale, Xq, s_x, stream));
-  EpiParams ep{};
-  ep.M = M; ep.N = N; ep.K = K; ep.Y = Y;
-  ep.bias = static_cast<const uint16_t*>(bias);
-  const bool bf = (xdt == QLIN_BF16);
-  if (wmode == QLIN_W_FP8_TENSOR) {
-    ep.x_scale = x_scale;
-    ep.w_scale = static_cast<const float*>(w_scale);
-    if (bf) QLIN_TRY((launch_gemm<1, EPI_FP8_TENSOR, __nv_bfloat16>(Xq, Wq, ep, st, 3)));
-    else QLIN_TRY((launch_gemm<1, EPI_FP8_TENSOR, __half>(Xq, Wq, ep, st, 4)));
-  } else {
-    ep.s_x = s_x;
-    ep.s_w_bf16 = static_cast<const uint16_t*>(w_scale);
-    if (bf) QLIN_TRY((launch_gemm<1, EPI_FP8_ROWCOL, __nv_bfloat16>(Xq, Wq, ep, st, 5)));
-    else QLIN_TRY((launch_gemm<1, EPI_FP8_ROWCOL, __half>(Xq, Wq, ep, st, 6)));
-  }
-  return ok();
+  return qlin_fp8_gemm(xdt, M, K, Xq, s_x, Wq, w_scale, wmode, N, x_scale, bias, Y, stream);
 }
 
 }  // extern "C"

@@ -146,6 +146,9 @@ PREP_CASES = [
     ("boundary", 40, 64, [(0, 3, 6.0), (1, 5, 6.03125), (2, 7, -6.03125), (3, 9, -6.0)]),
     ("many", 130, 1024, [(i % 130, (i * 37) % 1024, 7.0 + i) for i in range(150)]),
     ("none", 77, 512, []),
+    # rows 1 and 2 have their largest sub-threshold value in outlier column 5
+    ("recompute", 64, 128, [(0, 5, 9.0), (1, 5, 5.9), (2, 5, -5.95), (3, 9, 6.0), (4, 9, 3.5)]),
+    ("wide", 96, 12288, [(0, 17, 40.0), (1, 17, 5.5), (50, 9000, -7.0), (95, 12287, 6.5)]),
 ]
 
 
@@ -239,6 +242,10 @@ def test_int8_forward_tiny_workload(q):
     (333, 520, 1024, [(i, (i * 13) % 1024, 9.0) for i in range(0, 333, 7)]),
     (1, 1, 16, [(0, 3, 7.0)]),
     (257, 129, 64, []),
+    (300, 520, 512, [(i * 3, 40 * i + 1, 6.5 + i) for i in range(12)]),        # 9..16 outliers
+    (300, 520, 512, [(i * 3, 16 * i + 3, -6.5 - i) for i in range(30)]),       # 17..32 outliers
+    (300, 520, 512, [(i * 3, 16 * i + 3, -6.5 - i) for i in range(32)]),       # exactly 32
+    (300, 520, 512, [(i * 3, 15 * i + 3, -6.5 - i) for i in range(33)]),       # 33: global path
 ])
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
 def test_int8_forward_ragged(q, M, N, K, outl, dtype):
