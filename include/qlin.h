@@ -193,6 +193,35 @@ QLIN_API qlin_status qlin_int8_gemm_i32(const int8_t *Xq, const int8_t *Wq, int6
 QLIN_API qlin_status qlin_fp8_prep(const void *X, qlin_dtype xdt, int64_t M, int64_t K,
                           const float *x_scale, uint8_t *Xq, float *s_x, void *stream);
 
+/* ---------------- LLM.int8 forward with built-in scratch ------------------------------ */
+
+/* Size of the library's built-in scratch array (64 MiB per device). */
+#define QLIN_NOALLOC_SCRATCH_BYTES (64LL * 1024 * 1024)
+
+/* The same LLM.int8 forward as qlin_int8_outlier_forward, for callers that
+ * cannot allocate device memory where they run the layer (for example a
+ * plugin whose host framework owns all device allocations, or a
+ * latency-critical path that must not call cudaMalloc, which can synchronise
+ * the device). It takes no workspace: its scratch is a file-scope device
+ * array of QLIN_NOALLOC_SCRATCH_BYTES inside the library, which every GPU
+ * that loads the library holds until the process exits. The model-card pages
+ * have no counterpart of this entry point.
+ *   - Shapes whose qlin_workspace_bytes(QLIN_OP_INT8_OUTLIER, M, N, K) exceeds
+ *     QLIN_NOALLOC_SCRATCH_BYTES are rejected with QLIN_ERR_UNSUPPORTED and a
+ *     message; nothing is enqueued. Arguments are otherwise validated as in
+ *     qlin_int8_outlier_forward.
+ *   - It calls no cudaMalloc, cudaFree or other allocating routine.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress); make that first call before any stream capture.
+ *   - Every call uses the same array and finds the previous call's contents
+ *     in it; the parts that must start at zero are cleared on the call's
+ *     stream. Calls ordered on one stream are safe; calls that may overlap on
+ *     the GPU (different streams or host threads) race on the array. */
+QLIN_API qlin_status qlin_int8_outlier_forward_noalloc(const void *X, qlin_dtype xdt, int64_t M, int64_t K,
+                                              const int8_t *Wq, const float *w_scale, int64_t N,
+                                              float threshold, const void *bias, void *Y,
+                                              void *stream);
+
 /* ---------------- status ------------------------------------------------------------ */
 
 /* Reads (and with reset != 0 clears) the device status word of the current

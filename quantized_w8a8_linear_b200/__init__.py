@@ -53,6 +53,7 @@ def _load() -> ctypes.CDLL:
         "qlin_int8_outlier_forward": (st, [P, i32, i64, i64, P, P, i64, f32, P, P, P, sz, P]),
         "qlin_fp8_forward": (st, [P, i32, i64, i64, P, P, i32, i64, P, P, P, P, sz, P]),
         "qlin_int8_outlier_prepare": (st, [P, i32, i64, i64, P, P, i64, f32, P, sz, P]),
+        "qlin_int8_outlier_forward_noalloc": (st, [P, i32, i64, i64, P, P, i64, f32, P, P, P]),
         "qlin_int8_outlier_gemm": (st, [i32, i64, i64, P, P, i64, P, P, P, sz, P]),
         "qlin_fp8_gemm": (st, [i32, i64, i64, P, P, P, P, i32, i64, P, P, P, P]),
         "qlin_int8_prep": (st, [P, i32, i64, i64, f32, P, P, P, P, P, P, i64, P, sz, P]),
@@ -183,6 +184,19 @@ def qlin_int8_outlier_forward(X: torch.Tensor, Wq: torch.Tensor, w_scale: torch.
         ws = workspace(QLIN_OP_INT8_OUTLIER, M, N, K, X.device)
     _check(lib.qlin_int8_outlier_forward(_ptr(X), _dt(X), M, K, _ptr(Wq), _ptr(w_scale), N, float(threshold),
                                          _ptr(bias), _ptr(Y), _ptr(ws), ws.numel(), _stream(X.device)))
+    return Y
+
+
+def qlin_int8_outlier_forward_noalloc(X: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tensor,
+                                      threshold: float = 6.0, bias: Optional[torch.Tensor] = None,
+                                      Y: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """LLM.int8 linear with the library's built-in scratch (no workspace argument)."""
+    M, K = X.shape
+    N = Wq.shape[0]
+    if Y is None:
+        Y = torch.empty((M, N), dtype=X.dtype, device=X.device)
+    _check(lib.qlin_int8_outlier_forward_noalloc(_ptr(X), _dt(X), M, K, _ptr(Wq), _ptr(w_scale), N,
+                                                 float(threshold), _ptr(bias), _ptr(Y), _stream(X.device)))
     return Y
 
 

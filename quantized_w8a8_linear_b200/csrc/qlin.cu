@@ -650,3 +650,62 @@ qlin_status qlin_fp8_forward(const void* X, qlin_dtype xdt, int64_t M, int64_t K
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// LLM.int8 forward without caller-provided scratch.
+//
+// Some callers cannot allocate device memory at the point where they run the
+// layer: a plugin whose host framework owns every allocation and gives the
+// plugin no allocator, or a latency-critical path where a cudaMalloc (which
+// may synchronise the device) is not acceptable. For them the scratch of the
+// LLM.int8 forward lives in this file-scope device array, created with the
+// module: every GPU that loads the library holds these bytes until the
+// process exits. All calls share it, and it keeps the previous call's
+// contents; the prepare stage clears the parts that must start at zero
+// (barrier counter, outlier count, outlier bitmap) on the stream of each
+// call, so calls that are ordered on one stream are correct, while calls
+// that may overlap on the GPU (other streams, other host threads) race on it.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) uint8_t g_noalloc_scratch[QLIN_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[16] = {};
+
+// Device address of g_noalloc_scratch on the current device, looked up once
+// per device (in host code the array's name is only a host-side stand-in).
+qlin_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 16) return fail(QLIN_ERR_CUDA, "cudaGetDevice failed");
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr)
+      return fail(QLIN_ERR_CUDA, "cudaGetSymbolAddress(no-alloc scratch): %s", cudaGetErrorString(e));
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return QLIN_OK;
+}
+}  // namespace
+
+extern "C" qlin_status qlin_int8_outlier_forward_noalloc(const void* X, qlin_dtype xdt, int64_t M, int64_t K,
+                                                         const int8_t* Wq, const float* w_scale, int64_t N,
+                                                         float threshold, const void* bias, void* Y, void* stream) {
+  QLIN_TRY(check_common(X, xdt, M, K, N));
+  if (M == 0 || N == 0) return ok();
+  const size_t need = qlin_workspace_bytes(QLIN_OP_INT8_OUTLIER, M, N, K);
+  if (need > static_cast<size_t>(QLIN_NOALLOC_SCRATCH_BYTES))
+    return fail(QLIN_ERR_UNSUPPORTED,
+                "qlin_int8_outlier_forward_noalloc: M=%lld N=%lld K=%lld needs %zu bytes of scratch, more than the "
+                "%lld bytes of its built-in array; use qlin_int8_outlier_forward with a workspace",
+                static_cast<long long>(M), static_cast<long long>(N), static_cast<long long>(K), need,
+                static_cast<long long>(QLIN_NOALLOC_SCRATCH_BYTES));
+  void* ws = nullptr;
+  QLIN_TRY(noalloc_scratch(&ws));
+  return qlin_int8_outlier_forward(X, xdt, M, K, Wq, w_scale, N, threshold, bias, Y, ws,
+                                   static_cast<size_t>(QLIN_NOALLOC_SCRATCH_BYTES), stream);
+}
+
+
