@@ -54,6 +54,8 @@ def parse_args():
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU-baseline sample budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", action="store_true", help="skip the FP8 workloads")
+    ap.add_argument("--workload", default=WORKLOAD,
+                    help="workload timed as the main line (default: the 1024^2 LLM.int8 DiT MLP)")
     return ap.parse_args()
 
 
@@ -358,12 +360,15 @@ def run_reference(args):
     return 0
 
 
-def workload_config():
-    return {"workload": "LLM.int8 DiT MLP at 1024^2: up [4352x3072]x[12288x3072]^T + down "
-                        "[4352x12288]x[3072x12288]^T, bf16, threshold 6.0",
-            "name": WORKLOAD, "tokens": 4352, "hidden": 3072, "mlp": 12288, "threshold": 6.0,
-            "l2": "flushed before every timed step (256 MiB write, outside the timed events)",
-            "parallelism": "replicas"}
+def workload_config(name=WORKLOAD, wl=None):
+    l2 = "flushed before every timed step (256 MiB write, outside the timed events)"
+    if name == WORKLOAD:
+        return {"workload": "LLM.int8 DiT MLP at 1024^2: up [4352x3072]x[12288x3072]^T + down "
+                            "[4352x12288]x[3072x12288]^T, bf16, threshold 6.0",
+                "name": WORKLOAD, "tokens": 4352, "hidden": 3072, "mlp": 12288, "threshold": 6.0,
+                "l2": l2, "parallelism": "replicas"}
+    shapes = " + ".join(f"{l.name} [{l.M}x{l.K}]x[{l.N}x{l.K}]^T" for l in wl.linears)
+    return {"workload": f"{wl.mode}: {shapes}", "name": name, "l2": l2, "parallelism": "replicas"}
 
 
 # ---------------------------------------------------------------------------
@@ -389,7 +394,7 @@ def main():
     import quantized_w8a8_linear_b200 as q
     import workloads
 
-    wl = workloads.get_workload(WORKLOAD)
+    wl = workloads.get_workload(args.workload)
     runs = [LinearRun(q, wl, lin, i, device) for i, lin in enumerate(wl.linears)]
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     torch.cuda.synchronize()
@@ -465,7 +470,7 @@ def main():
 
     # -------- CPU baseline (rank 0, N = 1) --------
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload == WORKLOAD:
         import oracle
         data = [(r.X_cpu, r.W_cpu, r.lin) for r in runs]
         sample = OracleSample(data)
@@ -482,7 +487,7 @@ def main():
             "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
             "warmup": max(3, args.warmup), "ms_per_step": ms_per_step, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "int8", "data": "synthetic",
-            "config": workload_config(), "impl": "qlin",
+            "config": workload_config(args.workload, wl), "impl": "qlin",
             "pct_of_int8_peak": 100.0 * value / world / peak_tops,
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": sum(r.launches() for r in runs) * args.steps,
