@@ -165,6 +165,28 @@ QLIN_API qlin_status qlin_fp8_gemm(qlin_dtype xdt, int64_t M, int64_t K, const u
                           qlin_wmode wmode, int64_t N, const float *x_scale, const void *bias,
                           void *Y, void *stream);
 
+/* W4A8 forward (Qwen-Image-fni8 page, "Format": int4 per-group weights,
+ * int8 activations, fp32 scales; group 128 along K):
+ *   activations: per-token int8, s_x[i] = absmax_i / 127 (no outlier split);
+ *   C_g = sum over the 128 columns of group g of Xq * Wq4 (int32, exact; the
+ *         int4 weights are unpacked to int8 in shared memory and contracted
+ *         with tcgen05 kind::i8, one TMEM accumulator per group);
+ *   Y   = dtype(s_x[i] * sum_g w_scale[j,g] * C_g + bias[j]), the group sum in
+ *         fp32 in ascending g.
+ * Wq4 uint8 [N, K/2] and w_scale fp32 [N, K/128] from
+ * qlin_quantize_weight(QLIN_W_INT4_G128). K must be a multiple of 128.
+ * workspace: qlin_workspace_bytes(QLIN_OP_W4A8, M, N, K). */
+QLIN_API qlin_status qlin_w4a8_forward(const void *X, qlin_dtype xdt, int64_t M, int64_t K,
+                              const uint8_t *Wq4, const float *w_scale, int64_t N,
+                              const void *bias, void *Y, void *workspace, size_t ws_bytes,
+                              void *stream);
+
+/* The GEMM stage of qlin_w4a8_forward, on int8 codes Xq [M,K] and fp32 s_x [M]
+ * (qlin_int8_prep with the threshold off writes them). */
+QLIN_API qlin_status qlin_w4a8_gemm(qlin_dtype xdt, int64_t M, int64_t K, const int8_t *Xq,
+                           const float *s_x, const uint8_t *Wq4, const float *w_scale,
+                           int64_t N, const void *bias, void *Y, void *stream);
+
 /* ---------------- parity exports: the same kernels, intermediates written out ------ */
 
 /* LLM.int8 activation prep alone. Outputs: Xq int8 [M,K]; s_x fp32 [M];
@@ -187,6 +209,12 @@ QLIN_API qlin_status qlin_outlier_weights(const int8_t *Wq, const float *w_scale
 /* Raw int8 GEMM: C[M,N] int32 = Xq[M,K] Wq[N,K]^T, exact (|C| <= K*127^2). */
 QLIN_API qlin_status qlin_int8_gemm_i32(const int8_t *Xq, const int8_t *Wq, int64_t M, int64_t N,
                                int64_t K, int32_t *C, void *stream);
+
+/* The int32 group partials C_g [M,N] of one group (0 <= group < K/128) as the
+ * W4A8 GEMM computes them (parity export; the same kernel, its output stage
+ * replaced by the export). */
+QLIN_API qlin_status qlin_w4a8_group_i32(const int8_t *Xq, const uint8_t *Wq4, int64_t M, int64_t N,
+                                int64_t K, int group, int32_t *C, void *stream);
 
 /* FP8 activation prep alone: Xq e4m3 [M,K]; s_x fp32 [M] (dynamic mode,
  * x_scale == NULL; ignored and may be NULL in static mode). */

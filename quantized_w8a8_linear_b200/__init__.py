@@ -56,6 +56,9 @@ def _load() -> ctypes.CDLL:
         "qlin_int8_outlier_forward_noalloc": (st, [P, i32, i64, i64, P, P, i64, f32, P, P, P]),
         "qlin_int8_outlier_gemm": (st, [i32, i64, i64, P, P, i64, P, P, P, sz, P]),
         "qlin_fp8_gemm": (st, [i32, i64, i64, P, P, P, P, i32, i64, P, P, P, P]),
+        "qlin_w4a8_forward": (st, [P, i32, i64, i64, P, P, i64, P, P, P, sz, P]),
+        "qlin_w4a8_gemm": (st, [i32, i64, i64, P, P, P, P, i64, P, P, P]),
+        "qlin_w4a8_group_i32": (st, [P, P, i64, i64, i64, i32, P, P]),
         "qlin_int8_prep": (st, [P, i32, i64, i64, f32, P, P, P, P, P, P, i64, P, sz, P]),
         "qlin_outlier_weights": (st, [P, P, i64, i64, P, P, i32, P, i64, P]),
         "qlin_int8_gemm_i32": (st, [P, P, i64, i64, i64, P, P]),
@@ -246,6 +249,44 @@ def qlin_fp8_forward(X: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tensor, w
     _check(lib.qlin_fp8_forward(_ptr(X), _dt(X), M, K, _ptr(Wq), _ptr(w_scale), wmode, N, _ptr(x_scale),
                                 _ptr(bias), _ptr(Y), _ptr(ws), ws.numel(), _stream(X.device)))
     return Y
+
+
+def qlin_w4a8_forward(X: torch.Tensor, Wq4: torch.Tensor, w_scale: torch.Tensor,
+                      bias: Optional[torch.Tensor] = None, Y: Optional[torch.Tensor] = None,
+                      ws: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """W4A8 linear: int4 per-group-128 weights, per-token int8 activations."""
+    M, K = X.shape
+    N = Wq4.shape[0]
+    if Y is None:
+        Y = torch.empty((M, N), dtype=X.dtype, device=X.device)
+    if ws is None:
+        ws = workspace(QLIN_OP_W4A8, M, N, K, X.device)
+    _check(lib.qlin_w4a8_forward(_ptr(X), _dt(X), M, K, _ptr(Wq4), _ptr(w_scale), N, _ptr(bias), _ptr(Y),
+                                 _ptr(ws), ws.numel(), _stream(X.device)))
+    return Y
+
+
+def qlin_w4a8_gemm(Xq: torch.Tensor, s_x: torch.Tensor, Wq4: torch.Tensor, w_scale: torch.Tensor,
+                   dtype: torch.dtype, bias: Optional[torch.Tensor] = None,
+                   Y: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """GEMM stage of the W4A8 forward on int8 codes and per-token scales."""
+    M, K = Xq.shape
+    N = Wq4.shape[0]
+    if Y is None:
+        Y = torch.empty((M, N), dtype=dtype, device=Xq.device)
+    dt = QLIN_BF16 if dtype == torch.bfloat16 else QLIN_F16
+    _check(lib.qlin_w4a8_gemm(dt, M, K, _ptr(Xq), _ptr(s_x), _ptr(Wq4), _ptr(w_scale), N, _ptr(bias), _ptr(Y),
+                              _stream(Xq.device)))
+    return Y
+
+
+def qlin_w4a8_group_i32(Xq: torch.Tensor, Wq4: torch.Tensor, group: int) -> torch.Tensor:
+    """int32 partials C_g [M,N] of one group, as the W4A8 GEMM computes them (parity export)."""
+    M, K = Xq.shape
+    N = Wq4.shape[0]
+    C = torch.empty((M, N), dtype=torch.int32, device=Xq.device)
+    _check(lib.qlin_w4a8_group_i32(_ptr(Xq), _ptr(Wq4), M, N, K, int(group), _ptr(C), _stream(Xq.device)))
+    return C
 
 
 def qlin_int8_prep(X: torch.Tensor, threshold: float = 6.0):

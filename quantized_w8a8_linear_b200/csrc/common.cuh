@@ -84,6 +84,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Barrier among a group of threads on an mbarrier whose arrival count is the
+// group's thread count, so that the wait is bounded like every other wait.
+__device__ __forceinline__ bool epi_bar(uint64_t* bar, uint32_t& phase, volatile int* abort_flag) {
+  mbar_arrive(bar);
+  const bool ok = mbar_wait(bar, phase, abort_flag);
+  phase ^= 1u;
+  return ok;
+}
+
 // ---------------------------------------------------------------------------
 // TMA (tiled, 2D, no multicast)
 // ---------------------------------------------------------------------------

@@ -67,14 +67,6 @@ struct EpiStage {
   uint32_t wo[BN][16];
 };
 
-// Barrier among the epilogue threads, on an mbarrier (arrival count = the
-// epilogue thread count) so that the wait is bounded like every other wait.
-__device__ __forceinline__ bool epi_bar(uint64_t* bar, uint32_t& phase, volatile int* abort_flag) {
-  mbar_arrive(bar);
-  const bool ok = mbar_wait(bar, phase, abort_flag);
-  phase ^= 1u;
-  return ok;
-}
 
 template <typename TOut, int EPI, int BN>
 __device__ __forceinline__ void epi_stage(const EpiParams& p, EpiStage<BN>& es, int64_t n_base, int et, int cn,

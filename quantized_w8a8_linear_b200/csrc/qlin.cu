@@ -17,6 +17,7 @@
 #include "../../include/qlin.h"
 #include "common.cuh"
 #include "gemm.cuh"
+#include "gemm_w4a8.cuh"
 #include "prep.cuh"
 
 using namespace qlin;
@@ -325,6 +326,7 @@ size_t qlin_workspace_bytes(qlin_op op, int64_t M, int64_t N, int64_t K) {
     case QLIN_OP_INT8_PREP:
       return int8_layout(nullptr, M, N, K, false).total;
     case QLIN_OP_FP8:
+    case QLIN_OP_W4A8:
       return static_cast<size_t>(round_up(M * K, 256) + round_up(4 * M, 256));
     case QLIN_OP_QUANTIZE_WEIGHT:
       return 256;
@@ -650,6 +652,124 @@ qlin_status qlin_fp8_forward(const void* X, qlin_dtype xdt, int64_t M, int64_t K
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// W4A8
+// ---------------------------------------------------------------------------
+namespace {
+
+qlin_status make_tmap_bytes(CUtensorMap* m, const void* base, int64_t rows, int64_t row_bytes, int box_inner,
+                            int box_rows, CUtensorMapSwizzle sw) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc;
+  qlin_status s = get_encode(&enc);
+  if (s != QLIN_OK) return s;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(QLIN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return QLIN_OK;
+}
+
+template <typename TOut>
+qlin_status launch_w4a8(const int8_t* Xq, const uint8_t* Wq4, const W4Params& wp, cudaStream_t st) {
+  DeviceInfo* d;
+  qlin_status s = device_info(&d);
+  if (s != QLIN_OK) return s;
+  CUtensorMap ta, tb;
+  if ((s = make_tmap_bytes(&ta, Xq, wp.M, wp.K, W4_G, W4_BM, CU_TENSOR_MAP_SWIZZLE_128B)) != QLIN_OK) return s;
+  if ((s = make_tmap_bytes(&tb, Wq4, wp.N, wp.K / 2, W4_G / 2, W4_BN, CU_TENSOR_MAP_SWIZZLE_NONE)) != QLIN_OK)
+    return s;
+  auto kern = k_gemm_w4a8<TOut>;
+  static bool attr_set[16] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 16 && !attr_set[dev]) {
+    s = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, W4Smem::TOTAL),
+                   "cudaFuncSetAttribute");
+    if (s != QLIN_OK) return s;
+    attr_set[dev] = true;
+  }
+  const int64_t tiles = ((wp.M + W4_BM - 1) / W4_BM) * ((wp.N + W4_BN - 1) / W4_BN);
+  const int grid = static_cast<int>(tiles < d->sms ? tiles : d->sms);
+  kern<<<grid, W4_THREADS, W4Smem::TOTAL, st>>>(ta, tb, wp);
+  return check_cuda(cudaGetLastError(), "k_gemm_w4a8 launch");
+}
+
+qlin_status check_w4(const void* Xq, const void* Wq4, const float* w_scale, int64_t M, int64_t N, int64_t K) {
+  if (M < 0 || N < 0) return fail(QLIN_ERR_INVALID_ARG, "negative size");
+  if (K <= 0 || K % W4_G != 0) return fail(QLIN_ERR_ALIGNMENT, "W4A8 needs K a positive multiple of 128");
+  if (K > kMaxK) return fail(QLIN_ERR_UNSUPPORTED, "K too large");
+  if (M == 0 || N == 0) return QLIN_OK;
+  QLIN_REQ_PTR(Xq, "Xq");
+  QLIN_REQ_PTR(Wq4, "Wq4");
+  QLIN_REQ_PTR(w_scale, "w_scale");
+  return QLIN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+qlin_status qlin_w4a8_gemm(qlin_dtype xdt, int64_t M, int64_t K, const int8_t* Xq, const float* s_x,
+                           const uint8_t* Wq4, const float* w_scale, int64_t N, const void* bias, void* Y,
+                           void* stream) {
+  if (xdt != QLIN_F16 && xdt != QLIN_BF16) return fail(QLIN_ERR_INVALID_ARG, "bad dtype");
+  QLIN_TRY(check_w4(Xq, Wq4, w_scale, M, N, K));
+  if (M == 0 || N == 0) return ok();
+  QLIN_REQ_PTR(s_x, "s_x");
+  QLIN_REQ_PTR(Y, "Y");
+  if (bias != nullptr && !aligned16(bias)) return fail(QLIN_ERR_ALIGNMENT, "bias is not 16-byte aligned");
+  W4Params wp{};
+  wp.M = M; wp.N = N; wp.K = K; wp.Y = Y; wp.s_x = s_x; wp.s_w = w_scale;
+  wp.bias = static_cast<const uint16_t*>(bias); wp.dbg = nullptr; wp.dbg_group = -1;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (xdt == QLIN_BF16) QLIN_TRY(launch_w4a8<__nv_bfloat16>(Xq, Wq4, wp, st));
+  else QLIN_TRY(launch_w4a8<__half>(Xq, Wq4, wp, st));
+  return ok();
+}
+
+qlin_status qlin_w4a8_group_i32(const int8_t* Xq, const uint8_t* Wq4, int64_t M, int64_t N, int64_t K, int group,
+                                int32_t* C, void* stream) {
+  if (M < 0 || N < 0) return fail(QLIN_ERR_INVALID_ARG, "negative size");
+  if (K <= 0 || K % W4_G != 0) return fail(QLIN_ERR_ALIGNMENT, "W4A8 needs K a positive multiple of 128");
+  if (K > kMaxK) return fail(QLIN_ERR_UNSUPPORTED, "K too large");
+  if (group < 0 || group >= K / W4_G) return fail(QLIN_ERR_INVALID_ARG, "group out of range");
+  if (M == 0 || N == 0) return ok();
+  QLIN_REQ_PTR(Xq, "Xq");
+  QLIN_REQ_PTR(Wq4, "Wq4");
+  QLIN_REQ_PTR(C, "C");
+  W4Params wp{};
+  wp.M = M; wp.N = N; wp.K = K; wp.Y = nullptr; wp.s_x = nullptr; wp.s_w = nullptr; wp.bias = nullptr;
+  wp.dbg = C; wp.dbg_group = group;
+  QLIN_TRY(launch_w4a8<__nv_bfloat16>(Xq, Wq4, wp, static_cast<cudaStream_t>(stream)));
+  return ok();
+}
+
+qlin_status qlin_w4a8_forward(const void* X, qlin_dtype xdt, int64_t M, int64_t K, const uint8_t* Wq4,
+                              const float* w_scale, int64_t N, const void* bias, void* Y, void* workspace,
+                              size_t ws_bytes, void* stream) {
+  QLIN_TRY(check_common(X, xdt, M, K, N));
+  if (K % W4_G != 0) return fail(QLIN_ERR_ALIGNMENT, "W4A8 needs K a multiple of 128");
+  if (M == 0 || N == 0) return ok();
+  if (workspace == nullptr || ws_bytes < qlin_workspace_bytes(QLIN_OP_W4A8, M, N, K))
+    return fail(QLIN_ERR_WORKSPACE, "workspace too small");
+  QLIN_REQ_PTR(workspace, "workspace");
+  int8_t* Xq = static_cast<int8_t*>(workspace);
+  float* s_x = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + round_up(M * K, 256));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (xdt == QLIN_BF16)
+    QLIN_TRY(launch_rowquant<__nv_bfloat16, 0, false>(X, M, K, reinterpret_cast<uint8_t*>(Xq), s_x, nullptr, st));
+  else
+    QLIN_TRY(launch_rowquant<__half, 0, false>(X, M, K, reinterpret_cast<uint8_t*>(Xq), s_x, nullptr, st));
+  return qlin_w4a8_gemm(xdt, M, K, Xq, s_x, Wq4, w_scale, N, bias, Y, stream);
+}
+
+}  // extern "C"
+
 
 // ---------------------------------------------------------------------------
 // LLM.int8 forward without caller-provided scratch.

@@ -388,3 +388,60 @@ def test_fp8_dynamic_text_encoder_full_size(q, li):
     rows = sample_rows(lin.M, n=12, seed=li, must=[0, 5])
     r = oracle.fp8_forward(X, rq, rs, x_scale=None, rows=rows)
     assert_rows_close(Y, r, rows=rows, extra=EXTRA_FP8, what=lin.name)
+
+
+# ---------------------------------------------------------------------------
+# W4A8: int4 per-group-128 weights, per-token int8 activations
+# ---------------------------------------------------------------------------
+
+def _unpack_int4(packed: np.ndarray, K: int) -> np.ndarray:
+    lo = (packed & 0x0F).astype(np.int16)
+    hi = (packed >> 4).astype(np.int16)
+    q = np.empty((packed.shape[0], K), np.int64)
+    q[:, 0::2] = np.where(lo >= 8, lo - 16, lo)
+    q[:, 1::2] = np.where(hi >= 8, hi - 16, hi)
+    return q
+
+
+@pytest.mark.parametrize("M,N,K", [(64, 128, 128), (200, 300, 256), (129, 257, 1024), (333, 520, 3072)])
+def test_w4a8_group_int32_exact(q, M, N, K):
+    X = rand_x(M, K, M + K)
+    W = rand_w(N, K, N + K)
+    Wq4, sw = q.qlin_quantize_weight(dev(W), q.QLIN_W_INT4_G128)
+    p = q.qlin_int8_prep(dev(X), 0.0)
+    Xq = p["Xq"]
+    u = _unpack_int4(Wq4.cpu().numpy(), K)
+    xq = Xq.cpu().numpy().astype(np.int64)
+    for g in sorted({0, K // 128 - 1, (K // 128) // 2}):
+        C = q.qlin_w4a8_group_i32(Xq, Wq4, g).cpu().numpy().astype(np.int64)
+        sl = slice(g * 128, (g + 1) * 128)
+        assert np.array_equal(C, xq[:, sl] @ u[:, sl].T), g
+
+
+@pytest.mark.parametrize("M,N,K", [(64, 128, 128), (200, 300, 256), (129, 257, 1024), (333, 520, 3072)])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+def test_w4a8_forward(q, M, N, K, dtype):
+    X = rand_x(M, K, M + 2 * K, dtype, [(1, 5, 30.0)])
+    W = rand_w(N, K, N + 3, dtype)
+    bias = (torch.randn(N, generator=torch.Generator().manual_seed(4)) * 0.1).to(dtype)
+    Wq4, sw = q.qlin_quantize_weight(dev(W), q.QLIN_W_INT4_G128)
+    rq, rs = oracle.quantize_weight(W, "int4_g128")
+    assert np.array_equal(Wq4.cpu().numpy(), rq) and np.array_equal(sw.cpu().numpy(), rs)
+    Y = q.qlin_w4a8_forward(dev(X), Wq4, sw, bias=dev(bias))
+    r = oracle.w4a8_forward(X, rq, rs, group=128, bias=bias)
+    assert_rows_close(Y, r, extra=EXTRA_FP8, what=f"w4a8 {M}x{N}x{K}")
+
+
+def test_w4a8_dit2048_mlp_up_full_size(q):
+    """One DiT block's MLP up-projection at 2048^2 (16640 tokens), full size,
+    outputs on a sample of rows."""
+    wl = workloads.get_workload("dit2048_block_w4a8")
+    lin = wl.linears[2]
+    X, W, bias = workloads.make_linear(wl, lin, index=2)
+    Wq4, sw = q.qlin_quantize_weight(dev(W), q.QLIN_W_INT4_G128)
+    rq, rs = oracle.quantize_weight(W, "int4_g128")
+    assert np.array_equal(Wq4.cpu().numpy(), rq) and np.array_equal(sw.cpu().numpy(), rs)
+    Y = q.qlin_w4a8_forward(dev(X), Wq4, sw)
+    rows = sample_rows(lin.M, n=8, seed=5)
+    r = oracle.w4a8_forward(X, rq, rs, group=128, rows=rows)
+    assert_rows_close(Y, r, rows=rows, extra=EXTRA_FP8, what="w4a8 2048^2 up")
