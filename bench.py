@@ -53,7 +53,7 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU-baseline sample budget")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-secondary", action="store_true", help="skip the FP8 workloads")
+    ap.add_argument("--no-secondary", action="store_true", help="skip the secondary workloads")
     ap.add_argument("--workload", default=WORKLOAD,
                     help="workload timed as the main line (default: the 1024^2 LLM.int8 DiT MLP)")
     return ap.parse_args()
@@ -180,6 +180,11 @@ class LinearRun:
             self.ws = torch.empty(n, dtype=torch.uint8, device=device)
             # algorithmic prep bytes: X read (2 B) + Xq write (1 B) per element
             self.prep_bytes = 3.0 * M * K
+        elif self.mode == "w4a8":
+            self.Wq, self.s_w = q.qlin_quantize_weight(Wd, q.QLIN_W_INT4_G128)
+            self.Xq = torch.empty((M, K), dtype=torch.int8, device=device)
+            self.s_x = torch.empty((M,), dtype=torch.float32, device=device)
+            self.prep_bytes = 3.0 * M * K
         else:
             wmode = q.QLIN_W_FP8_TENSOR if self.mode == "fp8_static" else q.QLIN_W_FP8_CHANNEL
             self.wmode = wmode
@@ -196,6 +201,8 @@ class LinearRun:
         q = self.q
         if self.mode == "int8_outlier":
             q.qlin_int8_outlier_prepare(self.X, self.Wq, self.s_w, 6.0, self.ws)
+        elif self.mode == "w4a8":
+            q.qlin_w4a8_prep(self.X, self.Xq, self.s_x)
         else:
             q._check(q.lib.qlin_fp8_prep(q._ptr(self.X), q._dt(self.X), self.M, self.K, q._ptr(self.x_scale),
                                          q._ptr(self.Xq), q._ptr(self.s_x), q._stream(self.X.device)))
@@ -204,6 +211,8 @@ class LinearRun:
         q = self.q
         if self.mode == "int8_outlier":
             q.qlin_int8_outlier_gemm(self.dtype, self.M, self.K, self.Wq, self.s_w, self.Y, self.ws)
+        elif self.mode == "w4a8":
+            q.qlin_w4a8_gemm(self.Xq, self.s_x, self.Wq, self.s_w, self.dtype, Y=self.Y)
         else:
             q.qlin_fp8_gemm(self.Xq, self.s_x, self.Wq, self.s_w, self.wmode, self.dtype, x_scale=self.x_scale,
                             Y=self.Y)
@@ -451,10 +460,10 @@ def main():
     e2e = {"value": ops_step / (e2e_ms * 1e-3) / 1e12 * world, "unit": "TOPS", "h2d_bytes_per_step": h2d,
            "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
-    # -------- secondary workloads (FP8), rank-local, reported beside --------
+    # -------- secondary workloads (FP8, 2048^2 DiT block), rank-local, reported beside --------
     secondary = {}
     if not args.no_secondary:
-        for name in ("dit1024_fp8_static_qkv", "te_fp8_dynamic_mlp"):
+        for name in ("dit1024_fp8_static_qkv", "te_fp8_dynamic_mlp", "dit2048_block_int8", "dit2048_block_w4a8"):
             w2 = workloads.get_workload(name)
             r2 = [LinearRun(q, w2, lin, i, device) for i, lin in enumerate(w2.linears)]
             steps2 = max(20, args.steps // 5)
@@ -464,7 +473,13 @@ def main():
             secondary[name] = {"TOPS": steps2 * ops2 / (tot2 * 1e-3) / 1e12,
                                "gemm_TOPS": steps2 * ops2 / (sum(g2) * 1e-3) / 1e12,
                                "gemm_frac_of_peak": steps2 * ops2 / (sum(g2) * 1e-3) / 1e12 / peak_tops,
-                               "ms_per_step": tot2 / steps2}
+                               "ms_per_step": tot2 / steps2,
+                               "prep_GBps": steps2 * sum(r.prep_bytes for r in r2) / (sum(p2) * 1e-3) / 1e9,
+                               "gemm_TOPS_per_linear": {r.lin.name: steps2 * r.ops / (g * 1e-3) / 1e12
+                                                        for r, g in zip(r2, g2)}}
+            blocks = w2.extra.get("blocks") if w2.extra else None
+            if blocks:
+                secondary[name]["ms_per_sweep_of_%d_blocks" % blocks] = blocks * tot2 / steps2
             del r2
             torch.cuda.empty_cache()
 

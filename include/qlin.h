@@ -181,8 +181,14 @@ QLIN_API qlin_status qlin_w4a8_forward(const void *X, qlin_dtype xdt, int64_t M,
                               const void *bias, void *Y, void *workspace, size_t ws_bytes,
                               void *stream);
 
+/* The activation stage of qlin_w4a8_forward: per-token int8 codes Xq [M,K]
+ * (round-half-even of X * (1/s_x), IEEE fp32) and fp32 scales s_x [M] =
+ * absmax_i / 127, written to caller memory; one HBM-bound kernel. */
+QLIN_API qlin_status qlin_w4a8_prep(const void *X, qlin_dtype xdt, int64_t M, int64_t K, int8_t *Xq,
+                           float *s_x, void *stream);
+
 /* The GEMM stage of qlin_w4a8_forward, on int8 codes Xq [M,K] and fp32 s_x [M]
- * (qlin_int8_prep with the threshold off writes them). */
+ * (qlin_w4a8_prep, or qlin_int8_prep with the threshold off, writes them). */
 QLIN_API qlin_status qlin_w4a8_gemm(qlin_dtype xdt, int64_t M, int64_t K, const int8_t *Xq,
                            const float *s_x, const uint8_t *Wq4, const float *w_scale,
                            int64_t N, const void *bias, void *Y, void *stream);
@@ -205,6 +211,16 @@ QLIN_API qlin_status qlin_int8_prep(const void *X, qlin_dtype xdt, int64_t M, in
 QLIN_API qlin_status qlin_outlier_weights(const int8_t *Wq, const float *w_scale, int64_t N, int64_t K,
                                  const int32_t *O, const int32_t *count, qlin_dtype dt,
                                  void *W_O, int64_t ostride, void *stream);
+
+/* The int32 accumulator of qlin_int8_outlier_gemm, written out instead of Y:
+ * C[M,N] = sum over non-outlier columns k of Xq[m,k] * Wq[n,k], exact, from
+ * the workspace a qlin_int8_outlier_prepare call on the same stream filled
+ * (ixim/Image21-INT8, "Quantization": the int8 part of the decomposition).
+ * The same kernel as the fused forward with its output stage replaced: the
+ * MMA sums all K columns and the epilogue subtracts the outlier columns'
+ * products in int32. */
+QLIN_API qlin_status qlin_int8_outlier_gemm_i32(int64_t M, int64_t K, const int8_t *Wq, int64_t N,
+                                       int32_t *C, void *workspace, size_t ws_bytes, void *stream);
 
 /* Raw int8 GEMM: C[M,N] int32 = Xq[M,K] Wq[N,K]^T, exact (|C| <= K*127^2). */
 QLIN_API qlin_status qlin_int8_gemm_i32(const int8_t *Xq, const int8_t *Wq, int64_t M, int64_t N,

@@ -55,9 +55,11 @@ def _load() -> ctypes.CDLL:
         "qlin_int8_outlier_prepare": (st, [P, i32, i64, i64, P, P, i64, f32, P, sz, P]),
         "qlin_int8_outlier_forward_noalloc": (st, [P, i32, i64, i64, P, P, i64, f32, P, P, P]),
         "qlin_int8_outlier_gemm": (st, [i32, i64, i64, P, P, i64, P, P, P, sz, P]),
+        "qlin_int8_outlier_gemm_i32": (st, [i64, i64, P, i64, P, P, sz, P]),
         "qlin_fp8_gemm": (st, [i32, i64, i64, P, P, P, P, i32, i64, P, P, P, P]),
         "qlin_w4a8_forward": (st, [P, i32, i64, i64, P, P, i64, P, P, P, sz, P]),
         "qlin_w4a8_gemm": (st, [i32, i64, i64, P, P, P, P, i64, P, P, P]),
+        "qlin_w4a8_prep": (st, [P, i32, i64, i64, P, P, P]),
         "qlin_w4a8_group_i32": (st, [P, P, i64, i64, i64, i32, P, P]),
         "qlin_int8_prep": (st, [P, i32, i64, i64, f32, P, P, P, P, P, P, i64, P, sz, P]),
         "qlin_outlier_weights": (st, [P, P, i64, i64, P, P, i32, P, i64, P]),
@@ -222,6 +224,15 @@ def qlin_int8_outlier_gemm(dtype: torch.dtype, M: int, K: int, Wq: torch.Tensor,
     return Y
 
 
+def qlin_int8_outlier_gemm_i32(M: int, K: int, Wq: torch.Tensor, ws: torch.Tensor) -> torch.Tensor:
+    """int32 accumulator of the LLM.int8 GEMM without the outlier columns, from
+    the workspace a prepare call filled (parity export of the same kernel)."""
+    N = Wq.shape[0]
+    C = torch.empty((M, N), dtype=torch.int32, device=Wq.device)
+    _check(lib.qlin_int8_outlier_gemm_i32(M, K, _ptr(Wq), N, _ptr(C), _ptr(ws), ws.numel(), _stream(Wq.device)))
+    return C
+
+
 def qlin_fp8_gemm(Xq: torch.Tensor, s_x: Optional[torch.Tensor], Wq: torch.Tensor, w_scale: torch.Tensor,
                   wmode: int, dtype: torch.dtype, x_scale: Optional[torch.Tensor] = None,
                   bias: Optional[torch.Tensor] = None, Y: Optional[torch.Tensor] = None) -> torch.Tensor:
@@ -264,6 +275,17 @@ def qlin_w4a8_forward(X: torch.Tensor, Wq4: torch.Tensor, w_scale: torch.Tensor,
     _check(lib.qlin_w4a8_forward(_ptr(X), _dt(X), M, K, _ptr(Wq4), _ptr(w_scale), N, _ptr(bias), _ptr(Y),
                                  _ptr(ws), ws.numel(), _stream(X.device)))
     return Y
+
+
+def qlin_w4a8_prep(X: torch.Tensor, Xq: Optional[torch.Tensor] = None, s_x: Optional[torch.Tensor] = None):
+    """Activation stage of the W4A8 forward: per-token int8 codes and fp32 scales."""
+    M, K = X.shape
+    if Xq is None:
+        Xq = torch.empty((M, K), dtype=torch.int8, device=X.device)
+    if s_x is None:
+        s_x = torch.empty((M,), dtype=torch.float32, device=X.device)
+    _check(lib.qlin_w4a8_prep(_ptr(X), _dt(X), M, K, _ptr(Xq), _ptr(s_x), _stream(X.device)))
+    return Xq, s_x
 
 
 def qlin_w4a8_gemm(Xq: torch.Tensor, s_x: torch.Tensor, Wq4: torch.Tensor, w_scale: torch.Tensor,

@@ -23,7 +23,9 @@
 
 namespace qlin {
 
-enum EpiKind { EPI_I32 = 0, EPI_INT8_OUTLIER = 1, EPI_FP8_TENSOR = 2, EPI_FP8_ROWCOL = 3 };
+// EPI_INT8_OUTLIER_I32: the int32 accumulator of the LLM.int8 path after the
+// outlier-column correction, written out (parity export of the same kernel).
+enum EpiKind { EPI_I32 = 0, EPI_INT8_OUTLIER = 1, EPI_FP8_TENSOR = 2, EPI_FP8_ROWCOL = 3, EPI_INT8_OUTLIER_I32 = 4 };
 
 constexpr int GEMM_BM = 128;
 constexpr int GEMM_BK = 128;                 // bytes (= elements) per stage along K
@@ -43,6 +45,12 @@ struct EpiParams {
   const uint16_t* X_O;        // [M, ostride] outlier activations
   const uint16_t* W_O;        // [N, ostride] dequantised outlier weights
   int64_t ostride;
+  // LLM.int8: the int8 operands and the outlier columns. The A operand may
+  // hold non-zero codes in outlier columns; the epilogue subtracts their
+  // exact int32 contribution sum_o Xq[m,O[o]] * Wq[n,O[o]] from the accumulator.
+  const int8_t* Xq;           // [M,K]
+  const int8_t* Wq;           // [N,K]
+  const int32_t* O;           // [K] ascending outlier columns, first *count valid
 };
 
 template <int BN, int STAGES>
@@ -50,22 +58,34 @@ struct GemmSmem {
   static constexpr int A_BYTES = GEMM_BM * GEMM_BK;
   static constexpr int B_BYTES = BN * GEMM_BK;
   static constexpr int TILE_BYTES = STAGES * (A_BYTES + B_BYTES);
-  static constexpr int EPI_BYTES = static_cast<int>(sizeof(float) * 2 * BN + sizeof(uint32_t) * 16 * BN);
+  static constexpr int EPI_BYTES = static_cast<int>(sizeof(float) * 2 * BN + sizeof(uint32_t) * (16 + 8) * BN);
   static constexpr int BAR_BYTES = 8 * (2 * STAGES + 4 + 2) + 16;
   static constexpr int TOTAL = 1024 + TILE_BYTES + EPI_BYTES + BAR_BYTES;   // 1024: alignment slack
 };
 
 // Per-tile epilogue data staged in shared memory by the epilogue warps:
 // column scales, bias, and (LLM.int8) the tile's slice of the dequantised
-// outlier weight columns, up to 32 outliers as packed 16-bit pairs. All
-// lanes of a warp read the same word (a broadcast), so there are no bank
-// conflicts.
+// outlier weight columns, up to 32 outliers as packed 16-bit pairs, and the
+// int8 weight codes of those columns, 4 to a word. All lanes of a warp read
+// the same word (a broadcast), so there are no bank conflicts.
 template <int BN>
 struct EpiStage {
   float sw[BN];
   float bias[BN];
   uint32_t wo[BN][16];
+  uint32_t wq[BN][8];
 };
+
+// Four int8 codes of row `base` at outlier columns O[o0..o0+3] packed into a
+// word (0 beyond cnt).
+__device__ __forceinline__ uint32_t gather_codes4(const int8_t* __restrict__ base, const int32_t* __restrict__ O,
+                                                  int o0, int cnt) {
+  uint32_t w = 0;
+#pragma unroll
+  for (int e = 0; e < 4; ++e)
+    if (o0 + e < cnt) w |= static_cast<uint32_t>(static_cast<uint8_t>(__ldg(base + __ldg(O + o0 + e)))) << (8 * e);
+  return w;
+}
 
 
 template <typename TOut, int EPI, int BN>
@@ -82,7 +102,7 @@ __device__ __forceinline__ void epi_stage(const EpiParams& p, EpiStage<BN>& es, 
     es.sw[j] = sw;
     es.bias[j] = b;
   }
-  if (cn > 0) {
+  if (cn > 0 && EPI == EPI_INT8_OUTLIER) {
     const int nq = cn / 8;   // 16-byte quads of 8 outlier values per column
     for (int idx = et; idx < BN * nq; idx += 32 * GEMM_EPI_WARPS) {
       const int j = idx / nq, qd = idx - j * nq;
@@ -92,31 +112,58 @@ __device__ __forceinline__ void epi_stage(const EpiParams& p, EpiStage<BN>& es, 
       *reinterpret_cast<uint4*>(&es.wo[j][qd * 4]) = v;
     }
   }
-}
-
-template <typename TOut>
-__device__ __forceinline__ void store_chunk(const EpiParams& p, const float (&acc)[32], int64_t row, int64_t n0) {
-  const int64_t N = p.N;
-  uint16_t* y = reinterpret_cast<uint16_t*>(p.Y) + row * N + n0;
-  if (n0 + 32 <= N && (N & 7) == 0) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      uint4 v;
-      v.x = pack2<TOut>(acc[8 * i + 0], acc[8 * i + 1]);
-      v.y = pack2<TOut>(acc[8 * i + 2], acc[8 * i + 3]);
-      v.z = pack2<TOut>(acc[8 * i + 4], acc[8 * i + 5]);
-      v.w = pack2<TOut>(acc[8 * i + 6], acc[8 * i + 7]);
-      reinterpret_cast<uint4*>(y)[i] = v;
+  if (cn > 0) {
+    const int nw = cn / 4;
+    for (int idx = et; idx < BN * nw; idx += 32 * GEMM_EPI_WARPS) {
+      const int j = idx / nw, w = idx - j * nw;
+      const int64_t n = n_base + j;
+      es.wq[j][w] = n < p.N ? gather_codes4(p.Wq + n * p.K, p.O, 4 * w, cnt) : 0u;
     }
-  } else {
-#pragma unroll
-    for (int j = 0; j < 32; ++j)
-      if (n0 + j < N) y[j] = from_f<TOut>(acc[j]);
   }
 }
 
+// CW outputs (16-bit pairs, the lower column in the low half) to Y[row, n0..].
+template <int CW>
+__device__ __forceinline__ void store_chunk(const EpiParams& p, const uint32_t (&out)[CW / 2], int64_t row,
+                                            int64_t n0) {
+  const int64_t N = p.N;
+  uint16_t* y = reinterpret_cast<uint16_t*>(p.Y) + row * N + n0;
+  if (n0 + CW <= N && (N & 7) == 0) {
+#pragma unroll
+    for (int i = 0; i < CW / 8; ++i)
+      reinterpret_cast<uint4*>(y)[i] = make_uint4(out[4 * i], out[4 * i + 1], out[4 * i + 2], out[4 * i + 3]);
+  } else {
+#pragma unroll
+    for (int j = 0; j < CW; ++j)
+      if (n0 + j < N) y[j] = static_cast<uint16_t>(out[j >> 1] >> (16 * (j & 1)));
+  }
+}
+
+// LLM.int8 accumulator of (row, n) without the outlier columns:
+// acc - sum_o Xq[row,O[o]] * Wq[n,O[o]], exact in int32. xq: the row's codes
+// in the outlier columns, 4 to a word; the weight codes come from the stage
+// (CN > 0) or from global memory (CN < 0).
+template <int CN, int BN, int NXQ>
+__device__ __forceinline__ int32_t corrected(const EpiParams& p, const EpiStage<BN>& es, const uint32_t (&xq)[NXQ],
+                                             uint32_t acc, int64_t row, int64_t n, int jj, int cnt) {
+  int32_t c32 = static_cast<int32_t>(acc);
+  if constexpr (CN > 0) {
+#pragma unroll
+    for (int w = 0; w < CN / 4; ++w) c32 -= __dp4a(static_cast<int>(xq[w]), static_cast<int>(es.wq[jj][w]), 0);
+  }
+  if constexpr (CN < 0) {
+    if (n < p.N)
+      for (int o = 0; o < cnt; ++o) {
+        const int k = __ldg(p.O + o);
+        c32 -= static_cast<int32_t>(__ldg(p.Xq + row * p.K + k)) * static_cast<int32_t>(__ldg(p.Wq + n * p.K + k));
+      }
+  }
+  return c32;
+}
+
 // One accumulator tile, one thread per row: TMEM -> registers in chunks of
-// 32 columns, then y = acc * scales (+ outlier part) + bias -> Y.
+// CW columns (32; 16 where the outlier operands take the registers), then
+// y = acc * scales (+ outlier part) + bias -> Y.
 // CN: outlier columns handled from shared memory (0, 8, 16 or 32; a bucket
 // >= the count, zero-padded); CN < 0: more than 32 outliers, the weight
 // columns are read from global memory (correct for any count, not fast).
@@ -125,12 +172,18 @@ __device__ __forceinline__ void epi_tile(const EpiParams& p, const EpiStage<BN>&
                                          bool row_ok, int64_t n_base, float sx, float alpha, int cnt) {
   constexpr int NX = CN > 0 ? CN : 1;
   float xo[NX];
+  uint32_t xq[(NX + 3) / 4];   // this row's codes in the outlier columns, 4 to a word
 #pragma unroll
   for (int i = 0; i < NX; ++i) xo[i] = 0.0f;
+#pragma unroll
+  for (int i = 0; i < (NX + 3) / 4; ++i) xq[i] = 0u;
   if constexpr (CN > 0) {
 #pragma unroll
+    for (int w = 0; w < CN / 4; ++w)
+      if (row_ok && 4 * w < cnt) xq[w] = gather_codes4(p.Xq + row * p.K, p.O, 4 * w, cnt);
+#pragma unroll
     for (int qd = 0; qd < CN / 8; ++qd) {
-      if (row_ok && qd * 8 < cnt) {
+      if (EPI == EPI_INT8_OUTLIER && row_ok && qd * 8 < cnt) {
         uint16_t h[8];
         unpack8(*reinterpret_cast<const uint4*>(p.X_O + row * p.ostride + qd * 8), h);
 #pragma unroll
@@ -138,32 +191,40 @@ __device__ __forceinline__ void epi_tile(const EpiParams& p, const EpiStage<BN>&
       }
     }
   }
+  constexpr int CW = (CN == 32 || CN < 0) ? 16 : 32;
 #pragma unroll 1
-  for (int c = 0; c < BN / 32; ++c) {
-    uint32_t r[32];
+  for (int c = 0; c < BN / CW; ++c) {
+    uint32_t r[CW];
     __syncwarp();
-    tmem_ld32(t_row + static_cast<uint32_t>(c * 32), r);
+    tmem_ld(t_row + static_cast<uint32_t>(c * CW), r);
     tmem_ld_wait();
-    const int64_t n0 = n_base + c * 32;
+    const int64_t n0 = n_base + c * CW;
     if (row_ok && n0 < p.N) {
-      if constexpr (EPI == EPI_I32) {
-        int32_t* y = reinterpret_cast<int32_t*>(p.Y) + row * p.N + n0;
-        if (n0 + 32 <= p.N && (p.N & 3) == 0) {
+      if constexpr (EPI == EPI_I32 || EPI == EPI_INT8_OUTLIER_I32) {
+        if constexpr (EPI == EPI_INT8_OUTLIER_I32) {
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
+          for (int j = 0; j < CW; ++j)
+            r[j] = static_cast<uint32_t>(corrected<CN>(p, es, xq, r[j], row, n0 + j, c * CW + j, cnt));
+        }
+        int32_t* y = reinterpret_cast<int32_t*>(p.Y) + row * p.N + n0;
+        if (n0 + CW <= p.N && (p.N & 3) == 0) {
+#pragma unroll
+          for (int i = 0; i < CW / 4; ++i)
             reinterpret_cast<int4*>(y)[i] = make_int4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
         } else {
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
+          for (int j = 0; j < CW; ++j)
             if (n0 + j < p.N) y[j] = static_cast<int32_t>(r[j]);
         }
       } else {
-        float acc[32];
+        uint32_t out[CW / 2];   // the chunk's outputs as packed 16-bit pairs
+        float prev = 0.0f;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int jj = c * 32 + j;
+        for (int j = 0; j < CW; ++j) {
+          const int jj = c * CW + j;
           float a;
-          if constexpr (EPI == EPI_INT8_OUTLIER) a = static_cast<float>(static_cast<int32_t>(r[j])) * (sx * es.sw[jj]);
+          if constexpr (EPI == EPI_INT8_OUTLIER)
+            a = static_cast<float>(corrected<CN>(p, es, xq, r[j], row, n0 + j, jj, cnt)) * (sx * es.sw[jj]);
           else if constexpr (EPI == EPI_FP8_TENSOR) a = __uint_as_float(r[j]) * alpha;
           else a = __uint_as_float(r[j]) * (sx * es.sw[jj]);
           if constexpr (CN > 0) {
@@ -186,9 +247,11 @@ __device__ __forceinline__ void epi_tile(const EpiParams& p, const EpiStage<BN>&
               }
             }
           }
-          acc[j] = a + es.bias[jj];
+          a += es.bias[jj];
+          if (j & 1) out[j >> 1] = pack2<TOut>(prev, a);
+          else prev = a;
         }
-        store_chunk<TOut>(p, acc, row, n0);
+        store_chunk<CW>(p, out, row, n0);
       }
     }
   }
@@ -317,7 +380,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     const int et = threadIdx.x - 64;
     int cnt = 0;
     float alpha = 0.0f;
-    if constexpr (EPI == EPI_INT8_OUTLIER) cnt = *p.count;
+    if constexpr (EPI == EPI_INT8_OUTLIER || EPI == EPI_INT8_OUTLIER_I32) cnt = *p.count;
     if constexpr (EPI == EPI_FP8_TENSOR) alpha = __ldg(p.x_scale) * __ldg(p.w_scale);
     const int cn = cnt == 0 ? 0 : cnt <= 8 ? 8 : cnt <= 16 ? 16 : cnt <= 32 ? 32 : -1;
     int acc = 0;
@@ -339,7 +402,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       float sx = 0.0f;
       if constexpr (EPI == EPI_INT8_OUTLIER || EPI == EPI_FP8_ROWCOL) sx = row_ok ? __ldg(p.s_x + row) : 0.0f;
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
-      if constexpr (EPI == EPI_INT8_OUTLIER) {
+      if constexpr (EPI == EPI_INT8_OUTLIER || EPI == EPI_INT8_OUTLIER_I32) {
         if (cn == 0) epi_tile<TOut, EPI, BN, 0>(p, es, t_row, row, row_ok, n_base, sx, alpha, cnt);
         else if (cn == 8) epi_tile<TOut, EPI, BN, 8>(p, es, t_row, row, row_ok, n_base, sx, alpha, cnt);
         else if (cn == 16) epi_tile<TOut, EPI, BN, 16>(p, es, t_row, row, row_ok, n_base, sx, alpha, cnt);

@@ -5,6 +5,7 @@
 //     every token of the call), excludes them from the row absmax, copies
 //     them exactly into X_O and writes the outlier weight columns W_O;
 //   * k_gather_wo: dequantised outlier weight columns (standalone)
+//   * k_zero_outlier_cols: zero codes of the outlier columns (standalone)
 //     W_O[j,o] = dtype(fp32(Wq[j,O[o]]) * s_w[j]) (the weight.to(dtype) *
 //     weight_scale rule of the Text-Encoder-FP8 page, "Format");
 //   * k_fp8_static: per-tensor static E4M3 activation codes;
@@ -174,6 +175,7 @@ struct PrepArgs {
   int32_t* O;          // [K]  ascending outlier columns (written by CTA 0)
   int32_t* count;      // [1]
   uint32_t* sync;      // grid barrier counter (zero on entry for OUTL)
+  uint32_t* rowctr;    // next-row counter (zero on entry), or nullptr for a static row split
   uint16_t* X_O;
   int64_t ostride;
   WoGather wo;
@@ -280,8 +282,17 @@ __global__ void __launch_bounds__(RQ_THREADS, 3) k_prep_rows(const T* __restrict
   // staging: [PF_DEPTH][V][RQ_THREADS] 16-byte vectors, each thread only
   // touches its own column, so cp.async.wait_group alone orders it
   uint4* stage = reinterpret_cast<uint4*>(psm + ((OUTL ? 2 * NW : 0) + 3) / 4 * 4);
+  // rows: taken one at a time from a global counter (balances the units when
+  // rows cost different amounts), or split statically. The unit's leader keeps
+  // a ring of the unit's next row indices in shared memory, three ahead.
   const int64_t first = static_cast<int64_t>(blockIdx.x) * units + unit;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * units;
+  __shared__ long long rowq[RQ_WARPS][4];
+  long long* myq = rowq[unit];
+  auto grab = [&](int k) -> long long {
+    return a.rowctr != nullptr ? static_cast<long long>(atomicAdd(a.rowctr, 1u))
+                               : static_cast<long long>(first + static_cast<int64_t>(k) * stride);
+  };
   auto issue = [&](int64_t r, int slot) {
     const uint4* xr = reinterpret_cast<const uint4*>(X + (r < M ? r : 0) * K);
 #pragma unroll
@@ -291,11 +302,25 @@ __global__ void __launch_bounds__(RQ_THREADS, 3) k_prep_rows(const T* __restrict
     }
     cp_async_commit();
   };
+  static_assert(PF_DEPTH <= 3, "the row ring holds the current row and three more");
+  if (ut == 0) {
+    myq[0] = grab(0);
+    myq[1] = grab(1);
+    myq[2] = grab(2);
+  }
+  if (rw == 1) __syncwarp();
+  else asm volatile("bar.sync %0, %1;" ::"r"(1 + unit), "r"(UT) : "memory");
 #pragma unroll
-  for (int d = 0; d < PF_DEPTH - 1; ++d) issue(first + d * stride, d);
+  for (int d = 0; d < PF_DEPTH - 1; ++d) issue(myq[d], d);
   int slot = 0;
-  for (int64_t row = first; row < M; row += stride) {
-    issue(row + (PF_DEPTH - 1) * stride, (slot + PF_DEPTH - 1) % PF_DEPTH);
+  for (int t = 0;; ++t) {
+    const int64_t row = myq[t & 3];
+    if (row >= M) break;
+    issue(myq[(t + PF_DEPTH - 1) & 3], (slot + PF_DEPTH - 1) % PF_DEPTH);
+    // the slot read two iterations ago is free; every thread of the unit has
+    // passed that iteration's barrier (unit_max) since reading it
+    if (ut == 0) myq[(t + 3) & 3] = grab(t + 3);
+    if (rw == 1) __syncwarp();
     cp_async_wait<PF_DEPTH - 1>();   // this thread's copies of `row` have landed
     uint4 cur[V];
 #pragma unroll
@@ -433,7 +458,6 @@ __global__ void __launch_bounds__(RQ_THREADS, 3) k_prep_rows(const T* __restrict
       if (o < cnt) {
         const int k = outlier_col(sflags, swpre, NW, o);
         h = reinterpret_cast<const uint16_t*>(xr)[k];
-        a.Q[row * K + k] = 0;
         const uint32_t ah = h & 0x7FFFu;
         if (ah <= a.thr_bits) mo = max(mo, ah);
       }
@@ -498,6 +522,18 @@ __global__ void __launch_bounds__(256) k_gather_wo(const int8_t* __restrict__ Wq
 
 // Static per-tensor E4M3 codes: Xq = e4m3(x * (1 / *x_scale)); all-zero
 // codes if the scale is 0. Grid-stride over 8-element vectors.
+// The codes of the outlier columns set to 0 in Q [M,K] (a warp per row). The
+// fused forward never needs this: its GEMM takes those codes as 0 on its own.
+__global__ void __launch_bounds__(256) k_zero_outlier_cols(int8_t* __restrict__ Q, int64_t M, int64_t K,
+                                                         const int32_t* __restrict__ O,
+                                                         const int32_t* __restrict__ count_ptr) {
+  const int cnt = *count_ptr;
+  const int lane = threadIdx.x & 31;
+  for (int64_t row = static_cast<int64_t>(blockIdx.x) * 8 + (threadIdx.x >> 5); row < M;
+       row += static_cast<int64_t>(gridDim.x) * 8)
+    for (int o = lane; o < cnt; o += 32) Q[row * K + __ldg(O + o)] = 0;
+}
+
 template <typename T>
 __global__ void __launch_bounds__(256) k_fp8_static(const T* __restrict__ X, int64_t nvec,
                                                   const float* __restrict__ x_scale, uint8_t* __restrict__ Q) {

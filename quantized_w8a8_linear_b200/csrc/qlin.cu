@@ -224,6 +224,7 @@ qlin_status launch_rowquant(const void* X, int64_t rows, int64_t K, uint8_t* Q, 
 struct Int8Ws {
   uint32_t* sync;     // [1]  grid barrier counter of the prep kernel
   int32_t* count;     // [1]
+  uint32_t* rowctr;   // [1]  next-row counter of the prep kernel
   uint32_t* flags;    // [NW]
   int32_t* O;         // [K]
   float* s_x;         // [M]
@@ -232,7 +233,7 @@ struct Int8Ws {
   uint16_t* X_O;      // [M,ostride]
   uint16_t* W_O;      // [N,ostride]
   int64_t ostride;
-  size_t memset_bytes;  // zeroed each call: sync, count, flags
+  size_t memset_bytes;  // zeroed each call: sync, count, rowctr, flags
   size_t total;
 };
 
@@ -249,6 +250,7 @@ Int8Ws int8_layout(void* base, int64_t M, int64_t N, int64_t K, bool with_gemm_p
   uint8_t* hdr = take(16 + 4 * NW);
   w.sync = reinterpret_cast<uint32_t*>(hdr);
   w.count = reinterpret_cast<int32_t*>(hdr ? hdr + 4 : nullptr);
+  w.rowctr = reinterpret_cast<uint32_t*>(hdr ? hdr + 8 : nullptr);
   w.flags = reinterpret_cast<uint32_t*>(hdr ? hdr + 16 : nullptr);
   w.memset_bytes = static_cast<size_t>(16 + 4 * NW);
   w.O = reinterpret_cast<int32_t*>(take(4 * K));
@@ -277,7 +279,8 @@ qlin_status int8_prep_impl(const void* X, int64_t M, int64_t K, float thr, const
     PrepArgs a{};
     a.M = M; a.K = K; a.thr = thr; a.thr_bits = threshold_bits<T>(thr);
     a.Q = reinterpret_cast<uint8_t*>(Xq); a.s_f32 = s_x; a.amax_bits = w.amax;
-    a.flags = w.flags; a.O = w.O; a.count = w.count; a.sync = w.sync; a.X_O = X_O; a.ostride = ostride; a.wo = wo;
+    a.flags = w.flags; a.O = w.O; a.count = w.count; a.sync = w.sync; a.X_O = X_O;
+    a.rowctr = M < (int64_t{1} << 31) ? w.rowctr : nullptr; a.ostride = ostride; a.wo = wo;
     return launch_prep<T, 0, false, true>(X, a, st);
   }
   return launch_rowquant<T, 0, false>(X, M, K, reinterpret_cast<uint8_t*>(Xq), s_x, nullptr, st);
@@ -463,6 +466,13 @@ qlin_status qlin_int8_prep(const void* X, qlin_dtype xdt, int64_t M, int64_t K, 
                ? int8_prep_impl<__nv_bfloat16>(X, M, K, threshold, w, Xq, s_x, static_cast<uint16_t*>(X_O), ostride,
                                                st)
                : int8_prep_impl<__half>(X, M, K, threshold, w, Xq, s_x, static_cast<uint16_t*>(X_O), ostride, st));
+  if (decomposition_on(threshold) && M > 0) {
+    // the prep leaves the sub-threshold codes of outlier columns in place (the
+    // GEMM masks them); this export returns the decomposed Xq with them at 0
+    const int64_t want = (M + 7) / 8, cap = static_cast<int64_t>(d->sms) * 8;
+    k_zero_outlier_cols<<<static_cast<unsigned>(want < cap ? want : cap), 256, 0, st>>>(Xq, M, K, w.O, w.count);
+    QLIN_TRY(check_cuda(cudaGetLastError(), "k_zero_outlier_cols launch"));
+  }
   const int64_t NW = (K + 31) / 32;
   QLIN_TRY(check_cuda(cudaMemcpyAsync(flags, w.flags, 4 * NW, cudaMemcpyDeviceToDevice, st), "copy flags"));
   QLIN_TRY(check_cuda(cudaMemcpyAsync(count, w.count, 4, cudaMemcpyDeviceToDevice, st), "copy count"));
@@ -553,8 +563,28 @@ qlin_status qlin_int8_outlier_gemm(qlin_dtype xdt, int64_t M, int64_t K, const i
   ep.M = M; ep.N = N; ep.K = K; ep.Y = Y;
   ep.s_x = w.s_x; ep.s_w = w_scale; ep.bias = static_cast<const uint16_t*>(bias);
   ep.count = w.count; ep.X_O = w.X_O; ep.W_O = w.W_O; ep.ostride = w.ostride;
+  ep.Xq = w.Xq; ep.Wq = Wq; ep.O = w.O;
   if (xdt == QLIN_BF16) QLIN_TRY((launch_gemm<0, EPI_INT8_OUTLIER, __nv_bfloat16>(w.Xq, Wq, ep, st, 1)));
   else QLIN_TRY((launch_gemm<0, EPI_INT8_OUTLIER, __half>(w.Xq, Wq, ep, st, 2)));
+  return ok();
+}
+
+qlin_status qlin_int8_outlier_gemm_i32(int64_t M, int64_t K, const int8_t* Wq, int64_t N, int32_t* C,
+                                       void* workspace, size_t ws_bytes, void* stream) {
+  if (M < 0 || N < 0) return fail(QLIN_ERR_INVALID_ARG, "negative size");
+  if (K <= 0 || K % 16 != 0) return fail(QLIN_ERR_ALIGNMENT, "K must be a positive multiple of 16");
+  if (K > kMaxK) return fail(QLIN_ERR_UNSUPPORTED, "K too large");
+  if (M == 0 || N == 0) return ok();
+  QLIN_REQ_PTR(Wq, "Wq");
+  QLIN_REQ_PTR(C, "C");
+  if (workspace == nullptr || ws_bytes < qlin_workspace_bytes(QLIN_OP_INT8_OUTLIER, M, N, K))
+    return fail(QLIN_ERR_WORKSPACE, "workspace too small");
+  QLIN_REQ_PTR(workspace, "workspace");
+  Int8Ws w = int8_layout(workspace, M, N, K, true);
+  EpiParams ep{};
+  ep.M = M; ep.N = N; ep.K = K; ep.Y = C;
+  ep.count = w.count; ep.Xq = w.Xq; ep.Wq = Wq; ep.O = w.O;
+  QLIN_TRY((launch_gemm<0, EPI_INT8_OUTLIER_I32, __nv_bfloat16>(w.Xq, Wq, ep, static_cast<cudaStream_t>(stream), 7)));
   return ok();
 }
 
@@ -749,6 +779,18 @@ qlin_status qlin_w4a8_group_i32(const int8_t* Xq, const uint8_t* Wq4, int64_t M,
   return ok();
 }
 
+qlin_status qlin_w4a8_prep(const void* X, qlin_dtype xdt, int64_t M, int64_t K, int8_t* Xq, float* s_x,
+                           void* stream) {
+  QLIN_TRY(check_common(X, xdt, M, K, 0));
+  if (M == 0) return ok();
+  QLIN_REQ_PTR(Xq, "Xq");
+  QLIN_REQ_PTR(s_x, "s_x");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (xdt == QLIN_BF16)
+    return launch_rowquant<__nv_bfloat16, 0, false>(X, M, K, reinterpret_cast<uint8_t*>(Xq), s_x, nullptr, st);
+  return launch_rowquant<__half, 0, false>(X, M, K, reinterpret_cast<uint8_t*>(Xq), s_x, nullptr, st);
+}
+
 qlin_status qlin_w4a8_forward(const void* X, qlin_dtype xdt, int64_t M, int64_t K, const uint8_t* Wq4,
                               const float* w_scale, int64_t N, const void* bias, void* Y, void* workspace,
                               size_t ws_bytes, void* stream) {
@@ -760,11 +802,7 @@ qlin_status qlin_w4a8_forward(const void* X, qlin_dtype xdt, int64_t M, int64_t 
   QLIN_REQ_PTR(workspace, "workspace");
   int8_t* Xq = static_cast<int8_t*>(workspace);
   float* s_x = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + round_up(M * K, 256));
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (xdt == QLIN_BF16)
-    QLIN_TRY(launch_rowquant<__nv_bfloat16, 0, false>(X, M, K, reinterpret_cast<uint8_t*>(Xq), s_x, nullptr, st));
-  else
-    QLIN_TRY(launch_rowquant<__half, 0, false>(X, M, K, reinterpret_cast<uint8_t*>(Xq), s_x, nullptr, st));
+  QLIN_TRY(qlin_w4a8_prep(X, xdt, M, K, Xq, s_x, stream));
   return qlin_w4a8_gemm(xdt, M, K, Xq, s_x, Wq4, w_scale, N, bias, Y, stream);
 }
 

@@ -206,6 +206,30 @@ def test_int8_gemm_i32_exact(q, M, N, K):
     assert np.array_equal(C, ref)
 
 
+@pytest.mark.parametrize("M,N,K,outl", [
+    (200, 300, 208, []),                                                     # no outlier
+    (200, 300, 208, [(5, 7, 8.0), (199, 200, -30.0), (6, 7, 5.0)]),          # <= 8
+    (300, 520, 512, [(i * 3, 40 * i + 1, 6.5 + i) for i in range(12)]),      # 9..16
+    (300, 520, 512, [(i * 3, 16 * i + 3, -6.5 - i) for i in range(32)]),     # 17..32
+    (300, 520, 512, [(i * 3, 15 * i + 3, -6.5 - i) for i in range(33)]),     # > 32: global path
+    (130, 260, 3072, [(0, 2, 9.0), (1, 2, 5.99), (2, 3071, -6.01), (3, 1500, 5.5)]),
+])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+def test_int8_outlier_gemm_int32_exact(q, M, N, K, outl, dtype):
+    """The fused path's int32 accumulator (the MMA sums every column, the
+    epilogue takes the outlier columns' products back out) equals the
+    oracle's int8 part, sum over k not in O of Xq Wq, exactly."""
+    X = rand_x(M, K, M + 5 * N, dtype, outl)
+    W = rand_w(N, K, M + 5 * N, dtype)
+    Wq, s_w = q.qlin_quantize_weight(dev(W), q.QLIN_W_INT8_ROW)
+    ws = q.workspace(q.QLIN_OP_INT8_OUTLIER, M, N, K, "cuda")
+    q.qlin_int8_outlier_prepare(dev(X), Wq, s_w, THR, ws)
+    C = q.qlin_int8_outlier_gemm_i32(M, K, Wq, ws).cpu().numpy().astype(np.int64)
+    r = oracle.int8_outlier_prep(X, THR)
+    ref = r["Xq"].astype(np.int64) @ Wq.cpu().numpy().astype(np.int64).T
+    assert np.array_equal(C, ref)
+
+
 def test_int8_gemm_i32_extremes(q):
     # every code at +-127 at K = 12288: |C| = 12288 * 127^2 = 198,193,152
     K = 12288
@@ -401,6 +425,19 @@ def _unpack_int4(packed: np.ndarray, K: int) -> np.ndarray:
     q[:, 0::2] = np.where(lo >= 8, lo - 16, lo)
     q[:, 1::2] = np.where(hi >= 8, hi - 16, hi)
     return q
+
+
+@pytest.mark.parametrize("M,K", [(64, 128), (129, 1024), (333, 3072), (7, 12288)])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+def test_w4a8_prep_parity(q, M, K, dtype):
+    """W4A8 activations: per-token int8 with no outlier split, i.e. the
+    LLM.int8 prep with the decomposition off."""
+    X = rand_x(M, K, 3 * M + K, dtype, [(0, 5, 40.0), (M - 1, K - 1, -9.0)])
+    Xq, s_x = q.qlin_w4a8_prep(dev(X))
+    r = oracle.int8_outlier_prep(X, float("inf"))
+    assert r["count"] == 0
+    assert np.array_equal(Xq.cpu().numpy(), r["Xq"])
+    assert np.array_equal(s_x.cpu().numpy(), r["s_x"])
 
 
 @pytest.mark.parametrize("M,N,K", [(64, 128, 128), (200, 300, 256), (129, 257, 1024), (333, 520, 3072)])
