@@ -3,22 +3,31 @@
 //   C[M,N] = A[M,K] B[N,K]^T, A and B 8-bit (int8 -> int32 with kind::i8, or
 //   E4M3 -> fp32 with kind::f8f6f4), both K-major in global memory.
 //
-// Roles (one CTA per SM, 6 warps):
-//   warp 0      TMA producer: 128x128-byte A tiles and BNx128-byte B tiles,
+// Roles (one CTA per SM, 12 warps = 3 warpgroups; the third gives most of
+// its registers to the first two with setmaxnreg):
+//   warp 8      TMA producer: 128x128-byte A tiles and BNx128-byte B tiles,
 //               128B-swizzled, into a STAGES-deep shared-memory ring;
-//   warp 1      MMA issuer: allocates all 512 TMEM columns (two BN-column
+//   warp 9      MMA issuer: allocates all 512 TMEM columns (two BN-column
 //               accumulators), issues 4 UMMAs (K = 32 each) per stage and
 //               commits stage release / accumulator-ready to mbarriers;
-//   warps 2-5   epilogue: tcgen05.ld of their 32-lane quarter, fused dequant
-//               (row x column scales), the floating-point outlier part of
-//               LLM.int8 as a rank-|O| update on CUDA cores, bias, rounding,
-//               and the store of Y. The second accumulator lets the epilogue
-//               of tile t overlap the main loop of tile t+1.
+//   warps 10-11 idle;
+//   warps 0-7   epilogue, two groups of four warps; group g takes columns
+//               [g*BN/2, (g+1)*BN/2) of every tile, so two warps share each
+//               TMEM lane quarter and hide each other's latencies. Each warp
+//               reads its 32-lane quarter with tcgen05.ld (the next chunk in
+//               flight while the current one is processed) and does the fused
+//               dequant (row x column scales), for LLM.int8 the exact
+//               removal of the outlier columns' int8 products and the
+//               floating-point outlier part as a rank-|O| update, the bias,
+//               rounding and the store of Y. With two accumulators the
+//               epilogue of tile t overlaps the main loop of tile t+1.
 // Tiles are handed out round-robin (tile = blockIdx.x + i * gridDim.x) with
 // the M index fastest, so CTAs running together share the same weight tile.
 // Out-of-range rows and K columns are zero-filled by TMA; stores are
 // predicated on M and N.
 #pragma once
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace qlin {
@@ -29,12 +38,29 @@ enum EpiKind { EPI_I32 = 0, EPI_INT8_OUTLIER = 1, EPI_FP8_TENSOR = 2, EPI_FP8_RO
 
 constexpr int GEMM_BM = 128;
 constexpr int GEMM_BK = 128;                 // bytes (= elements) per stage along K
-constexpr int GEMM_EPI_WARPS = 4;
-constexpr int GEMM_THREADS = 64 + 32 * GEMM_EPI_WARPS;
+constexpr int GEMM_EPI_WARPS = 4;            // per group: one per TMEM lane quarter
+constexpr int GEMM_EPI_GROUPS = 2;           // one per TMEM accumulator
+constexpr int GEMM_EPI_THREADS = 32 * GEMM_EPI_WARPS;
+constexpr int GEMM_EPI_ALL = GEMM_EPI_WARPS * GEMM_EPI_GROUPS;   // warps 0..7
+constexpr int GEMM_WARP_TMA = GEMM_EPI_ALL;
+constexpr int GEMM_WARP_MMA = GEMM_EPI_ALL + 1;
+constexpr int GEMM_THREADS = 32 * (GEMM_EPI_ALL + 4);
+// Register split (setmaxnreg): the launch gives every thread the kernel's
+// register count R; the producer warpgroup drops to GEMM_REGS_LOW and the two
+// epilogue warpgroups rise to GEMM_REGS_HIGH. That fits the block's pool when
+// 128 (R - LOW) >= 256 (HIGH - R), i.e. R >= GEMM_REGS_MIN_LAUNCH; the launch
+// checks R against it.
+constexpr int GEMM_REGS_LOW = 56;
+constexpr int GEMM_REGS_HIGH = 208;
+constexpr int GEMM_REGS_MIN_LAUNCH = 160;
+static_assert(128 * (GEMM_REGS_MIN_LAUNCH - GEMM_REGS_LOW) >= 256 * (GEMM_REGS_HIGH - GEMM_REGS_MIN_LAUNCH),
+              "register split must fit the launch pool");
+constexpr int GEMM_CW = 16;                  // accumulator columns per tcgen05.ld in the epilogue
+constexpr int GEMM_OUTL_STAGED = 16;         // outlier counts up to this take the staged fast path
 
 struct EpiParams {
   int64_t M, N, K;
-  void* Y;                    // [M,N]: int32 (EPI_I32) or 16-bit output dtype
+  void* Y;                    // [M,N]: int32 (EPI_I32, EPI_INT8_OUTLIER_I32) or 16-bit output dtype
   const float* s_x;           // [M] per-token scale
   const float* s_w;           // [N] fp32 per-channel weight scale
   const uint16_t* s_w_bf16;   // [N] bf16 per-channel weight scale
@@ -45,90 +71,129 @@ struct EpiParams {
   const uint16_t* X_O;        // [M, ostride] outlier activations
   const uint16_t* W_O;        // [N, ostride] dequantised outlier weights
   int64_t ostride;
-  // LLM.int8: the int8 operands and the outlier columns. The A operand may
-  // hold non-zero codes in outlier columns; the epilogue subtracts their
-  // exact int32 contribution sum_o Xq[m,O[o]] * Wq[n,O[o]] from the accumulator.
+  // LLM.int8: the A operand may hold non-zero codes in outlier columns; the
+  // epilogue subtracts their exact int32 contribution
+  // sum_o Xq[m,O[o]] * Wq[n,O[o]] from the accumulator. Counts up to
+  // GEMM_OUTL_STAGED read the codes from the compact copies XqO / WqO (16 per
+  // row, zero-padded); larger counts gather them from Xq / Wq through O.
   const int8_t* Xq;           // [M,K]
   const int8_t* Wq;           // [N,K]
   const int32_t* O;           // [K] ascending outlier columns, first *count valid
+  const int8_t* XqO;          // [M,16]
+  const int8_t* WqO;          // [N,16]
+  // 16-bit Y written through the kernel's Y tensor map (TMA stores of 32-row x
+  // 16-column boxes from shared memory) instead of per-thread stores
+  int tma_y;
 };
+
+constexpr int GEMM_YBOX_BYTES = 32 * GEMM_CW * 2;   // one warp's 32 rows x 16 columns of 16-bit Y
+
+// Per-tile column data staged in shared memory by an epilogue group, one
+// 64-byte record per column, read with 16-byte broadcasts (all lanes of a
+// warp read the same address, so no bank conflicts and few wavefronts; the
+// tensor core reads its operands from the same shared memory):
+//   q[0] = {column scale (fp32), bias (fp32), WqO[n,0..3], WqO[n,4..7]}
+//   q[1] = W_O[n, 0..7]    (16-bit)
+//   q[2] = {WqO[n,8..11], WqO[n,12..15], 0, 0}
+//   q[3] = W_O[n, 8..15]   (16-bit)
+// Only q[0] is read without outliers, q[0..1] for up to 8 outlier columns.
+template <int BN>
+struct EpiStage {
+  uint4 q[BN][4];
+};
+
+// Packed fp32 fused multiply-add: two IEEE fmas per instruction.
+__device__ __forceinline__ unsigned long long fma_f32x2(unsigned long long a, unsigned long long b,
+                                                        unsigned long long c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ unsigned long long f32x2_of(uint32_t lo, uint32_t hi) {
+  return static_cast<unsigned long long>(lo) | (static_cast<unsigned long long>(hi) << 32);
+}
 
 template <int BN, int STAGES>
 struct GemmSmem {
   static constexpr int A_BYTES = GEMM_BM * GEMM_BK;
   static constexpr int B_BYTES = BN * GEMM_BK;
   static constexpr int TILE_BYTES = STAGES * (A_BYTES + B_BYTES);
-  static constexpr int EPI_BYTES = static_cast<int>(sizeof(float) * 2 * BN + sizeof(uint32_t) * (16 + 8) * BN);
-  static constexpr int BAR_BYTES = 8 * (2 * STAGES + 4 + 2) + 16;
-  static constexpr int TOTAL = 1024 + TILE_BYTES + EPI_BYTES + BAR_BYTES;   // 1024: alignment slack
+  static constexpr int EPI_BYTES = static_cast<int>(sizeof(EpiStage<BN / GEMM_EPI_GROUPS>)) * GEMM_EPI_GROUPS;
+  // Y staging for the TMA stores: two boxes per epilogue warp
+  static constexpr int Y_BYTES = GEMM_EPI_WARPS * GEMM_EPI_GROUPS * 2 * GEMM_YBOX_BYTES;
+  // full[STAGES], empty[STAGES], tfull[2], tempty[2], drain, epi[GROUPS]; tmem slot, abort flag
+  static constexpr int BAR_BYTES = 8 * (2 * STAGES + 4 + 1 + GEMM_EPI_GROUPS) + 16;
+  static constexpr int TOTAL = 1024 + TILE_BYTES + EPI_BYTES + Y_BYTES + BAR_BYTES;   // 1024: alignment slack
+  static_assert(TILE_BYTES % 1024 == 0 && EPI_BYTES % 1024 == 0, "the Y staging boxes stay 1024-byte aligned");
 };
-
-// Per-tile epilogue data staged in shared memory by the epilogue warps:
-// column scales, bias, and (LLM.int8) the tile's slice of the dequantised
-// outlier weight columns, up to 32 outliers as packed 16-bit pairs, and the
-// int8 weight codes of those columns, 4 to a word. All lanes of a warp read
-// the same word (a broadcast), so there are no bank conflicts.
-template <int BN>
-struct EpiStage {
-  float sw[BN];
-  float bias[BN];
-  uint32_t wo[BN][16];
-  uint32_t wq[BN][8];
-};
-
-// Four int8 codes of row `base` at outlier columns O[o0..o0+3] packed into a
-// word (0 beyond cnt).
-__device__ __forceinline__ uint32_t gather_codes4(const int8_t* __restrict__ base, const int32_t* __restrict__ O,
-                                                  int o0, int cnt) {
-  uint32_t w = 0;
-#pragma unroll
-  for (int e = 0; e < 4; ++e)
-    if (o0 + e < cnt) w |= static_cast<uint32_t>(static_cast<uint8_t>(__ldg(base + __ldg(O + o0 + e)))) << (8 * e);
-  return w;
-}
-
 
 template <typename TOut, int EPI, int BN>
-__device__ __forceinline__ void epi_stage(const EpiParams& p, EpiStage<BN>& es, int64_t n_base, int et, int cn,
-                                          int cnt) {
-  for (int j = et; j < BN; j += 32 * GEMM_EPI_WARPS) {
-    const int64_t n = n_base + j;
-    float sw = 0.0f, b = 0.0f;
+__device__ __forceinline__ void epi_stage(const EpiParams& p, EpiStage<BN>& es, int64_t n_base, int et, int cn) {
+  constexpr int PER = BN / GEMM_EPI_THREADS;
+  constexpr bool OUTL = EPI == EPI_INT8_OUTLIER || EPI == EPI_INT8_OUTLIER_I32;
+  float sw[PER], b[PER];
+  uint4 wo0[PER], wo1[PER], wq[PER];
+  // every load first, then every store: one memory round trip per tile
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int64_t n = n_base + et + i * GEMM_EPI_THREADS;
+    sw[i] = 0.0f;
+    b[i] = 0.0f;
+    wo0[i] = wo1[i] = wq[i] = make_uint4(0u, 0u, 0u, 0u);
     if (n < p.N) {
-      if constexpr (EPI == EPI_INT8_OUTLIER) sw = __ldg(p.s_w + n);
-      if constexpr (EPI == EPI_FP8_ROWCOL) sw = to_f<__nv_bfloat16>(__ldg(p.s_w_bf16 + n));
-      if (p.bias != nullptr) b = to_f<TOut>(__ldg(p.bias + n));
-    }
-    es.sw[j] = sw;
-    es.bias[j] = b;
-  }
-  if (cn > 0 && EPI == EPI_INT8_OUTLIER) {
-    const int nq = cn / 8;   // 16-byte quads of 8 outlier values per column
-    for (int idx = et; idx < BN * nq; idx += 32 * GEMM_EPI_WARPS) {
-      const int j = idx / nq, qd = idx - j * nq;
-      const int64_t n = n_base + j;
-      uint4 v = make_uint4(0u, 0u, 0u, 0u);
-      if (n < p.N && qd * 8 < cnt) v = __ldg(reinterpret_cast<const uint4*>(p.W_O + n * p.ostride + qd * 8));
-      *reinterpret_cast<uint4*>(&es.wo[j][qd * 4]) = v;
-    }
-  }
-  if (cn > 0) {
-    const int nw = cn / 4;
-    for (int idx = et; idx < BN * nw; idx += 32 * GEMM_EPI_WARPS) {
-      const int j = idx / nw, w = idx - j * nw;
-      const int64_t n = n_base + j;
-      es.wq[j][w] = n < p.N ? gather_codes4(p.Wq + n * p.K, p.O, 4 * w, cnt) : 0u;
+      if constexpr (EPI == EPI_INT8_OUTLIER) sw[i] = __ldg(p.s_w + n);
+      if constexpr (EPI == EPI_FP8_ROWCOL) sw[i] = to_f<__nv_bfloat16>(__ldg(p.s_w_bf16 + n));
+      if constexpr (EPI == EPI_INT8_OUTLIER || EPI == EPI_FP8_TENSOR || EPI == EPI_FP8_ROWCOL)
+        if (p.bias != nullptr) b[i] = to_f<TOut>(__ldg(p.bias + n));
+      if constexpr (OUTL) {
+        if (cn > 0) {
+          wq[i] = __ldg(reinterpret_cast<const uint4*>(p.WqO + n * 16));
+          if constexpr (EPI == EPI_INT8_OUTLIER) {
+            const uint4* w = reinterpret_cast<const uint4*>(p.W_O + n * p.ostride);
+            wo0[i] = __ldg(w);
+            if (cn > 8) wo1[i] = __ldg(w + 1);
+          }
+        }
+      }
     }
   }
+#pragma unroll
+  for (int i = 0; i < PER; ++i) {
+    const int j = et + i * GEMM_EPI_THREADS;
+    es.q[j][0] = make_uint4(__float_as_uint(sw[i]), __float_as_uint(b[i]), wq[i].x, wq[i].y);
+    if constexpr (OUTL) {
+      es.q[j][1] = wo0[i];
+      es.q[j][2] = make_uint4(wq[i].z, wq[i].w, 0u, 0u);
+      es.q[j][3] = wo1[i];
+    }
+  }
+}
+
+// fp32 pair (lo, hi) of two packed 16-bit values
+template <typename T>
+__device__ __forceinline__ unsigned long long f32x2_of16(uint32_t w) {
+  if constexpr (std::is_same<T, __nv_bfloat16>::value) return f32x2_of(w << 16, w & 0xFFFF0000u);
+  else return f32x2_of(__float_as_uint(__half2float(__ushort_as_half(static_cast<unsigned short>(w & 0xFFFFu)))),
+                       __float_as_uint(__half2float(__ushort_as_half(static_cast<unsigned short>(w >> 16)))));
 }
 
 // CW outputs (16-bit pairs, the lower column in the low half) to Y[row, n0..].
+// v8: Y is 32-byte aligned and N a multiple of 16, so every 16-column chunk is
+// one aligned 32-byte sector, written with one 256-bit store.
 template <int CW>
 __device__ __forceinline__ void store_chunk(const EpiParams& p, const uint32_t (&out)[CW / 2], int64_t row,
-                                            int64_t n0) {
+                                            int64_t n0, bool v8) {
   const int64_t N = p.N;
   uint16_t* y = reinterpret_cast<uint16_t*>(p.Y) + row * N + n0;
-  if (n0 + CW <= N && (N & 7) == 0) {
+  if (v8 && n0 + CW <= N) {
+    static_assert(CW % 16 == 0, "256-bit stores take 16 columns");
+#pragma unroll
+    for (int i = 0; i < CW / 16; ++i)
+      asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(y + 16 * i), "r"(out[8 * i]),
+                   "r"(out[8 * i + 1]), "r"(out[8 * i + 2]), "r"(out[8 * i + 3]), "r"(out[8 * i + 4]),
+                   "r"(out[8 * i + 5]), "r"(out[8 * i + 6]), "r"(out[8 * i + 7])
+                   : "memory");
+  } else if (n0 + CW <= N && (N & 7) == 0) {
 #pragma unroll
     for (int i = 0; i < CW / 8; ++i)
       reinterpret_cast<uint4*>(y)[i] = make_uint4(out[4 * i], out[4 * i + 1], out[4 * i + 2], out[4 * i + 3]);
@@ -139,140 +204,210 @@ __device__ __forceinline__ void store_chunk(const EpiParams& p, const uint32_t (
   }
 }
 
-// LLM.int8 accumulator of (row, n) without the outlier columns:
-// acc - sum_o Xq[row,O[o]] * Wq[n,O[o]], exact in int32. xq: the row's codes
-// in the outlier columns, 4 to a word; the weight codes come from the stage
-// (CN > 0) or from global memory (CN < 0).
-template <int CN, int BN, int NXQ>
-__device__ __forceinline__ int32_t corrected(const EpiParams& p, const EpiStage<BN>& es, const uint32_t (&xq)[NXQ],
-                                             uint32_t acc, int64_t row, int64_t n, int jj, int cnt) {
-  int32_t c32 = static_cast<int32_t>(acc);
-  if constexpr (CN > 0) {
+// CW int32 outputs to Y[row, n0..].
+template <int CW>
+__device__ __forceinline__ void store_chunk_i32(const EpiParams& p, const uint32_t (&r)[CW], int64_t row,
+                                                int64_t n0) {
+  int32_t* y = reinterpret_cast<int32_t*>(p.Y) + row * p.N + n0;
+  if (n0 + CW <= p.N && (p.N & 3) == 0) {
 #pragma unroll
-    for (int w = 0; w < CN / 4; ++w) c32 -= __dp4a(static_cast<int>(xq[w]), static_cast<int>(es.wq[jj][w]), 0);
+    for (int i = 0; i < CW / 4; ++i)
+      reinterpret_cast<int4*>(y)[i] = make_int4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
+  } else {
+#pragma unroll
+    for (int j = 0; j < CW; ++j)
+      if (n0 + j < p.N) y[j] = static_cast<int32_t>(r[j]);
   }
-  if constexpr (CN < 0) {
-    if (n < p.N)
-      for (int o = 0; o < cnt; ++o) {
-        const int k = __ldg(p.O + o);
-        c32 -= static_cast<int32_t>(__ldg(p.Xq + row * p.K + k)) * static_cast<int32_t>(__ldg(p.Wq + n * p.K + k));
-      }
-  }
-  return c32;
 }
 
-// One accumulator tile, one thread per row: TMEM -> registers in chunks of
-// CW columns (32; 16 where the outlier operands take the registers), then
-// y = acc * scales (+ outlier part) + bias -> Y.
-// CN: outlier columns handled from shared memory (0, 8, 16 or 32; a bucket
-// >= the count, zero-padded); CN < 0: more than 32 outliers, the weight
-// columns are read from global memory (correct for any count, not fast).
+// One chunk of GEMM_CW accumulator columns of one row: r -> Y[row, n0..).
+// CN: outlier columns (0, 8 or 16: a bucket >= the count, the staged operands
+// zero-padded) or -1 (more than 16: gathered from global memory, correct for
+// any count, not fast).
+// 16-bit outputs are returned in `out` (the caller stores them); int32
+// outputs are stored here.
+template <typename TOut, int EPI, int BN, int CN, int NX, int NQ>
+__device__ __forceinline__ void epi_chunk(const EpiParams& p, const EpiStage<BN>& es, uint32_t (&r)[GEMM_CW], int c,
+                                          int64_t row, int64_t n_base, float sx, float alpha, int cnt,
+                                          const float (&xo)[NX], const unsigned long long (&xp)[8],
+                                          const uint32_t (&nxq)[NQ], uint32_t (&out)[GEMM_CW / 2]) {
+  constexpr bool OUTL = EPI == EPI_INT8_OUTLIER || EPI == EPI_INT8_OUTLIER_I32;
+  const int64_t n0 = n_base + c * GEMM_CW;
+  float prev = 0.0f;
+#pragma unroll
+  for (int j = 0; j < GEMM_CW; ++j) {
+    const uint4 q0 = es.q[c * GEMM_CW + j][0];
+    int32_t acc = static_cast<int32_t>(r[j]);
+    if constexpr (OUTL) {
+      // the accumulator without the outlier columns' products, exact in int32
+      if constexpr (CN > 0) {
+        acc = __dp4a(static_cast<int>(nxq[0]), static_cast<int>(q0.z), acc);
+        acc = __dp4a(static_cast<int>(nxq[1]), static_cast<int>(q0.w), acc);
+        if constexpr (CN > 8) {
+          const uint4 q2 = es.q[c * GEMM_CW + j][2];
+          acc = __dp4a(static_cast<int>(nxq[2]), static_cast<int>(q2.x), acc);
+          acc = __dp4a(static_cast<int>(nxq[3]), static_cast<int>(q2.y), acc);
+        }
+      }
+      if constexpr (CN < 0) {
+        if (n0 + j < p.N)
+          for (int o = 0; o < cnt; ++o) {
+            const int k = __ldg(p.O + o);
+            acc -= static_cast<int32_t>(__ldg(p.Xq + row * p.K + k)) *
+                   static_cast<int32_t>(__ldg(p.Wq + (n0 + j) * p.K + k));
+          }
+      }
+    }
+    if constexpr (EPI == EPI_I32 || EPI == EPI_INT8_OUTLIER_I32) {
+      r[j] = static_cast<uint32_t>(acc);
+    } else {
+      const float sw = __uint_as_float(q0.x), bias = __uint_as_float(q0.y);
+      float a;
+      if constexpr (EPI == EPI_INT8_OUTLIER) a = fmaf(static_cast<float>(acc), sx * sw, bias);
+      else if constexpr (EPI == EPI_FP8_TENSOR) a = fmaf(__uint_as_float(r[j]), alpha, bias);
+      else a = fmaf(__uint_as_float(r[j]), sx * sw, bias);
+      if constexpr (EPI == EPI_INT8_OUTLIER && CN > 0) {
+        // floating-point outlier part: sum_o X_O[row,o] W_O[n,o], outlier pairs per packed fma
+        const uint4 q1 = es.q[c * GEMM_CW + j][1];
+        unsigned long long t = fma_f32x2(xp[0], f32x2_of16<TOut>(q1.x), 0ull);
+        t = fma_f32x2(xp[1], f32x2_of16<TOut>(q1.y), t);
+        t = fma_f32x2(xp[2], f32x2_of16<TOut>(q1.z), t);
+        t = fma_f32x2(xp[3], f32x2_of16<TOut>(q1.w), t);
+        if constexpr (CN > 8) {
+          const uint4 q3 = es.q[c * GEMM_CW + j][3];
+          t = fma_f32x2(xp[4], f32x2_of16<TOut>(q3.x), t);
+          t = fma_f32x2(xp[5], f32x2_of16<TOut>(q3.y), t);
+          t = fma_f32x2(xp[6], f32x2_of16<TOut>(q3.z), t);
+          t = fma_f32x2(xp[7], f32x2_of16<TOut>(q3.w), t);
+        }
+        a += __uint_as_float(static_cast<uint32_t>(t)) + __uint_as_float(static_cast<uint32_t>(t >> 32));
+      }
+      if constexpr (EPI == EPI_INT8_OUTLIER && CN < 0) {
+        if (n0 + j < p.N)
+          for (int o0 = 0; o0 < cnt; o0 += 8) {
+            uint16_t xh[8], wh[8];
+            unpack8(__ldg(reinterpret_cast<const uint4*>(p.X_O + row * p.ostride + o0)), xh);
+            unpack8(__ldg(reinterpret_cast<const uint4*>(p.W_O + (n0 + j) * p.ostride + o0)), wh);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) a = fmaf(to_f<TOut>(xh[e]), to_f<TOut>(wh[e]), a);
+          }
+      }
+      if (j & 1) out[j >> 1] = pack2<TOut>(prev, a);
+      else prev = a;
+    }
+  }
+  if constexpr (EPI == EPI_I32 || EPI == EPI_INT8_OUTLIER_I32) store_chunk_i32<GEMM_CW>(p, r, row, n0);
+}
+
+// One accumulator tile, one thread per row (its TMEM lane): the row's
+// operands first, then the accumulator in chunks of GEMM_CW columns with the
+// next chunk's tcgen05.ld in flight while the current one is processed.
 template <typename TOut, int EPI, int BN, int CN>
 __device__ __forceinline__ void epi_tile(const EpiParams& p, const EpiStage<BN>& es, uint32_t t_row, int64_t row,
-                                         bool row_ok, int64_t n_base, float sx, float alpha, int cnt) {
+                                         bool row_ok, int64_t n_base, float alpha, int cnt, const CUtensorMap* tmY,
+                                         uint8_t* ybox, int64_t row0) {
   constexpr int NX = CN > 0 ? CN : 1;
+  constexpr int NQ = CN > 0 ? CN / 4 : 1;
   float xo[NX];
-  uint32_t xq[(NX + 3) / 4];   // this row's codes in the outlier columns, 4 to a word
+  uint32_t nxq[NQ];   // minus the row's codes in the outlier columns, 4 to a word
 #pragma unroll
   for (int i = 0; i < NX; ++i) xo[i] = 0.0f;
 #pragma unroll
-  for (int i = 0; i < (NX + 3) / 4; ++i) xq[i] = 0u;
-  if constexpr (CN > 0) {
+  for (int i = 0; i < NQ; ++i) nxq[i] = 0u;
+  float sx = 0.0f;
+  if (row_ok) {
+    if constexpr (EPI == EPI_INT8_OUTLIER || EPI == EPI_FP8_ROWCOL) sx = __ldg(p.s_x + row);
+    if constexpr (CN > 0) {
+      const uint4 q4 = __ldg(reinterpret_cast<const uint4*>(p.XqO + row * 16));
+      nxq[0] = __vsub4(0u, q4.x);   // codes lie in [-127, 127]: negation is exact
+      nxq[1] = __vsub4(0u, q4.y);
+      if constexpr (CN > 8) {
+        nxq[2] = __vsub4(0u, q4.z);
+        nxq[3] = __vsub4(0u, q4.w);
+      }
+      if constexpr (EPI == EPI_INT8_OUTLIER) {
 #pragma unroll
-    for (int w = 0; w < CN / 4; ++w)
-      if (row_ok && 4 * w < cnt) xq[w] = gather_codes4(p.Xq + row * p.K, p.O, 4 * w, cnt);
+        for (int qd = 0; qd < CN / 8; ++qd) {
+          uint16_t h[8];
+          unpack8(__ldg(reinterpret_cast<const uint4*>(p.X_O + row * p.ostride + qd * 8)), h);
 #pragma unroll
-    for (int qd = 0; qd < CN / 8; ++qd) {
-      if (EPI == EPI_INT8_OUTLIER && row_ok && qd * 8 < cnt) {
-        uint16_t h[8];
-        unpack8(*reinterpret_cast<const uint4*>(p.X_O + row * p.ostride + qd * 8), h);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) xo[qd * 8 + e] = to_f<TOut>(h[e]);
+          for (int e = 0; e < 8; ++e) xo[qd * 8 + e] = to_f<TOut>(h[e]);
+        }
       }
     }
   }
-  constexpr int CW = (CN == 32 || CN < 0) ? 16 : 32;
-#pragma unroll 1
-  for (int c = 0; c < BN / CW; ++c) {
-    uint32_t r[CW];
-    __syncwarp();
-    tmem_ld(t_row + static_cast<uint32_t>(c * CW), r);
-    tmem_ld_wait();
-    const int64_t n0 = n_base + c * CW;
-    if (row_ok && n0 < p.N) {
-      if constexpr (EPI == EPI_I32 || EPI == EPI_INT8_OUTLIER_I32) {
-        if constexpr (EPI == EPI_INT8_OUTLIER_I32) {
+  unsigned long long xp[8];   // the row's outlier values as fp32 pairs
 #pragma unroll
-          for (int j = 0; j < CW; ++j)
-            r[j] = static_cast<uint32_t>(corrected<CN>(p, es, xq, r[j], row, n0 + j, c * CW + j, cnt));
+  for (int i = 0; i < 8; ++i) xp[i] = f32x2_of(__float_as_uint(xo[(2 * i) % NX]), __float_as_uint(xo[(2 * i + 1) % NX]));
+  const bool v8 = (reinterpret_cast<uintptr_t>(p.Y) & 31u) == 0 && (p.N & 15) == 0;
+  constexpr int NCH = BN / GEMM_CW;
+  static_assert(NCH % 2 == 0, "chunks are processed in pairs");
+  const int lane = threadIdx.x & 31;
+  // one chunk: compute, then store (TMA box from shared memory, or per-thread stores)
+  auto chunk = [&](uint32_t (&r)[GEMM_CW], int c) {
+    const int64_t n0 = n_base + c * GEMM_CW;
+    if (n0 >= p.N) return;   // warp-uniform
+    uint32_t out[GEMM_CW / 2];
+#pragma unroll
+    for (int i = 0; i < GEMM_CW / 2; ++i) out[i] = 0u;
+    if (row_ok) epi_chunk<TOut, EPI, BN, CN>(p, es, r, c, row, n_base, sx, alpha, cnt, xo, xp, nxq, out);
+    if constexpr (EPI != EPI_I32 && EPI != EPI_INT8_OUTLIER_I32) {
+      if (p.tma_y) {
+        uint8_t* box = ybox + (c & 1) * GEMM_YBOX_BYTES;
+        if (lane == 0) bulk_wait_read<1>();   // the box's previous store has read it
+        __syncwarp();
+        // row `lane` of the box, 128B-pattern swizzle of the 32-byte rows (SWIZZLE_32B:
+        // 16-byte half h sits at h ^ bit 2 of the row): conflict-free quarter-warp writes
+        const uint32_t base = smem_u32(box) + static_cast<uint32_t>(lane) * 32u;
+        const uint32_t x = ((static_cast<uint32_t>(lane) >> 2) & 1u) << 4;
+        st_shared_v4(base + x, out[0], out[1], out[2], out[3]);
+        st_shared_v4(base + (16u ^ x), out[4], out[5], out[6], out[7]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(tmY, box, static_cast<int32_t>(n0), static_cast<int32_t>(row0));
+          bulk_commit();
         }
-        int32_t* y = reinterpret_cast<int32_t*>(p.Y) + row * p.N + n0;
-        if (n0 + CW <= p.N && (p.N & 3) == 0) {
-#pragma unroll
-          for (int i = 0; i < CW / 4; ++i)
-            reinterpret_cast<int4*>(y)[i] = make_int4(r[4 * i], r[4 * i + 1], r[4 * i + 2], r[4 * i + 3]);
-        } else {
-#pragma unroll
-          for (int j = 0; j < CW; ++j)
-            if (n0 + j < p.N) y[j] = static_cast<int32_t>(r[j]);
-        }
-      } else {
-        uint32_t out[CW / 2];   // the chunk's outputs as packed 16-bit pairs
-        float prev = 0.0f;
-#pragma unroll
-        for (int j = 0; j < CW; ++j) {
-          const int jj = c * CW + j;
-          float a;
-          if constexpr (EPI == EPI_INT8_OUTLIER)
-            a = static_cast<float>(corrected<CN>(p, es, xq, r[j], row, n0 + j, jj, cnt)) * (sx * es.sw[jj]);
-          else if constexpr (EPI == EPI_FP8_TENSOR) a = __uint_as_float(r[j]) * alpha;
-          else a = __uint_as_float(r[j]) * (sx * es.sw[jj]);
-          if constexpr (CN > 0) {
-#pragma unroll
-            for (int qd = 0; qd < CN / 8; ++qd) {
-              uint16_t h[8];
-              unpack8(*reinterpret_cast<const uint4*>(&es.wo[jj][qd * 4]), h);
-#pragma unroll
-              for (int e = 0; e < 8; ++e) a = fmaf(xo[qd * 8 + e], to_f<TOut>(h[e]), a);
-            }
-          }
-          if constexpr (CN < 0) {
-            for (int o0 = 0; o0 < cnt; o0 += 8) {
-              uint16_t xh[8], wh[8];
-              unpack8(*reinterpret_cast<const uint4*>(p.X_O + row * p.ostride + o0), xh);
-              if (n0 + j < p.N) {
-                unpack8(__ldg(reinterpret_cast<const uint4*>(p.W_O + (n0 + j) * p.ostride + o0)), wh);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) a = fmaf(to_f<TOut>(xh[e]), to_f<TOut>(wh[e]), a);
-              }
-            }
-          }
-          a += es.bias[jj];
-          if (j & 1) out[j >> 1] = pack2<TOut>(prev, a);
-          else prev = a;
-        }
-        store_chunk<CW>(p, out, row, n0);
+      } else if (row_ok) {
+        store_chunk<GEMM_CW>(p, out, row, n0, v8);
       }
     }
+  };
+  uint32_t ra[GEMM_CW], rb[GEMM_CW];
+  __syncwarp();
+  tmem_ld16(t_row, ra);
+#pragma unroll 1
+  for (int c = 0; c < NCH; c += 2) {
+    __syncwarp();
+    tmem_wait16(ra);
+    tmem_ld16(t_row + static_cast<uint32_t>((c + 1) * GEMM_CW), rb);
+    chunk(ra, c);
+    __syncwarp();
+    tmem_wait16(rb);
+    if (c + 2 < NCH) tmem_ld16(t_row + static_cast<uint32_t>((c + 2) * GEMM_CW), ra);
+    chunk(rb, c + 1);
   }
 }
 
 template <int KIND, int EPI, typename TOut, int BN, int STAGES>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
-    k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const EpiParams p) {
+    k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+           const __grid_constant__ CUtensorMap tmY, const EpiParams p) {
   using L = GemmSmem<BN, STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + STAGES * L::A_BYTES;
-  EpiStage<BN>& es = *reinterpret_cast<EpiStage<BN>*>(smem + L::TILE_BYTES);
-  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + L::TILE_BYTES + L::EPI_BYTES);
+  constexpr int BNG = BN / GEMM_EPI_GROUPS;   // columns per epilogue group
+  EpiStage<BNG>* estage = reinterpret_cast<EpiStage<BNG>*>(smem + L::TILE_BYTES);   // [GEMM_EPI_GROUPS]
+  uint8_t* ystage = smem + L::TILE_BYTES + L::EPI_BYTES;   // [epilogue warp][2] boxes
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + L::TILE_BYTES + L::EPI_BYTES + L::Y_BYTES);
   uint64_t* empty_bar = full_bar + STAGES;
   uint64_t* tfull_bar = empty_bar + STAGES;     // [2]
   uint64_t* tempty_bar = tfull_bar + 2;         // [2]
   uint64_t* drain_bar = tempty_bar + 2;         // [1]
-  uint64_t* epi_mbar = drain_bar + 1;           // [1]
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(epi_mbar + 1);
+  uint64_t* epi_mbar = drain_bar + 1;           // [GEMM_EPI_GROUPS]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(epi_mbar + GEMM_EPI_GROUPS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -290,18 +425,18 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tfull_bar[b], 1);
-      mbar_init(&tempty_bar[b], GEMM_EPI_WARPS);
+      mbar_init(&tempty_bar[b], GEMM_EPI_WARPS * GEMM_EPI_GROUPS);
     }
     mbar_init(drain_bar, 1);
-    mbar_init(epi_mbar, 32 * GEMM_EPI_WARPS);
+    for (int g = 0; g < GEMM_EPI_GROUPS; ++g) mbar_init(&epi_mbar[g], GEMM_EPI_THREADS);
     *abort_flag = 0;
     fence_mbarrier_init();
   }
-  if (warp == 0 && lane == 0) {
+  if (warp == GEMM_WARP_TMA && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
   }
-  if (warp == 1) {
+  if (warp == GEMM_WARP_MMA) {
     tmem_alloc(tmem_slot, 2 * BN);
     tmem_relinquish();
   }
@@ -309,8 +444,11 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-
-  if (warp == 0) {
+  // each role's register budget is set inside its branch: code after a merge
+  // would be held to the lower of the two
+  if (warp >= GEMM_EPI_ALL) {
+  setmaxnreg_dec<GEMM_REGS_LOW>();
+  if (warp == GEMM_WARP_TMA) {
     if (lane == 0) {
       // ---------------- TMA producer ----------------
       int stage = 0;
@@ -340,7 +478,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         }
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == GEMM_WARP_MMA) {
     if (lane == 0) {
       // ---------------- MMA issuer ----------------
       constexpr uint32_t idesc = KIND == 0 ? idesc_i8(GEMM_BM, BN) : idesc_e4m3(GEMM_BM, BN);
@@ -374,52 +512,61 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       const uint64_t t0 = globaltimer();
       while (!mbar_try_wait(a, 0) && globaltimer() - t0 < g_wait_timeout_ns) {}
     }
+  }
   } else {
-    // ---------------- epilogue ----------------
+    setmaxnreg_inc<GEMM_REGS_HIGH>();
+    // ---------------- epilogue: group g takes columns [g*BNG, (g+1)*BNG) of every tile ----------------
+    const int g = warp / GEMM_EPI_WARPS;
     const int q = warp & 3;   // TMEM lane quarter this warp may access
-    const int et = threadIdx.x - 64;
+    const int et = threadIdx.x - g * GEMM_EPI_THREADS;
+    EpiStage<BNG>& es = estage[g];
+    uint8_t* ybox = ystage + warp * 2 * GEMM_YBOX_BYTES;
     int cnt = 0;
     float alpha = 0.0f;
     if constexpr (EPI == EPI_INT8_OUTLIER || EPI == EPI_INT8_OUTLIER_I32) cnt = *p.count;
     if constexpr (EPI == EPI_FP8_TENSOR) alpha = __ldg(p.x_scale) * __ldg(p.w_scale);
-    const int cn = cnt == 0 ? 0 : cnt <= 8 ? 8 : cnt <= 16 ? 16 : cnt <= 32 ? 32 : -1;
+    const int cn = cnt == 0 ? 0 : cnt <= 8 ? 8 : cnt <= GEMM_OUTL_STAGED ? 16 : -1;
     int acc = 0;
     uint32_t acc_phase = 0;
     uint32_t bar_phase = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
       const int mb = tile % num_m, nb = tile / num_m;
-      const int64_t n_base = static_cast<int64_t>(nb) * BN;
+      const int64_t n_base = static_cast<int64_t>(nb) * BN + g * BNG;
       if constexpr (EPI != EPI_I32) {
-        // the previous tile's readers are done with the staging area
-        if (!epi_bar(epi_mbar, bar_phase, abort_flag)) break;
-        epi_stage<TOut, EPI, BN>(p, es, n_base, et, cn, cnt);
-        if (!epi_bar(epi_mbar, bar_phase, abort_flag)) break;
+        // the group's readers of the previous tile are done with its staging area
+        if (!epi_bar(&epi_mbar[g], bar_phase, abort_flag)) break;
+        epi_stage<TOut, EPI, BNG>(p, es, n_base, et, cn);
+        if (!epi_bar(&epi_mbar[g], bar_phase, abort_flag)) break;
       }
       if (!mbar_wait(&tfull_bar[acc], acc_phase, abort_flag)) break;
       tc_fence_after();
       const int64_t row = static_cast<int64_t>(mb) * GEMM_BM + q * 32 + lane;
       const bool row_ok = row < M;
-      float sx = 0.0f;
-      if constexpr (EPI == EPI_INT8_OUTLIER || EPI == EPI_FP8_ROWCOL) sx = row_ok ? __ldg(p.s_x + row) : 0.0f;
-      const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN);
+      const uint32_t t_row =
+          tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN + g * BNG);
       if constexpr (EPI == EPI_INT8_OUTLIER || EPI == EPI_INT8_OUTLIER_I32) {
-        if (cn == 0) epi_tile<TOut, EPI, BN, 0>(p, es, t_row, row, row_ok, n_base, sx, alpha, cnt);
-        else if (cn == 8) epi_tile<TOut, EPI, BN, 8>(p, es, t_row, row, row_ok, n_base, sx, alpha, cnt);
-        else if (cn == 16) epi_tile<TOut, EPI, BN, 16>(p, es, t_row, row, row_ok, n_base, sx, alpha, cnt);
-        else if (cn == 32) epi_tile<TOut, EPI, BN, 32>(p, es, t_row, row, row_ok, n_base, sx, alpha, cnt);
-        else epi_tile<TOut, EPI, BN, -1>(p, es, t_row, row, row_ok, n_base, sx, alpha, cnt);
+        if (cn == 0) epi_tile<TOut, EPI, BNG, 0>(p, es, t_row, row, row_ok, n_base, alpha, cnt, &tmY, ybox,
+                                                           row - lane);
+        else if (cn == 8) epi_tile<TOut, EPI, BNG, 8>(p, es, t_row, row, row_ok, n_base, alpha, cnt, &tmY, ybox,
+                                                           row - lane);
+        else if (cn == 16) epi_tile<TOut, EPI, BNG, 16>(p, es, t_row, row, row_ok, n_base, alpha, cnt, &tmY, ybox,
+                                                           row - lane);
+        else epi_tile<TOut, EPI, BNG, -1>(p, es, t_row, row, row_ok, n_base, alpha, cnt, &tmY, ybox,
+                                                           row - lane);
       } else {
-        epi_tile<TOut, EPI, BN, 0>(p, es, t_row, row, row_ok, n_base, sx, alpha, cnt);
+        epi_tile<TOut, EPI, BNG, 0>(p, es, t_row, row, row_ok, n_base, alpha, cnt, &tmY, ybox,
+                                                           row - lane);
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tempty_bar[acc]);
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
+    if (lane == 0) bulk_wait<0>();   // this warp's Y stores are complete before the CTA exits
   }
 
   __syncthreads();
-  if (warp == 1) {
+  if (warp == GEMM_WARP_MMA) {
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem_base, 2 * BN);

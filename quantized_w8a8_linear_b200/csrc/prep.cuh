@@ -87,7 +87,14 @@ struct WoGather {
   int64_t N;
   const int32_t* O;
   uint16_t* W_O;
+  int8_t* WqO;   // [N, OUTL_CODES] weight codes of the first outlier columns, or nullptr
 };
+
+// Outlier counts up to OUTL_CODES also get compact int8 copies of the codes in
+// their columns (Xq[:,O] and Wq[:,O], zero-padded to OUTL_CODES per row), so
+// that the GEMM epilogue can take those columns' products back out without
+// gathering from Xq and Wq.
+constexpr int OUTL_CODES = 16;
 
 // Round-half-even of an fp32 value in (-2^22, 2^22) to an integer, read from
 // the low byte of t + 1.5 * 2^23: the add rounds to nearest even, and within
@@ -178,6 +185,7 @@ struct PrepArgs {
   uint32_t* rowctr;    // next-row counter (zero on entry), or nullptr for a static row split
   uint16_t* X_O;
   int64_t ostride;
+  int8_t* XqO;         // [M, OUTL_CODES] codes of the first outlier columns (count <= OUTL_CODES), or nullptr
   WoGather wo;
 };
 
@@ -465,6 +473,12 @@ __global__ void __launch_bounds__(RQ_THREADS, 3) k_prep_rows(const T* __restrict
     }
     mo = __reduce_max_sync(0xffffffffu, mo);
     const uint32_t mb = __ldcg(a.amax_bits + row);
+    if (a.XqO != nullptr && cnt <= OUTL_CODES && lane < OUTL_CODES) {
+      // the codes pass 1 left in the outlier columns (a requantised row gets 0 there)
+      int8_t c = 0;
+      if (lane < cnt && mo < mb) c = static_cast<int8_t>(__ldcg(a.Q + row * K + outlier_col(sflags, swpre, NW, lane)));
+      a.XqO[row * OUTL_CODES + lane] = c;
+    }
     if (mo >= mb) {
       // the pass-1 absmax may sit in an outlier column: requantise exactly
       uint32_t m = 0;
@@ -501,6 +515,15 @@ __global__ void __launch_bounds__(RQ_THREADS, 3) k_prep_rows(const T* __restrict
       if (o < cnt)
         val = __fmul_rn(static_cast<float>(a.wo.Wq[j * K + outlier_col(sflags, swpre, NW, o)]), __ldg(a.wo.s_w + j));
       a.wo.W_O[j * a.ostride + o] = from_f<T>(val);
+    }
+    if (a.wo.WqO != nullptr && cnt <= OUTL_CODES) {
+      const int64_t tq = a.wo.N * OUTL_CODES;
+      for (int64_t t = static_cast<int64_t>(blockIdx.x) * RQ_THREADS + tid; t < tq;
+           t += static_cast<int64_t>(gridDim.x) * RQ_THREADS) {
+        const int64_t j = t / OUTL_CODES;
+        const int o = static_cast<int>(t - j * OUTL_CODES);
+        a.wo.WqO[t] = o < cnt ? a.wo.Wq[j * K + outlier_col(sflags, swpre, NW, o)] : int8_t{0};
+      }
     }
   }
 }

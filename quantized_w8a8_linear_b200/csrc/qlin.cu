@@ -109,21 +109,53 @@ qlin_status make_tmap_k128(CUtensorMap* m, const void* base, int64_t rows, int64
   return QLIN_OK;
 }
 
+// 16-bit row-major Y [M, N] for the GEMM's TMA stores: box 16 columns x 32
+// rows, 32-byte swizzle (the epilogue writes its staging boxes in that layout).
+qlin_status make_tmap_y16(CUtensorMap* m, void* Y, int64_t M, int64_t N) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc;
+  qlin_status s = get_encode(&enc);
+  if (s != QLIN_OK) return s;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(N), static_cast<cuuint64_t>(M)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(N * 2)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(GEMM_CW), 32u};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, Y, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(QLIN_ERR_CUDA, "cuTensorMapEncodeTiled (Y) failed (%d)", static_cast<int>(r));
+  return QLIN_OK;
+}
+
 // ---- GEMM launch ------------------------------------------------------------
 constexpr int kBN = 256;
 constexpr int kStages = 4;
 
 template <int KIND, int EPI, typename TOut>
-qlin_status launch_gemm(const void* A, const void* B, const EpiParams& ep, cudaStream_t st, int attr_slot) {
+qlin_status launch_gemm(const void* A, const void* B, EpiParams ep, cudaStream_t st, int attr_slot) {
   DeviceInfo* d;
   qlin_status s = device_info(&d);
   if (s != QLIN_OK) return s;
-  CUtensorMap ta, tb;
+  CUtensorMap ta, tb, ty;
   if ((s = make_tmap_k128(&ta, A, ep.M, ep.K, GEMM_BM)) != QLIN_OK) return s;
   if ((s = make_tmap_k128(&tb, B, ep.N, ep.K, kBN)) != QLIN_OK) return s;
+  std::memset(&ty, 0, sizeof(ty));
+  ep.tma_y = 0;
+  // 16-bit Y goes out through TMA when its rows are 16-byte multiples and it is 16-byte aligned
+  constexpr bool y16 = EPI != EPI_I32 && EPI != EPI_INT8_OUTLIER_I32;
+  if (y16 && ep.N % 8 == 0 && aligned16(ep.Y)) {
+    if ((s = make_tmap_y16(&ty, ep.Y, ep.M, ep.N)) != QLIN_OK) return s;
+    ep.tma_y = 1;
+  }
   auto kern = k_gemm<KIND, EPI, TOut, kBN, kStages>;
   constexpr int smem = GemmSmem<kBN, kStages>::TOTAL;
   if (!d->gemm_attr_set[attr_slot]) {
+    // the kernel's warpgroups trade registers with setmaxnreg: the launch
+    // register count must leave enough in the block's pool for the split
+    cudaFuncAttributes fa{};
+    s = check_cuda(cudaFuncGetAttributes(&fa, kern), "cudaFuncGetAttributes");
+    if (s != QLIN_OK) return s;
+    if (fa.numRegs < GEMM_REGS_MIN_LAUNCH || fa.numRegs > GEMM_REGS_HIGH)
+      return fail(QLIN_ERR_UNSUPPORTED, "k_gemm was built with %d registers per thread; the register split needs %d..%d",
+                  fa.numRegs, GEMM_REGS_MIN_LAUNCH, GEMM_REGS_HIGH);
     s = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
                    "cudaFuncSetAttribute");
     if (s != QLIN_OK) return s;
@@ -131,7 +163,7 @@ qlin_status launch_gemm(const void* A, const void* B, const EpiParams& ep, cudaS
   }
   const int64_t tiles = ((ep.M + GEMM_BM - 1) / GEMM_BM) * ((ep.N + kBN - 1) / kBN);
   const int grid = static_cast<int>(tiles < d->sms ? tiles : d->sms);
-  kern<<<grid, GEMM_THREADS, smem, st>>>(ta, tb, ep);
+  kern<<<grid, GEMM_THREADS, smem, st>>>(ta, tb, ty, ep);
   return check_cuda(cudaGetLastError(), "k_gemm launch");
 }
 
@@ -232,6 +264,8 @@ struct Int8Ws {
   int8_t* Xq;         // [M,K]
   uint16_t* X_O;      // [M,ostride]
   uint16_t* W_O;      // [N,ostride]
+  int8_t* XqO;        // [M,OUTL_CODES]
+  int8_t* WqO;        // [N,OUTL_CODES]
   int64_t ostride;
   size_t memset_bytes;  // zeroed each call: sync, count, rowctr, flags
   size_t total;
@@ -261,6 +295,8 @@ Int8Ws int8_layout(void* base, int64_t M, int64_t N, int64_t K, bool with_gemm_p
     w.Xq = reinterpret_cast<int8_t*>(take(static_cast<size_t>(M * K)));
     w.X_O = reinterpret_cast<uint16_t*>(take(static_cast<size_t>(2 * M * w.ostride)));
     w.W_O = reinterpret_cast<uint16_t*>(take(static_cast<size_t>(2 * N * w.ostride)));
+    w.XqO = reinterpret_cast<int8_t*>(take(static_cast<size_t>(M * OUTL_CODES)));
+    w.WqO = reinterpret_cast<int8_t*>(take(static_cast<size_t>(N * OUTL_CODES)));
   }
   w.total = off;
   return w;
@@ -271,7 +307,7 @@ bool decomposition_on(float thr) { return thr > 0.0f && !std::isinf(thr); }
 template <typename T>
 qlin_status int8_prep_impl(const void* X, int64_t M, int64_t K, float thr, const Int8Ws& w, int8_t* Xq, float* s_x,
                            uint16_t* X_O, int64_t ostride, cudaStream_t st,
-                           WoGather wo = WoGather{nullptr, nullptr, 0, nullptr, nullptr}) {
+                           WoGather wo = WoGather{nullptr, nullptr, 0, nullptr, nullptr, nullptr}) {
   qlin_status s = check_cuda(cudaMemsetAsync(w.sync, 0, w.memset_bytes, st), "cudaMemsetAsync");
   if (s != QLIN_OK) return s;
   if (M == 0) return QLIN_OK;
@@ -280,7 +316,8 @@ qlin_status int8_prep_impl(const void* X, int64_t M, int64_t K, float thr, const
     a.M = M; a.K = K; a.thr = thr; a.thr_bits = threshold_bits<T>(thr);
     a.Q = reinterpret_cast<uint8_t*>(Xq); a.s_f32 = s_x; a.amax_bits = w.amax;
     a.flags = w.flags; a.O = w.O; a.count = w.count; a.sync = w.sync; a.X_O = X_O;
-    a.rowctr = M < (int64_t{1} << 31) ? w.rowctr : nullptr; a.ostride = ostride; a.wo = wo;
+    a.rowctr = M < (int64_t{1} << 31) ? w.rowctr : nullptr;
+    a.XqO = w.XqO; a.ostride = ostride; a.wo = wo;
     return launch_prep<T, 0, false, true>(X, a, st);
   }
   return launch_rowquant<T, 0, false>(X, M, K, reinterpret_cast<uint8_t*>(Xq), s_x, nullptr, st);
@@ -535,7 +572,7 @@ qlin_status qlin_int8_outlier_prepare(const void* X, qlin_dtype xdt, int64_t M, 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   Int8Ws w = int8_layout(workspace, M, N, K, true);
   const bool bf = (xdt == QLIN_BF16);
-  const WoGather wo{Wq, w_scale, N, w.O, w.W_O};
+  const WoGather wo{Wq, w_scale, N, w.O, w.W_O, w.WqO};
   QLIN_TRY(bf ? int8_prep_impl<__nv_bfloat16>(X, M, K, threshold, w, w.Xq, w.s_x, w.X_O, w.ostride, st, wo)
               : int8_prep_impl<__half>(X, M, K, threshold, w, w.Xq, w.s_x, w.X_O, w.ostride, st, wo));
   (void)d;
@@ -563,7 +600,7 @@ qlin_status qlin_int8_outlier_gemm(qlin_dtype xdt, int64_t M, int64_t K, const i
   ep.M = M; ep.N = N; ep.K = K; ep.Y = Y;
   ep.s_x = w.s_x; ep.s_w = w_scale; ep.bias = static_cast<const uint16_t*>(bias);
   ep.count = w.count; ep.X_O = w.X_O; ep.W_O = w.W_O; ep.ostride = w.ostride;
-  ep.Xq = w.Xq; ep.Wq = Wq; ep.O = w.O;
+  ep.Xq = w.Xq; ep.Wq = Wq; ep.O = w.O; ep.XqO = w.XqO; ep.WqO = w.WqO;
   if (xdt == QLIN_BF16) QLIN_TRY((launch_gemm<0, EPI_INT8_OUTLIER, __nv_bfloat16>(w.Xq, Wq, ep, st, 1)));
   else QLIN_TRY((launch_gemm<0, EPI_INT8_OUTLIER, __half>(w.Xq, Wq, ep, st, 2)));
   return ok();
@@ -583,7 +620,7 @@ qlin_status qlin_int8_outlier_gemm_i32(int64_t M, int64_t K, const int8_t* Wq, i
   Int8Ws w = int8_layout(workspace, M, N, K, true);
   EpiParams ep{};
   ep.M = M; ep.N = N; ep.K = K; ep.Y = C;
-  ep.count = w.count; ep.Xq = w.Xq; ep.Wq = Wq; ep.O = w.O;
+  ep.count = w.count; ep.Xq = w.Xq; ep.Wq = Wq; ep.O = w.O; ep.XqO = w.XqO; ep.WqO = w.WqO;
   QLIN_TRY((launch_gemm<0, EPI_INT8_OUTLIER_I32, __nv_bfloat16>(w.Xq, Wq, ep, static_cast<cudaStream_t>(stream), 7)));
   return ok();
 }
