@@ -159,10 +159,13 @@ __device__ __forceinline__ uint32_t keep_mask(uint32_t om, int i) {
 //            the host before the launch; all CTAs are co-resident);
 //   compact  every CTA scans the bitmap into shared memory (per-word prefix
 //            counts); CTA 0 writes the ascending list O and the count;
-//   fix-up   per row, one warp reads the row's values in the O columns:
-//            copies them to X_O (zero-padded to a multiple of 8), sets their
-//            codes to 0, and if the largest of them that is <= thr reaches
-//            the kept absmax, requantises the whole row with the exact absmax;
+//   fix-up   per row, one warp reads the row's values in the O columns and
+//            copies them to X_O (zero-padded to a multiple of 8) and, for up
+//            to OUTL_CODES columns, the codes pass 1 left there to XqO (the
+//            GEMM takes those codes' products back out, so Xq keeps them); if
+//            the largest of the values that is <= thr reaches the kept
+//            absmax, the row is requantised with the exact absmax (by the
+//            whole CTA, from shared memory), its outlier codes then 0;
 //   W_O      the dequantised outlier weight columns (wo.N > 0).
 // ---------------------------------------------------------------------------
 constexpr int RQ_THREADS = 256;
@@ -292,7 +295,7 @@ __global__ void __launch_bounds__(RQ_THREADS, 3) k_prep_rows(const T* __restrict
   uint4* stage = reinterpret_cast<uint4*>(psm + ((OUTL ? 2 * NW : 0) + 3) / 4 * 4);
   // rows: taken one at a time from a global counter (balances the units when
   // rows cost different amounts), or split statically. The unit's leader keeps
-  // a ring of the unit's next row indices in shared memory, three ahead.
+  // a ring of the unit's next row indices in shared memory, two ahead.
   const int64_t first = static_cast<int64_t>(blockIdx.x) * units + unit;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * units;
   __shared__ long long rowq[RQ_WARPS][4];
@@ -310,11 +313,10 @@ __global__ void __launch_bounds__(RQ_THREADS, 3) k_prep_rows(const T* __restrict
     }
     cp_async_commit();
   };
-  static_assert(PF_DEPTH <= 3, "the row ring holds the current row and three more");
+  static_assert(PF_DEPTH == 2, "rows are taken two ahead: the one in flight and the next");
   if (ut == 0) {
     myq[0] = grab(0);
     myq[1] = grab(1);
-    myq[2] = grab(2);
   }
   if (rw == 1) __syncwarp();
   else asm volatile("bar.sync %0, %1;" ::"r"(1 + unit), "r"(UT) : "memory");
@@ -325,9 +327,10 @@ __global__ void __launch_bounds__(RQ_THREADS, 3) k_prep_rows(const T* __restrict
     const int64_t row = myq[t & 3];
     if (row >= M) break;
     issue(myq[(t + PF_DEPTH - 1) & 3], (slot + PF_DEPTH - 1) % PF_DEPTH);
-    // the slot read two iterations ago is free; every thread of the unit has
-    // passed that iteration's barrier (unit_max) since reading it
-    if (ut == 0) myq[(t + 3) & 3] = grab(t + 3);
+    // slot (t+2)&3 was last read two iterations ago, before that iteration's
+    // barrier (unit_max); its new row is first read at iteration t+1
+    // (prefetch), after this iteration's barrier
+    if (ut == 0) myq[(t + 2) & 3] = grab(t + 2);
     if (rw == 1) __syncwarp();
     cp_async_wait<PF_DEPTH - 1>();   // this thread's copies of `row` have landed
     uint4 cur[V];
@@ -457,6 +460,21 @@ __global__ void __launch_bounds__(RQ_THREADS, 3) k_prep_rows(const T* __restrict
   const int pad = (cnt + 7) & ~7;
 
   // ---------------- fix-up: one warp per row ----------------
+  constexpr int RQ_LIST = 32;
+  __shared__ long long rq_rows[RQ_LIST];
+  __shared__ int rq_n;
+  if (tid == 0) rq_n = 0;
+  __syncthreads();
+  // a vector of the row with its outlier columns' entries zeroed
+  auto masked_vec = [&](const T* xr, int64_t idx) -> uint4 {
+    uint4 x = ld_nc_v4(reinterpret_cast<const uint4*>(xr) + idx);
+    const uint32_t omv = (sflags[idx >> 2] >> ((idx & 3) * 8)) & 0xFFu;
+    x.x &= keep_mask(omv, 0);
+    x.y &= keep_mask(omv, 1);
+    x.z &= keep_mask(omv, 2);
+    x.w &= keep_mask(omv, 3);
+    return x;
+  };
   for (int64_t row = static_cast<int64_t>(blockIdx.x) * RQ_WARPS + warp; row < M;
        row += static_cast<int64_t>(gridDim.x) * RQ_WARPS) {
     const T* xr = X + row * K;
@@ -480,28 +498,67 @@ __global__ void __launch_bounds__(RQ_THREADS, 3) k_prep_rows(const T* __restrict
       a.XqO[row * OUTL_CODES + lane] = c;
     }
     if (mo >= mb) {
-      // the pass-1 absmax may sit in an outlier column: requantise exactly
-      uint32_t m = 0;
-      for (int64_t idx = lane; idx < KV; idx += 32) {
-        uint4 x = ld_nc_v4(reinterpret_cast<const uint4*>(xr) + idx);
-        const uint32_t omv = (sflags[idx >> 2] >> ((idx & 3) * 8)) & 0xFFu;
-        x.x &= keep_mask(omv, 0);
-        x.y &= keep_mask(omv, 1);
-        x.z &= keep_mask(omv, 2);
-        x.w &= keep_mask(omv, 3);
-        m = vec_absmax2<T>(m, x);
-      }
-      m = __reduce_max_sync(0xffffffffu, pair_max_bits(m));
-      const float s = to_f<T>(static_cast<uint16_t>(m)) / QMAX;
-      if (lane == 0) a.s_f32[row] = s;
-      const float inv = 1.0f / s;
-      const bool zero = (s == 0.0f), fast = s >= 1.17549435e-38f;
-      for (int64_t idx = lane; idx < KV; idx += 32) {
-        const uint4 x = ld_nc_v4(reinterpret_cast<const uint4*>(xr) + idx);
-        const uint32_t omv = (sflags[idx >> 2] >> ((idx & 3) * 8)) & 0xFFu;
-        *reinterpret_cast<uint2*>(a.Q + row * K + idx * 8) = quant_vec<T, CODE>(x, omv, inv, fast, zero);
+      // the pass-1 absmax may sit in an outlier column: requantise exactly,
+      // by the whole CTA below (a row is up to 64 KB: one warp alone would
+      // take tens of microseconds), or by this warp if the list is full
+      int slot = 0;
+      if (lane == 0) slot = atomicAdd(&rq_n, 1);
+      slot = __shfl_sync(0xffffffffu, slot, 0);
+      if (slot < RQ_LIST) {
+        if (lane == 0) rq_rows[slot] = row;
+      } else {
+        uint32_t m = 0;
+        for (int64_t idx = lane; idx < KV; idx += 32) m = vec_absmax2<T>(m, masked_vec(xr, idx));
+        m = __reduce_max_sync(0xffffffffu, pair_max_bits(m));
+        const float s = to_f<T>(static_cast<uint16_t>(m)) / QMAX;
+        if (lane == 0) a.s_f32[row] = s;
+        const float inv = 1.0f / s;
+        const bool zero = (s == 0.0f), fast = s >= 1.17549435e-38f;
+        for (int64_t idx = lane; idx < KV; idx += 32) {
+          const uint4 x = ld_nc_v4(reinterpret_cast<const uint4*>(xr) + idx);
+          const uint32_t omv = (sflags[idx >> 2] >> ((idx & 3) * 8)) & 0xFFu;
+          *reinterpret_cast<uint2*>(a.Q + row * K + idx * 8) = quant_vec<T, CODE>(x, omv, inv, fast, zero);
+        }
       }
     }
+  }
+  __syncthreads();
+  // the CTA's listed rows, each read once into the pass-1 staging area (which
+  // holds at least one row), then reduced and quantised from there
+  const int nrq = min(rq_n, RQ_LIST);
+  for (int i = 0; i < nrq; ++i) {
+    const int64_t row = rq_rows[i];
+    const uint4* xr = reinterpret_cast<const uint4*>(X + row * K);
+    for (int idx = tid; idx < KV; idx += RQ_THREADS) cp_async16(&stage[idx], xr + idx, true);
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncthreads();
+    uint32_t m = 0;
+    for (int idx = tid; idx < KV; idx += RQ_THREADS) {
+      uint4 x = stage[idx];
+      const uint32_t omv = (sflags[idx >> 2] >> ((idx & 3) * 8)) & 0xFFu;
+      x.x &= keep_mask(omv, 0);
+      x.y &= keep_mask(omv, 1);
+      x.z &= keep_mask(omv, 2);
+      x.w &= keep_mask(omv, 3);
+      m = vec_absmax2<T>(m, x);
+    }
+    m = __reduce_max_sync(0xffffffffu, pair_max_bits(m));
+    if (lane == 0) red[0][warp] = m;
+    __syncthreads();
+    m = 0;
+#pragma unroll
+    for (int w = 0; w < RQ_WARPS; ++w) m = max(m, red[0][w]);
+    const float s = to_f<T>(static_cast<uint16_t>(m)) / QMAX;
+    if (tid == 0) a.s_f32[row] = s;
+    const float inv = 1.0f / s;
+    const bool zero = (s == 0.0f), fast = s >= 1.17549435e-38f;
+    for (int idx = tid; idx < KV; idx += RQ_THREADS) {
+      const uint32_t omv = (sflags[idx >> 2] >> ((idx & 3) * 8)) & 0xFFu;
+      *reinterpret_cast<uint2*>(a.Q + row * K + static_cast<int64_t>(idx) * 8) =
+          quant_vec<T, CODE>(stage[idx], omv, inv, fast, zero);
+    }
+    __syncthreads();   // stage and red are reused by the next row
   }
 
   // ---------------- outlier weight columns ----------------
