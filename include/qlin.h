@@ -237,6 +237,12 @@ QLIN_API qlin_status qlin_w4a8_group_i32(const int8_t *Xq, const uint8_t *Wq4, i
 QLIN_API qlin_status qlin_fp8_prep(const void *X, qlin_dtype xdt, int64_t M, int64_t K,
                           const float *x_scale, uint8_t *Xq, float *s_x, void *stream);
 
+/* The E4M3 conversion every FP8 kernel uses (cvt.rn.satfinite.e4m3x2.f32),
+ * applied to n fp32 values t: codes[i] = round-to-nearest-even E4M3 of t[i],
+ * saturating to +-448 (Text-Encoder-FP8 page, "How it was tested": 3-bit
+ * mantissa). Parity export; n >= 0, no alignment requirement. */
+QLIN_API qlin_status qlin_e4m3_encode_f32(const float *t, uint8_t *codes, int64_t n, void *stream);
+
 /* ---------------- LLM.int8 forward with built-in scratch ------------------------------ */
 
 /* Size of the library's built-in scratch array (64 MiB per device). */

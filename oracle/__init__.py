@@ -59,6 +59,9 @@ def lib() -> ctypes.CDLL:
             "orc_e4m3_decode": (ctypes.c_double, [ctypes.c_uint8]),
             "orc_e4m3_encode": (ctypes.c_uint8, [f32]),
             "orc_e4m3_encode_search": (ctypes.c_uint8, [f32]),
+            "orc_e4m3_encode_bits": (ctypes.c_uint8, [f32]),
+            "orc_e4m3_compare_encoders": (ctypes.c_int64, [ctypes.c_uint64, ctypes.c_uint64]),
+            "orc_e4m3_encode_range": (None, [ctypes.c_uint64, ctypes.c_uint64, P]),
             "orc_q_int8": (i32, [f32, f32]),
             "orc_q_int4": (i32, [f32, f32]),
             "orc_q_e4m3": (ctypes.c_uint8, [f32, f32]),
@@ -148,6 +151,23 @@ def e4m3_encode(t: float) -> int:
 
 def e4m3_encode_search(t: float) -> int:
     return lib().orc_e4m3_encode_search(float(t))
+
+
+def e4m3_encode_bits(t: float) -> int:
+    """Third encoder, integer arithmetic on the fp32 bit fields (pins e4m3_encode)."""
+    return lib().orc_e4m3_encode_bits(float(t))
+
+
+def e4m3_compare_encoders(lo: int, count: int) -> int:
+    """Mismatches of e4m3_encode vs e4m3_encode_bits over fp32 bit patterns [lo, lo+count)."""
+    return int(lib().orc_e4m3_compare_encoders(int(lo), int(count)))
+
+
+def e4m3_encode_range(lo: int, count: int) -> np.ndarray:
+    """e4m3_encode of the floats with bit patterns lo .. lo+count-1."""
+    out = np.empty((count,), np.uint8)
+    lib().orc_e4m3_encode_range(int(lo), int(count), _p(out))
+    return out
 
 
 def q_int8(v: float, inv: float) -> int:

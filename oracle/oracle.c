@@ -178,6 +178,68 @@ uint8_t orc_e4m3_encode_search(float t) {
     return sign | (uint8_t)best;
 }
 
+/* A third E4M3 encoder, integer arithmetic on the fp32 bit fields (round
+ * to nearest even by shifting the 24-bit significand with a round bit and a
+ * sticky bit), used only to pin orc_e4m3_encode over all 2^32 inputs. */
+static uint32_t rne_shift(uint32_t x, int s) {
+    if (s <= 0) return x;
+    if (s > 31) return 0;
+    uint32_t q = x >> s;
+    uint32_t r = (x >> (s - 1)) & 1u;
+    uint32_t sticky = x & ((1u << (s - 1)) - 1u);
+    if (r && (sticky || (q & 1u))) ++q;
+    return q;
+}
+
+uint8_t orc_e4m3_encode_bits(float t) {
+    uint32_t u;
+    memcpy(&u, &t, 4);
+    const uint8_t sign = (uint8_t)((u >> 24) & 0x80u);
+    const uint32_t a = u & 0x7fffffffu;
+    if (a > 0x7f800000u) return 0x7f;           /* NaN */
+    if (a >= 0x7f800000u) return sign | 0x7e;   /* +-inf saturates */
+    const int E = (int)(a >> 23) - 127;         /* fp32 subnormals have E = -127 */
+    const uint32_t sig = (a >> 23) ? ((a & 0x7fffffu) | 0x800000u) : (a & 0x7fffffu);
+    if (E > 8) return sign | 0x7e;
+    if (E < -6) {
+        /* e4m3 subnormal: the code is round(|t| / 2^-9), |t| = sig * 2^(E - 23) */
+        const int sh = (E == -127) ? 23 + 126 - 9 : 23 - (E + 9);
+        const uint32_t q = rne_shift(sig, sh);   /* 0..8; 8 is the smallest normal, code 0x08 */
+        return sign | (uint8_t)q;
+    }
+    uint32_t q = rne_shift(sig, 20);            /* 4 significant bits: 8..16 */
+    int e = E;
+    if (q == 16u) { q = 8u; ++e; }
+    const int field = e + 7;
+    if (field > 15 || (field == 15 && q - 8u == 7u)) return sign | 0x7e;   /* above 448 */
+    return sign | (uint8_t)((field << 3) | (int)(q - 8u));
+}
+
+/* Mismatches between orc_e4m3_encode and orc_e4m3_encode_bits over the fp32
+ * bit patterns [lo, lo + count). */
+int64_t orc_e4m3_compare_encoders(uint64_t lo, uint64_t count) {
+    int64_t bad = 0;
+#pragma omp parallel for reduction(+ : bad) schedule(static)
+    for (int64_t i = 0; i < (int64_t)count; ++i) {
+        const uint32_t bits = (uint32_t)(lo + (uint64_t)i);
+        float t;
+        memcpy(&t, &bits, 4);
+        if (orc_e4m3_encode(t) != orc_e4m3_encode_bits(t)) ++bad;
+    }
+    return bad;
+}
+
+/* codes[i] = orc_e4m3_encode(float with bit pattern lo + i), i < count. */
+void orc_e4m3_encode_range(uint64_t lo, uint64_t count, uint8_t *codes) {
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < (int64_t)count; ++i) {
+        const uint32_t bits = (uint32_t)(lo + (uint64_t)i);
+        float t;
+        memcpy(&t, &bits, 4);
+        codes[i] = orc_e4m3_encode(t);
+    }
+}
+
 /* ------------------------------------------------------------------ */
 /* Quantiser Q(v, s): s = absmax / QMAX, inv = 1 / s, t = v * inv.     */
 /* ------------------------------------------------------------------ */

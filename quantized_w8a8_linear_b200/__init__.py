@@ -65,6 +65,7 @@ def _load() -> ctypes.CDLL:
         "qlin_outlier_weights": (st, [P, P, i64, i64, P, P, i32, P, i64, P]),
         "qlin_int8_gemm_i32": (st, [P, P, i64, i64, i64, P, P]),
         "qlin_fp8_prep": (st, [P, i32, i64, i64, P, P, P, P]),
+        "qlin_e4m3_encode_f32": (st, [P, P, i64, P]),
         "qlin_get_device_status": (st, [P, i32]),
         "qlin_set_wait_timeout_ns": (st, [ctypes.c_uint64]),
         "qlin_last_error_string": (ctypes.c_char_p, []),
@@ -356,6 +357,15 @@ def qlin_fp8_prep(X: torch.Tensor, x_scale: Optional[torch.Tensor] = None):
     s_x = torch.empty((M,), dtype=torch.float32, device=X.device)
     _check(lib.qlin_fp8_prep(_ptr(X), _dt(X), M, K, _ptr(x_scale), _ptr(Xq), _ptr(s_x), _stream(X.device)))
     return Xq, s_x
+
+
+def qlin_e4m3_encode_f32(t: torch.Tensor, codes: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """E4M3 codes of fp32 values with the device conversion the FP8 kernels use (parity export)."""
+    t = t.reshape(-1)
+    if codes is None:
+        codes = torch.empty(t.shape, dtype=torch.uint8, device=t.device)
+    _check(lib.qlin_e4m3_encode_f32(_ptr(t), _ptr(codes), t.numel(), _stream(t.device)))
+    return codes
 
 
 def qlin_get_device_status(reset: bool = False) -> int:

@@ -102,16 +102,6 @@ struct EpiStage {
   uint4 q[BN][4];
 };
 
-// Packed fp32 fused multiply-add: two IEEE fmas per instruction.
-__device__ __forceinline__ unsigned long long fma_f32x2(unsigned long long a, unsigned long long b,
-                                                        unsigned long long c) {
-  unsigned long long d;
-  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-  return d;
-}
-__device__ __forceinline__ unsigned long long f32x2_of(uint32_t lo, uint32_t hi) {
-  return static_cast<unsigned long long>(lo) | (static_cast<unsigned long long>(hi) << 32);
-}
 
 template <int BN, int STAGES>
 struct GemmSmem {

@@ -16,7 +16,10 @@
 //                writes), then hand the stage to the MMA;
 //   warps 4-11   promotion + epilogue, two warps per 32-lane TMEM quarter,
 //                each with 64 columns: per group, int32 -> fp32 (exact: |C_g|
-//                <= 128*127*7 < 2^22) and sum += s_w[j,g] * C_g in registers;
+//                <= 128*127*7 < 2^22) and sum += s_w[j,g] * C_g in registers
+//                (packed f32x2 arithmetic); the next group's accumulator is
+//                read from TMEM while this one is promoted, and an accumulator
+//                is handed back to the MMA as soon as it has been read;
 //                after the last group, y = s_x[i] * sum + bias -> Y.
 // All waits are bounded (common.cuh).
 #pragma once
@@ -30,6 +33,14 @@ constexpr int W4_CONV_WARPS = 2, W4_PROMO_WARPS = 8;
 constexpr int W4_THREADS = 32 * (2 + W4_CONV_WARPS + W4_PROMO_WARPS);
 constexpr int W4_ACC = 4;                             // TMEM group accumulators (4 x 128 columns)
 constexpr int W4_SWIN = 32;                           // groups per staged window of weight scales
+// Register split (setmaxnreg): warpgroup 0 (producer, MMA, converters) drops
+// to W4_REGS_LOW, the promotion warpgroups rise to W4_REGS_HIGH. It fits the
+// block's pool when 128 (R - LOW) >= 256 (HIGH - R) for the launch count R.
+constexpr int W4_REGS_LOW = 64;
+constexpr int W4_REGS_HIGH = 216;
+constexpr int W4_REGS_MIN_LAUNCH = 166;
+static_assert(128 * (W4_REGS_MIN_LAUNCH - W4_REGS_LOW) >= 256 * (W4_REGS_HIGH - W4_REGS_MIN_LAUNCH),
+              "register split must fit the launch pool");
 
 struct W4Params {
   int64_t M, N, K;
@@ -122,6 +133,8 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
+  if (warp < 2 + W4_CONV_WARPS) {
+  setmaxnreg_dec<W4_REGS_LOW>();
   if (warp == 0) {
     if (lane == 0) {
       // ---------------- TMA producer ----------------
@@ -209,7 +222,9 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
       }
       if (!ok) break;
     }
+  }
   } else {
+    setmaxnreg_inc<W4_REGS_HIGH>();
     // ---------------- promotion + epilogue ----------------
     const int pw = warp - (2 + W4_CONV_WARPS);   // 0..7
     const int q = warp & 3;                      // TMEM lane quarter
@@ -218,14 +233,45 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
     int buf = 0;
     uint32_t buf_phase = 0, bar_phase = 0;
     bool ok = true;
+    // TMEM address of this warp's lane quarter, columns c0 + 32h of accumulator buffer b
+    auto taddr = [&](int b, int h) {
+      return tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * W4_BN + c0 + 32 * h);
+    };
+    uint32_t rx[32], ry[32];   // half 0 and half 1 of a group's 64 columns
     for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
       const int mb = tile % num_m, nb = tile / num_m;
       const int64_t n_base = static_cast<int64_t>(nb) * W4_BN;
       const int64_t row = static_cast<int64_t>(mb) * W4_BM + q * 32 + lane;
       const bool row_ok = row < M;
-      float acc[64];
+      unsigned long long acc[32];   // 64 fp32 sums as pairs
 #pragma unroll
-      for (int j = 0; j < 64; ++j) acc[j] = 0.0f;
+      for (int j = 0; j < 32; ++j) acc[j] = 0ull;
+      // acc[16h..16h+15] += s_w[., g] * float(C_g) for half h of the warp's columns
+      auto promote = [&](int g, int h, const uint32_t (&r)[32]) {
+        const float2* sw = reinterpret_cast<const float2*>(s_win + (g % W4_SWIN) * W4_BN + c0 + 32 * h);
+        // int32 -> fp32: |C| < 2^22, so C + 1.5*2^23 is exact as a float and subtracting gives C
+        const unsigned long long magic = f32x2_of(__float_as_uint(-12582912.0f), __float_as_uint(-12582912.0f));
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const unsigned long long c =
+              add_f32x2(f32x2_of(static_cast<uint32_t>(static_cast<int32_t>(r[2 * j]) + 0x4B400000),
+                                 static_cast<uint32_t>(static_cast<int32_t>(r[2 * j + 1]) + 0x4B400000)),
+                        magic);
+          const float2 s2 = sw[j];
+          acc[16 * h + j] = fma_f32x2(f32x2_of(__float_as_uint(s2.x), __float_as_uint(s2.y)), c, acc[16 * h + j]);
+        }
+        if (p.dbg != nullptr && g == p.dbg_group && row_ok) {
+          for (int j = 0; j < 32; ++j) {
+            const int64_t n = n_base + c0 + 32 * h + j;
+            if (n < N) p.dbg[row * N + n] = static_cast<int32_t>(r[j]);
+          }
+        }
+      };
+      // half 0 of group 0
+      if (!mbar_wait(&gfull_bar[buf], buf_phase, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      __syncwarp();
+      tmem_ld32(taddr(buf, 0), rx);
       for (int g = 0; g < G; ++g) {
         if (g % W4_SWIN == 0) {
           // stage the weight scales of groups [g, g + W4_SWIN) for the tile's columns
@@ -237,35 +283,31 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
           }
           if (!epi_bar(promo_bar, bar_phase, abort_flag)) { ok = false; break; }
         }
-        if (!mbar_wait(&gfull_bar[buf], buf_phase, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(buf * W4_BN);
-        const float* sw = s_win + (g % W4_SWIN) * W4_BN + c0;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t r[32];
-          __syncwarp();
-          tmem_ld32(t_row + static_cast<uint32_t>(c0 + 32 * h), r);
-          tmem_ld_wait();
-          // int32 -> fp32: |C| < 2^22, so C + 1.5*2^23 is exact and subtracting gives C
-#pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const float c = __fsub_rn(__int_as_float(static_cast<int32_t>(r[j]) + 0x4B400000), 12582912.0f);
-            acc[32 * h + j] = fmaf(sw[32 * h + j], c, acc[32 * h + j]);
-          }
-          if (p.dbg != nullptr && g == p.dbg_group && row_ok) {
-            for (int j = 0; j < 32; ++j) {
-              const int64_t n = n_base + c0 + 32 * h + j;
-              if (n < N) p.dbg[row * N + n] = static_cast<int32_t>(r[j]);
-            }
-          }
-        }
+        // half 0 landed; half 1 of the same buffer in flight while half 0 is promoted
+        __syncwarp();
+        tmem_wait_regs32(rx);
+        tmem_ld32(taddr(buf, 1), ry);
+        promote(g, 0, rx);
+        __syncwarp();
+        tmem_wait_regs32(ry);
+        // both halves read: the buffer goes back to the MMA
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&gempty_bar[buf]);
         if (++buf == W4_ACC) { buf = 0; buf_phase ^= 1u; }
+        // half 0 of the next group in flight while half 1 is promoted
+        if (g + 1 < G) {
+          if (!mbar_wait(&gfull_bar[buf], buf_phase, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          __syncwarp();
+          tmem_ld32(taddr(buf, 0), rx);
+        }
+        promote(g, 1, ry);
       }
-      if (!ok) break;
+      if (!ok) {
+        tmem_ld_wait();   // no TMEM load of this warp is left in flight when the CTA winds down
+        break;
+      }
       if (row_ok && p.dbg == nullptr) {
         const float sx = __ldg(p.s_x + row);
 #pragma unroll
@@ -277,7 +319,9 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
           for (int j = 0; j < 32; ++j) {
             const int64_t n = n0 + j;
             const float b = (p.bias != nullptr && n < N) ? to_f<TOut>(__ldg(p.bias + n)) : 0.0f;
-            y[j] = sx * acc[32 * h + j] + b;
+            const unsigned long long a2 = acc[16 * h + j / 2];
+            const float a = __uint_as_float(static_cast<uint32_t>((j & 1) ? (a2 >> 32) : a2));
+            y[j] = sx * a + b;
           }
           uint16_t* yp = reinterpret_cast<uint16_t*>(p.Y) + row * N + n0;
           if (n0 + 32 <= N && (N & 7) == 0) {

@@ -602,6 +602,18 @@ __global__ void __launch_bounds__(256) k_gather_wo(const int8_t* __restrict__ Wq
 
 // Static per-tensor E4M3 codes: Xq = e4m3(x * (1 / *x_scale)); all-zero
 // codes if the scale is 0. Grid-stride over 8-element vectors.
+// E4M3 codes of n fp32 values (grid-stride, two per conversion).
+__global__ void __launch_bounds__(256) k_e4m3_encode(const float* __restrict__ t, uint8_t* __restrict__ codes,
+                                                   int64_t n) {
+  for (int64_t i = 2 * (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x); i < n;
+       i += 2 * static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float a = t[i], b = i + 1 < n ? t[i + 1] : 0.0f;
+    const uint32_t c = e4m3x2(a, b);
+    codes[i] = static_cast<uint8_t>(c & 0xFFu);
+    if (i + 1 < n) codes[i + 1] = static_cast<uint8_t>(c >> 8);
+  }
+}
+
 // The codes of the outlier columns set to 0 in Q [M,K] (a warp per row). The
 // fused forward never needs this: its GEMM takes those codes as 0 on its own.
 __global__ void __launch_bounds__(256) k_zero_outlier_cols(int8_t* __restrict__ Q, int64_t M, int64_t K,

@@ -636,6 +636,18 @@ qlin_status qlin_int8_outlier_forward(const void* X, qlin_dtype xdt, int64_t M, 
   return qlin_int8_outlier_gemm(xdt, M, K, Wq, w_scale, N, bias, Y, workspace, ws_bytes, stream);
 }
 
+qlin_status qlin_e4m3_encode_f32(const float* t, uint8_t* codes, int64_t n, void* stream) {
+  if (n < 0) return fail(QLIN_ERR_INVALID_ARG, "negative size");
+  if (n == 0) return ok();
+  QLIN_REQ_PTR(t, "t");
+  QLIN_REQ_PTR(codes, "codes");
+  DeviceInfo* d;
+  QLIN_TRY(device_info(&d));
+  const int64_t want = (n + 511) / 512, cap = static_cast<int64_t>(d->sms) * 16;
+  k_e4m3_encode<<<static_cast<unsigned>(want < cap ? want : cap), 256, 0, static_cast<cudaStream_t>(stream)>>>(t, codes, n);
+  return check_cuda(cudaGetLastError(), "k_e4m3_encode launch");
+}
+
 qlin_status qlin_fp8_prep(const void* X, qlin_dtype xdt, int64_t M, int64_t K, const float* x_scale, uint8_t* Xq,
                           float* s_x, void* stream) {
   QLIN_TRY(check_common(X, xdt, M, K, 0));
@@ -755,6 +767,14 @@ qlin_status launch_w4a8(const int8_t* Xq, const uint8_t* Wq4, const W4Params& wp
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 16 && !attr_set[dev]) {
+    // the warpgroups trade registers with setmaxnreg: the launch register
+    // count must leave enough in the block's pool for the split
+    cudaFuncAttributes fa{};
+    s = check_cuda(cudaFuncGetAttributes(&fa, kern), "cudaFuncGetAttributes");
+    if (s != QLIN_OK) return s;
+    if (fa.numRegs < W4_REGS_MIN_LAUNCH || fa.numRegs > W4_REGS_HIGH)
+      return fail(QLIN_ERR_UNSUPPORTED, "k_gemm_w4a8 was built with %d registers per thread; the register split needs %d..%d",
+                  fa.numRegs, W4_REGS_MIN_LAUNCH, W4_REGS_HIGH);
     s = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, W4Smem::TOTAL),
                    "cudaFuncSetAttribute");
     if (s != QLIN_OK) return s;

@@ -80,6 +80,20 @@ def test_e4m3_codes_every_boundary(q):
         assert np.array_equal(codes.cpu().numpy(), ref), dtype
 
 
+def test_e4m3_device_conversion_all_finite_fp32(q):
+    """The conversion every FP8 kernel uses, on all 2^32 fp32 bit patterns,
+    against the oracle's encoder. Non-finite inputs are outside the reading
+    (the pages leave them unspecified), so NaN and infinity are skipped."""
+    chunk = 1 << 26
+    for lo in range(0, 1 << 32, chunk):
+        bits = torch.arange(lo, lo + chunk, dtype=torch.int64, device="cuda").to(torch.int32)
+        codes = q.qlin_e4m3_encode_f32(bits.view(torch.float32)).cpu().numpy()
+        ref = oracle.e4m3_encode_range(lo, chunk)
+        u = np.arange(lo, lo + chunk, dtype=np.uint64)
+        finite = ((u >> 23) & 0xFF) != 0xFF
+        assert np.array_equal(codes[finite], ref[finite]), hex(lo)
+
+
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
 def test_all_16bit_values_int8_and_e4m3(q, dtype):
     # every finite 16-bit pattern, one row per block of 2048, dynamic scales

@@ -173,3 +173,13 @@ def test_massive_activation_values_in_bf16():
     assert oracle.e4m3_scale(12992.0) == 29.0
     assert oracle.q_e4m3(12992.0, 1.0 / 29.0) == 0x7E
     assert math.isclose(oracle.e4m3_scale(9024.0), 9024.0 / 448.0, rel_tol=1e-7)
+
+
+def test_e4m3_encoder_matches_bitfield_encoder_on_all_fp32():
+    """Exhaustive pin of the E4M3 encoder: every one of the 2^32 fp32 bit
+    patterns gives the same code from the grid-rounding encoder (double
+    arithmetic) and from an integer encoder on the fp32 bit fields (round bit
+    and sticky bit on the 24-bit significand)."""
+    chunk = 1 << 28
+    for lo in range(0, 1 << 32, chunk):
+        assert oracle.e4m3_compare_encoders(lo, chunk) == 0, hex(lo)
