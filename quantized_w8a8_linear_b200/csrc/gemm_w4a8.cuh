@@ -5,15 +5,16 @@
 //   C_g[i,j] = sum_{k in group g} Xq[i,k] * Wq4[j,k]          (int32, exact)
 //   Y[i,j]   = dtype( s_x[i] * sum_g s_w[j,g] * C_g[i,j] + bias[j] )
 //
-// Roles (one CTA per SM, 12 warps, persistent over 128x128 output tiles):
+// Roles (one CTA per SM, 16 warps, persistent over 128x128 output tiles):
 //   warp 0       TMA producer: the int8 A tile (128 x 128 B) and the packed
 //                int4 B tile (128 rows x 64 B) of one group per stage;
 //   warp 1       MMA issuer: TMEM holds four 128-column int32 group
 //                accumulators; each group is 4 x tcgen05.mma kind::i8 (K=32)
 //                into a fresh accumulator;
-//   warps 2-3    converters: unpack the int4 B tile to int8 in the 128-byte
-//                swizzled K-major layout the MMA reads (the same layout TMA
+//   warps 2-3,   converters: unpack the int4 B tile to int8 in the 128-byte
+//   12-13        swizzled K-major layout the MMA reads (the same layout TMA
 //                writes), then hand the stage to the MMA;
+//   warps 14-15  idle;
 //   warps 4-11   promotion + epilogue, two warps per 32-lane TMEM quarter,
 //                each with 64 columns: per group, int32 -> fp32 (exact: |C_g|
 //                <= 128*127*7 < 2^22) and sum += s_w[j,g] * C_g in registers
@@ -29,17 +30,18 @@ namespace qlin {
 
 constexpr int W4_BM = 128, W4_BN = 128, W4_G = 128;   // tile rows, tile columns, group (= K per stage)
 constexpr int W4_STAGES = 4;
-constexpr int W4_CONV_WARPS = 2, W4_PROMO_WARPS = 8;
-constexpr int W4_THREADS = 32 * (2 + W4_CONV_WARPS + W4_PROMO_WARPS);
+constexpr int W4_CONV_WARPS = 4, W4_PROMO_WARPS = 8;
+constexpr int W4_THREADS = 512;   // 16 warps: 4 warpgroups (see the role list above)
 constexpr int W4_ACC = 4;                             // TMEM group accumulators (4 x 128 columns)
 constexpr int W4_SWIN = 32;                           // groups per staged window of weight scales
-// Register split (setmaxnreg): warpgroup 0 (producer, MMA, converters) drops
-// to W4_REGS_LOW, the promotion warpgroups rise to W4_REGS_HIGH. It fits the
-// block's pool when 128 (R - LOW) >= 256 (HIGH - R) for the launch count R.
-constexpr int W4_REGS_LOW = 64;
+// Register split (setmaxnreg): warpgroups 0 and 3 (producer, MMA, converters)
+// drop to W4_REGS_LOW, the promotion warpgroups 1 and 2 rise to W4_REGS_HIGH.
+// It fits the block's pool when 2 * 128 (R - LOW) >= 256 (HIGH - R) for the
+// launch count R.
+constexpr int W4_REGS_LOW = 40;
 constexpr int W4_REGS_HIGH = 216;
-constexpr int W4_REGS_MIN_LAUNCH = 166;
-static_assert(128 * (W4_REGS_MIN_LAUNCH - W4_REGS_LOW) >= 256 * (W4_REGS_HIGH - W4_REGS_MIN_LAUNCH),
+constexpr int W4_REGS_MIN_LAUNCH = 128;
+static_assert(2 * 128 * (W4_REGS_MIN_LAUNCH - W4_REGS_LOW) >= 256 * (W4_REGS_HIGH - W4_REGS_MIN_LAUNCH),
               "register split must fit the launch pool");
 
 struct W4Params {
@@ -63,13 +65,19 @@ struct W4Smem {
 };
 
 // 32 signed int4 (16 packed bytes, even k in the low nibble) -> 32 int8.
+// Per byte: 0x80 | (nibble ^ 8) is 0x80 + (t + 8) for the nibble's value t,
+// so subtracting 8 borrows from no neighbour and leaves 0x80 + t, and
+// flipping bit 7 gives t in two's complement.
+__device__ __forceinline__ uint32_t sext_nibbles(uint32_t nib4) {   // four nibbles in the low halves of 4 bytes
+  return ((((nib4 & 0x0F0F0F0Fu) ^ 0x88888888u) - 0x08080808u) ^ 0x80808080u);
+}
 __device__ __forceinline__ void unpack_int4x32(const uint4& p, uint4& lo16, uint4& hi16) {
   const uint32_t w[4] = {p.x, p.y, p.z, p.w};
   uint32_t o[8];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const uint32_t l = __vsub4((w[i] & 0x0F0F0F0Fu) ^ 0x08080808u, 0x08080808u);          // even k
-    const uint32_t h = __vsub4(((w[i] >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u, 0x08080808u);   // odd k
+    const uint32_t l = sext_nibbles(w[i]);        // even k
+    const uint32_t h = sext_nibbles(w[i] >> 4);   // odd k
     o[2 * i] = __byte_perm(l, h, 0x5140);
     o[2 * i + 1] = __byte_perm(l, h, 0x7362);
   }
@@ -133,7 +141,7 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp < 2 + W4_CONV_WARPS) {
+  if (warp < 4 || warp >= 12) {
   setmaxnreg_dec<W4_REGS_LOW>();
   if (warp == 0) {
     if (lane == 0) {
@@ -194,9 +202,9 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
       const uint64_t t0 = globaltimer();
       while (!mbar_try_wait(a, 0) && globaltimer() - t0 < g_wait_timeout_ns) {}
     }
-  } else if (warp < 2 + W4_CONV_WARPS) {
+  } else if (warp == 2 || warp == 3 || warp == 12 || warp == 13) {
     // ---------------- converters: packed int4 -> swizzled int8 ----------------
-    const int ct = threadIdx.x - 64;   // 0..127
+    const int ct = warp < 4 ? threadIdx.x - 64 : threadIdx.x - 384 + 64;   // 0..127
     int stage = 0;
     uint32_t phase = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
@@ -226,10 +234,10 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
   } else {
     setmaxnreg_inc<W4_REGS_HIGH>();
     // ---------------- promotion + epilogue ----------------
-    const int pw = warp - (2 + W4_CONV_WARPS);   // 0..7
+    const int pw = warp - 4;                     // 0..7
     const int q = warp & 3;                      // TMEM lane quarter
     const int c0 = (pw >> 2) * 64;               // this warp's first column of the tile
-    const int pt = threadIdx.x - 32 * (2 + W4_CONV_WARPS);   // 0..255
+    const int pt = threadIdx.x - 128;            // 0..255
     int buf = 0;
     uint32_t buf_phase = 0, bar_phase = 0;
     bool ok = true;
@@ -237,7 +245,7 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
     auto taddr = [&](int b, int h) {
       return tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * W4_BN + c0 + 32 * h);
     };
-    uint32_t rx[32], ry[32];   // half 0 and half 1 of a group's 64 columns
+    uint32_t ra0[32], ra1[32], rb0[32], rb1[32];   // two groups' 64 columns (halves 0 and 1)
     for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
       const int mb = tile % num_m, nb = tile / num_m;
       const int64_t n_base = static_cast<int64_t>(nb) * W4_BN;
@@ -267,12 +275,30 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
           }
         }
       };
-      // half 0 of group 0
-      if (!mbar_wait(&gfull_bar[buf], buf_phase, abort_flag)) { ok = false; break; }
-      tc_fence_after();
-      __syncwarp();
-      tmem_ld32(taddr(buf, 0), rx);
-      for (int g = 0; g < G; ++g) {
+      // Groups alternate between register sets a and b: group g+1's loads are
+      // issued right after group g's have landed and fly while g is promoted
+      // (tcgen05.wait::ld waits for all of a thread's loads, so the overlap is
+      // one group deep). An accumulator goes back to the MMA once it is read.
+      auto fetch = [&](uint32_t (&r0)[32], uint32_t (&r1)[32]) -> bool {
+        if (!mbar_wait(&gfull_bar[buf], buf_phase, abort_flag)) return false;
+        tc_fence_after();
+        __syncwarp();
+        tmem_ld32(taddr(buf, 0), r0);
+        tmem_ld32(taddr(buf, 1), r1);
+        return true;
+      };
+      auto landed = [&](uint32_t (&r0)[32], uint32_t (&r1)[32]) {
+        __syncwarp();
+        tmem_wait_regs32(r0);
+        tmem_wait_regs32(r1);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&gempty_bar[buf]);
+        if (++buf == W4_ACC) { buf = 0; buf_phase ^= 1u; }
+      };
+      static_assert(W4_SWIN % 2 == 0, "scale windows start on even groups (register set a)");
+      if (!fetch(ra0, ra1)) { ok = false; break; }
+      for (int g = 0; g < G; g += 2) {
         if (g % W4_SWIN == 0) {
           // stage the weight scales of groups [g, g + W4_SWIN) for the tile's columns
           if (!epi_bar(promo_bar, bar_phase, abort_flag)) { ok = false; break; }
@@ -283,26 +309,15 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
           }
           if (!epi_bar(promo_bar, bar_phase, abort_flag)) { ok = false; break; }
         }
-        // half 0 landed; half 1 of the same buffer in flight while half 0 is promoted
-        __syncwarp();
-        tmem_wait_regs32(rx);
-        tmem_ld32(taddr(buf, 1), ry);
-        promote(g, 0, rx);
-        __syncwarp();
-        tmem_wait_regs32(ry);
-        // both halves read: the buffer goes back to the MMA
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&gempty_bar[buf]);
-        if (++buf == W4_ACC) { buf = 0; buf_phase ^= 1u; }
-        // half 0 of the next group in flight while half 1 is promoted
-        if (g + 1 < G) {
-          if (!mbar_wait(&gfull_bar[buf], buf_phase, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          __syncwarp();
-          tmem_ld32(taddr(buf, 0), rx);
-        }
-        promote(g, 1, ry);
+        landed(ra0, ra1);
+        if (g + 1 < G && !fetch(rb0, rb1)) { ok = false; break; }
+        promote(g, 0, ra0);
+        promote(g, 1, ra1);
+        if (g + 1 >= G) break;
+        landed(rb0, rb1);
+        if (g + 2 < G && !fetch(ra0, ra1)) { ok = false; break; }
+        promote(g + 1, 0, rb0);
+        promote(g + 1, 1, rb1);
       }
       if (!ok) {
         tmem_ld_wait();   // no TMEM load of this warp is left in flight when the CTA winds down
