@@ -119,7 +119,7 @@ struct GemmSmem {
 
 template <typename TOut, int EPI, int BN>
 __device__ __forceinline__ void epi_stage(const EpiParams& p, EpiStage<BN>& es, int64_t n_base, int et, int cn) {
-  constexpr int PER = BN / GEMM_EPI_THREADS;
+  constexpr int PER = BN >= GEMM_EPI_THREADS ? BN / GEMM_EPI_THREADS : 1;   // columns per thread
   constexpr bool OUTL = EPI == EPI_INT8_OUTLIER || EPI == EPI_INT8_OUTLIER_I32;
   float sw[PER], b[PER];
   uint4 wo0[PER], wo1[PER], wq[PER];
@@ -127,10 +127,11 @@ __device__ __forceinline__ void epi_stage(const EpiParams& p, EpiStage<BN>& es, 
 #pragma unroll
   for (int i = 0; i < PER; ++i) {
     const int64_t n = n_base + et + i * GEMM_EPI_THREADS;
+    const bool mine = et + i * GEMM_EPI_THREADS < BN;
     sw[i] = 0.0f;
     b[i] = 0.0f;
     wo0[i] = wo1[i] = wq[i] = make_uint4(0u, 0u, 0u, 0u);
-    if (n < p.N) {
+    if (mine && n < p.N) {
       if constexpr (EPI == EPI_INT8_OUTLIER) sw[i] = __ldg(p.s_w + n);
       if constexpr (EPI == EPI_FP8_ROWCOL) sw[i] = to_f<__nv_bfloat16>(__ldg(p.s_w_bf16 + n));
       if constexpr (EPI == EPI_INT8_OUTLIER || EPI == EPI_FP8_TENSOR || EPI == EPI_FP8_ROWCOL)
@@ -150,6 +151,7 @@ __device__ __forceinline__ void epi_stage(const EpiParams& p, EpiStage<BN>& es, 
 #pragma unroll
   for (int i = 0; i < PER; ++i) {
     const int j = et + i * GEMM_EPI_THREADS;
+    if (j >= BN) continue;
     es.q[j][0] = make_uint4(__float_as_uint(sw[i]), __float_as_uint(b[i]), wq[i].x, wq[i].y);
     if constexpr (OUTL) {
       es.q[j][1] = wo0[i];
