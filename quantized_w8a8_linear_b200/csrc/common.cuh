@@ -251,6 +251,18 @@ __device__ __forceinline__ uint64_t sdesc_k128(uint32_t saddr) {
   return d;
 }
 
+// The same for a K-major tile of 32-byte rows in the 32B-swizzle layout
+// (8-row groups of 256 bytes; swizzle mode 6 = 32B).
+__device__ __forceinline__ uint64_t sdesc_k32(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>(1u) << 16;
+  d |= static_cast<uint64_t>(256u >> 4) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  d |= static_cast<uint64_t>(6u) << 61;
+  return d;
+}
+
 // Instruction descriptors (dense, K-major A and B, no negation):
 // bits 4-5 D format, 7-9 A format, 10-12 B format, 17-22 N>>3, 24-28 M>>4.
 __host__ __device__ constexpr uint32_t idesc_i8(int M, int N) {

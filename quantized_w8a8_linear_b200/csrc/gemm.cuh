@@ -56,7 +56,8 @@ constexpr int GEMM_REGS_MIN_LAUNCH = 160;
 static_assert(128 * (GEMM_REGS_MIN_LAUNCH - GEMM_REGS_LOW) >= 256 * (GEMM_REGS_HIGH - GEMM_REGS_MIN_LAUNCH),
               "register split must fit the launch pool");
 constexpr int GEMM_CW = 16;                  // accumulator columns per tcgen05.ld in the epilogue
-constexpr int GEMM_OUTL_STAGED = 16;         // outlier counts up to this take the staged fast path
+constexpr int GEMM_OUTL_STAGED = 16;         // outlier counts up to this take the staged fp part in the epilogue
+constexpr int GEMM_CORR_K = 32;              // outlier counts up to this take their int8 products out with one MMA
 
 struct EpiParams {
   int64_t M, N, K;
@@ -71,16 +72,17 @@ struct EpiParams {
   const uint16_t* X_O;        // [M, ostride] outlier activations
   const uint16_t* W_O;        // [N, ostride] dequantised outlier weights
   int64_t ostride;
-  // LLM.int8: the A operand may hold non-zero codes in outlier columns; the
-  // epilogue subtracts their exact int32 contribution
-  // sum_o Xq[m,O[o]] * Wq[n,O[o]] from the accumulator. Counts up to
-  // GEMM_OUTL_STAGED read the codes from the compact copies XqO / WqO (16 per
-  // row, zero-padded); larger counts gather them from Xq / Wq through O.
+  // LLM.int8: the A operand may hold non-zero codes in outlier columns, whose
+  // exact int32 contribution sum_o Xq[m,O[o]] * Wq[n,O[o]] leaves the
+  // accumulator: for counts up to GEMM_CORR_K by one more MMA per tile over
+  // the compact copies -Xq[:,O] and Wq[:,O] (the kernel's tmXc / tmWc tensor
+  // maps, [M,32] and [N,32], zero-padded); for larger counts in the epilogue,
+  // gathered from Xq / Wq through O.
   const int8_t* Xq;           // [M,K]
   const int8_t* Wq;           // [N,K]
   const int32_t* O;           // [K] ascending outlier columns, first *count valid
-  const int8_t* XqO;          // [M,16]
-  const int8_t* WqO;          // [N,16]
+  const int8_t* XqO;          // [M,32] -Xq[:,O] (host side: source of tmXc)
+  const int8_t* WqO;          // [N,32] Wq[:,O] (host side: source of tmWc)
   // 16-bit Y written through the kernel's Y tensor map (TMA stores of 32-row x
   // 16-column boxes from shared memory) instead of per-thread stores
   int tma_y;
@@ -89,17 +91,16 @@ struct EpiParams {
 constexpr int GEMM_YBOX_BYTES = 32 * GEMM_CW * 2;   // one warp's 32 rows x 16 columns of 16-bit Y
 
 // Per-tile column data staged in shared memory by an epilogue group, one
-// 64-byte record per column, read with 16-byte broadcasts (all lanes of a
+// 48-byte record per column, read with 16-byte broadcasts (all lanes of a
 // warp read the same address, so no bank conflicts and few wavefronts; the
 // tensor core reads its operands from the same shared memory):
-//   q[0] = {column scale (fp32), bias (fp32), WqO[n,0..3], WqO[n,4..7]}
+//   q[0] = {column scale (fp32), bias (fp32), 0, 0}
 //   q[1] = W_O[n, 0..7]    (16-bit)
-//   q[2] = {WqO[n,8..11], WqO[n,12..15], 0, 0}
-//   q[3] = W_O[n, 8..15]   (16-bit)
+//   q[2] = W_O[n, 8..15]   (16-bit)
 // Only q[0] is read without outliers, q[0..1] for up to 8 outlier columns.
 template <int BN>
 struct EpiStage {
-  uint4 q[BN][4];
+  uint4 q[BN][3];
 };
 
 
@@ -122,7 +123,7 @@ __device__ __forceinline__ void epi_stage(const EpiParams& p, EpiStage<BN>& es, 
   constexpr int PER = BN >= GEMM_EPI_THREADS ? BN / GEMM_EPI_THREADS : 1;   // columns per thread
   constexpr bool OUTL = EPI == EPI_INT8_OUTLIER || EPI == EPI_INT8_OUTLIER_I32;
   float sw[PER], b[PER];
-  uint4 wo0[PER], wo1[PER], wq[PER];
+  uint4 wo0[PER], wo1[PER];
   // every load first, then every store: one memory round trip per tile
 #pragma unroll
   for (int i = 0; i < PER; ++i) {
@@ -130,7 +131,7 @@ __device__ __forceinline__ void epi_stage(const EpiParams& p, EpiStage<BN>& es, 
     const bool mine = et + i * GEMM_EPI_THREADS < BN;
     sw[i] = 0.0f;
     b[i] = 0.0f;
-    wo0[i] = wo1[i] = wq[i] = make_uint4(0u, 0u, 0u, 0u);
+    wo0[i] = wo1[i] = make_uint4(0u, 0u, 0u, 0u);
     if (mine && n < p.N) {
       if constexpr (EPI == EPI_INT8_OUTLIER) sw[i] = __ldg(p.s_w + n);
       if constexpr (EPI == EPI_FP8_ROWCOL) sw[i] = to_f<__nv_bfloat16>(__ldg(p.s_w_bf16 + n));
@@ -138,7 +139,6 @@ __device__ __forceinline__ void epi_stage(const EpiParams& p, EpiStage<BN>& es, 
         if (p.bias != nullptr) b[i] = to_f<TOut>(__ldg(p.bias + n));
       if constexpr (OUTL) {
         if (cn > 0) {
-          wq[i] = __ldg(reinterpret_cast<const uint4*>(p.WqO + n * 16));
           if constexpr (EPI == EPI_INT8_OUTLIER) {
             const uint4* w = reinterpret_cast<const uint4*>(p.W_O + n * p.ostride);
             wo0[i] = __ldg(w);
@@ -152,11 +152,10 @@ __device__ __forceinline__ void epi_stage(const EpiParams& p, EpiStage<BN>& es, 
   for (int i = 0; i < PER; ++i) {
     const int j = et + i * GEMM_EPI_THREADS;
     if (j >= BN) continue;
-    es.q[j][0] = make_uint4(__float_as_uint(sw[i]), __float_as_uint(b[i]), wq[i].x, wq[i].y);
+    es.q[j][0] = make_uint4(__float_as_uint(sw[i]), __float_as_uint(b[i]), 0u, 0u);
     if constexpr (OUTL) {
       es.q[j][1] = wo0[i];
-      es.q[j][2] = make_uint4(wq[i].z, wq[i].w, 0u, 0u);
-      es.q[j][3] = wo1[i];
+      es.q[j][2] = wo1[i];
     }
   }
 }
@@ -218,11 +217,11 @@ __device__ __forceinline__ void store_chunk_i32(const EpiParams& p, const uint32
 // any count, not fast).
 // 16-bit outputs are returned in `out` (the caller stores them); int32
 // outputs are stored here.
-template <typename TOut, int EPI, int BN, int CN, int NX, int NQ>
+template <typename TOut, int EPI, int BN, int CN, int NX>
 __device__ __forceinline__ void epi_chunk(const EpiParams& p, const EpiStage<BN>& es, uint32_t (&r)[GEMM_CW], int c,
                                           int64_t row, int64_t n_base, float sx, float alpha, int cnt,
                                           const float (&xo)[NX], const unsigned long long (&xp)[8],
-                                          const uint32_t (&nxq)[NQ], uint32_t (&out)[GEMM_CW / 2]) {
+                                          uint32_t (&out)[GEMM_CW / 2]) {
   constexpr bool OUTL = EPI == EPI_INT8_OUTLIER || EPI == EPI_INT8_OUTLIER_I32;
   const int64_t n0 = n_base + c * GEMM_CW;
   float prev = 0.0f;
@@ -230,25 +229,15 @@ __device__ __forceinline__ void epi_chunk(const EpiParams& p, const EpiStage<BN>
   for (int j = 0; j < GEMM_CW; ++j) {
     const uint4 q0 = es.q[c * GEMM_CW + j][0];
     int32_t acc = static_cast<int32_t>(r[j]);
-    if constexpr (OUTL) {
-      // the accumulator without the outlier columns' products, exact in int32
-      if constexpr (CN > 0) {
-        acc = __dp4a(static_cast<int>(nxq[0]), static_cast<int>(q0.z), acc);
-        acc = __dp4a(static_cast<int>(nxq[1]), static_cast<int>(q0.w), acc);
-        if constexpr (CN > 8) {
-          const uint4 q2 = es.q[c * GEMM_CW + j][2];
-          acc = __dp4a(static_cast<int>(nxq[2]), static_cast<int>(q2.x), acc);
-          acc = __dp4a(static_cast<int>(nxq[3]), static_cast<int>(q2.y), acc);
+    if constexpr (OUTL && CN < 0) {
+      // more outlier columns than the correction MMA takes: their products
+      // leave the accumulator here, exact in int32
+      if (cnt > GEMM_CORR_K && n0 + j < p.N)
+        for (int o = 0; o < cnt; ++o) {
+          const int k = __ldg(p.O + o);
+          acc -= static_cast<int32_t>(__ldg(p.Xq + row * p.K + k)) *
+                 static_cast<int32_t>(__ldg(p.Wq + (n0 + j) * p.K + k));
         }
-      }
-      if constexpr (CN < 0) {
-        if (n0 + j < p.N)
-          for (int o = 0; o < cnt; ++o) {
-            const int k = __ldg(p.O + o);
-            acc -= static_cast<int32_t>(__ldg(p.Xq + row * p.K + k)) *
-                   static_cast<int32_t>(__ldg(p.Wq + (n0 + j) * p.K + k));
-          }
-      }
     }
     if constexpr (EPI == EPI_I32 || EPI == EPI_INT8_OUTLIER_I32) {
       r[j] = static_cast<uint32_t>(acc);
@@ -266,7 +255,7 @@ __device__ __forceinline__ void epi_chunk(const EpiParams& p, const EpiStage<BN>
         t = fma_f32x2(xp[2], f32x2_of16<TOut>(q1.z), t);
         t = fma_f32x2(xp[3], f32x2_of16<TOut>(q1.w), t);
         if constexpr (CN > 8) {
-          const uint4 q3 = es.q[c * GEMM_CW + j][3];
+          const uint4 q3 = es.q[c * GEMM_CW + j][2];
           t = fma_f32x2(xp[4], f32x2_of16<TOut>(q3.x), t);
           t = fma_f32x2(xp[5], f32x2_of16<TOut>(q3.y), t);
           t = fma_f32x2(xp[6], f32x2_of16<TOut>(q3.z), t);
@@ -299,24 +288,13 @@ __device__ __forceinline__ void epi_tile(const EpiParams& p, const EpiStage<BN>&
                                          bool row_ok, int64_t n_base, float alpha, int cnt, const CUtensorMap* tmY,
                                          uint8_t* ybox, int64_t row0) {
   constexpr int NX = CN > 0 ? CN : 1;
-  constexpr int NQ = CN > 0 ? CN / 4 : 1;
   float xo[NX];
-  uint32_t nxq[NQ];   // minus the row's codes in the outlier columns, 4 to a word
 #pragma unroll
   for (int i = 0; i < NX; ++i) xo[i] = 0.0f;
-#pragma unroll
-  for (int i = 0; i < NQ; ++i) nxq[i] = 0u;
   float sx = 0.0f;
   if (row_ok) {
     if constexpr (EPI == EPI_INT8_OUTLIER || EPI == EPI_FP8_ROWCOL) sx = __ldg(p.s_x + row);
     if constexpr (CN > 0) {
-      const uint4 q4 = __ldg(reinterpret_cast<const uint4*>(p.XqO + row * 16));
-      nxq[0] = __vsub4(0u, q4.x);   // codes lie in [-127, 127]: negation is exact
-      nxq[1] = __vsub4(0u, q4.y);
-      if constexpr (CN > 8) {
-        nxq[2] = __vsub4(0u, q4.z);
-        nxq[3] = __vsub4(0u, q4.w);
-      }
       if constexpr (EPI == EPI_INT8_OUTLIER) {
 #pragma unroll
         for (int qd = 0; qd < CN / 8; ++qd) {
@@ -342,7 +320,7 @@ __device__ __forceinline__ void epi_tile(const EpiParams& p, const EpiStage<BN>&
     uint32_t out[GEMM_CW / 2];
 #pragma unroll
     for (int i = 0; i < GEMM_CW / 2; ++i) out[i] = 0u;
-    if (row_ok) epi_chunk<TOut, EPI, BN, CN>(p, es, r, c, row, n_base, sx, alpha, cnt, xo, xp, nxq, out);
+    if (row_ok) epi_chunk<TOut, EPI, BN, CN>(p, es, r, c, row, n_base, sx, alpha, cnt, xo, xp, out);
     if constexpr (EPI != EPI_I32 && EPI != EPI_INT8_OUTLIER_I32) {
       if (p.tma_y) {
         uint8_t* box = ybox + (c & 1) * GEMM_YBOX_BYTES;
@@ -384,7 +362,8 @@ __device__ __forceinline__ void epi_tile(const EpiParams& p, const EpiStage<BN>&
 template <int KIND, int EPI, typename TOut, int BN, int STAGES>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-           const __grid_constant__ CUtensorMap tmY, const EpiParams p) {
+           const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmXc,
+           const __grid_constant__ CUtensorMap tmWc, const EpiParams p) {
   using L = GemmSmem<BN, STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -409,6 +388,13 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   const int num_n = static_cast<int>((N + BN - 1) / BN);
   const int num_tiles = num_m * num_n;
   const int num_kb = static_cast<int>((K + GEMM_BK - 1) / GEMM_BK);
+  // LLM.int8 with 1..GEMM_CORR_K outlier columns: each tile ends with one more
+  // stage, (-Xq[:,O]) x Wq[:,O]^T with K = 32, added to the accumulator
+  bool corr = false;
+  if constexpr (EPI == EPI_INT8_OUTLIER || EPI == EPI_INT8_OUTLIER_I32) {
+    const int c = *p.count;
+    corr = c > 0 && c <= GEMM_CORR_K;
+  }
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -457,6 +443,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           issued |= 1u << stage;
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
+        if (ok && corr) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full_bar[stage], (GEMM_BM + BN) * GEMM_CORR_K);
+          tma_load_2d(sA + stage * L::A_BYTES, &tmXc, &full_bar[stage], 0, mb * GEMM_BM);
+          tma_load_2d(sB + stage * L::B_BYTES, &tmWc, &full_bar[stage], 0, nb * BN);
+          issued |= 1u << stage;
+          if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
       }
       if (!ok) {
         // aborted: wait (bounded) for the copies still in flight before the CTA exits
@@ -493,6 +487,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             umma<KIND>(d_tmem, adesc + 2u * k, bdesc + 2u * k, idesc, (kb | k) != 0 ? 1u : 0u);
           umma_commit(&empty_bar[stage]);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+        }
+        if (ok && corr) {
+          if (!mbar_wait(&full_bar[stage], phase, abort_flag)) {
+            ok = false;
+          } else {
+            tc_fence_after();
+            umma<KIND>(d_tmem, sdesc_k32(smem_u32(sA + stage * L::A_BYTES)), sdesc_k32(smem_u32(sB + stage * L::B_BYTES)),
+                       idesc, 1u);
+            umma_commit(&empty_bar[stage]);
+            if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+          }
         }
         if (!ok) break;
         umma_commit(&tfull_bar[acc]);

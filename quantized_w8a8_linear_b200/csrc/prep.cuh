@@ -87,14 +87,14 @@ struct WoGather {
   int64_t N;
   const int32_t* O;
   uint16_t* W_O;
-  int8_t* WqO;   // [N, OUTL_CODES] weight codes of the first outlier columns, or nullptr
+  int8_t* WqO;   // [N, OUTL_CODES] weight codes of the outlier columns (count <= OUTL_CODES), or nullptr
 };
 
 // Outlier counts up to OUTL_CODES also get compact int8 copies of the codes in
-// their columns (Xq[:,O] and Wq[:,O], zero-padded to OUTL_CODES per row), so
-// that the GEMM epilogue can take those columns' products back out without
-// gathering from Xq and Wq.
-constexpr int OUTL_CODES = 16;
+// their columns, zero-padded to OUTL_CODES per row: -Xq[:,O] and Wq[:,O]. The
+// GEMM adds their product to its accumulator with one more MMA (K = 32),
+// which takes those columns' products back out of the full-K contraction.
+constexpr int OUTL_CODES = 32;
 
 // Round-half-even of an fp32 value in (-2^22, 2^22) to an integer, read from
 // the low byte of t + 1.5 * 2^23: the add rounds to nearest even, and within
@@ -161,8 +161,8 @@ __device__ __forceinline__ uint32_t keep_mask(uint32_t om, int i) {
 //            counts); CTA 0 writes the ascending list O and the count;
 //   fix-up   per row, one warp reads the row's values in the O columns and
 //            copies them to X_O (zero-padded to a multiple of 8) and, for up
-//            to OUTL_CODES columns, the codes pass 1 left there to XqO (the
-//            GEMM takes those codes' products back out, so Xq keeps them); if
+//            to OUTL_CODES columns, minus the codes pass 1 left there to XqO
+//            (the GEMM takes those codes' products back out, so Xq keeps them); if
 //            the largest of the values that is <= thr reaches the kept
 //            absmax, the row is requantised with the exact absmax (by the
 //            whole CTA, from shared memory), its outlier codes then 0;
@@ -188,7 +188,7 @@ struct PrepArgs {
   uint32_t* rowctr;    // next-row counter (zero on entry), or nullptr for a static row split
   uint16_t* X_O;
   int64_t ostride;
-  int8_t* XqO;         // [M, OUTL_CODES] codes of the first outlier columns (count <= OUTL_CODES), or nullptr
+  int8_t* XqO;         // [M, OUTL_CODES] minus the codes in the outlier columns (count <= OUTL_CODES), or nullptr
   WoGather wo;
 };
 
@@ -492,10 +492,10 @@ __global__ void __launch_bounds__(RQ_THREADS, 3) k_prep_rows(const T* __restrict
     mo = __reduce_max_sync(0xffffffffu, mo);
     const uint32_t mb = __ldcg(a.amax_bits + row);
     if (a.XqO != nullptr && cnt <= OUTL_CODES && lane < OUTL_CODES) {
-      // the codes pass 1 left in the outlier columns (a requantised row gets 0 there)
+      // minus the codes pass 1 left in the outlier columns (a requantised row has 0 there)
       int8_t c = 0;
       if (lane < cnt && mo < mb) c = static_cast<int8_t>(__ldcg(a.Q + row * K + outlier_col(sflags, swpre, NW, lane)));
-      a.XqO[row * OUTL_CODES + lane] = c;
+      a.XqO[row * OUTL_CODES + lane] = static_cast<int8_t>(-c);   // codes lie in [-127, 127]
     }
     if (mo >= mb) {
       // the pass-1 absmax may sit in an outlier column: requantise exactly,

@@ -132,12 +132,25 @@ qlin_status make_tmap_y16(CUtensorMap* m, void* Y, int64_t M, int64_t N) {
 // text-encoder gate projection, 192 wide tiles in two waves, ran as fast as
 // with 384 narrow ones in three; its down projection, 64 wide tiles, gained
 // a quarter from 128 narrow ones).
+qlin_status make_tmap_bytes(CUtensorMap* m, const void* base, int64_t rows, int64_t row_bytes, int box_inner,
+                            int box_rows, CUtensorMapSwizzle sw);
+static_assert(OUTL_CODES == GEMM_CORR_K, "the prep's compact outlier codes feed the GEMM's correction MMA");
+
 template <int KIND, int EPI, typename TOut, int BN, int STAGES>
 qlin_status launch_gemm_bn(const CUtensorMap& ta, const void* B, EpiParams ep, const CUtensorMap& ty,
                            DeviceInfo* d, cudaStream_t st, int attr_slot) {
   qlin_status s;
-  CUtensorMap tb;
+  CUtensorMap tb, txc, twc;
   if ((s = make_tmap_k128(&tb, B, ep.N, ep.K, BN)) != QLIN_OK) return s;
+  std::memset(&txc, 0, sizeof(txc));
+  std::memset(&twc, 0, sizeof(twc));
+  if constexpr (EPI == EPI_INT8_OUTLIER || EPI == EPI_INT8_OUTLIER_I32) {
+    // -Xq[:,O] [M,32] and Wq[:,O] [N,32] for the correction MMA (32B swizzle)
+    if ((s = make_tmap_bytes(&txc, ep.XqO, ep.M, GEMM_CORR_K, GEMM_CORR_K, GEMM_BM, CU_TENSOR_MAP_SWIZZLE_32B)) != QLIN_OK)
+      return s;
+    if ((s = make_tmap_bytes(&twc, ep.WqO, ep.N, GEMM_CORR_K, GEMM_CORR_K, BN, CU_TENSOR_MAP_SWIZZLE_32B)) != QLIN_OK)
+      return s;
+  }
   auto kern = k_gemm<KIND, EPI, TOut, BN, STAGES>;
   constexpr int smem = GemmSmem<BN, STAGES>::TOTAL;
   static_assert(smem <= 227 * 1024, "k_gemm shared memory");
@@ -157,7 +170,7 @@ qlin_status launch_gemm_bn(const CUtensorMap& ta, const void* B, EpiParams ep, c
   }
   const int64_t tiles = ((ep.M + GEMM_BM - 1) / GEMM_BM) * ((ep.N + BN - 1) / BN);
   const int grid = static_cast<int>(tiles < d->sms ? tiles : d->sms);
-  kern<<<grid, GEMM_THREADS, smem, st>>>(ta, tb, ty, ep);
+  kern<<<grid, GEMM_THREADS, smem, st>>>(ta, tb, ty, txc, twc, ep);
   return check_cuda(cudaGetLastError(), "k_gemm launch");
 }
 
