@@ -259,6 +259,52 @@ def time_steps(runs, steps, warmup, flush):
     return prep, gemm
 
 
+def time_whole(runs, steps, warmup, flush):
+    """Device time of `steps` whole steps (every linear's prepare + gemm, no
+    events in between), replayed from one CUDA graph when the launches can be
+    captured. L2 flushed before each step outside the events. Returns
+    (total ms, "graph" | "stream")."""
+    import torch
+    st = torch.cuda.current_stream()
+    replay = None
+    mode = "stream"
+    try:
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream()
+        side.wait_stream(st)
+        with torch.cuda.stream(side):
+            with torch.cuda.graph(g, stream=side):
+                for r in runs:
+                    r.forward()
+        st.wait_stream(side)
+        torch.cuda.synchronize()
+        replay = g.replay
+        mode = "graph"
+    except Exception:
+        torch.cuda.synchronize()
+
+    def one():
+        if replay is not None:
+            replay()
+        else:
+            for r in runs:
+                r.forward()
+    for _ in range(warmup):
+        flush.zero_()
+        one()
+    torch.cuda.synchronize()
+    evs = []
+    for _ in range(steps):
+        flush.zero_()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        one()
+        e1.record(st)
+        evs.append((e0, e1))
+    torch.cuda.synchronize()
+    return sum(a.elapsed_time(b) for a, b in evs), mode
+
+
 def time_e2e(runs, steps):
     """Same work through the public one-call forward with host buffers:
     pinned H2D of every input, forward, D2H of every output, per step."""
@@ -415,13 +461,16 @@ def main():
     clocks = ClockSampler(local)
     clocks.start()
     t_wall0 = time.perf_counter()
+    # whole steps (the headline), then the same steps with an event between
+    # every stage (the per-kernel split and the roofline)
+    whole_ms, step_mode = time_whole(runs, args.steps, max(3, args.warmup), flush)
     prep_ms, gemm_ms = time_steps(runs, args.steps, max(3, args.warmup), flush)
     t_wall = time.perf_counter() - t_wall0
     clk = clocks.stop()
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    total_ms = sum(prep_ms) + sum(gemm_ms)
+    total_ms = whole_ms
     t_max = torch.tensor([total_ms], dtype=torch.float64, device=device)
     if world > 1:
         dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
@@ -507,6 +556,8 @@ def main():
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
             "gpu_launches": sum(r.launches() for r in runs) * args.steps,
             "clocks": clk, "kernels": kernels, "secondary": secondary, "wall_s_timed_region": t_wall,
+            "timing": {"value": f"whole steps with no event between stages ({step_mode} replay)",
+                       "kernels": "a second pass of the same steps with an event between every stage"},
         }
         print(json.dumps(line), flush=True)
     if world > 1:
