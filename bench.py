@@ -226,6 +226,24 @@ class LinearRun:
         return 2
 
 
+def max_over_ranks(value, device, world):
+    """The largest of the ranks' values (all_reduce MAX over the default
+    process group); the local value when there is one rank."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tops(world, steps, ops_step, total_ms_max):
+    """Throughput of all ranks together: each rank ran `steps` steps of
+    `ops_step` ops; the job took the slowest rank's time."""
+    return world * steps * ops_step / (total_ms_max * 1e-3) / 1e12
+
+
 def time_steps(runs, steps, warmup, flush):
     """Device time of `steps` steps (each: every linear's prepare + gemm), L2
     flushed before each step outside the events. Returns per-part sums (ms)."""
@@ -470,14 +488,9 @@ def main():
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    total_ms = whole_ms
-    t_max = torch.tensor([total_ms], dtype=torch.float64, device=device)
-    if world > 1:
-        dist.all_reduce(t_max, op=dist.ReduceOp.MAX)
-    total_ms_max = float(t_max.item())
-
+    total_ms_max = max_over_ranks(whole_ms, device, world)
     ops_step = sum(r.ops for r in runs)
-    value = world * args.steps * ops_step / (total_ms_max * 1e-3) / 1e12
+    value = whole_job_tops(world, args.steps, ops_step, total_ms_max)
     ms_per_step = total_ms_max / args.steps
 
     # -------- roofline of the dominant kernel (the tcgen05 GEMM) --------
