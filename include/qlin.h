@@ -199,7 +199,8 @@ QLIN_API qlin_status qlin_w4a8_gemm(qlin_dtype xdt, int64_t M, int64_t K, const 
  * flags uint32 [ceil(K/32)] (bit k%32 of word k/32 set iff column k is an
  * outlier); O int32 [K] (ascending outlier columns, first *count valid);
  * count int32 [1]; X_O [M, ostride] in xdt (X[:,O], zero-padded to a multiple
- * of 8 columns; ostride >= round_up(K,8), a multiple of 8).
+ * of 8 columns, and to 16 columns when 1 <= count <= 16; ostride >=
+ * round_up(K,8), a multiple of 8).
  * workspace: qlin_workspace_bytes(QLIN_OP_INT8_PREP, M, 0, K). */
 QLIN_API qlin_status qlin_int8_prep(const void *X, qlin_dtype xdt, int64_t M, int64_t K, float threshold,
                            int8_t *Xq, float *s_x, uint32_t *flags, int32_t *O, int32_t *count,

@@ -217,11 +217,11 @@ __device__ __forceinline__ void store_chunk_i32(const EpiParams& p, const uint32
 // any count, not fast).
 // 16-bit outputs are returned in `out` (the caller stores them); int32
 // outputs are stored here.
-template <typename TOut, int EPI, int BN, int CN, int NX>
-__device__ __forceinline__ void epi_chunk(const EpiParams& p, const EpiStage<BN>& es, uint32_t (&r)[GEMM_CW], int c,
-                                          int64_t row, int64_t n_base, float sx, float alpha, int cnt,
-                                          const float (&xo)[NX], const unsigned long long (&xp)[8],
-                                          uint32_t (&out)[GEMM_CW / 2]) {
+template <typename TOut, int EPI, int BN, int CN, int NX, bool FTM>
+__device__ __forceinline__ void epi_chunk(const EpiParams& p, const EpiStage<BN>& es, uint32_t (&r)[GEMM_CW],
+                                          const uint32_t (&f)[GEMM_CW], int c, int64_t row, int64_t n_base, float sx,
+                                          float alpha, int cnt, const float (&xo)[NX],
+                                          const unsigned long long (&xp)[8], uint32_t (&out)[GEMM_CW / 2]) {
   constexpr bool OUTL = EPI == EPI_INT8_OUTLIER || EPI == EPI_INT8_OUTLIER_I32;
   const int64_t n0 = n_base + c * GEMM_CW;
   float prev = 0.0f;
@@ -247,6 +247,7 @@ __device__ __forceinline__ void epi_chunk(const EpiParams& p, const EpiStage<BN>
       if constexpr (EPI == EPI_INT8_OUTLIER) a = fmaf(static_cast<float>(acc), sx * sw, bias);
       else if constexpr (EPI == EPI_FP8_TENSOR) a = fmaf(__uint_as_float(r[j]), alpha, bias);
       else a = fmaf(__uint_as_float(r[j]), sx * sw, bias);
+      if constexpr (FTM) a += __uint_as_float(f[j]);   // the fp outlier part, from its TMEM accumulator
       if constexpr (EPI == EPI_INT8_OUTLIER && CN > 0) {
         // floating-point outlier part: sum_o X_O[row,o] W_O[n,o], outlier pairs per packed fma
         const uint4 q1 = es.q[c * GEMM_CW + j][1];
@@ -283,10 +284,12 @@ __device__ __forceinline__ void epi_chunk(const EpiParams& p, const EpiStage<BN>
 // One accumulator tile, one thread per row (its TMEM lane): the row's
 // operands first, then the accumulator in chunks of GEMM_CW columns with the
 // next chunk's tcgen05.ld in flight while the current one is processed.
-template <typename TOut, int EPI, int BN, int CN>
+// FTM: the fp outlier part was computed by the tensor core into a second
+// accumulator at t_row_f; the epilogue adds it instead of computing it.
+template <typename TOut, int EPI, int BN, int CN, bool FTM = false>
 __device__ __forceinline__ void epi_tile(const EpiParams& p, const EpiStage<BN>& es, uint32_t t_row, int64_t row,
                                          bool row_ok, int64_t n_base, float alpha, int cnt, const CUtensorMap* tmY,
-                                         uint8_t* ybox, int64_t row0) {
+                                         uint8_t* ybox, int64_t row0, uint32_t t_row_f = 0) {
   constexpr int NX = CN > 0 ? CN : 1;
   float xo[NX];
 #pragma unroll
@@ -314,13 +317,13 @@ __device__ __forceinline__ void epi_tile(const EpiParams& p, const EpiStage<BN>&
   static_assert(NCH % 2 == 0, "chunks are processed in pairs");
   const int lane = threadIdx.x & 31;
   // one chunk: compute, then store (TMA box from shared memory, or per-thread stores)
-  auto chunk = [&](uint32_t (&r)[GEMM_CW], int c) {
+  auto chunk = [&](uint32_t (&r)[GEMM_CW], const uint32_t (&f)[GEMM_CW], int c) {
     const int64_t n0 = n_base + c * GEMM_CW;
     if (n0 >= p.N) return;   // warp-uniform
     uint32_t out[GEMM_CW / 2];
 #pragma unroll
     for (int i = 0; i < GEMM_CW / 2; ++i) out[i] = 0u;
-    if (row_ok) epi_chunk<TOut, EPI, BN, CN>(p, es, r, c, row, n_base, sx, alpha, cnt, xo, xp, out);
+    if (row_ok) epi_chunk<TOut, EPI, BN, CN, NX, FTM>(p, es, r, f, c, row, n_base, sx, alpha, cnt, xo, xp, out);
     if constexpr (EPI != EPI_I32 && EPI != EPI_INT8_OUTLIER_I32) {
       if (p.tma_y) {
         uint8_t* box = ybox + (c & 1) * GEMM_YBOX_BYTES;
@@ -344,18 +347,26 @@ __device__ __forceinline__ void epi_tile(const EpiParams& p, const EpiStage<BN>&
     }
   };
   uint32_t ra[GEMM_CW], rb[GEMM_CW];
+  uint32_t fa[GEMM_CW], fb[GEMM_CW];   // the fp outlier part (FTM); unused otherwise
   __syncwarp();
   tmem_ld16(t_row, ra);
+  if constexpr (FTM) tmem_ld16(t_row_f, fa);
 #pragma unroll 1
   for (int c = 0; c < NCH; c += 2) {
     __syncwarp();
     tmem_wait16(ra);
+    if constexpr (FTM) tmem_wait16(fa);
     tmem_ld16(t_row + static_cast<uint32_t>((c + 1) * GEMM_CW), rb);
-    chunk(ra, c);
+    if constexpr (FTM) tmem_ld16(t_row_f + static_cast<uint32_t>((c + 1) * GEMM_CW), fb);
+    chunk(ra, fa, c);
     __syncwarp();
     tmem_wait16(rb);
-    if (c + 2 < NCH) tmem_ld16(t_row + static_cast<uint32_t>((c + 2) * GEMM_CW), ra);
-    chunk(rb, c + 1);
+    if constexpr (FTM) tmem_wait16(fb);
+    if (c + 2 < NCH) {
+      tmem_ld16(t_row + static_cast<uint32_t>((c + 2) * GEMM_CW), ra);
+      if constexpr (FTM) tmem_ld16(t_row_f + static_cast<uint32_t>((c + 2) * GEMM_CW), fa);
+    }
+    chunk(rb, fb, c + 1);
   }
 }
 
@@ -363,7 +374,8 @@ template <int KIND, int EPI, typename TOut, int BN, int STAGES>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
     k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
            const __grid_constant__ CUtensorMap tmY, const __grid_constant__ CUtensorMap tmXc,
-           const __grid_constant__ CUtensorMap tmWc, const EpiParams p) {
+           const __grid_constant__ CUtensorMap tmWc, const __grid_constant__ CUtensorMap tmXo,
+           const __grid_constant__ CUtensorMap tmWo, const EpiParams p) {
   using L = GemmSmem<BN, STAGES>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -395,6 +407,17 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     const int c = *p.count;
     corr = c > 0 && c <= GEMM_CORR_K;
   }
+  // FT (LLM.int8, 128-wide tiles): TMEM also holds two fp32 accumulators for
+  // the fp outlier part. With 1..16 outlier columns the extra stage carries
+  // X_O and W_O (16 columns each, zero-padded) as well, and one kind::f16 MMA
+  // (K = 16) computes X_O W_O^T there, so the epilogue only adds it.
+  constexpr bool FT = EPI == EPI_INT8_OUTLIER && BN == 128;
+  constexpr int TMEM_COLS = FT ? 4 * BN : 2 * BN;
+  bool fmma = false;
+  if constexpr (FT) {
+    const int c = *p.count;
+    fmma = c > 0 && c <= GEMM_OUTL_STAGED;
+  }
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -415,7 +438,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     tma_prefetch_desc(&tmB);
   }
   if (warp == GEMM_WARP_MMA) {
-    tmem_alloc(tmem_slot, 2 * BN);
+    tmem_alloc(tmem_slot, TMEM_COLS);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -445,9 +468,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         }
         if (ok && corr) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
-          mbar_arrive_expect_tx(&full_bar[stage], (GEMM_BM + BN) * GEMM_CORR_K);
+          mbar_arrive_expect_tx(&full_bar[stage], (GEMM_BM + BN) * GEMM_CORR_K * (fmma ? 2 : 1));
           tma_load_2d(sA + stage * L::A_BYTES, &tmXc, &full_bar[stage], 0, mb * GEMM_BM);
           tma_load_2d(sB + stage * L::B_BYTES, &tmWc, &full_bar[stage], 0, nb * BN);
+          if (fmma) {
+            // X_O and W_O, 16 two-byte columns = 32-byte rows, after the codes
+            tma_load_2d(sA + stage * L::A_BYTES + GEMM_BM * GEMM_CORR_K, &tmXo, &full_bar[stage], 0, mb * GEMM_BM);
+            tma_load_2d(sB + stage * L::B_BYTES + BN * GEMM_CORR_K, &tmWo, &full_bar[stage], 0, nb * BN);
+          }
           issued |= 1u << stage;
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
@@ -495,6 +523,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
             tc_fence_after();
             umma<KIND>(d_tmem, sdesc_k32(smem_u32(sA + stage * L::A_BYTES)), sdesc_k32(smem_u32(sB + stage * L::B_BYTES)),
                        idesc, 1u);
+            if (fmma) {
+              constexpr uint32_t idesc_f = idesc_f16(GEMM_BM, BN, std::is_same<TOut, __nv_bfloat16>::value);
+              umma<2>(tmem_base + static_cast<uint32_t>(2 * BN + acc * BN),
+                      sdesc_k32(smem_u32(sA + stage * L::A_BYTES + GEMM_BM * GEMM_CORR_K)),
+                      sdesc_k32(smem_u32(sB + stage * L::B_BYTES + BN * GEMM_CORR_K)), idesc_f, 0u);
+            }
             umma_commit(&empty_bar[stage]);
             if (++stage == STAGES) { stage = 0; phase ^= 1u; }
           }
@@ -532,7 +566,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       if constexpr (EPI != EPI_I32) {
         // the group's readers of the previous tile are done with its staging area
         if (!epi_bar(&epi_mbar[g], bar_phase, abort_flag)) break;
-        epi_stage<TOut, EPI, BNG>(p, es, n_base, et, cn);
+        epi_stage<TOut, EPI, BNG>(p, es, n_base, et, FT && cn > 0 && cnt <= GEMM_OUTL_STAGED ? 0 : cn);
         if (!epi_bar(&epi_mbar[g], bar_phase, abort_flag)) break;
       }
       if (!mbar_wait(&tfull_bar[acc], acc_phase, abort_flag)) break;
@@ -541,7 +575,14 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       const bool row_ok = row < M;
       const uint32_t t_row =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN + g * BNG);
-      if constexpr (EPI == EPI_INT8_OUTLIER || EPI == EPI_INT8_OUTLIER_I32) {
+      if constexpr (FT) {
+        const uint32_t t_row_f = t_row + static_cast<uint32_t>(2 * BN);
+        if (cn == 0) epi_tile<TOut, EPI, BNG, 0>(p, es, t_row, row, row_ok, n_base, alpha, cnt, &tmY, ybox, row - lane);
+        else if (cnt <= GEMM_OUTL_STAGED)
+          epi_tile<TOut, EPI, BNG, 0, true>(p, es, t_row, row, row_ok, n_base, alpha, cnt, &tmY, ybox, row - lane,
+                                            t_row_f);
+        else epi_tile<TOut, EPI, BNG, -1>(p, es, t_row, row, row_ok, n_base, alpha, cnt, &tmY, ybox, row - lane);
+      } else if constexpr (EPI == EPI_INT8_OUTLIER || EPI == EPI_INT8_OUTLIER_I32) {
         if (cn == 0) epi_tile<TOut, EPI, BNG, 0>(p, es, t_row, row, row_ok, n_base, alpha, cnt, &tmY, ybox,
                                                            row - lane);
         else if (cn == 8) epi_tile<TOut, EPI, BNG, 8>(p, es, t_row, row, row_ok, n_base, alpha, cnt, &tmY, ybox,
@@ -566,7 +607,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   if (warp == GEMM_WARP_MMA) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, 2 * BN);
+    tmem_dealloc(tmem_base, TMEM_COLS);
   }
 }
 

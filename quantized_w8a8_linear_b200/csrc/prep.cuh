@@ -95,6 +95,7 @@ struct WoGather {
 // GEMM adds their product to its accumulator with one more MMA (K = 32),
 // which takes those columns' products back out of the full-K contraction.
 constexpr int OUTL_CODES = 32;
+constexpr int OUTL_FP_MMA_K = 16;
 
 // Round-half-even of an fp32 value in (-2^22, 2^22) to an integer, read from
 // the low byte of t + 1.5 * 2^23: the add rounds to nearest even, and within
@@ -160,7 +161,7 @@ __device__ __forceinline__ uint32_t keep_mask(uint32_t om, int i) {
 //   compact  every CTA scans the bitmap into shared memory (per-word prefix
 //            counts); CTA 0 writes the ascending list O and the count;
 //   fix-up   per row, one warp reads the row's values in the O columns and
-//            copies them to X_O (zero-padded to a multiple of 8) and, for up
+//            copies them to X_O (zero-padded to a multiple of 8, or to 16) and, for up
 //            to OUTL_CODES columns, minus the codes pass 1 left there to XqO
 //            (the GEMM takes those codes' products back out, so Xq keeps them); if
 //            the largest of the values that is <= thr reaches the kept
@@ -457,7 +458,9 @@ __global__ void __launch_bounds__(RQ_THREADS, 3) k_prep_rows(const T* __restrict
   if (blockIdx.x == 0 && tid == 0) *a.count = cnt;
   __syncthreads();
   if (cnt == 0) return;
-  const int pad = (cnt + 7) & ~7;
+  // X_O and W_O are zero-padded to a multiple of 8 columns, and to 16 for up
+  // to 16 outlier columns (one K = 16 tensor-core step of the fp part)
+  const int pad = cnt <= OUTL_FP_MMA_K ? OUTL_FP_MMA_K : (cnt + 7) & ~7;
 
   // ---------------- fix-up: one warp per row ----------------
   constexpr int RQ_LIST = 32;

@@ -133,22 +133,34 @@ qlin_status make_tmap_y16(CUtensorMap* m, void* Y, int64_t M, int64_t N) {
 // with 384 narrow ones in three; its down projection, 64 wide tiles, gained
 // a quarter from 128 narrow ones).
 qlin_status make_tmap_bytes(CUtensorMap* m, const void* base, int64_t rows, int64_t row_bytes, int box_inner,
-                            int box_rows, CUtensorMapSwizzle sw);
+                            int box_rows, CUtensorMapSwizzle sw, int64_t stride_bytes = 0);
 static_assert(OUTL_CODES == GEMM_CORR_K, "the prep's compact outlier codes feed the GEMM's correction MMA");
 
 template <int KIND, int EPI, typename TOut, int BN, int STAGES>
 qlin_status launch_gemm_bn(const CUtensorMap& ta, const void* B, EpiParams ep, const CUtensorMap& ty,
                            DeviceInfo* d, cudaStream_t st, int attr_slot) {
   qlin_status s;
-  CUtensorMap tb, txc, twc;
+  CUtensorMap tb, txc, twc, txo, two;
   if ((s = make_tmap_k128(&tb, B, ep.N, ep.K, BN)) != QLIN_OK) return s;
   std::memset(&txc, 0, sizeof(txc));
   std::memset(&twc, 0, sizeof(twc));
+  std::memset(&txo, 0, sizeof(txo));
+  std::memset(&two, 0, sizeof(two));
   if constexpr (EPI == EPI_INT8_OUTLIER || EPI == EPI_INT8_OUTLIER_I32) {
     // -Xq[:,O] [M,32] and Wq[:,O] [N,32] for the correction MMA (32B swizzle)
     if ((s = make_tmap_bytes(&txc, ep.XqO, ep.M, GEMM_CORR_K, GEMM_CORR_K, GEMM_BM, CU_TENSOR_MAP_SWIZZLE_32B)) != QLIN_OK)
       return s;
     if ((s = make_tmap_bytes(&twc, ep.WqO, ep.N, GEMM_CORR_K, GEMM_CORR_K, BN, CU_TENSOR_MAP_SWIZZLE_32B)) != QLIN_OK)
+      return s;
+  }
+  if constexpr (EPI == EPI_INT8_OUTLIER && BN == 128) {
+    // X_O [M,16] and W_O [N,16] (16-bit, first 16 of ostride columns, zero
+    // past the count) for the fp outlier MMA (32B swizzle)
+    constexpr int FB = GEMM_OUTL_STAGED * 2;
+    if ((s = make_tmap_bytes(&txo, ep.X_O, ep.M, FB, FB, GEMM_BM, CU_TENSOR_MAP_SWIZZLE_32B, 2 * ep.ostride)) !=
+        QLIN_OK)
+      return s;
+    if ((s = make_tmap_bytes(&two, ep.W_O, ep.N, FB, FB, BN, CU_TENSOR_MAP_SWIZZLE_32B, 2 * ep.ostride)) != QLIN_OK)
       return s;
   }
   auto kern = k_gemm<KIND, EPI, TOut, BN, STAGES>;
@@ -170,7 +182,7 @@ qlin_status launch_gemm_bn(const CUtensorMap& ta, const void* B, EpiParams ep, c
   }
   const int64_t tiles = ((ep.M + GEMM_BM - 1) / GEMM_BM) * ((ep.N + BN - 1) / BN);
   const int grid = static_cast<int>(tiles < d->sms ? tiles : d->sms);
-  kern<<<grid, GEMM_THREADS, smem, st>>>(ta, tb, ty, txc, twc, ep);
+  kern<<<grid, GEMM_THREADS, smem, st>>>(ta, tb, ty, txc, twc, txo, two, ep);
   return check_cuda(cudaGetLastError(), "k_gemm launch");
 }
 
@@ -773,13 +785,14 @@ qlin_status qlin_fp8_forward(const void* X, qlin_dtype xdt, int64_t M, int64_t K
 // ---------------------------------------------------------------------------
 namespace {
 
+// A 2-D byte tensor [rows, row_bytes] (row pitch stride_bytes, or row_bytes when 0).
 qlin_status make_tmap_bytes(CUtensorMap* m, const void* base, int64_t rows, int64_t row_bytes, int box_inner,
-                            int box_rows, CUtensorMapSwizzle sw) {
+                            int box_rows, CUtensorMapSwizzle sw, int64_t stride_bytes) {
   PFN_cuTensorMapEncodeTiled_v12000 enc;
   qlin_status s = get_encode(&enc);
   if (s != QLIN_OK) return s;
   cuuint64_t dims[2] = {static_cast<cuuint64_t>(row_bytes), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(stride_bytes > 0 ? stride_bytes : row_bytes)};
   cuuint32_t box[2] = {static_cast<cuuint32_t>(box_inner), static_cast<cuuint32_t>(box_rows)};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
