@@ -284,6 +284,21 @@ QLIN_API qlin_status qlin_get_device_status(int32_t *status, int reset);
  * 2e9). Synchronous; call it outside stream capture. */
 QLIN_API qlin_status qlin_set_wait_timeout_ns(uint64_t ns);
 
+/* Work schedule of the LLM.int8 GEMMs (qlin_int8_outlier_forward / _gemm /
+ * _gemm_i32), process-wide, read at each launch:
+ *   0  automatic (default): whole output tiles handed out round-robin, or
+ *      stream-K when a cost model predicts a gain of 5% or more (few tiles
+ *      over a long K: the split-K case);
+ *   1  whole tiles only;
+ *   2  stream-K whenever the shape has more than one k-block iteration in
+ *      total, down to one iteration per CTA (exercises cut tiles; slow).
+ * Under stream-K each CTA takes an equal contiguous range of the
+ * tiles x k-blocks iterations; a tile cut between CTAs is summed from int32
+ * partial accumulators in the workspace, so the int32 accumulator (and Y, for
+ * the same tile width) is the same bit for bit under every schedule. No CTA
+ * waits for another. QLIN_ERR_INVALID_ARG for another mode. */
+QLIN_API qlin_status qlin_set_gemm_schedule(int mode);
+
 /* Message for the last error returned on the calling thread ("" if none). */
 QLIN_API const char *qlin_last_error_string(void);
 

@@ -68,6 +68,7 @@ def _load() -> ctypes.CDLL:
         "qlin_e4m3_encode_f32": (st, [P, P, i64, P]),
         "qlin_get_device_status": (st, [P, i32]),
         "qlin_set_wait_timeout_ns": (st, [ctypes.c_uint64]),
+        "qlin_set_gemm_schedule": (st, [ctypes.c_int]),
         "qlin_last_error_string": (ctypes.c_char_p, []),
         "qlin_version": (i32, []),
     }
@@ -376,6 +377,11 @@ def qlin_get_device_status(reset: bool = False) -> int:
 
 def qlin_set_wait_timeout_ns(ns: int) -> None:
     _check(lib.qlin_set_wait_timeout_ns(int(ns)))
+
+
+def qlin_set_gemm_schedule(mode: int) -> None:
+    """0 automatic, 1 whole tiles only, 2 stream-K wherever possible (int8 GEMMs)."""
+    _check(lib.qlin_set_gemm_schedule(int(mode)))
 
 
 __all__ = [n for n in dir() if n.startswith(("qlin_", "QLIN_"))] + ["QlinError", "workspace", "lib"]

@@ -21,8 +21,9 @@
 //               floating-point outlier part as a rank-|O| update, the bias,
 //               rounding and the store of Y. With two accumulators the
 //               epilogue of tile t overlaps the main loop of tile t+1.
-// Tiles are handed out round-robin (tile = blockIdx.x + i * gridDim.x) with
-// the M index fastest, so CTAs running together share the same weight tile.
+// Tiles are handed out round-robin (tile = blockIdx.x + i * gridDim.x) in
+// bands of group_m m-blocks, M fastest within a band, so that the CTAs running
+// together share few A and B tiles in L2 (or under stream-K, below).
 // Out-of-range rows and K columns are zero-filled by TMA; stores are
 // predicated on M and N.
 #pragma once
@@ -58,6 +59,22 @@ static_assert(128 * (GEMM_REGS_MIN_LAUNCH - GEMM_REGS_LOW) >= 256 * (GEMM_REGS_H
 constexpr int GEMM_CW = 16;                  // accumulator columns per tcgen05.ld in the epilogue
 constexpr int GEMM_OUTL_STAGED = 16;         // outlier counts up to this take the staged fp part in the epilogue
 constexpr int GEMM_CORR_K = 32;              // outlier counts up to this take their int8 products out with one MMA
+// Stream-K (kind::i8, 128 x 256 tiles): at most this many CTAs (partial slots
+// in the workspace: two per CTA), each with at least GEMM_SK_MIN_ITERS k-blocks
+// unless forced. A cut tile costs its parties about GEMM_SK_COST_KB k-blocks of
+// main loop (measured: 4 us to write a partial and fence it, 3 us to add one),
+// and the CTAs' k offsets drift apart, so fewer A and B tiles are shared in
+// L2; the automatic choice takes stream-K only for a gain of 5% or more.
+constexpr int GEMM_SK_MAX_CTAS = 160;
+constexpr int GEMM_SK_BN = 256;
+constexpr int GEMM_SK_MIN_ITERS = 8;
+constexpr int GEMM_SK_COST_KB = 24;
+// The LLM.int8 epilogue of a 128 x 256 tile takes about as long as this many
+// k-blocks of its main loop (measured: 18K cycles against 0.7K per k-block).
+constexpr int GEMM_EPI_KB = 26;
+// Tile bands (tile_mn): 16 m-blocks, so 148 tiles in flight share 16 A tiles
+// and about 9 B tiles.
+constexpr int GEMM_GROUP_M = 16;
 
 struct EpiParams {
   int64_t M, N, K;
@@ -86,7 +103,179 @@ struct EpiParams {
   // 16-bit Y written through the kernel's Y tensor map (TMA stores of 32-row x
   // 16-column boxes from shared memory) instead of per-thread stores
   int tma_y;
+  // Stream-K schedule (kind::i8 only): the T = tiles x k-blocks iterations are
+  // cut into gridDim.x equal contiguous ranges, one per CTA, so that no SM
+  // idles through a partial last wave. A tile cut between CTAs is finished by
+  // exactly one of them from the others' int32 partial accumulators (exact).
+  int sk;
+  int sk_dp_tiles;     // tiles [0, sk_dp_tiles) go whole and round-robin; stream-K covers the rest
+  int32_t* sk_count;   // [tiles][GEMM_EPI_GROUPS] arrival counters: zero on entry, left zero
+  int32_t* sk_part;    // [2 * gridDim.x][BN/4][128][4] int32 partial accumulators
+  // Tile order: tile t lies in band t / (group_m * num_n) of group_m m-blocks
+  // (the last band may be narrower), m fastest within the band; so the tiles
+  // in flight together share few A and B tiles. 0: one band of all m-blocks.
+  int group_m;
 };
+
+__device__ __forceinline__ void tile_mn(int t, int num_m, int num_n, int group_m, int& mb, int& nb) {
+  const int gm = group_m > 0 && group_m < num_m ? group_m : num_m;
+  const int band = t / (gm * num_n);
+  const int m0 = band * gm;
+  const int h = num_m - m0 < gm ? num_m - m0 : gm;   // m-blocks in this band
+  const int r = t - band * gm * num_n;
+  mb = m0 + r % h;
+  nb = r / h;
+}
+
+// One CTA's share of the work as segments (tile, k-blocks [kb0, kb1)): whole
+// tiles round-robin; under stream-K only the tiles below sk_dp_tiles (whole
+// waves), then, of the T = (tiles - sk_dp_tiles) x KB iterations of the
+// remaining tiles, [b T / G, (b+1) T / G) (b = blockIdx.x, G = gridDim.x) cut
+// at tile boundaries. Such a range may start with the tail of a tile that an
+// earlier CTA began (a contributor segment) and end with the head of a tile
+// (kb0 = 0, the owner segment); tiles in between are whole.
+struct Seg {
+  int tile, kb0, kb1;
+};
+__device__ __forceinline__ int64_t sk_begin(int b, int G, int64_t T) { return static_cast<int64_t>(b) * T / G; }
+struct SegIter {
+  int64_t pos, end;
+  int tile, dp_end, KB;
+  int head_kb1;   // > 0: the range's cut last tile, taken first (k-blocks [0, head_kb1))
+  bool sk;
+  __device__ __forceinline__ SegIter(bool sk_, int num_tiles, int dp_tiles, int KB_)
+      : tile(static_cast<int>(blockIdx.x)), dp_end(sk_ ? dp_tiles : num_tiles), KB(KB_), head_kb1(0), sk(sk_) {
+    const int64_t base = static_cast<int64_t>(dp_end) * KB_;
+    const int64_t T = static_cast<int64_t>(num_tiles) * KB_ - base;
+    pos = sk_ ? base + sk_begin(blockIdx.x, gridDim.x, T) : 0;
+    end = sk_ ? base + sk_begin(blockIdx.x + 1, gridDim.x, T) : 0;
+    if (sk_) {
+      // A cut head goes before the rest of the range, so that the epilogues
+      // of both cut tiles overlap the main loop of whole ones (a short head
+      // last would queue its epilogue behind the previous tile's).
+      const int64_t last0 = (end - 1) / KB_ * KB_;   // first iteration of the range's last tile
+      if (end - last0 < KB_ && last0 > pos) {
+        head_kb1 = static_cast<int>(end - last0);
+        end = last0;
+      }
+    }
+  }
+  __device__ __forceinline__ bool next(Seg& s) {
+    if (tile < dp_end) {
+      s.tile = tile;
+      s.kb0 = 0;
+      s.kb1 = KB;
+      tile += gridDim.x;
+      return true;
+    }
+    if (!sk) return false;
+    if (head_kb1 > 0) {
+      s.tile = static_cast<int>(end / KB);
+      s.kb0 = 0;
+      s.kb1 = head_kb1;
+      head_kb1 = 0;
+      return true;
+    }
+    if (pos >= end) return false;
+    s.tile = static_cast<int>(pos / KB);
+    s.kb0 = static_cast<int>(pos - static_cast<int64_t>(s.tile) * KB);
+    const int64_t left = end - pos;
+    s.kb1 = left < KB - s.kb0 ? s.kb0 + static_cast<int>(left) : KB;
+    pos += s.kb1 - s.kb0;
+    return true;
+  }
+};
+// The CTAs that hold parts of a cut tile: the owner ob (its range holds the
+// tile's first iteration) and the contributors ob+1 .. ob+nc (their ranges
+// start inside the tile). Their partial slots: 2c for contributor c, 2ob+1
+// for the owner.
+__device__ __forceinline__ void sk_parties(int tile, int KB, int num_tiles, int dp_tiles, int& ob, int& nc) {
+  const int G = gridDim.x;
+  const int64_t T = static_cast<int64_t>(num_tiles - dp_tiles) * KB;
+  const int64_t x0 = static_cast<int64_t>(tile - dp_tiles) * KB, x1 = x0 + KB;
+  int b = static_cast<int>(x0 * G / T);
+  if (b > G - 1) b = G - 1;
+  while (b > 0 && sk_begin(b, G, T) > x0) --b;
+  while (b + 1 < G && sk_begin(b + 1, G, T) <= x0) ++b;
+  ob = b;
+  int c = b + 1;
+  while (c < G && sk_begin(c, G, T) < x1) ++c;
+  nc = c - b - 1;
+}
+
+// Partial-slot traffic of an epilogue group: its BNG columns of one TMEM
+// accumulator, 64 columns (4 tcgen05.ld of 16) at a time. Slot layout
+// [BN/4 column quads][128 rows] of int4: thread `row` moves its row's quads
+// and every warp-wide 16-byte access covers 512 contiguous bytes.
+template <int BN, int BNG>
+__device__ __forceinline__ void sk_store_partial(int32_t* slot, uint32_t t_row, int g, int row_in_tile) {
+  constexpr int NCH = BNG / GEMM_CW;
+  static_assert(NCH % 4 == 0, "partials move in groups of four chunks");
+  int4* dst = reinterpret_cast<int4*>(slot) + static_cast<int64_t>(g * NCH) * 4 * GEMM_BM + row_in_tile;
+#pragma unroll 1
+  for (int c0 = 0; c0 < NCH; c0 += 4) {
+    uint32_t r[4][GEMM_CW];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) tmem_ld16(t_row + static_cast<uint32_t>((c0 + i) * GEMM_CW), r[i]);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) tmem_wait16(r[i]);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int v = 0; v < 4; ++v)
+        __stcg(dst + static_cast<int64_t>((c0 + i) * 4 + v) * GEMM_BM,
+               make_int4(r[i][4 * v], r[i][4 * v + 1], r[i][4 * v + 2], r[i][4 * v + 3]));
+  }
+}
+// Adds the other parties' partial slots to the group's columns of the TMEM
+// accumulator (int32: exact in any order). Parties q = 0..nc: the owner ob
+// (q = 0, slot 2ob+1) and the contributors ob+q (slot 2(ob+q)); self_q is
+// this CTA's own party, whose part is already in TMEM.
+template <int BN, int BNG>
+__device__ __forceinline__ void sk_add_partials(const int32_t* part, int ob, int nc, int self_q, uint32_t t_row,
+                                                int g, int row_in_tile) {
+  constexpr int NCH = BNG / GEMM_CW;
+  constexpr int64_t SLOT_V4 = static_cast<int64_t>(GEMM_BM) * BN / 4;
+  const int4* src0 = reinterpret_cast<const int4*>(part) + static_cast<int64_t>(g * NCH) * 4 * GEMM_BM + row_in_tile;
+#pragma unroll 1
+  for (int c0 = 0; c0 < NCH; c0 += 4) {
+    uint32_t r[4][GEMM_CW];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) tmem_ld16(t_row + static_cast<uint32_t>((c0 + i) * GEMM_CW), r[i]);
+    bool waited = false;
+#pragma unroll 1
+    for (int q = 0; q <= nc; ++q) {
+      if (q == self_q) continue;
+      const int slot = q == 0 ? 2 * ob + 1 : 2 * (ob + q);
+      const int4* src = src0 + slot * SLOT_V4 + static_cast<int64_t>(c0) * 4 * GEMM_BM;
+      int4 v[4][4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) v[i][j] = __ldcg(src + static_cast<int64_t>(i * 4 + j) * GEMM_BM);
+      if (!waited) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) tmem_wait16(r[i]);
+        waited = true;
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          r[i][4 * j] += static_cast<uint32_t>(v[i][j].x);
+          r[i][4 * j + 1] += static_cast<uint32_t>(v[i][j].y);
+          r[i][4 * j + 2] += static_cast<uint32_t>(v[i][j].z);
+          r[i][4 * j + 3] += static_cast<uint32_t>(v[i][j].w);
+        }
+    }
+    if (!waited)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) tmem_wait16(r[i]);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) tmem_st16(t_row + static_cast<uint32_t>((c0 + i) * GEMM_CW), r[i]);
+  }
+  tmem_st_wait();
+}
 
 constexpr int GEMM_YBOX_BYTES = 32 * GEMM_CW * 2;   // one warp's 32 rows x 16 columns of 16-bit Y
 
@@ -392,6 +581,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   uint64_t* epi_mbar = drain_bar + 1;           // [GEMM_EPI_GROUPS]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(epi_mbar + GEMM_EPI_GROUPS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* sk_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);   // [GEMM_EPI_GROUPS]
+  static_assert(GEMM_EPI_GROUPS <= 2, "the barrier area's 16 tail bytes hold the TMEM slot, abort and sk flags");
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -418,6 +609,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     const int c = *p.count;
     fmma = c > 0 && c <= GEMM_OUTL_STAGED;
   }
+  // stream-K: int32 partials only (exact), and not with the FT accumulators,
+  // which only the tile's owner segment computes
+  constexpr bool SK_OK = KIND == 0 && !FT;
+  const bool sk = SK_OK && p.sk != 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -456,9 +651,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       uint32_t phase = 0;
       uint32_t issued = 0;   // bit s: stage s has a load in flight that nobody consumed yet
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-        const int mb = tile % num_m, nb = tile / num_m;
-        for (int kb = 0; kb < num_kb; ++kb) {
+      SegIter its(sk, num_tiles, p.sk_dp_tiles, num_kb);
+      Seg sg;
+      while (ok && its.next(sg)) {
+        int mb, nb;
+        tile_mn(sg.tile, num_m, num_n, p.group_m, mb, nb);
+        for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
           mbar_arrive_expect_tx(&full_bar[stage], L::A_BYTES + L::B_BYTES);
           tma_load_2d(sA + stage * L::A_BYTES, &tmA, &full_bar[stage], kb * GEMM_BK, mb * GEMM_BM);
@@ -466,7 +664,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           issued |= 1u << stage;
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
-        if (ok && corr) {
+        if (ok && corr && sg.kb0 == 0) {   // the tile's owner segment
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
           mbar_arrive_expect_tx(&full_bar[stage], (GEMM_BM + BN) * GEMM_CORR_K * (fmma ? 2 : 1));
           tma_load_2d(sA + stage * L::A_BYTES, &tmXc, &full_bar[stage], 0, mb * GEMM_BM);
@@ -501,22 +699,24 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+      SegIter its(sk, num_tiles, p.sk_dp_tiles, num_kb);
+      Seg sg;
+      while (ok && its.next(sg)) {
         if (!mbar_wait(&tempty_bar[acc], acc_phase ^ 1u, abort_flag)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
-        for (int kb = 0; kb < num_kb; ++kb) {
+        for (int kb = sg.kb0; kb < sg.kb1; ++kb) {
           if (!mbar_wait(&full_bar[stage], phase, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint64_t adesc = sdesc_k128(smem_u32(sA + stage * L::A_BYTES));
           const uint64_t bdesc = sdesc_k128(smem_u32(sB + stage * L::B_BYTES));
 #pragma unroll
           for (int k = 0; k < GEMM_BK / 32; ++k)
-            umma<KIND>(d_tmem, adesc + 2u * k, bdesc + 2u * k, idesc, (kb | k) != 0 ? 1u : 0u);
+            umma<KIND>(d_tmem, adesc + 2u * k, bdesc + 2u * k, idesc, (kb != sg.kb0 || k != 0) ? 1u : 0u);
           umma_commit(&empty_bar[stage]);
           if (++stage == STAGES) { stage = 0; phase ^= 1u; }
         }
-        if (ok && corr) {
+        if (ok && corr && sg.kb0 == 0) {
           if (!mbar_wait(&full_bar[stage], phase, abort_flag)) {
             ok = false;
           } else {
@@ -560,40 +760,86 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     uint32_t bar_phase = 0;
-    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-      const int mb = tile % num_m, nb = tile / num_m;
+    SegIter its(sk, num_tiles, p.sk_dp_tiles, num_kb);
+    Seg sg;
+    while (its.next(sg)) {
+      int mb, nb;
+      tile_mn(sg.tile, num_m, num_n, p.group_m, mb, nb);
       const int64_t n_base = static_cast<int64_t>(nb) * BN + g * BNG;
-      if constexpr (EPI != EPI_I32) {
-        // the group's readers of the previous tile are done with its staging area
-        if (!epi_bar(&epi_mbar[g], bar_phase, abort_flag)) break;
-        epi_stage<TOut, EPI, BNG>(p, es, n_base, et, FT && cn > 0 && cnt <= GEMM_OUTL_STAGED ? 0 : cn);
-        if (!epi_bar(&epi_mbar[g], bar_phase, abort_flag)) break;
-      }
-      if (!mbar_wait(&tfull_bar[acc], acc_phase, abort_flag)) break;
-      tc_fence_after();
       const int64_t row = static_cast<int64_t>(mb) * GEMM_BM + q * 32 + lane;
       const bool row_ok = row < M;
       const uint32_t t_row =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN + g * BNG);
-      if constexpr (FT) {
-        const uint32_t t_row_f = t_row + static_cast<uint32_t>(2 * BN);
-        if (cn == 0) epi_tile<TOut, EPI, BNG, 0>(p, es, t_row, row, row_ok, n_base, alpha, cnt, &tmY, ybox, row - lane);
-        else if (cnt <= GEMM_OUTL_STAGED)
-          epi_tile<TOut, EPI, BNG, 0, true>(p, es, t_row, row, row_ok, n_base, alpha, cnt, &tmY, ybox, row - lane,
-                                            t_row_f);
-        else epi_tile<TOut, EPI, BNG, -1>(p, es, t_row, row, row_ok, n_base, alpha, cnt, &tmY, ybox, row - lane);
-      } else if constexpr (EPI == EPI_INT8_OUTLIER || EPI == EPI_INT8_OUTLIER_I32) {
-        if (cn == 0) epi_tile<TOut, EPI, BNG, 0>(p, es, t_row, row, row_ok, n_base, alpha, cnt, &tmY, ybox,
-                                                           row - lane);
-        else if (cn == 8) epi_tile<TOut, EPI, BNG, 8>(p, es, t_row, row, row_ok, n_base, alpha, cnt, &tmY, ybox,
-                                                           row - lane);
-        else if (cn == 16) epi_tile<TOut, EPI, BNG, 16>(p, es, t_row, row, row_ok, n_base, alpha, cnt, &tmY, ybox,
-                                                           row - lane);
-        else epi_tile<TOut, EPI, BNG, -1>(p, es, t_row, row, row_ok, n_base, alpha, cnt, &tmY, ybox,
-                                                           row - lane);
+      bool doer = true;   // this group writes the tile's Y
+      if (!(sk && (sg.kb0 != 0 || sg.kb1 != num_kb))) {
+        if constexpr (EPI != EPI_I32) {
+          // the group's readers of the previous tile are done with its staging area
+          if (!epi_bar(&epi_mbar[g], bar_phase, abort_flag)) break;
+          epi_stage<TOut, EPI, BNG>(p, es, n_base, et, FT && cn > 0 && cnt <= GEMM_OUTL_STAGED ? 0 : cn);
+          if (!epi_bar(&epi_mbar[g], bar_phase, abort_flag)) break;
+        }
+        if (!mbar_wait(&tfull_bar[acc], acc_phase, abort_flag)) break;
+        tc_fence_after();
       } else {
-        epi_tile<TOut, EPI, BNG, 0>(p, es, t_row, row, row_ok, n_base, alpha, cnt, &tmY, ybox,
-                                                           row - lane);
+        // A cut tile (stream-K). Every party but one leaves its int32 partial
+        // in its slot and counts itself in; the one that finishes the tile is
+        // the owner if all contributors have arrived when its own part is
+        // done (then it writes no partial), else the last to arrive. Nobody
+        // waits for another CTA.
+        if (!mbar_wait(&tfull_bar[acc], acc_phase, abort_flag)) break;
+        tc_fence_after();
+        int ob, nc;
+        sk_parties(sg.tile, num_kb, num_tiles, p.sk_dp_tiles, ob, nc);
+        const int self_q = static_cast<int>(blockIdx.x) - ob;   // 0: the owner
+        int* ctr = p.sk_count + static_cast<int64_t>(sg.tile) * GEMM_EPI_GROUPS + g;
+        const int row_in_tile = q * 32 + lane;
+        bool fast = false;
+        if (self_q == 0) {
+          if (et == 0) sk_flag[g] = ld_acquire_gpu(ctr) == nc ? 1 : 0;
+          if (!epi_bar(&epi_mbar[g], bar_phase, abort_flag)) break;
+          fast = sk_flag[g] != 0;
+        }
+        if (!fast) {
+          const int64_t slot = 2 * static_cast<int64_t>(blockIdx.x) + (self_q == 0 ? 1 : 0);
+          sk_store_partial<BN, BNG>(p.sk_part + slot * (GEMM_BM * BN), t_row, g, row_in_tile);
+          __threadfence();
+          if (!epi_bar(&epi_mbar[g], bar_phase, abort_flag)) break;
+          if (et == 0) sk_flag[g] = atom_add_acq_rel_gpu(ctr, 1) == nc ? 1 : 0;   // the (nc+1)-th arrival
+          if (!epi_bar(&epi_mbar[g], bar_phase, abort_flag)) break;
+          doer = sk_flag[g] != 0;
+        }
+        if (doer) {
+          __threadfence();
+          if (et == 0) *ctr = 0;   // every other party has counted itself in: ready for the next launch
+          sk_add_partials<BN, BNG>(p.sk_part, ob, nc, self_q, t_row, g, row_in_tile);
+          if constexpr (EPI != EPI_I32) {
+            if (!epi_bar(&epi_mbar[g], bar_phase, abort_flag)) break;
+            epi_stage<TOut, EPI, BNG>(p, es, n_base, et, cn);
+            if (!epi_bar(&epi_mbar[g], bar_phase, abort_flag)) break;
+          }
+        }
+      }
+      if (doer) {
+        if constexpr (FT) {
+          const uint32_t t_row_f = t_row + static_cast<uint32_t>(2 * BN);
+          if (cn == 0) epi_tile<TOut, EPI, BNG, 0>(p, es, t_row, row, row_ok, n_base, alpha, cnt, &tmY, ybox, row - lane);
+          else if (cnt <= GEMM_OUTL_STAGED)
+            epi_tile<TOut, EPI, BNG, 0, true>(p, es, t_row, row, row_ok, n_base, alpha, cnt, &tmY, ybox, row - lane,
+                                              t_row_f);
+          else epi_tile<TOut, EPI, BNG, -1>(p, es, t_row, row, row_ok, n_base, alpha, cnt, &tmY, ybox, row - lane);
+        } else if constexpr (EPI == EPI_INT8_OUTLIER || EPI == EPI_INT8_OUTLIER_I32) {
+          if (cn == 0) epi_tile<TOut, EPI, BNG, 0>(p, es, t_row, row, row_ok, n_base, alpha, cnt, &tmY, ybox,
+                                                             row - lane);
+          else if (cn == 8) epi_tile<TOut, EPI, BNG, 8>(p, es, t_row, row, row_ok, n_base, alpha, cnt, &tmY, ybox,
+                                                             row - lane);
+          else if (cn == 16) epi_tile<TOut, EPI, BNG, 16>(p, es, t_row, row, row_ok, n_base, alpha, cnt, &tmY, ybox,
+                                                             row - lane);
+          else epi_tile<TOut, EPI, BNG, -1>(p, es, t_row, row, row_ok, n_base, alpha, cnt, &tmY, ybox,
+                                                             row - lane);
+        } else {
+          epi_tile<TOut, EPI, BNG, 0>(p, es, t_row, row, row_ok, n_base, alpha, cnt, &tmY, ybox,
+                                                             row - lane);
+        }
       }
       tc_fence_before();
       __syncwarp();

@@ -7,6 +7,8 @@
 // synchronised inside a forward.
 #include <cudaTypedefs.h>
 
+#include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -131,14 +133,16 @@ qlin_status make_tmap_y16(CUtensorMap* m, void* Y, int64_t M, int64_t N) {
 // twice the operand bytes per MAC and are counted at 75% (measured: the
 // text-encoder gate projection, 192 wide tiles in two waves, ran as fast as
 // with 384 narrow ones in three; its down projection, 64 wide tiles, gained
-// a quarter from 128 narrow ones).
+// a quarter from 128 narrow ones). The int8 GEMMs with a workspace may run
+// 128 x 256 tiles under stream-K instead, when the last wave of whole tiles
+// would leave many SMs idle.
 qlin_status make_tmap_bytes(CUtensorMap* m, const void* base, int64_t rows, int64_t row_bytes, int box_inner,
                             int box_rows, CUtensorMapSwizzle sw, int64_t stride_bytes = 0);
 static_assert(OUTL_CODES == GEMM_CORR_K, "the prep's compact outlier codes feed the GEMM's correction MMA");
 
 template <int KIND, int EPI, typename TOut, int BN, int STAGES>
 qlin_status launch_gemm_bn(const CUtensorMap& ta, const void* B, EpiParams ep, const CUtensorMap& ty,
-                           DeviceInfo* d, cudaStream_t st, int attr_slot) {
+                           DeviceInfo* d, cudaStream_t st, int attr_slot, int grid_ctas = 0) {
   qlin_status s;
   CUtensorMap tb, txc, twc, txo, two;
   if ((s = make_tmap_k128(&tb, B, ep.N, ep.K, BN)) != QLIN_OK) return s;
@@ -181,19 +185,26 @@ qlin_status launch_gemm_bn(const CUtensorMap& ta, const void* B, EpiParams ep, c
     d->gemm_attr_set[attr_slot] = true;
   }
   const int64_t tiles = ((ep.M + GEMM_BM - 1) / GEMM_BM) * ((ep.N + BN - 1) / BN);
-  const int grid = static_cast<int>(tiles < d->sms ? tiles : d->sms);
+  const int grid = grid_ctas > 0 ? grid_ctas : static_cast<int>(tiles < d->sms ? tiles : d->sms);
   kern<<<grid, GEMM_THREADS, smem, st>>>(ta, tb, ty, txc, twc, txo, two, ep);
   return check_cuda(cudaGetLastError(), "k_gemm launch");
 }
 
-// Fraction of the SMs' tile slots a launch fills (tiles over waves x SMs).
-double wave_fill(int64_t tiles, int sms) {
-  const int64_t waves = (tiles + sms - 1) / sms;
-  return waves == 0 ? 1.0 : static_cast<double>(tiles) / static_cast<double>(waves * sms);
-}
+// Work schedule of the int8 GEMMs (qlin_set_gemm_schedule): 0 automatic,
+// 1 whole tiles only, 2 stream-K wherever the workspace has partial slots.
+std::atomic<int> g_gemm_schedule{0};
 
+// Tile width and schedule. Costs are in k-blocks of 128 x 256 main loop on the
+// busiest SM. Tile width: whole 128 x 256 tiles take ceil(tiles / SMs) * KB,
+// whole 128 x 128 tiles ceil(tiles / SMs) * KB * 2/3 (half the work at 75% of
+// the rate). Stream-K (int8 with a workspace; sk_cap = the CTAs its partial
+// slots serve, 0: none) keeps all but the last two waves of whole tiles and
+// cuts the rest into equal ranges: it pays when the main loop, not the
+// epilogue, bounds a tile (each CTA still runs an epilogue per tile it
+// finishes, GEMM_EPI_KB each, and its ranges add up to two more).
 template <int KIND, int EPI, typename TOut>
-qlin_status launch_gemm(const void* A, const void* B, EpiParams ep, cudaStream_t st, int attr_slot) {
+qlin_status launch_gemm(const void* A, const void* B, EpiParams ep, cudaStream_t st, int attr_slot,
+                        int sk_cap = 0) {
   DeviceInfo* d;
   qlin_status s = device_info(&d);
   if (s != QLIN_OK) return s;
@@ -208,9 +219,39 @@ qlin_status launch_gemm(const void* A, const void* B, EpiParams ep, cudaStream_t
     ep.tma_y = 1;
   }
   const int64_t mt = (ep.M + GEMM_BM - 1) / GEMM_BM;
-  const double f256 = wave_fill(mt * ((ep.N + 255) / 256), d->sms);
-  const double f128 = 0.75 * wave_fill(mt * ((ep.N + 127) / 128), d->sms);
-  if (f128 > f256)
+  const int64_t sms = d->sms;
+  const int64_t kb = (ep.K + GEMM_BK - 1) / GEMM_BK;
+  const int64_t t256 = mt * ((ep.N + 255) / 256), t128 = mt * ((ep.N + 127) / 128);
+  const double dp256 = static_cast<double>((t256 + sms - 1) / sms * kb);
+  const double dp128 = static_cast<double>((t128 + sms - 1) / sms * kb) * (2.0 / 3.0);
+  ep.sk = 0;
+  ep.sk_dp_tiles = 0;
+  ep.group_m = GEMM_GROUP_M;
+  const int mode = g_gemm_schedule.load(std::memory_order_relaxed);
+  if constexpr (KIND == 0) {
+    const int64_t G0 = std::min<int64_t>(sms, sk_cap);
+    if (G0 >= 2 && mode != 1 && ep.sk_count != nullptr && ep.sk_part != nullptr) {
+      const int64_t W = t256 / G0;                      // whole waves
+      const int64_t dp_tiles = W >= 1 ? (W - 1) * G0 : 0;
+      const int64_t tail = (t256 - dp_tiles) * kb;      // iterations cut into ranges
+      const int64_t G = W >= 1 ? G0 : std::min<int64_t>(G0, tail / (mode == 2 ? 1 : GEMM_SK_MIN_ITERS));
+      if (G >= 2) {
+        const int64_t per = (tail + G - 1) / G;
+        const int64_t segs = (per + kb - 1) / kb + 1;   // a cut tail, whole tiles, a cut head
+        const double main = static_cast<double>((W >= 1 ? (W - 1) * kb : 0) + per + GEMM_SK_COST_KB);
+        const double epi = (static_cast<double>(W >= 1 ? W - 1 : 0) + segs - 0.5) * GEMM_EPI_KB;
+        const double dpc256 = static_cast<double>((t256 + sms - 1) / sms) * std::max<double>(kb, GEMM_EPI_KB);
+        const double dpc128 =
+            static_cast<double>((t128 + sms - 1) / sms) * std::max<double>(kb * (2.0 / 3.0), GEMM_EPI_KB / 2.0);
+        if (mode == 2 || std::max(main, epi) < 0.95 * std::min(dpc256, dpc128)) {
+          ep.sk = 1;
+          ep.sk_dp_tiles = static_cast<int>(dp_tiles);
+          return launch_gemm_bn<KIND, EPI, TOut, 256, 4>(ta, B, ep, ty, d, st, 2 * attr_slot, static_cast<int>(G));
+        }
+      }
+    }
+  }
+  if (dp128 < dp256)
     return launch_gemm_bn<KIND, EPI, TOut, 128, 6>(ta, B, ep, ty, d, st, 2 * attr_slot + 1);
   return launch_gemm_bn<KIND, EPI, TOut, 256, 4>(ta, B, ep, ty, d, st, 2 * attr_slot);
 }
@@ -314,10 +355,21 @@ struct Int8Ws {
   uint16_t* W_O;      // [N,ostride]
   int8_t* XqO;        // [M,OUTL_CODES]
   int8_t* WqO;        // [N,OUTL_CODES]
+  int32_t* sk_count;  // [128x256 tiles][GEMM_EPI_GROUPS] stream-K arrival counters
+  int32_t* sk_part;   // [sk_ctas * 2][128 * 256] stream-K partial accumulators
+  int sk_ctas;        // CTAs the partial slots serve
   int64_t ostride;
-  size_t memset_bytes;  // zeroed each call: sync, count, rowctr, flags
+  size_t memset_bytes;  // zeroed each call: sync, count, rowctr, flags, sk_count
   size_t total;
 };
+
+// Stream-K capacity of a GEMM: min(GEMM_SK_MAX_CTAS, iterations of its
+// 128 x 256 tiles) CTAs.
+int64_t sk_tiles(int64_t M, int64_t N) { return ((M + GEMM_BM - 1) / GEMM_BM) * ((N + GEMM_SK_BN - 1) / GEMM_SK_BN); }
+int sk_capacity(int64_t M, int64_t N, int64_t K) {
+  const int64_t T = sk_tiles(M, N) * ((K + GEMM_BK - 1) / GEMM_BK);
+  return static_cast<int>(T < GEMM_SK_MAX_CTAS ? T : GEMM_SK_MAX_CTAS);
+}
 
 Int8Ws int8_layout(void* base, int64_t M, int64_t N, int64_t K, bool with_gemm_parts) {
   Int8Ws w{};
@@ -329,12 +381,14 @@ Int8Ws int8_layout(void* base, int64_t M, int64_t N, int64_t K, bool with_gemm_p
     return r;
   };
   const int64_t NW = (K + 31) / 32;
-  uint8_t* hdr = take(16 + 4 * NW);
+  const int64_t nctr = with_gemm_parts ? GEMM_EPI_GROUPS * sk_tiles(M, N) : 0;
+  uint8_t* hdr = take(16 + 4 * NW + 4 * nctr);
   w.sync = reinterpret_cast<uint32_t*>(hdr);
   w.count = reinterpret_cast<int32_t*>(hdr ? hdr + 4 : nullptr);
   w.rowctr = reinterpret_cast<uint32_t*>(hdr ? hdr + 8 : nullptr);
   w.flags = reinterpret_cast<uint32_t*>(hdr ? hdr + 16 : nullptr);
-  w.memset_bytes = static_cast<size_t>(16 + 4 * NW);
+  w.sk_count = reinterpret_cast<int32_t*>(hdr && nctr > 0 ? hdr + 16 + 4 * NW : nullptr);
+  w.memset_bytes = static_cast<size_t>(16 + 4 * NW + 4 * nctr);
   w.O = reinterpret_cast<int32_t*>(take(4 * K));
   w.ostride = round_up(K, 8);
   w.amax = reinterpret_cast<uint16_t*>(take(2 * M));
@@ -345,6 +399,9 @@ Int8Ws int8_layout(void* base, int64_t M, int64_t N, int64_t K, bool with_gemm_p
     w.W_O = reinterpret_cast<uint16_t*>(take(static_cast<size_t>(2 * N * w.ostride)));
     w.XqO = reinterpret_cast<int8_t*>(take(static_cast<size_t>(M * OUTL_CODES)));
     w.WqO = reinterpret_cast<int8_t*>(take(static_cast<size_t>(N * OUTL_CODES)));
+    w.sk_ctas = sk_capacity(M, N, K);
+    w.sk_part = reinterpret_cast<int32_t*>(
+        take(static_cast<size_t>(2 * w.sk_ctas) * GEMM_BM * GEMM_SK_BN * sizeof(int32_t)));
   }
   w.total = off;
   return w;
@@ -433,6 +490,12 @@ qlin_status qlin_get_device_status(int32_t* status, int reset) {
     const int z = 0;
     QLIN_TRY(check_cuda(cudaMemcpyToSymbol(qlin::g_status, &z, sizeof(int)), "cudaMemcpyToSymbol"));
   }
+  return ok();
+}
+
+qlin_status qlin_set_gemm_schedule(int mode) {
+  if (mode < 0 || mode > 2) return fail(QLIN_ERR_INVALID_ARG, "schedule mode must be 0, 1 or 2 (got %d)", mode);
+  g_gemm_schedule.store(mode, std::memory_order_relaxed);
   return ok();
 }
 
@@ -649,8 +712,9 @@ qlin_status qlin_int8_outlier_gemm(qlin_dtype xdt, int64_t M, int64_t K, const i
   ep.s_x = w.s_x; ep.s_w = w_scale; ep.bias = static_cast<const uint16_t*>(bias);
   ep.count = w.count; ep.X_O = w.X_O; ep.W_O = w.W_O; ep.ostride = w.ostride;
   ep.Xq = w.Xq; ep.Wq = Wq; ep.O = w.O; ep.XqO = w.XqO; ep.WqO = w.WqO;
-  if (xdt == QLIN_BF16) QLIN_TRY((launch_gemm<0, EPI_INT8_OUTLIER, __nv_bfloat16>(w.Xq, Wq, ep, st, 1)));
-  else QLIN_TRY((launch_gemm<0, EPI_INT8_OUTLIER, __half>(w.Xq, Wq, ep, st, 2)));
+  ep.sk_count = w.sk_count; ep.sk_part = w.sk_part;
+  if (xdt == QLIN_BF16) QLIN_TRY((launch_gemm<0, EPI_INT8_OUTLIER, __nv_bfloat16>(w.Xq, Wq, ep, st, 1, w.sk_ctas)));
+  else QLIN_TRY((launch_gemm<0, EPI_INT8_OUTLIER, __half>(w.Xq, Wq, ep, st, 2, w.sk_ctas)));
   return ok();
 }
 
@@ -669,7 +733,9 @@ qlin_status qlin_int8_outlier_gemm_i32(int64_t M, int64_t K, const int8_t* Wq, i
   EpiParams ep{};
   ep.M = M; ep.N = N; ep.K = K; ep.Y = C;
   ep.count = w.count; ep.Xq = w.Xq; ep.Wq = Wq; ep.O = w.O; ep.XqO = w.XqO; ep.WqO = w.WqO;
-  QLIN_TRY((launch_gemm<0, EPI_INT8_OUTLIER_I32, __nv_bfloat16>(w.Xq, Wq, ep, static_cast<cudaStream_t>(stream), 7)));
+  ep.sk_count = w.sk_count; ep.sk_part = w.sk_part;
+  QLIN_TRY((launch_gemm<0, EPI_INT8_OUTLIER_I32, __nv_bfloat16>(w.Xq, Wq, ep, static_cast<cudaStream_t>(stream), 7,
+                                                                 w.sk_ctas)));
   return ok();
 }
 

@@ -55,6 +55,26 @@ def test_workspace_sizes(q):
     assert q.qlin_workspace_bytes(q.QLIN_OP_INT8_OUTLIER, M, N, 0) == 0
 
 
+def test_workspace_holds_stream_k_slots(q):
+    # two 128 x 256 int32 partial slots per stream-K CTA (at most 160 CTAs,
+    # at most one per k-block iteration) on top of the other arrays
+    M, N, K = 4352, 12288, 3072
+    ws = q.qlin_workspace_bytes(q.QLIN_OP_INT8_OUTLIER, M, N, K)
+    assert ws >= M * K + 2 * M * K + 2 * N * K + 2 * 160 * 128 * 256 * 4
+    M, N, K = 64, 256, 256   # 1 tile x 2 k-blocks: 2 CTAs at most
+    small = q.qlin_workspace_bytes(q.QLIN_OP_INT8_OUTLIER, M, N, K)
+    base = M * K + 2 * M * K + 2 * N * K
+    assert base + 2 * 2 * 128 * 256 * 4 <= small < base + 2 * 2 * 128 * 256 * 4 + (1 << 16)
+
+
+def test_gemm_schedule_modes(q):
+    for mode in (0, 1, 2):
+        assert q.lib.qlin_set_gemm_schedule(mode) == q.QLIN_OK
+    assert q.lib.qlin_set_gemm_schedule(3) == q.QLIN_ERR_INVALID_ARG
+    assert b"schedule" in q.lib.qlin_last_error_string()
+    assert q.lib.qlin_set_gemm_schedule(0) == q.QLIN_OK
+
+
 @pytest.mark.parametrize("K,dt,expect", [(15, 1, 3), (0, 1, 3), (32784, 1, 2), (64, 7, 1)])
 def test_host_validation_rejects_before_launch(q, K, dt, expect):
     # X pointer is a fake aligned address: validation fails before any use

@@ -206,8 +206,9 @@ def test_outlier_weights_parity(q, dtype):
 # int8 tcgen05 GEMM: int32 accumulators bit-exact
 # ---------------------------------------------------------------------------
 
+# (2500, 600, 128): 20 m-blocks, a band of 16 and a narrower last band of 4
 GEMM_SHAPES = [(64, 512, 256), (128, 256, 128), (200, 300, 208), (1, 1, 16), (129, 257, 16),
-               (333, 600, 1024), (512, 768, 3072), (16, 48, 12288)]
+               (333, 600, 1024), (512, 768, 3072), (16, 48, 12288), (2500, 600, 128)]
 
 
 @pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
@@ -242,6 +243,76 @@ def test_int8_outlier_gemm_int32_exact(q, M, N, K, outl, dtype):
     r = oracle.int8_outlier_prep(X, THR)
     ref = r["Xq"].astype(np.int64) @ Wq.cpu().numpy().astype(np.int64).T
     assert np.array_equal(C, ref)
+
+
+# Stream-K: the int32 accumulator of a tile cut between CTAs is the sum of
+# their partials, so it stays exact under every schedule. Schedule 2 cuts the
+# work down to one k-block per CTA: (300, 520, 512) has 9 tiles of 4 k-blocks
+# (each tile in 4 CTAs), (130, 260, 3072) 4 tiles of 24 (each in 24 CTAs),
+# (1000, 1100, 2048) 40 tiles of 16 over 148 CTAs (ranges of 4-5 k-blocks
+# that start and end inside tiles); (2048, 5120, 256) has 320 tiles, more
+# than two waves: the first 148 go whole, the other 172 are cut into ranges.
+SK_CASES = [
+    (300, 520, 512, []),
+    (300, 520, 512, [(i * 3, 40 * i + 1, 6.5 + i) for i in range(12)]),
+    (300, 520, 512, [(i * 3, 16 * i + 3, -6.5 - i) for i in range(32)]),
+    (300, 520, 512, [(i * 3, 15 * i + 3, -6.5 - i) for i in range(33)]),
+    (130, 260, 3072, [(0, 2, 9.0), (1, 2, 5.99), (2, 3071, -6.01), (3, 1500, 5.5)]),
+    (1000, 1100, 2048, [(i * 7, (i * 131) % 2048, 7.0 + i) for i in range(20)]),
+    (2048, 5120, 256, [(i * 50, (i * 37) % 256, -7.0 - i) for i in range(10)]),
+]
+
+
+@pytest.fixture
+def schedule(q):
+    yield q.qlin_set_gemm_schedule
+    q.qlin_set_gemm_schedule(0)
+
+
+@pytest.mark.parametrize("mode", [1, 2])
+@pytest.mark.parametrize("M,N,K,outl", SK_CASES)
+def test_int8_outlier_gemm_int32_exact_any_schedule(q, schedule, mode, M, N, K, outl):
+    X = rand_x(M, K, M + 5 * N, torch.bfloat16, outl)
+    W = rand_w(N, K, M + 5 * N)
+    Wq, s_w = q.qlin_quantize_weight(dev(W), q.QLIN_W_INT8_ROW)
+    ws = q.workspace(q.QLIN_OP_INT8_OUTLIER, M, N, K, "cuda")
+    schedule(mode)
+    q.qlin_int8_outlier_prepare(dev(X), Wq, s_w, THR, ws)
+    C1 = q.qlin_int8_outlier_gemm_i32(M, K, Wq, ws).cpu().numpy().astype(np.int64)
+    # a second launch on the same workspace: the arrival counters were left at zero
+    C2 = q.qlin_int8_outlier_gemm_i32(M, K, Wq, ws).cpu().numpy().astype(np.int64)
+    r = oracle.int8_outlier_prep(X, THR)
+    # |sum| < 2^31, so the float64 product is exact
+    ref = (r["Xq"].astype(np.float64) @ Wq.cpu().numpy().astype(np.float64).T).astype(np.int64)
+    assert np.array_equal(C1, ref)
+    assert np.array_equal(C2, ref)
+
+
+@pytest.mark.parametrize("M,N,K,outl", SK_CASES)
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+def test_int8_forward_stream_k(q, schedule, M, N, K, outl, dtype):
+    X = rand_x(M, K, M + N, dtype, outl)
+    W = rand_w(N, K, M + N, dtype)
+    bias = (torch.randn(N, generator=torch.Generator().manual_seed(2)) * 0.1).to(dtype)
+    schedule(2)
+    Y, r = run_int8_forward(q, X, W, bias)
+    assert_rows_close(Y, r, what=f"stream-K {M}x{N}x{K}")
+    if len(outl) == 0 or len(outl) > 16:
+        # same per-element arithmetic as whole 128 x 256 tiles: equal bit for bit
+        schedule(1)
+        Y1, _ = run_int8_forward(q, X, W, bias)
+        assert np.array_equal(as_bits(Y), as_bits(Y1))
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+def test_int8_forward_split_k_automatic(q, dtype):
+    """One 128 x 256 tile over K = 16384: the automatic schedule cuts its 128
+    k-blocks over 16 CTAs (stream-K as split-K)."""
+    M, N, K = 128, 256, 16384
+    X = rand_x(M, K, 77, dtype, [(3, 100, 9.0), (90, 16000, -7.5)])
+    W = rand_w(N, K, 77, dtype)
+    Y, r = run_int8_forward(q, X, W)
+    assert_rows_close(Y, r, what="split-K")
 
 
 def test_int8_gemm_i32_extremes(q):
