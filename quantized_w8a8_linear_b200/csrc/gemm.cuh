@@ -3,17 +3,19 @@
 //   C[M,N] = A[M,K] B[N,K]^T, A and B 8-bit (int8 -> int32 with kind::i8, or
 //   E4M3 -> fp32 with kind::f8f6f4), both K-major in global memory.
 //
-// Roles (one CTA per SM, 12 warps = 3 warpgroups; the third gives most of
-// its registers to the first two with setmaxnreg):
-//   warp 8      TMA producer: 128x128-byte A tiles and BNx128-byte B tiles,
+// Roles (one CTA per SM, 20 warps = 5 warpgroups; the last gives most of its
+// registers to the first four with setmaxnreg):
+//   warp 16     TMA producer: 128x128-byte A tiles and BNx128-byte B tiles,
 //               128B-swizzled, into a STAGES-deep shared-memory ring;
-//   warp 9      MMA issuer: allocates all 512 TMEM columns (two BN-column
+//   warp 17     MMA issuer: allocates all 512 TMEM columns (two BN-column
 //               accumulators), issues 4 UMMAs (K = 32 each) per stage and
 //               commits stage release / accumulator-ready to mbarriers;
-//   warps 10-11 idle;
-//   warps 0-7   epilogue, two groups of four warps; group g takes columns
-//               [g*BN/2, (g+1)*BN/2) of every tile, so two warps share each
-//               TMEM lane quarter and hide each other's latencies. Each warp
+//   warps 18-19 idle;
+//   warps 0-15  epilogue, four groups of four warps; group g takes columns
+//               [g*BN/4, (g+1)*BN/4) of every tile, so four warps share each
+//               TMEM lane quarter and hide each other's latencies (the
+//               epilogue is latency-bound: shared-memory broadcasts, packed
+//               fp32 chains, tcgen05.ld and the Y stores). Each warp
 //               reads its 32-lane quarter with tcgen05.ld (the next chunk in
 //               flight while the current one is processed) and does the fused
 //               dequant (row x column scales), for LLM.int8 the exact
@@ -40,21 +42,22 @@ enum EpiKind { EPI_I32 = 0, EPI_INT8_OUTLIER = 1, EPI_FP8_TENSOR = 2, EPI_FP8_RO
 constexpr int GEMM_BM = 128;
 constexpr int GEMM_BK = 128;                 // bytes (= elements) per stage along K
 constexpr int GEMM_EPI_WARPS = 4;            // per group: one per TMEM lane quarter
-constexpr int GEMM_EPI_GROUPS = 2;           // one per TMEM accumulator
+constexpr int GEMM_EPI_GROUPS = 4;           // column quarters of every accumulator tile
 constexpr int GEMM_EPI_THREADS = 32 * GEMM_EPI_WARPS;
-constexpr int GEMM_EPI_ALL = GEMM_EPI_WARPS * GEMM_EPI_GROUPS;   // warps 0..7
+constexpr int GEMM_EPI_ALL = GEMM_EPI_WARPS * GEMM_EPI_GROUPS;   // warps 0..15
 constexpr int GEMM_WARP_TMA = GEMM_EPI_ALL;
 constexpr int GEMM_WARP_MMA = GEMM_EPI_ALL + 1;
 constexpr int GEMM_THREADS = 32 * (GEMM_EPI_ALL + 4);
 // Register split (setmaxnreg): the launch gives every thread the kernel's
-// register count R; the producer warpgroup drops to GEMM_REGS_LOW and the two
-// epilogue warpgroups rise to GEMM_REGS_HIGH. That fits the block's pool when
-// 128 (R - LOW) >= 256 (HIGH - R), i.e. R >= GEMM_REGS_MIN_LAUNCH; the launch
-// checks R against it.
+// register count R (96 for 640 threads); the producer warpgroup drops to
+// GEMM_REGS_LOW and the four epilogue warpgroups rise to GEMM_REGS_HIGH. That
+// fits the block's pool when 128 (R - LOW) >= 512 (HIGH - R), i.e.
+// R >= GEMM_REGS_MIN_LAUNCH; the launch checks R against it.
 constexpr int GEMM_REGS_LOW = 56;
-constexpr int GEMM_REGS_HIGH = 208;
-constexpr int GEMM_REGS_MIN_LAUNCH = 160;
-static_assert(128 * (GEMM_REGS_MIN_LAUNCH - GEMM_REGS_LOW) >= 256 * (GEMM_REGS_HIGH - GEMM_REGS_MIN_LAUNCH),
+constexpr int GEMM_REGS_HIGH = 104;
+constexpr int GEMM_REGS_MIN_LAUNCH = 95;
+static_assert(128 * (GEMM_REGS_MIN_LAUNCH - GEMM_REGS_LOW) >=
+                  32 * GEMM_EPI_ALL * (GEMM_REGS_HIGH - GEMM_REGS_MIN_LAUNCH),
               "register split must fit the launch pool");
 constexpr int GEMM_CW = 16;                  // accumulator columns per tcgen05.ld in the epilogue
 constexpr int GEMM_OUTL_STAGED = 16;         // outlier counts up to this take the staged fp part in the epilogue
@@ -279,17 +282,17 @@ __device__ __forceinline__ void sk_add_partials(const int32_t* part, int ob, int
 
 constexpr int GEMM_YBOX_BYTES = 32 * GEMM_CW * 2;   // one warp's 32 rows x 16 columns of 16-bit Y
 
-// Per-tile column data staged in shared memory by an epilogue group, one
-// 48-byte record per column, read with 16-byte broadcasts (all lanes of a
-// warp read the same address, so no bank conflicts and few wavefronts; the
-// tensor core reads its operands from the same shared memory):
-//   q[0] = {column scale (fp32), bias (fp32), 0, 0}
-//   q[1] = W_O[n, 0..7]    (16-bit)
-//   q[2] = W_O[n, 8..15]   (16-bit)
-// Only q[0] is read without outliers, q[0..1] for up to 8 outlier columns.
+// Per-tile column data staged in shared memory by an epilogue group, read
+// with 16-byte broadcasts (all lanes of a warp read the same address, so no
+// bank conflicts and few wavefronts; the tensor core reads its operands from
+// the same shared memory):
+//   sb[i] = {scale(2i), scale(2i+1), bias(2i), bias(2i+1)} (fp32), a column pair
+//   wo[n] = {W_O[n, 0..7], W_O[n, 8..15]} (16-bit)
+// Only sb is read without outliers, wo[n][0] for up to 8 outlier columns.
 template <int BN>
 struct EpiStage {
-  uint4 q[BN][3];
+  float4 sb[BN / 2];
+  uint4 wo[BN][2];
 };
 
 
@@ -299,10 +302,10 @@ struct GemmSmem {
   static constexpr int B_BYTES = BN * GEMM_BK;
   static constexpr int TILE_BYTES = STAGES * (A_BYTES + B_BYTES);
   static constexpr int EPI_BYTES = static_cast<int>(sizeof(EpiStage<BN / GEMM_EPI_GROUPS>)) * GEMM_EPI_GROUPS;
-  // Y staging for the TMA stores: two boxes per epilogue warp
-  static constexpr int Y_BYTES = GEMM_EPI_WARPS * GEMM_EPI_GROUPS * 2 * GEMM_YBOX_BYTES;
-  // full[STAGES], empty[STAGES], tfull[2], tempty[2], drain, epi[GROUPS]; tmem slot, abort flag
-  static constexpr int BAR_BYTES = 8 * (2 * STAGES + 4 + 1 + GEMM_EPI_GROUPS) + 16;
+  // Y staging for the TMA stores: one box per epilogue warp
+  static constexpr int Y_BYTES = GEMM_EPI_ALL * GEMM_YBOX_BYTES;
+  // full[STAGES], empty[STAGES], tfull[2], tempty[2], drain, epi[GROUPS]; tmem slot, abort flag, sk flags
+  static constexpr int BAR_BYTES = 8 * (2 * STAGES + 4 + 1 + GEMM_EPI_GROUPS) + 32;
   static constexpr int TOTAL = 1024 + TILE_BYTES + EPI_BYTES + Y_BYTES + BAR_BYTES;   // 1024: alignment slack
   static_assert(TILE_BYTES % 1024 == 0 && EPI_BYTES % 1024 == 0, "the Y staging boxes stay 1024-byte aligned");
 };
@@ -337,14 +340,16 @@ __device__ __forceinline__ void epi_stage(const EpiParams& p, EpiStage<BN>& es, 
       }
     }
   }
+  float* sbf = reinterpret_cast<float*>(es.sb);
 #pragma unroll
   for (int i = 0; i < PER; ++i) {
     const int j = et + i * GEMM_EPI_THREADS;
     if (j >= BN) continue;
-    es.q[j][0] = make_uint4(__float_as_uint(sw[i]), __float_as_uint(b[i]), 0u, 0u);
+    sbf[(j >> 1) * 4 + (j & 1)] = sw[i];
+    sbf[(j >> 1) * 4 + 2 + (j & 1)] = b[i];
     if constexpr (OUTL) {
-      es.q[j][1] = wo0[i];
-      es.q[j][2] = wo1[i];
+      es.wo[j][0] = wo0[i];
+      es.wo[j][1] = wo1[i];
     }
   }
 }
@@ -414,9 +419,10 @@ __device__ __forceinline__ void epi_chunk(const EpiParams& p, const EpiStage<BN>
   constexpr bool OUTL = EPI == EPI_INT8_OUTLIER || EPI == EPI_INT8_OUTLIER_I32;
   const int64_t n0 = n_base + c * GEMM_CW;
   float prev = 0.0f;
+  float4 sbv = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
 #pragma unroll
   for (int j = 0; j < GEMM_CW; ++j) {
-    const uint4 q0 = es.q[c * GEMM_CW + j][0];
+    if ((j & 1) == 0) sbv = es.sb[(c * GEMM_CW + j) >> 1];
     int32_t acc = static_cast<int32_t>(r[j]);
     if constexpr (OUTL && CN < 0) {
       // more outlier columns than the correction MMA takes: their products
@@ -431,7 +437,7 @@ __device__ __forceinline__ void epi_chunk(const EpiParams& p, const EpiStage<BN>
     if constexpr (EPI == EPI_I32 || EPI == EPI_INT8_OUTLIER_I32) {
       r[j] = static_cast<uint32_t>(acc);
     } else {
-      const float sw = __uint_as_float(q0.x), bias = __uint_as_float(q0.y);
+      const float sw = (j & 1) ? sbv.y : sbv.x, bias = (j & 1) ? sbv.w : sbv.z;
       float a;
       if constexpr (EPI == EPI_INT8_OUTLIER) a = fmaf(static_cast<float>(acc), sx * sw, bias);
       else if constexpr (EPI == EPI_FP8_TENSOR) a = fmaf(__uint_as_float(r[j]), alpha, bias);
@@ -439,13 +445,13 @@ __device__ __forceinline__ void epi_chunk(const EpiParams& p, const EpiStage<BN>
       if constexpr (FTM) a += __uint_as_float(f[j]);   // the fp outlier part, from its TMEM accumulator
       if constexpr (EPI == EPI_INT8_OUTLIER && CN > 0) {
         // floating-point outlier part: sum_o X_O[row,o] W_O[n,o], outlier pairs per packed fma
-        const uint4 q1 = es.q[c * GEMM_CW + j][1];
+        const uint4 q1 = es.wo[c * GEMM_CW + j][0];
         unsigned long long t = fma_f32x2(xp[0], f32x2_of16<TOut>(q1.x), 0ull);
         t = fma_f32x2(xp[1], f32x2_of16<TOut>(q1.y), t);
         t = fma_f32x2(xp[2], f32x2_of16<TOut>(q1.z), t);
         t = fma_f32x2(xp[3], f32x2_of16<TOut>(q1.w), t);
         if constexpr (CN > 8) {
-          const uint4 q3 = es.q[c * GEMM_CW + j][2];
+          const uint4 q3 = es.wo[c * GEMM_CW + j][1];
           t = fma_f32x2(xp[4], f32x2_of16<TOut>(q3.x), t);
           t = fma_f32x2(xp[5], f32x2_of16<TOut>(q3.y), t);
           t = fma_f32x2(xp[6], f32x2_of16<TOut>(q3.z), t);
@@ -515,8 +521,8 @@ __device__ __forceinline__ void epi_tile(const EpiParams& p, const EpiStage<BN>&
     if (row_ok) epi_chunk<TOut, EPI, BN, CN, NX, FTM>(p, es, r, f, c, row, n_base, sx, alpha, cnt, xo, xp, out);
     if constexpr (EPI != EPI_I32 && EPI != EPI_INT8_OUTLIER_I32) {
       if (p.tma_y) {
-        uint8_t* box = ybox + (c & 1) * GEMM_YBOX_BYTES;
-        if (lane == 0) bulk_wait_read<1>();   // the box's previous store has read it
+        uint8_t* box = ybox;
+        if (lane == 0) bulk_wait_read<0>();   // the box's previous store has read it
         __syncwarp();
         // row `lane` of the box, 128B-pattern swizzle of the 32-byte rows (SWIZZLE_32B:
         // 16-byte half h sits at h ^ bit 2 of the row): conflict-free quarter-warp writes
@@ -572,7 +578,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   uint8_t* sB = smem + STAGES * L::A_BYTES;
   constexpr int BNG = BN / GEMM_EPI_GROUPS;   // columns per epilogue group
   EpiStage<BNG>* estage = reinterpret_cast<EpiStage<BNG>*>(smem + L::TILE_BYTES);   // [GEMM_EPI_GROUPS]
-  uint8_t* ystage = smem + L::TILE_BYTES + L::EPI_BYTES;   // [epilogue warp][2] boxes
+  uint8_t* ystage = smem + L::TILE_BYTES + L::EPI_BYTES;   // [epilogue warp] boxes
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + L::TILE_BYTES + L::EPI_BYTES + L::Y_BYTES);
   uint64_t* empty_bar = full_bar + STAGES;
   uint64_t* tfull_bar = empty_bar + STAGES;     // [2]
@@ -582,7 +588,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(epi_mbar + GEMM_EPI_GROUPS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* sk_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);   // [GEMM_EPI_GROUPS]
-  static_assert(GEMM_EPI_GROUPS <= 2, "the barrier area's 16 tail bytes hold the TMEM slot, abort and sk flags");
+  static_assert(GEMM_EPI_GROUPS <= 6, "the barrier area's 32 tail bytes hold the TMEM slot, abort and sk flags");
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -611,7 +617,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   }
   // stream-K: int32 partials only (exact), and not with the FT accumulators,
   // which only the tile's owner segment computes
-  constexpr bool SK_OK = KIND == 0 && !FT;
+  constexpr bool SK_OK = KIND == 0 && BN == GEMM_SK_BN;
   const bool sk = SK_OK && p.sk != 0;
 
   if (threadIdx.x == 0) {
@@ -751,7 +757,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     const int q = warp & 3;   // TMEM lane quarter this warp may access
     const int et = threadIdx.x - g * GEMM_EPI_THREADS;
     EpiStage<BNG>& es = estage[g];
-    uint8_t* ybox = ystage + warp * 2 * GEMM_YBOX_BYTES;
+    uint8_t* ybox = ystage + warp * GEMM_YBOX_BYTES;
     int cnt = 0;
     float alpha = 0.0f;
     if constexpr (EPI == EPI_INT8_OUTLIER || EPI == EPI_INT8_OUTLIER_I32) cnt = *p.count;
@@ -771,7 +777,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       const uint32_t t_row =
           tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * BN + g * BNG);
       bool doer = true;   // this group writes the tile's Y
-      if (!(sk && (sg.kb0 != 0 || sg.kb1 != num_kb))) {
+      bool split = false;
+      if constexpr (SK_OK) split = sk && (sg.kb0 != 0 || sg.kb1 != num_kb);
+      if (!split) {
         if constexpr (EPI != EPI_I32) {
           // the group's readers of the previous tile are done with its staging area
           if (!epi_bar(&epi_mbar[g], bar_phase, abort_flag)) break;
@@ -780,7 +788,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         }
         if (!mbar_wait(&tfull_bar[acc], acc_phase, abort_flag)) break;
         tc_fence_after();
-      } else {
+      } else if constexpr (SK_OK) {
         // A cut tile (stream-K). Every party but one leaves its int32 partial
         // in its slot and counts itself in; the one that finishes the tile is
         // the owner if all contributors have arrived when its own part is
