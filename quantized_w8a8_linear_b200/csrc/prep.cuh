@@ -96,6 +96,7 @@ struct WoGather {
 // which takes those columns' products back out of the full-K contraction.
 constexpr int OUTL_CODES = 32;
 constexpr int OUTL_FP_MMA_K = 16;
+constexpr int OUTL_LIST = 64;   // outlier counts up to this keep the column list in shared memory
 
 // Round-half-even of an fp32 value in (-2^22, 2^22) to an integer, read from
 // the low byte of t + 1.5 * 2^23: the add rounds to nearest even, and within
@@ -296,10 +297,10 @@ __global__ void __launch_bounds__(RQ_THREADS, 3) k_prep_rows(const T* __restrict
   uint4* stage = reinterpret_cast<uint4*>(psm + ((OUTL ? 2 * NW : 0) + 3) / 4 * 4);
   // rows: taken one at a time from a global counter (balances the units when
   // rows cost different amounts), or split statically. The unit's leader keeps
-  // a ring of the unit's next row indices in shared memory, two ahead.
+  // a ring of the unit's next row indices in shared memory, PF_DEPTH ahead.
   const int64_t first = static_cast<int64_t>(blockIdx.x) * units + unit;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * units;
-  __shared__ long long rowq[RQ_WARPS][4];
+  __shared__ long long rowq[RQ_WARPS][8];
   long long* myq = rowq[unit];
   auto grab = [&](int k) -> long long {
     return a.rowctr != nullptr ? static_cast<long long>(atomicAdd(a.rowctr, 1u))
@@ -314,24 +315,22 @@ __global__ void __launch_bounds__(RQ_THREADS, 3) k_prep_rows(const T* __restrict
     }
     cp_async_commit();
   };
-  static_assert(PF_DEPTH == 2, "rows are taken two ahead: the one in flight and the next");
-  if (ut == 0) {
-    myq[0] = grab(0);
-    myq[1] = grab(1);
-  }
+  static_assert(PF_DEPTH >= 2 && PF_DEPTH <= 7, "the row ring holds the rows in flight and the next");
+  if (ut == 0)
+    for (int d = 0; d < PF_DEPTH; ++d) myq[d] = grab(d);
   if (rw == 1) __syncwarp();
   else asm volatile("bar.sync %0, %1;" ::"r"(1 + unit), "r"(UT) : "memory");
 #pragma unroll
   for (int d = 0; d < PF_DEPTH - 1; ++d) issue(myq[d], d);
   int slot = 0;
   for (int t = 0;; ++t) {
-    const int64_t row = myq[t & 3];
+    const int64_t row = myq[t & 7];
     if (row >= M) break;
-    issue(myq[(t + PF_DEPTH - 1) & 3], (slot + PF_DEPTH - 1) % PF_DEPTH);
-    // slot (t+2)&3 was last read two iterations ago, before that iteration's
-    // barrier (unit_max); its new row is first read at iteration t+1
-    // (prefetch), after this iteration's barrier
-    if (ut == 0) myq[(t + 2) & 3] = grab(t + 2);
+    issue(myq[(t + PF_DEPTH - 1) & 7], (slot + PF_DEPTH - 1) % PF_DEPTH);
+    // ring entry (t+D)&7 last held row t+D-8, read at iteration t+D-8 < t
+    // before that iteration's barrier (unit_max); its new row is first read
+    // at iteration t+1 (prefetch), after this iteration's barrier
+    if (ut == 0) myq[(t + PF_DEPTH) & 7] = grab(t + PF_DEPTH);
     if (rw == 1) __syncwarp();
     cp_async_wait<PF_DEPTH - 1>();   // this thread's copies of `row` have landed
     uint4 cur[V];
@@ -439,18 +438,23 @@ __global__ void __launch_bounds__(RQ_THREADS, 3) k_prep_rows(const T* __restrict
     if (i < warp) base += warp_tot[i];
     cnt += warp_tot[i];
   }
+  // the ascending list O: in global memory (CTA 0) and, for up to OUTL_LIST
+  // columns, in every CTA's shared memory (lookups then take one load, not
+  // a search over the bitmap)
+  __shared__ int o_list[OUTL_LIST];
   int run = base + incl - local;
   for (int u = 0; u < per; ++u) {
     const int w = tid * per + u;
     if (w < NW) {
       swpre[w] = run;
-      if (blockIdx.x == 0) {
-        uint32_t bits = sflags[w];
-        int o = run;
-        while (bits) {
-          a.O[o++] = w * 32 + (__ffs(bits) - 1);
-          bits &= bits - 1;
-        }
+      uint32_t bits = sflags[w];
+      int o = run;
+      while (bits) {
+        const int col = w * 32 + (__ffs(bits) - 1);
+        if (blockIdx.x == 0) a.O[o] = col;
+        if (o < OUTL_LIST) o_list[o] = col;
+        ++o;
+        bits &= bits - 1;
       }
       run += __popc(sflags[w]);
     }
@@ -458,6 +462,7 @@ __global__ void __launch_bounds__(RQ_THREADS, 3) k_prep_rows(const T* __restrict
   if (blockIdx.x == 0 && tid == 0) *a.count = cnt;
   __syncthreads();
   if (cnt == 0) return;
+  auto ocol = [&](int o) -> int { return cnt <= OUTL_LIST ? o_list[o] : outlier_col(sflags, swpre, NW, o); };
   // X_O and W_O are zero-padded to a multiple of 8 columns, and to 16 for up
   // to 16 outlier columns (one K = 16 tensor-core step of the fp part)
   const int pad = cnt <= OUTL_FP_MMA_K ? OUTL_FP_MMA_K : (cnt + 7) & ~7;
@@ -485,7 +490,7 @@ __global__ void __launch_bounds__(RQ_THREADS, 3) k_prep_rows(const T* __restrict
     for (int o = lane; o < pad; o += 32) {
       uint16_t h = 0;
       if (o < cnt) {
-        const int k = outlier_col(sflags, swpre, NW, o);
+        const int k = ocol(o);
         h = reinterpret_cast<const uint16_t*>(xr)[k];
         const uint32_t ah = h & 0x7FFFu;
         if (ah <= a.thr_bits) mo = max(mo, ah);
@@ -497,7 +502,7 @@ __global__ void __launch_bounds__(RQ_THREADS, 3) k_prep_rows(const T* __restrict
     if (a.XqO != nullptr && cnt <= OUTL_CODES && lane < OUTL_CODES) {
       // minus the codes pass 1 left in the outlier columns (a requantised row has 0 there)
       int8_t c = 0;
-      if (lane < cnt && mo < mb) c = static_cast<int8_t>(__ldcg(a.Q + row * K + outlier_col(sflags, swpre, NW, lane)));
+      if (lane < cnt && mo < mb) c = static_cast<int8_t>(__ldcg(a.Q + row * K + ocol(lane)));
       a.XqO[row * OUTL_CODES + lane] = static_cast<int8_t>(-c);   // codes lie in [-127, 127]
     }
     if (mo >= mb) {
@@ -565,7 +570,43 @@ __global__ void __launch_bounds__(RQ_THREADS, 3) k_prep_rows(const T* __restrict
   }
 
   // ---------------- outlier weight columns ----------------
-  if (a.wo.N > 0) {
+  if (a.wo.N > 0 && a.wo.WqO != nullptr && cnt <= OUTL_CODES) {
+    // one thread per weight row: its codes in the O columns (independent
+    // loads, one round trip), then W_O[j, 0..pad) and WqO[j, 0..32) as
+    // 16-byte stores
+    for (int64_t j = static_cast<int64_t>(blockIdx.x) * RQ_THREADS + tid; j < a.wo.N;
+         j += static_cast<int64_t>(gridDim.x) * RQ_THREADS) {
+      const int8_t* wr = a.wo.Wq + j * K;
+      const float sw = __ldg(a.wo.s_w + j);
+      int8_t c[OUTL_CODES];
+#pragma unroll
+      for (int o = 0; o < OUTL_CODES; ++o) c[o] = o < cnt ? wr[o_list[o]] : int8_t{0};
+      uint32_t cw[OUTL_CODES / 4];
+#pragma unroll
+      for (int i = 0; i < OUTL_CODES / 4; ++i)
+        cw[i] = static_cast<uint32_t>(static_cast<uint8_t>(c[4 * i])) |
+                (static_cast<uint32_t>(static_cast<uint8_t>(c[4 * i + 1])) << 8) |
+                (static_cast<uint32_t>(static_cast<uint8_t>(c[4 * i + 2])) << 16) |
+                (static_cast<uint32_t>(static_cast<uint8_t>(c[4 * i + 3])) << 24);
+      uint4* q4 = reinterpret_cast<uint4*>(a.wo.WqO + j * OUTL_CODES);
+      q4[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+      q4[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+      uint4* w4 = reinterpret_cast<uint4*>(a.wo.W_O + j * a.ostride);
+#pragma unroll
+      for (int v = 0; v < OUTL_CODES / 8; ++v) {
+        if (v * 8 >= pad) break;
+        uint32_t h[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int o = v * 8 + 2 * e;
+          const uint32_t lo = from_f<T>(__fmul_rn(static_cast<float>(c[o]), sw));
+          const uint32_t hi = from_f<T>(__fmul_rn(static_cast<float>(c[o + 1]), sw));
+          h[e] = lo | (hi << 16);
+        }
+        w4[v] = make_uint4(h[0], h[1], h[2], h[3]);
+      }
+    }
+  } else if (a.wo.N > 0) {
     const int64_t total = a.wo.N * pad;
     for (int64_t t = static_cast<int64_t>(blockIdx.x) * RQ_THREADS + tid; t < total;
          t += static_cast<int64_t>(gridDim.x) * RQ_THREADS) {
@@ -573,7 +614,7 @@ __global__ void __launch_bounds__(RQ_THREADS, 3) k_prep_rows(const T* __restrict
       const int o = static_cast<int>(t - j * pad);
       float val = 0.0f;
       if (o < cnt)
-        val = __fmul_rn(static_cast<float>(a.wo.Wq[j * K + outlier_col(sflags, swpre, NW, o)]), __ldg(a.wo.s_w + j));
+        val = __fmul_rn(static_cast<float>(a.wo.Wq[j * K + ocol(o)]), __ldg(a.wo.s_w + j));
       a.wo.W_O[j * a.ostride + o] = from_f<T>(val);
     }
     if (a.wo.WqO != nullptr && cnt <= OUTL_CODES) {
@@ -582,7 +623,7 @@ __global__ void __launch_bounds__(RQ_THREADS, 3) k_prep_rows(const T* __restrict
            t += static_cast<int64_t>(gridDim.x) * RQ_THREADS) {
         const int64_t j = t / OUTL_CODES;
         const int o = static_cast<int>(t - j * OUTL_CODES);
-        a.wo.WqO[t] = o < cnt ? a.wo.Wq[j * K + outlier_col(sflags, swpre, NW, o)] : int8_t{0};
+        a.wo.WqO[t] = o < cnt ? a.wo.Wq[j * K + ocol(o)] : int8_t{0};
       }
     }
   }
