@@ -171,6 +171,32 @@ __device__ __forceinline__ unsigned long long add_f32x2(unsigned long long a, un
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
+__device__ __forceinline__ unsigned long long mul_f32x2(unsigned long long a, unsigned long long b) {
+  unsigned long long d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float lo_f(unsigned long long v) { return __uint_as_float(static_cast<uint32_t>(v)); }
+__device__ __forceinline__ float hi_f(unsigned long long v) { return __uint_as_float(static_cast<uint32_t>(v >> 32)); }
+
+// acc + x.lo * w.lo + x.hi * w.hi for packed 16-bit pairs x, w (bf16 or
+// fp16), as two mixed-precision fmas: each takes its 16-bit operands exactly
+// and rounds once to fp32, like fp32 fmaf on the widened values.
+template <bool BF16>
+__device__ __forceinline__ float fma2_mixed(uint32_t x, uint32_t w, float acc) {
+  float d;
+  if constexpr (BF16)
+    asm("{\n\t.reg .b16 xl, xh, wl, wh;\n\t"
+        "mov.b32 {xl, xh}, %1;\n\tmov.b32 {wl, wh}, %2;\n\t"
+        "fma.rn.f32.bf16 %0, xl, wl, %3;\n\tfma.rn.f32.bf16 %0, xh, wh, %0;\n\t}"
+        : "=f"(d) : "r"(x), "r"(w), "f"(acc));
+  else
+    asm("{\n\t.reg .b16 xl, xh, wl, wh;\n\t"
+        "mov.b32 {xl, xh}, %1;\n\tmov.b32 {wl, wh}, %2;\n\t"
+        "fma.rn.f32.f16 %0, xl, wl, %3;\n\tfma.rn.f32.f16 %0, xh, wh, %0;\n\t}"
+        : "=f"(d) : "r"(x), "r"(w), "f"(acc));
+  return d;
+}
 
 // tcgen05.wait::ld naming 32 loaded registers, so that no use of them can be
 // scheduled before the wait.

@@ -354,14 +354,6 @@ __device__ __forceinline__ void epi_stage(const EpiParams& p, EpiStage<BN>& es, 
   }
 }
 
-// fp32 pair (lo, hi) of two packed 16-bit values
-template <typename T>
-__device__ __forceinline__ unsigned long long f32x2_of16(uint32_t w) {
-  if constexpr (std::is_same<T, __nv_bfloat16>::value) return f32x2_of(w << 16, w & 0xFFFF0000u);
-  else return f32x2_of(__float_as_uint(__half2float(__ushort_as_half(static_cast<unsigned short>(w & 0xFFFFu)))),
-                       __float_as_uint(__half2float(__ushort_as_half(static_cast<unsigned short>(w >> 16)))));
-}
-
 // CW outputs (16-bit pairs, the lower column in the low half) to Y[row, n0..].
 // v8: Y is 32-byte aligned and N a multiple of 16, so every 16-column chunk is
 // one aligned 32-byte sector, written with one 256-bit store.
@@ -411,66 +403,95 @@ __device__ __forceinline__ void store_chunk_i32(const EpiParams& p, const uint32
 // any count, not fast).
 // 16-bit outputs are returned in `out` (the caller stores them); int32
 // outputs are stored here.
-template <typename TOut, int EPI, int BN, int CN, int NX, bool FTM>
+template <typename TOut, int EPI, int BN, int CN, int XR, bool FTM>
 __device__ __forceinline__ void epi_chunk(const EpiParams& p, const EpiStage<BN>& es, uint32_t (&r)[GEMM_CW],
                                           const uint32_t (&f)[GEMM_CW], int c, int64_t row, int64_t n_base, float sx,
-                                          float alpha, int cnt, const float (&xo)[NX],
-                                          const unsigned long long (&xp)[8], uint32_t (&out)[GEMM_CW / 2]) {
+                                          float alpha, int cnt, const uint32_t (&xr)[XR],
+                                          uint32_t (&out)[GEMM_CW / 2]) {
   constexpr bool OUTL = EPI == EPI_INT8_OUTLIER || EPI == EPI_INT8_OUTLIER_I32;
+  constexpr bool BF = std::is_same<TOut, __nv_bfloat16>::value;
   const int64_t n0 = n_base + c * GEMM_CW;
-  float prev = 0.0f;
-  float4 sbv = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  // column pairs (j, j+1): one staged record, packed dequant arithmetic
 #pragma unroll
-  for (int j = 0; j < GEMM_CW; ++j) {
-    if ((j & 1) == 0) sbv = es.sb[(c * GEMM_CW + j) >> 1];
-    int32_t acc = static_cast<int32_t>(r[j]);
+  for (int j = 0; j < GEMM_CW; j += 2) {
+    int32_t acc[2] = {static_cast<int32_t>(r[j]), static_cast<int32_t>(r[j + 1])};
     if constexpr (OUTL && CN < 0) {
       // more outlier columns than the correction MMA takes: their products
       // leave the accumulator here, exact in int32
-      if (cnt > GEMM_CORR_K && n0 + j < p.N)
-        for (int o = 0; o < cnt; ++o) {
-          const int k = __ldg(p.O + o);
-          acc -= static_cast<int32_t>(__ldg(p.Xq + row * p.K + k)) *
-                 static_cast<int32_t>(__ldg(p.Wq + (n0 + j) * p.K + k));
-        }
+#pragma unroll
+      for (int e = 0; e < 2; ++e)
+        if (cnt > GEMM_CORR_K && n0 + j + e < p.N)
+          for (int o = 0; o < cnt; ++o) {
+            const int k = __ldg(p.O + o);
+            acc[e] -= static_cast<int32_t>(__ldg(p.Xq + row * p.K + k)) *
+                      static_cast<int32_t>(__ldg(p.Wq + (n0 + j + e) * p.K + k));
+          }
     }
     if constexpr (EPI == EPI_I32 || EPI == EPI_INT8_OUTLIER_I32) {
-      r[j] = static_cast<uint32_t>(acc);
+      r[j] = static_cast<uint32_t>(acc[0]);
+      r[j + 1] = static_cast<uint32_t>(acc[1]);
     } else {
-      const float sw = (j & 1) ? sbv.y : sbv.x, bias = (j & 1) ? sbv.w : sbv.z;
-      float a;
-      if constexpr (EPI == EPI_INT8_OUTLIER) a = fmaf(static_cast<float>(acc), sx * sw, bias);
-      else if constexpr (EPI == EPI_FP8_TENSOR) a = fmaf(__uint_as_float(r[j]), alpha, bias);
-      else a = fmaf(__uint_as_float(r[j]), sx * sw, bias);
-      if constexpr (FTM) a += __uint_as_float(f[j]);   // the fp outlier part, from its TMEM accumulator
+      const float4 sbv = es.sb[(c * GEMM_CW + j) >> 1];   // {scale j, scale j+1, bias j, bias j+1}
+      const unsigned long long b2 = f32x2_of(__float_as_uint(sbv.z), __float_as_uint(sbv.w));
+      unsigned long long v;
+      if constexpr (EPI == EPI_FP8_TENSOR) {
+        v = fma_f32x2(f32x2_of(r[j], r[j + 1]), f32x2_of(__float_as_uint(alpha), __float_as_uint(alpha)), b2);
+      } else {
+        // acc * (s_x * s_w) + bias, as fmaf(acc, s_x * s_w, bias) per column
+        const unsigned long long s2 = mul_f32x2(f32x2_of(__float_as_uint(sx), __float_as_uint(sx)),
+                                                f32x2_of(__float_as_uint(sbv.x), __float_as_uint(sbv.y)));
+        const unsigned long long a2 =
+            EPI == EPI_INT8_OUTLIER
+                ? f32x2_of(__float_as_uint(static_cast<float>(acc[0])), __float_as_uint(static_cast<float>(acc[1])))
+                : f32x2_of(r[j], r[j + 1]);
+        v = fma_f32x2(a2, s2, b2);
+      }
+      float a0 = lo_f(v), a1 = hi_f(v);
+      if constexpr (FTM) {   // the fp outlier part, from its TMEM accumulator
+        a0 += __uint_as_float(f[j]);
+        a1 += __uint_as_float(f[j + 1]);
+      }
       if constexpr (EPI == EPI_INT8_OUTLIER && CN > 0) {
-        // floating-point outlier part: sum_o X_O[row,o] W_O[n,o], outlier pairs per packed fma
-        const uint4 q1 = es.wo[c * GEMM_CW + j][0];
-        unsigned long long t = fma_f32x2(xp[0], f32x2_of16<TOut>(q1.x), 0ull);
-        t = fma_f32x2(xp[1], f32x2_of16<TOut>(q1.y), t);
-        t = fma_f32x2(xp[2], f32x2_of16<TOut>(q1.z), t);
-        t = fma_f32x2(xp[3], f32x2_of16<TOut>(q1.w), t);
+        // floating-point outlier part: sum_o X_O[row,o] W_O[n,o], one
+        // mixed-precision fma per outlier column on the 16-bit values
+        const uint4 w0 = es.wo[c * GEMM_CW + j][0], w1 = es.wo[c * GEMM_CW + j + 1][0];
+        a0 = fma2_mixed<BF>(xr[0], w0.x, a0);
+        a1 = fma2_mixed<BF>(xr[0], w1.x, a1);
+        a0 = fma2_mixed<BF>(xr[1], w0.y, a0);
+        a1 = fma2_mixed<BF>(xr[1], w1.y, a1);
+        a0 = fma2_mixed<BF>(xr[2], w0.z, a0);
+        a1 = fma2_mixed<BF>(xr[2], w1.z, a1);
+        a0 = fma2_mixed<BF>(xr[3], w0.w, a0);
+        a1 = fma2_mixed<BF>(xr[3], w1.w, a1);
         if constexpr (CN > 8) {
-          const uint4 q3 = es.wo[c * GEMM_CW + j][1];
-          t = fma_f32x2(xp[4], f32x2_of16<TOut>(q3.x), t);
-          t = fma_f32x2(xp[5], f32x2_of16<TOut>(q3.y), t);
-          t = fma_f32x2(xp[6], f32x2_of16<TOut>(q3.z), t);
-          t = fma_f32x2(xp[7], f32x2_of16<TOut>(q3.w), t);
+          const uint4 u0 = es.wo[c * GEMM_CW + j][1], u1 = es.wo[c * GEMM_CW + j + 1][1];
+          a0 = fma2_mixed<BF>(xr[4], u0.x, a0);
+          a1 = fma2_mixed<BF>(xr[4], u1.x, a1);
+          a0 = fma2_mixed<BF>(xr[5], u0.y, a0);
+          a1 = fma2_mixed<BF>(xr[5], u1.y, a1);
+          a0 = fma2_mixed<BF>(xr[6], u0.z, a0);
+          a1 = fma2_mixed<BF>(xr[6], u1.z, a1);
+          a0 = fma2_mixed<BF>(xr[7], u0.w, a0);
+          a1 = fma2_mixed<BF>(xr[7], u1.w, a1);
         }
-        a += __uint_as_float(static_cast<uint32_t>(t)) + __uint_as_float(static_cast<uint32_t>(t >> 32));
       }
       if constexpr (EPI == EPI_INT8_OUTLIER && CN < 0) {
-        if (n0 + j < p.N)
-          for (int o0 = 0; o0 < cnt; o0 += 8) {
-            uint16_t xh[8], wh[8];
-            unpack8(__ldg(reinterpret_cast<const uint4*>(p.X_O + row * p.ostride + o0)), xh);
-            unpack8(__ldg(reinterpret_cast<const uint4*>(p.W_O + (n0 + j) * p.ostride + o0)), wh);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) a = fmaf(to_f<TOut>(xh[e]), to_f<TOut>(wh[e]), a);
-          }
+        for (int e = 0; e < 2; ++e) {
+          float a = e ? a1 : a0;
+          if (n0 + j + e < p.N)
+            for (int o0 = 0; o0 < cnt; o0 += 8) {
+              uint16_t xh[8], wh[8];
+              unpack8(__ldg(reinterpret_cast<const uint4*>(p.X_O + row * p.ostride + o0)), xh);
+              unpack8(__ldg(reinterpret_cast<const uint4*>(p.W_O + (n0 + j + e) * p.ostride + o0)), wh);
+#pragma unroll
+              for (int k = 0; k < 8; ++k) a = fmaf(to_f<TOut>(xh[k]), to_f<TOut>(wh[k]), a);
+            }
+          if (e) a1 = a;
+          else a0 = a;
+        }
       }
-      if (j & 1) out[j >> 1] = pack2<TOut>(prev, a);
-      else prev = a;
+      out[j >> 1] = pack2<TOut>(a0, a1);
     }
   }
   if constexpr (EPI == EPI_I32 || EPI == EPI_INT8_OUTLIER_I32) store_chunk_i32<GEMM_CW>(p, r, row, n0);
@@ -485,10 +506,10 @@ template <typename TOut, int EPI, int BN, int CN, bool FTM = false>
 __device__ __forceinline__ void epi_tile(const EpiParams& p, const EpiStage<BN>& es, uint32_t t_row, int64_t row,
                                          bool row_ok, int64_t n_base, float alpha, int cnt, const CUtensorMap* tmY,
                                          uint8_t* ybox, int64_t row0, uint32_t t_row_f = 0) {
-  constexpr int NX = CN > 0 ? CN : 1;
-  float xo[NX];
+  constexpr int XR = CN > 0 ? CN / 2 : 1;
+  uint32_t xr[XR];   // the row's outlier values X_O[row, 0..CN), 16-bit pairs
 #pragma unroll
-  for (int i = 0; i < NX; ++i) xo[i] = 0.0f;
+  for (int i = 0; i < XR; ++i) xr[i] = 0u;
   float sx = 0.0f;
   if (row_ok) {
     if constexpr (EPI == EPI_INT8_OUTLIER || EPI == EPI_FP8_ROWCOL) sx = __ldg(p.s_x + row);
@@ -496,17 +517,15 @@ __device__ __forceinline__ void epi_tile(const EpiParams& p, const EpiStage<BN>&
       if constexpr (EPI == EPI_INT8_OUTLIER) {
 #pragma unroll
         for (int qd = 0; qd < CN / 8; ++qd) {
-          uint16_t h[8];
-          unpack8(__ldg(reinterpret_cast<const uint4*>(p.X_O + row * p.ostride + qd * 8)), h);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) xo[qd * 8 + e] = to_f<TOut>(h[e]);
+          const uint4 u = __ldg(reinterpret_cast<const uint4*>(p.X_O + row * p.ostride + qd * 8));
+          xr[qd * 4] = u.x;
+          xr[qd * 4 + 1] = u.y;
+          xr[qd * 4 + 2] = u.z;
+          xr[qd * 4 + 3] = u.w;
         }
       }
     }
   }
-  unsigned long long xp[8];   // the row's outlier values as fp32 pairs
-#pragma unroll
-  for (int i = 0; i < 8; ++i) xp[i] = f32x2_of(__float_as_uint(xo[(2 * i) % NX]), __float_as_uint(xo[(2 * i + 1) % NX]));
   const bool v8 = (reinterpret_cast<uintptr_t>(p.Y) & 31u) == 0 && (p.N & 15) == 0;
   constexpr int NCH = BN / GEMM_CW;
   static_assert(NCH % 2 == 0, "chunks are processed in pairs");
@@ -518,7 +537,7 @@ __device__ __forceinline__ void epi_tile(const EpiParams& p, const EpiStage<BN>&
     uint32_t out[GEMM_CW / 2];
 #pragma unroll
     for (int i = 0; i < GEMM_CW / 2; ++i) out[i] = 0u;
-    if (row_ok) epi_chunk<TOut, EPI, BN, CN, NX, FTM>(p, es, r, f, c, row, n_base, sx, alpha, cnt, xo, xp, out);
+    if (row_ok) epi_chunk<TOut, EPI, BN, CN, XR, FTM>(p, es, r, f, c, row, n_base, sx, alpha, cnt, xr, out);
     if constexpr (EPI != EPI_I32 && EPI != EPI_INT8_OUTLIER_I32) {
       if (p.tma_y) {
         uint8_t* box = ybox;

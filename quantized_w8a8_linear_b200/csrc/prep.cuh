@@ -49,12 +49,6 @@ __device__ __forceinline__ uint32_t absmax2<__half>(uint32_t m, uint32_t x) {
   return d;
 }
 
-// Packed fp32 multiply (two IEEE round-to-nearest products per instruction).
-__device__ __forceinline__ unsigned long long mul_f32x2(unsigned long long a, unsigned long long b) {
-  unsigned long long d;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
 __device__ __forceinline__ unsigned long long pair_f32(uint32_t lo, uint32_t hi) {
   return static_cast<unsigned long long>(lo) | (static_cast<unsigned long long>(hi) << 32);
 }
