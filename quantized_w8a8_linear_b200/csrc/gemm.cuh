@@ -398,9 +398,9 @@ __device__ __forceinline__ void store_chunk_i32(const EpiParams& p, const uint32
 }
 
 // One chunk of GEMM_CW accumulator columns of one row: r -> Y[row, n0..).
-// CN: outlier columns (0, 8 or 16: a bucket >= the count, the staged operands
-// zero-padded) or -1 (more than 16: gathered from global memory, correct for
-// any count, not fast).
+// CN: outlier columns (0, 2, 4, 8 or 16: a bucket >= the count, the staged
+// operands zero-padded) or -1 (more than 16: gathered from global memory,
+// correct for any count, not fast).
 // 16-bit outputs are returned in `out` (the caller stores them); int32
 // outputs are stored here.
 template <typename TOut, int EPI, int BN, int CN, int XR, bool FTM>
@@ -457,12 +457,16 @@ __device__ __forceinline__ void epi_chunk(const EpiParams& p, const EpiStage<BN>
         const uint4 w0 = es.wo[c * GEMM_CW + j][0], w1 = es.wo[c * GEMM_CW + j + 1][0];
         a0 = fma2_mixed<BF>(xr[0], w0.x, a0);
         a1 = fma2_mixed<BF>(xr[0], w1.x, a1);
-        a0 = fma2_mixed<BF>(xr[1], w0.y, a0);
-        a1 = fma2_mixed<BF>(xr[1], w1.y, a1);
-        a0 = fma2_mixed<BF>(xr[2], w0.z, a0);
-        a1 = fma2_mixed<BF>(xr[2], w1.z, a1);
-        a0 = fma2_mixed<BF>(xr[3], w0.w, a0);
-        a1 = fma2_mixed<BF>(xr[3], w1.w, a1);
+        if constexpr (CN > 2) {
+          a0 = fma2_mixed<BF>(xr[1], w0.y, a0);
+          a1 = fma2_mixed<BF>(xr[1], w1.y, a1);
+        }
+        if constexpr (CN > 4) {
+          a0 = fma2_mixed<BF>(xr[2], w0.z, a0);
+          a1 = fma2_mixed<BF>(xr[2], w1.z, a1);
+          a0 = fma2_mixed<BF>(xr[3], w0.w, a0);
+          a1 = fma2_mixed<BF>(xr[3], w1.w, a1);
+        }
         if constexpr (CN > 8) {
           const uint4 u0 = es.wo[c * GEMM_CW + j][1], u1 = es.wo[c * GEMM_CW + j + 1][1];
           a0 = fma2_mixed<BF>(xr[4], u0.x, a0);
@@ -516,12 +520,12 @@ __device__ __forceinline__ void epi_tile(const EpiParams& p, const EpiStage<BN>&
     if constexpr (CN > 0) {
       if constexpr (EPI == EPI_INT8_OUTLIER) {
 #pragma unroll
-        for (int qd = 0; qd < CN / 8; ++qd) {
+        for (int qd = 0; qd < (CN + 7) / 8; ++qd) {
           const uint4 u = __ldg(reinterpret_cast<const uint4*>(p.X_O + row * p.ostride + qd * 8));
-          xr[qd * 4] = u.x;
-          xr[qd * 4 + 1] = u.y;
-          xr[qd * 4 + 2] = u.z;
-          xr[qd * 4 + 3] = u.w;
+          const uint32_t uw[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            if (qd * 4 + e < XR) xr[qd * 4 + e] = uw[e];
         }
       }
     }
@@ -781,7 +785,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     float alpha = 0.0f;
     if constexpr (EPI == EPI_INT8_OUTLIER || EPI == EPI_INT8_OUTLIER_I32) cnt = *p.count;
     if constexpr (EPI == EPI_FP8_TENSOR) alpha = __ldg(p.x_scale) * __ldg(p.w_scale);
-    const int cn = cnt == 0 ? 0 : cnt <= 8 ? 8 : cnt <= GEMM_OUTL_STAGED ? 16 : -1;
+    const int cn = cnt == 0 ? 0 : cnt <= 2 ? 2 : cnt <= 4 ? 4 : cnt <= 8 ? 8 : cnt <= GEMM_OUTL_STAGED ? 16 : -1;
     int acc = 0;
     uint32_t acc_phase = 0;
     uint32_t bar_phase = 0;
@@ -856,6 +860,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           else epi_tile<TOut, EPI, BNG, -1>(p, es, t_row, row, row_ok, n_base, alpha, cnt, &tmY, ybox, row - lane);
         } else if constexpr (EPI == EPI_INT8_OUTLIER || EPI == EPI_INT8_OUTLIER_I32) {
           if (cn == 0) epi_tile<TOut, EPI, BNG, 0>(p, es, t_row, row, row_ok, n_base, alpha, cnt, &tmY, ybox,
+                                                             row - lane);
+          else if (cn == 2) epi_tile<TOut, EPI, BNG, 2>(p, es, t_row, row, row_ok, n_base, alpha, cnt, &tmY, ybox,
+                                                             row - lane);
+          else if (cn == 4) epi_tile<TOut, EPI, BNG, 4>(p, es, t_row, row, row_ok, n_base, alpha, cnt, &tmY, ybox,
                                                              row - lane);
           else if (cn == 8) epi_tile<TOut, EPI, BNG, 8>(p, es, t_row, row, row_ok, n_base, alpha, cnt, &tmY, ybox,
                                                              row - lane);
