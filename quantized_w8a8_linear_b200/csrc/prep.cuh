@@ -568,8 +568,10 @@ __global__ void __launch_bounds__(RQ_THREADS, 3) k_prep_rows(const T* __restrict
     // one thread per weight row: its codes in the O columns (independent
     // loads, one round trip), then W_O[j, 0..pad) and WqO[j, 0..32) as
     // 16-byte stores
-    for (int64_t j = static_cast<int64_t>(blockIdx.x) * RQ_THREADS + tid; j < a.wo.N;
-         j += static_cast<int64_t>(gridDim.x) * RQ_THREADS) {
+    // rows go to warp w of every CTA before warp w+1 of any, so that the
+    // gather spreads over all CTAs (each finishes its own fix-up first)
+    const int64_t wg = static_cast<int64_t>(warp) * gridDim.x + blockIdx.x;
+    for (int64_t j = wg * 32 + lane; j < a.wo.N; j += static_cast<int64_t>(gridDim.x) * RQ_THREADS) {
       const int8_t* wr = a.wo.Wq + j * K;
       const float sw = __ldg(a.wo.s_w + j);
       int8_t c[OUTL_CODES];
