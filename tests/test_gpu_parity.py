@@ -116,7 +116,7 @@ def test_all_16bit_values_int8_and_e4m3(q, dtype):
 # weight quantisation (offline step)
 # ---------------------------------------------------------------------------
 
-@pytest.mark.parametrize("N,K", [(512, 256), (300, 208), (37, 4096)])
+@pytest.mark.parametrize("N,K", [(512, 256), (300, 208), (37, 4096), (33, 32768)])
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
 def test_quantize_weight_parity(q, N, K, dtype):
     W = rand_w(N, K, N + K, dtype)
@@ -163,6 +163,8 @@ PREP_CASES = [
     # rows 1 and 2 have their largest sub-threshold value in outlier column 5
     ("recompute", 64, 128, [(0, 5, 9.0), (1, 5, 5.9), (2, 5, -5.95), (3, 9, 6.0), (4, 9, 3.5)]),
     ("wide", 96, 12288, [(0, 17, 40.0), (1, 17, 5.5), (50, 9000, -7.0), (95, 12287, 6.5)]),
+    # the largest K the library takes (16 vectors per lane, rows of 64 KB)
+    ("max_k", 40, 32768, [(0, 17, 40.0), (39, 32767, -6.5), (20, 16384, 7.0), (21, 16384, 5.0)]),
 ]
 
 
@@ -182,7 +184,7 @@ def test_int8_prep_parity(q, name, M, K, outl, dtype):
     assert np.array_equal(p["Xq"].cpu().numpy(), r["Xq"])
     xo = as_bits(p["X_O"])
     assert np.array_equal(xo[:, :n], r["X_O"])
-    pad = (n + 7) // 8 * 8
+    pad = 16 if 1 <= n <= 16 else (n + 7) // 8 * 8   # zero padding the header documents
     assert np.all(xo[:, n:pad] == 0)
 
 
@@ -355,6 +357,7 @@ def test_int8_forward_tiny_workload(q):
     (300, 520, 512, [(i * 3, 16 * i + 3, -6.5 - i) for i in range(30)]),       # 17..32 outliers
     (300, 520, 512, [(i * 3, 16 * i + 3, -6.5 - i) for i in range(32)]),       # exactly 32
     (300, 520, 512, [(i * 3, 15 * i + 3, -6.5 - i) for i in range(33)]),       # 33: global path
+    (70, 264, 32768, [(0, 5, 9.0), (69, 32767, -8.0), (35, 20000, 6.5)]),      # the largest K
 ])
 @pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
 def test_int8_forward_ragged(q, M, N, K, outl, dtype):
@@ -451,7 +454,7 @@ def test_fp8_static_forward(q, M, N, K, dtype):
     assert_rows_close(Y, r, extra=EXTRA_FP8, what="fp8 static")
 
 
-@pytest.mark.parametrize("M,N,K", [(64, 512, 256), (200, 300, 208), (130, 4096, 12288)])
+@pytest.mark.parametrize("M,N,K", [(64, 512, 256), (200, 300, 208), (130, 4096, 12288), (70, 264, 32768)])
 def test_fp8_dynamic_forward(q, M, N, K):
     X = rand_x(M, K, M + 5, torch.bfloat16, [(0, 7, 12992.0), (5, 7, 9024.0)])
     W = rand_w(N, K, M + 5)
