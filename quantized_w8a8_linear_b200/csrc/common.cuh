@@ -108,6 +108,16 @@ __device__ __forceinline__ bool epi_bar(uint64_t* bar, uint32_t& phase, volatile
   return ok;
 }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start while the kernel before it finishes; griddep_wait
+// blocks until that kernel has completed and its writes are visible (a no-op
+// when there is none). griddep_launch_dependents lets the next such kernel be
+// scheduled before this one ends.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------------------
 // TMA (tiled, 2D, no multicast)
 // ---------------------------------------------------------------------------

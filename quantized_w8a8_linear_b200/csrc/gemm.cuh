@@ -622,22 +622,12 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   const int num_kb = static_cast<int>((K + GEMM_BK - 1) / GEMM_BK);
   // LLM.int8 with 1..GEMM_CORR_K outlier columns: each tile ends with one more
   // stage, (-Xq[:,O]) x Wq[:,O]^T with K = 32, added to the accumulator
-  bool corr = false;
-  if constexpr (EPI == EPI_INT8_OUTLIER || EPI == EPI_INT8_OUTLIER_I32) {
-    const int c = *p.count;
-    corr = c > 0 && c <= GEMM_CORR_K;
-  }
   // FT (LLM.int8, 128-wide tiles): TMEM also holds two fp32 accumulators for
   // the fp outlier part. With 1..16 outlier columns the extra stage carries
   // X_O and W_O (16 columns each, zero-padded) as well, and one kind::f16 MMA
   // (K = 16) computes X_O W_O^T there, so the epilogue only adds it.
   constexpr bool FT = EPI == EPI_INT8_OUTLIER && BN == 128;
   constexpr int TMEM_COLS = FT ? 4 * BN : 2 * BN;
-  bool fmma = false;
-  if constexpr (FT) {
-    const int c = *p.count;
-    fmma = c > 0 && c <= GEMM_OUTL_STAGED;
-  }
   // stream-K: int32 partials only (exact), and not with the FT accumulators,
   // which only the tile's owner segment computes
   constexpr bool SK_OK = KIND == 0 && BN == GEMM_SK_BN;
@@ -669,6 +659,20 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // Launched as a programmatic dependent of the kernel before it (the
+  // activation prep): everything above overlapped that kernel's tail; from
+  // here on its outputs are read, so wait until it has completed.
+  griddep_wait();
+  bool corr = false;
+  if constexpr (EPI == EPI_INT8_OUTLIER || EPI == EPI_INT8_OUTLIER_I32) {
+    const int c = *p.count;
+    corr = c > 0 && c <= GEMM_CORR_K;
+  }
+  bool fmma = false;
+  if constexpr (FT) {
+    const int c = *p.count;
+    fmma = c > 0 && c <= GEMM_OUTL_STAGED;
+  }
   // each role's register budget is set inside its branch: code after a merge
   // would be held to the lower of the two
   if (warp >= GEMM_EPI_ALL) {

@@ -256,6 +256,9 @@ __device__ __forceinline__ uint32_t pair_max_bits(uint32_t m2) {
 
 template <typename T, int V, int CODE, bool SCALE_BF16, bool OUTL>
 __global__ void __launch_bounds__(RQ_THREADS, 3) k_prep_rows(const T* __restrict__ X, const PrepArgs a) {
+  // the GEMM that follows may be scheduled now (it waits for this grid's
+  // completion before it reads anything this kernel writes)
+  griddep_launch_dependents();
   extern __shared__ uint32_t psm[];   // OUTL: sflags[NW], swpre[NW]
   __shared__ uint32_t red[2][RQ_WARPS];
   const int64_t M = a.M, K = a.K;

@@ -186,8 +186,20 @@ qlin_status launch_gemm_bn(const CUtensorMap& ta, const void* B, EpiParams ep, c
   }
   const int64_t tiles = ((ep.M + GEMM_BM - 1) / GEMM_BM) * ((ep.N + BN - 1) / BN);
   const int grid = grid_ctas > 0 ? grid_ctas : static_cast<int>(tiles < d->sms ? tiles : d->sms);
-  kern<<<grid, GEMM_THREADS, smem, st>>>(ta, tb, ty, txc, twc, txo, two, ep);
-  return check_cuda(cudaGetLastError(), "k_gemm launch");
+  // programmatic dependent launch: the CTAs may start (barrier set-up, TMEM
+  // allocation) while the kernel before them finishes; they wait for it with
+  // griddepcontrol.wait before touching its outputs
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(GEMM_THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return check_cuda(cudaLaunchKernelEx(&cfg, kern, ta, tb, ty, txc, twc, txo, two, ep), "k_gemm launch");
 }
 
 // Work schedule of the int8 GEMMs (qlin_set_gemm_schedule): 0 automatic,
