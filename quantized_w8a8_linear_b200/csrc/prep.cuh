@@ -672,6 +672,7 @@ __global__ void __launch_bounds__(256) k_zero_outlier_cols(int8_t* __restrict__ 
 template <typename T>
 __global__ void __launch_bounds__(256) k_fp8_static(const T* __restrict__ X, int64_t nvec,
                                                   const float* __restrict__ x_scale, uint8_t* __restrict__ Q) {
+  griddep_launch_dependents();   // the GEMM may be scheduled now (it waits for this grid to complete)
   const float s = __ldg(x_scale);
   const float inv = 1.0f / s;
   const bool zero = (s == 0.0f);
