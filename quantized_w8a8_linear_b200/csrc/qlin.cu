@@ -238,7 +238,10 @@ qlin_status launch_gemm(const void* A, const void* B, EpiParams ep, cudaStream_t
   const double dp128 = static_cast<double>((t128 + sms - 1) / sms * kb) * (2.0 / 3.0);
   ep.sk = 0;
   ep.sk_dp_tiles = 0;
-  ep.group_m = GEMM_GROUP_M;
+  // tile bands pay when A and B do not fit in L2 together (measured: the
+  // 2048^2 block linears, 59-240 MB of operands, gained 2-24%; the 1024^2 up
+  // projection, 51 MB, and the FP8 QKV, 41 MB, lost 1-2% to them)
+  ep.group_m = (ep.M + ep.N) * ep.K > (int64_t{56} << 20) ? GEMM_GROUP_M : 0;
   const int mode = g_gemm_schedule.load(std::memory_order_relaxed);
   if constexpr (KIND == 0) {
     const int64_t G0 = std::min<int64_t>(sms, sk_cap);
