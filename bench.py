@@ -500,12 +500,19 @@ def main():
     gemm_avg_ms = sum(gemm_ms) / gemm_launches
     gemm_ops_avg = ops_step / len(runs)
     achieved = gemm_ops_avg / (gemm_avg_ms * 1e-3) / 1e12
-    traffic, traffic_note = profiled_traffic("k_gemm_int8_outlier_dit1024")
+    # the ncu DRAM counters exist for the headline workload's GEMM only
+    traffic = None
+    if wl.name == "dit1024_int8_mlp":
+        traffic, _ = profiled_traffic("k_gemm_int8_outlier_dit1024")
+    kernel_name = {"int8_outlier": "k_gemm<kind::i8, LLM.int8 epilogue>",
+                   "w4a8": "k_gemm_w4a8<kind::i8, per-group promotion>",
+                   "fp8_static": "k_gemm<kind::f8f6f4, per-tensor epilogue>",
+                   "fp8_dynamic": "k_gemm<kind::f8f6f4, per-token x per-channel epilogue>"}.get(wl.mode, wl.mode)
+    unit_kind = "fp8 TFLOPS" if wl.mode.startswith("fp8") else "int8 TOPS"
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak_tops, "unit": "TFLOP/s",
-                "frac": achieved / peak_tops, "traffic": traffic,
-                "kernel": "k_gemm<kind::i8, LLM.int8 epilogue>",
+                "frac": achieved / peak_tops, "traffic": traffic, "kernel": kernel_name,
                 "peak_source": f"{peak_src} bf16 burst {peaks['bf16_tflops']} TFLOP/s x {INT8_PER_BF16} "
-                               f"(nominal int8:bf16 dense ratio); unit is int8 TOPS"}
+                               f"(nominal int8|fp8:bf16 dense ratio); unit is {unit_kind}"}
     hbm = float(peaks["hbm_gbs"])
     prep_bytes = sum(r.prep_bytes for r in runs)
     prep_gbs = prep_bytes * args.steps / (sum(prep_ms) * 1e-3) / 1e9
