@@ -84,6 +84,8 @@ def lib() -> ctypes.CDLL:
                                        P, P, P, P, P]),
             "orc_w4a8_forward": (None, [P, i32, i64, i64, P, P, i64, i64, P, P, i64,
                                         P, P, P, P, P]),
+            "orc_fp8_weight_only_dequant": (None, [P, P, i64, i64, P]),
+            "orc_fp8_weight_only_forward": (None, [P, i32, i64, i64, P, P, i64, P, P, i64, P, P]),
             "orc_num_threads": (i32, []),
         }
         for name, (res, args) in sig.items():
@@ -332,6 +334,33 @@ def fp8_forward(X, Wq, w_scale, x_scale: Optional[float] = None, bias=None,
     lib().orc_fp8_forward(_p(xb), dt, M, K, _p(Wq), wst, _p(wsb), N, xs, _p(bb), _p(r), nr,
                           _p(Xq), _p(s_x), _p(acc), _p(Y64), _p(Y))
     return dict(Xq=Xq, s_x=s_x, acc=acc, Y64=Y64, Y=Y, dt=dt)
+
+
+def fp8_weight_only_dequant(Wq, s_w_bits) -> np.ndarray:
+    """bf16 bits [N,K] of W_deq = bf16(decode(Wq) * s_w) (weight.to(bf16) * weight_scale)."""
+    Wq = _np(Wq, np.uint8)
+    N, K = Wq.shape
+    sw = np.ascontiguousarray(np.asarray(s_w_bits, dtype=np.uint16).reshape(-1))
+    out = np.zeros((N, K), np.uint16)
+    lib().orc_fp8_weight_only_dequant(_p(Wq), _p(sw), N, K, _p(out))
+    return out
+
+
+def fp8_weight_only_forward(X, Wq, s_w_bits, bias=None, rows: Optional[Sequence[int]] = None):
+    """Weight-only FP8 linear: Y = X W_deq^T + bias, activations unquantised.
+    s_w_bits: uint16 bf16 bits [N] (the [out,1] scale)."""
+    xb, dt = _bits16(X)
+    M, K = X.shape
+    Wq = _np(Wq, np.uint8)
+    N = Wq.shape[0]
+    sw = np.ascontiguousarray(np.asarray(s_w_bits, dtype=np.uint16).reshape(-1))
+    bb = None if bias is None else _bits16(bias)[0]
+    r, nr = _rows(rows)
+    R = M if r is None else nr
+    Y64 = np.zeros((R, N), np.float64)
+    Y = np.zeros((R, N), np.uint16)
+    lib().orc_fp8_weight_only_forward(_p(xb), dt, M, K, _p(Wq), _p(sw), N, _p(bb), _p(r), nr, _p(Y64), _p(Y))
+    return dict(Y64=Y64, Y=Y, dt=dt)
 
 
 # ---------------------------------------------------------------------------

@@ -562,6 +562,48 @@ void orc_fp8_forward(const uint16_t *X, int dt, int64_t M, int64_t K, const uint
 }
 
 /* ------------------------------------------------------------------ */
+/* Weight-only FP8 (Qwen-Image-2.1-Text-Encoder-FP8, section "Format":  */
+/* E4M3 weights with a bf16 scale per output channel, [out,1], and the  */
+/* dequant rule weight.to(bf16) * weight_scale; the activations stay    */
+/* in their 16-bit dtype).                                              */
+/* ------------------------------------------------------------------ */
+
+/* W_deq[j,k] = bf16(decode(Wq[j,k]) * s_w[j]): the e4m3 value widens to
+ * bf16 exactly (3 mantissa bits), the bf16 x bf16 product is exact in
+ * double, and the bf16 multiply rounds it once, to nearest even. */
+void orc_fp8_weight_only_dequant(const uint8_t *Wq, const uint16_t *s_w_bf16, int64_t N, int64_t K,
+                                 uint16_t *W_deq) {
+#pragma omp parallel for schedule(static)
+    for (int64_t j = 0; j < N; ++j) {
+        double s = orc_bf16_to_double(s_w_bf16[j]);
+        for (int64_t k = 0; k < K; ++k) W_deq[j * K + k] = orc_double_to_bf16(orc_e4m3_decode(Wq[j * K + k]) * s);
+    }
+}
+
+/* Y64[i,j] = sum_k X[i,k] * W_deq[j,k] + bias[j] in double (each product of
+ * two 16-bit values is exact); Y = Y64 rounded once to the activation dtype.
+ * W_deq is bf16 and X is bf16 or fp16, as the page's rule leaves them. */
+void orc_fp8_weight_only_forward(const uint16_t *X, int dt, int64_t M, int64_t K, const uint8_t *Wq,
+                                 const uint16_t *s_w_bf16, int64_t N, const uint16_t *bias,
+                                 const int64_t *rows, int64_t nrows, double *Y64, uint16_t *Y) {
+    uint16_t *Wd = (uint16_t *)malloc(sizeof(uint16_t) * (size_t)(N * K > 0 ? N * K : 1));
+    orc_fp8_weight_only_dequant(Wq, s_w_bf16, N, K, Wd);
+    if (!rows) nrows = M;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < nrows; ++r) {
+        int64_t i = rows ? rows[r] : r;
+        for (int64_t j = 0; j < N; ++j) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k) acc += widen(X[i * K + k], dt) * orc_bf16_to_double(Wd[j * K + k]);
+            if (bias) acc += widen(bias[j], dt);
+            if (Y64) Y64[r * N + j] = acc;
+            if (Y) Y[r * N + j] = narrow(acc, dt);
+        }
+    }
+    free(Wd);
+}
+
+/* ------------------------------------------------------------------ */
 /* W4A8: int4 per-group weights, int8 per-token activations.           */
 /* ------------------------------------------------------------------ */
 

@@ -295,6 +295,65 @@ def unpack_int4(packed, K):
     return q
 
 
+# ---------------------------------------------------------------------------
+# Weight-only FP8 (Text-Encoder-FP8 page, "Format": weight.to(bf16) * weight_scale,
+# activations unquantised)
+# ---------------------------------------------------------------------------
+
+def _finite_e4m3_codes(shape, seed):
+    g = np.random.default_rng(seed)
+    c = g.integers(0, 256, size=shape, dtype=np.uint8)
+    c[(c & 0x7F) == 0x7F] = 0x3C                       # no NaN codes
+    return c
+
+
+def test_fp8_weight_only_dequant_is_torch_rule():
+    """W_deq equals torch's own float8 cast and bf16 multiply, bit for bit,
+    on every code at several scales and on random codes and scales."""
+    codes = np.tile(np.arange(256, dtype=np.uint8), (6, 1))
+    codes[(codes & 0x7F) == 0x7F] = 0
+    scales = torch.tensor([1.0, 0.5, 3.0e-3, 1.0 / 448, 7.1875, 2.0 ** -20], dtype=torch.bfloat16)
+    g = torch.Generator().manual_seed(31)
+    rc = _finite_e4m3_codes((64, 96), 31)
+    rs = (torch.rand(64, generator=g) * 0.05 + 1e-4).to(torch.bfloat16)
+    for c, s in ((codes, scales), (rc, rs)):
+        bits = s.view(torch.int16).numpy().view(np.uint16)
+        got = oracle.fp8_weight_only_dequant(c, bits)
+        ref = (torch.from_numpy(c).view(torch.float8_e4m3fn).to(torch.bfloat16) * s[:, None])
+        assert np.array_equal(got, ref.view(torch.int16).numpy().view(np.uint16))
+
+
+def test_fp8_weight_only_unit_scale_is_plain_matmul():
+    """With all scales 1 the weights are the decoded codes, so Y64 is the
+    fp64 matmul of X with torch's decode of the codes."""
+    M, K, N = 12, 160, 20
+    X = rand_x(M, K, 32)
+    codes = _finite_e4m3_codes((N, K), 32)
+    ones = np.full((N,), 0x3F80, np.uint16)            # bf16 1.0
+    r = oracle.fp8_weight_only_forward(X, codes, ones)
+    ref = X.double().numpy() @ decode_e4m3_torch(codes).T
+    np.testing.assert_allclose(r["Y64"], ref, rtol=1e-12, atol=1e-12)
+
+
+def test_fp8_weight_only_closed_form_and_rounding():
+    """X = 1 and one code per row: Y64 = K * bf16(decode(c) * s) + bias, and
+    Y is Y64 rounded once to the activation dtype."""
+    M, K, N = 3, 64, 5
+    X = torch.ones((M, K), dtype=torch.bfloat16)
+    codes = np.zeros((N, K), np.uint8)
+    cvals = [0x38, 0x41, 0xC6, 0x01, 0x7E]             # 1, 2.25, -14, the smallest subnormal, 448
+    for j, c in enumerate(cvals):
+        codes[j, :] = c
+    s = torch.tensor([0.5, 0.0999, -3.0, 1024.0, 0.013], dtype=torch.bfloat16)
+    bias = torch.tensor([0.0, 1.5, -2.0, 0.25, 100.0], dtype=torch.bfloat16)
+    r = oracle.fp8_weight_only_forward(X, codes, s.view(torch.int16).numpy().view(np.uint16), bias=bias)
+    w = (torch.from_numpy(codes[:, :1]).view(torch.float8_e4m3fn).to(torch.bfloat16) * s[:, None]).double()
+    ref = K * w.numpy().reshape(-1) + bias.double().numpy()
+    assert np.array_equal(r["Y64"], np.tile(ref, (M, 1)))
+    y = torch.from_numpy(r["Y64"]).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(r["Y"], y)
+
+
 def test_int4_pack_layout_and_range():
     W = rand_w(8, 256, 12)
     q, s = oracle.quantize_weight(W, "int4_g128")
