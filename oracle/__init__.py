@@ -84,6 +84,9 @@ def lib() -> ctypes.CDLL:
                                        P, P, P, P, P]),
             "orc_w4a8_forward": (None, [P, i32, i64, i64, P, P, i64, i64, P, P, i64,
                                         P, P, P, P, P]),
+            "orc_quantize_weight_int8_block": (None, [P, i32, i64, i64, i64, P, P]),
+            "orc_int8_block_forward": (None, [P, i32, i64, i64, P, P, i64, i64, P, P, i64,
+                                              P, P, P, P, P]),
             "orc_fp8_weight_only_dequant": (None, [P, P, i64, i64, P]),
             "orc_fp8_weight_only_forward": (None, [P, i32, i64, i64, P, P, i64, P, P, i64, P, P]),
             "orc_num_threads": (i32, []),
@@ -202,11 +205,11 @@ def absmax_scale(X, qmax: float) -> float:
 
 
 def quantize_weight(W, mode: str, group: int = 128):
-    """Offline weight quantisation. mode: int8_row | fp8_tensor | fp8_channel | int4_g128.
+    """Offline weight quantisation. mode: int8_row | fp8_tensor | fp8_channel | int4_g128 | int8_block.
 
     Returns (Wq, w_scale) as numpy arrays: int8 [N,K] + fp32 [N]; uint8 e4m3
     [N,K] + fp32 [1]; uint8 e4m3 [N,K] + uint16 bf16 bits [N]; uint8 packed
-    [N,K/2] + fp32 [N,K/group].
+    [N,K/2] + fp32 [N,K/group]; int8 [N,K] + fp32 [N,K/group] (block scales).
     """
     wb, dt = _bits16(W)
     N, K = W.shape
@@ -223,6 +226,11 @@ def quantize_weight(W, mode: str, group: int = 128):
         q = np.zeros((N, K), np.uint8)
         s = np.zeros((N,), np.uint16)
         L.orc_quantize_weight_fp8_channel(_p(wb), dt, N, K, _p(q), _p(s))
+    elif mode == "int8_block":
+        assert K % group == 0
+        q = np.zeros((N, K), np.int8)
+        s = np.zeros((N, K // group), np.float32)
+        L.orc_quantize_weight_int8_block(_p(wb), dt, N, K, group, _p(q), _p(s))
     elif mode == "int4_g128":
         assert K % group == 0
         q = np.zeros((N, K // 2), np.uint8)
@@ -385,3 +393,29 @@ def w4a8_forward(X, Wq4, s_w, group: int = 128, bias=None, rows: Optional[Sequen
     lib().orc_w4a8_forward(_p(xb), dt, M, K, _p(Wq4), _p(s_w), N, group, _p(bb), _p(r), nr,
                            _p(Xq), _p(s_x), _p(Cg), _p(Y64), _p(Y))
     return dict(Xq=Xq, s_x=s_x, Cg=Cg, Y64=Y64, Y=Y, dt=dt)
+
+
+# ---------------------------------------------------------------------------
+# Block-scaled int8 weights (one scale per 32 weights of a row)
+# ---------------------------------------------------------------------------
+
+def int8_block_forward(X, Wq, s_w, block: int = 32, bias=None, rows: Optional[Sequence[int]] = None,
+                       want_cb: bool = False):
+    """Y = s_x[i] * sum_b s_w[j,b] * C_b[i,j] + bias, per-token int8 activations,
+    int8 weights with fp32 scales [N, K/block]."""
+    xb, dt = _bits16(X)
+    M, K = X.shape
+    Wq = _np(Wq, np.int8)
+    s_w = _np(s_w, np.float32)
+    N = Wq.shape[0]
+    bb = None if bias is None else _bits16(bias)[0]
+    r, nr = _rows(rows)
+    R = M if r is None else nr
+    Xq = np.zeros((M, K), np.int8)
+    s_x = np.zeros((M,), np.float32)
+    Cb = np.zeros((R, N, K // block), np.int32) if want_cb else None
+    Y64 = np.zeros((R, N), np.float64)
+    Y = np.zeros((R, N), np.uint16)
+    lib().orc_int8_block_forward(_p(xb), dt, M, K, _p(Wq), _p(s_w), N, block, _p(bb), _p(r), nr,
+                                 _p(Xq), _p(s_x), _p(Cb), _p(Y64), _p(Y))
+    return dict(Xq=Xq, s_x=s_x, Cb=Cb, Y64=Y64, Y=Y, dt=dt)

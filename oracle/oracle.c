@@ -644,6 +644,69 @@ void orc_w4a8_forward(const uint16_t *X, int dt, int64_t M, int64_t K, const uin
     free(s_x);
 }
 
+/* ------------------------------------------------------------------ */
+/* Block-scaled int8 weights (Qwen-Image-2.1-Text-Encoder-FP8, section  */
+/* "How it was tested", where GGUF Q8_0 is compared: int8 codes, one    */
+/* scale for each run of 32 weights). The page fixes only the block of  */
+/* 32 along a weight row and the 8-bit codes; the scale and code rules  */
+/* are the quantiser Q above (s = absmax_block / 127, fp32), and the    */
+/* activations take the W4A8 mode's per-token int8 rows.                */
+/* ------------------------------------------------------------------ */
+
+/* One fp32 scale per (output channel j, block b of B consecutive k):
+ * s_w[j,b] = absmax_{k in b} |W[j,k]| / 127, Wq[j,k] = Q(W[j,k], s_w[j,b]). */
+void orc_quantize_weight_int8_block(const uint16_t *W, int dt, int64_t N, int64_t K, int64_t B,
+                                    int8_t *Wq, float *s_w) {
+    float *w = widen_all(W, dt, N * K);
+    int64_t nb = K / B;
+    for (int64_t j = 0; j < N; ++j) {
+        for (int64_t b = 0; b < nb; ++b) {
+            const float *wb = w + j * K + b * B;
+            float s = scale_of(absmax_range(wb, B), 127.0f);
+            float inv = recip(s);
+            s_w[j * nb + b] = s;
+            for (int64_t k = 0; k < B; ++k) Wq[j * K + b * B + k] = (int8_t)(s == 0.0f ? 0 : q_int(wb[k], inv, 127));
+        }
+    }
+    free(w);
+}
+
+/* Per block b of B columns:
+ *   C_b[i,j] = sum_{k in b} Xq[i,k] * Wq[j,k]  (int32)
+ *   Y64[i,j] = s_x[i] * sum_b s_w[j,b] * C_b[i,j] + bias[j],
+ * with Xq, s_x the per-token int8 rows over all K. */
+void orc_int8_block_forward(const uint16_t *X, int dt, int64_t M, int64_t K, const int8_t *Wq,
+                            const float *s_w, int64_t N, int64_t B, const uint16_t *bias,
+                            const int64_t *rows, int64_t nrows, int8_t *Xq_out, float *s_x_out,
+                            int32_t *Cb, double *Y64, uint16_t *Y) {
+    int8_t *Xq = (int8_t *)malloc((size_t)(M * K > 0 ? M * K : 1));
+    float *s_x = (float *)malloc(sizeof(float) * (size_t)(M > 0 ? M : 1));
+    orc_int8_outlier_prep(X, dt, M, K, 0.0f, Xq, s_x, NULL, NULL, NULL, NULL, 0);
+    if (Xq_out) memcpy(Xq_out, Xq, (size_t)(M * K));
+    if (s_x_out) memcpy(s_x_out, s_x, sizeof(float) * (size_t)M);
+    int64_t nb = K / B;
+    if (!rows) nrows = M;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < nrows; ++r) {
+        int64_t i = rows ? rows[r] : r;
+        for (int64_t j = 0; j < N; ++j) {
+            double acc = 0.0;
+            for (int64_t b = 0; b < nb; ++b) {
+                int64_t c = 0;
+                for (int64_t k = b * B; k < (b + 1) * B; ++k) c += (int64_t)Xq[i * K + k] * (int64_t)Wq[j * K + k];
+                if (Cb) Cb[(r * N + j) * nb + b] = (int32_t)c;
+                acc += (double)s_w[j * nb + b] * (double)c;
+            }
+            double y = (double)s_x[i] * acc;
+            if (bias) y += widen(bias[j], dt);
+            if (Y64) Y64[r * N + j] = y;
+            if (Y) Y[r * N + j] = narrow(y, dt);
+        }
+    }
+    free(Xq);
+    free(s_x);
+}
+
 int orc_num_threads(void) {
 #ifdef _OPENMP
     return omp_get_max_threads();

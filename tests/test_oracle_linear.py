@@ -412,3 +412,83 @@ def test_zero_rows_and_degenerate_scales():
     assert np.all(np.isfinite(p["s_x"])) and np.all(p["s_x"][[0, 2, 3]] > 0)
     xq, sx = oracle.fp8_dynamic_prep(X)
     assert sx[1] == 0.0 and np.all(xq[1] == 0)
+
+
+# ---------------------------------------------------------------------------
+# Block-scaled int8 weights: 8-bit codes with one scale per 32 weights of a
+# row (the text-encoder page's comparison with GGUF Q8_0)
+# ---------------------------------------------------------------------------
+
+def test_int8_block_of_whole_row_is_per_channel():
+    W = rand_w(12, 96, 21)
+    qb, sb = oracle.quantize_weight(W, "int8_block", group=96)
+    qr, sr = oracle.quantize_weight(W, "int8_row")
+    assert np.array_equal(qb, qr) and np.array_equal(sb[:, 0], sr)
+
+
+def test_int8_block_scales_follow_each_slice():
+    N, K, B = 9, 160, 32
+    W = rand_w(N, K, 22).float()
+    W[3, 64:96] = 0.0                                 # an all-zero block: scale 0, codes 0
+    W[5, 40] = 0.5                                    # one large weight moves only its own block
+    W = W.to(torch.bfloat16)
+    q, s = oracle.quantize_weight(W, "int8_block", group=B)
+    assert s.shape == (N, K // B)
+    assert s[3, 2] == 0.0 and np.all(q[3, 64:96] == 0)
+    for b in range(K // B):
+        qs, ss = oracle.quantize_weight(W[:, b * B:(b + 1) * B].contiguous(), "int8_row")
+        assert np.array_equal(q[:, b * B:(b + 1) * B], qs)
+        assert np.array_equal(s[:, b], ss)
+    assert np.abs(q).max() == 127 and q.min() >= -127
+    # the large weight sets its block's scale: 0.5 / 127 in fp32
+    assert s[5, 1] == np.float32(np.float32(0.5) / np.float32(127.0))
+
+
+def test_int8_block_equal_scales_reduce_to_vectorwise():
+    M, K, N, B = 7, 128, 11, 32
+    X = rand_x(M, K, 23)
+    g = torch.Generator().manual_seed(24)
+    W = torch.randn((N, K), generator=g) * 0.02
+    W.view(N, K // B, B)[:, :, 5] = -0.0625          # identical absmax in every block of a row
+    W = W.to(torch.bfloat16)
+    q, s = oracle.quantize_weight(W, "int8_block", group=B)
+    assert np.all(s == s[:, :1])
+    r = oracle.int8_block_forward(X, q, s, block=B, want_cb=True)
+    qr, sr = oracle.quantize_weight(W, "int8_row")
+    assert np.array_equal(q, qr) and np.array_equal(s[:, 0], sr)
+    v = oracle.int8_outlier_forward(X, qr, sr, 0.0)
+    assert np.array_equal(r["Cb"].sum(axis=2).astype(np.int64), v["C"].astype(np.int64))
+    np.testing.assert_allclose(r["Y64"], v["Y64"], rtol=1e-12, atol=0.0)
+    assert np.array_equal(r["Y"], v["Y"])
+
+
+def test_int8_block_forward_within_rounding_bound():
+    """|Y64 - (X W^T + b)| <= sum_k (|x| + s_x/2) * s_w/2 + |w| * s_x/2: each
+    code is its value rounded to the nearest step of its scale."""
+    M, K, N, B = 5, 192, 13, 32
+    X = rand_x(M, K, 25)
+    W = rand_w(N, K, 26)
+    bias = (torch.randn(N, generator=torch.Generator().manual_seed(27)) * 0.1).to(torch.bfloat16)
+    q, s = oracle.quantize_weight(W, "int8_block", group=B)
+    r = oracle.int8_block_forward(X, q, s, block=B, bias=bias, want_cb=True)
+    C = np.zeros((M, N, K // B), np.int64)
+    for b in range(K // B):
+        sl = slice(b * B, (b + 1) * B)
+        C[:, :, b] = r["Xq"][:, sl].astype(np.int64) @ q[:, sl].astype(np.int64).T
+    assert np.array_equal(r["Cb"].astype(np.int64), C)
+    x = X.double().numpy()
+    w = W.double().numpy()
+    exact = x @ w.T + bias.double().numpy()[None, :]
+    sx = r["s_x"].astype(np.float64)[:, None, None]
+    sw = np.repeat(s.astype(np.float64), B, axis=1)[None, :, :]
+    bound = ((np.abs(x)[:, None, :] + sx / 2) * sw / 2 + np.abs(w)[None, :, :] * sx / 2).sum(axis=2)
+    err = np.abs(r["Y64"] - exact)
+    assert np.all(err <= bound * (1 + 1e-6) + 1e-12)
+    # and the bound is not vacuous: the error is a small part of |Y|
+    assert np.linalg.norm(err) < 0.05 * np.linalg.norm(exact)
+    # a transposed block scale breaks the bound somewhere
+    s_bad = s.copy()
+    s_bad[:, [0, 1]] = s_bad[:, [1, 0]]
+    s_bad[:, 0] *= 3.0
+    bad = oracle.int8_block_forward(X, q, s_bad, block=B, bias=bias)
+    assert np.any(np.abs(bad["Y64"] - exact) > bound)
