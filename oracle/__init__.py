@@ -87,6 +87,7 @@ def lib() -> ctypes.CDLL:
             "orc_quantize_weight_int8_block": (None, [P, i32, i64, i64, i64, P, P]),
             "orc_int8_block_forward": (None, [P, i32, i64, i64, P, P, i64, i64, P, P, i64,
                                               P, P, P, P, P]),
+            "orc_fp_linear_forward": (None, [P, i32, i64, i64, P, i64, P, P, i64, P, P]),
             "orc_fp8_weight_only_dequant": (None, [P, P, i64, i64, P]),
             "orc_fp8_weight_only_forward": (None, [P, i32, i64, i64, P, P, i64, P, P, i64, P, P]),
             "orc_num_threads": (i32, []),
@@ -419,3 +420,24 @@ def int8_block_forward(X, Wq, s_w, block: int = 32, bias=None, rows: Optional[Se
     lib().orc_int8_block_forward(_p(xb), dt, M, K, _p(Wq), _p(s_w), N, block, _p(bb), _p(r), nr,
                                  _p(Xq), _p(s_x), _p(Cb), _p(Y64), _p(Y))
     return dict(Xq=Xq, s_x=s_x, Cb=Cb, Y64=Y64, Y=Y, dt=dt)
+
+
+# ---------------------------------------------------------------------------
+# Unquantised 16-bit linear (layers kept in fp16)
+# ---------------------------------------------------------------------------
+
+def fp_linear_forward(X, W, bias=None, rows: Optional[Sequence[int]] = None):
+    """Y = X W^T + bias with X, W (and bias) in one 16-bit dtype; Y64 exact in
+    fp64, Y rounded once to that dtype."""
+    xb, dt = _bits16(X)
+    wb, wdt = _bits16(W)
+    assert wdt == dt, "X and W must share a dtype"
+    M, K = X.shape
+    N = W.shape[0]
+    bb = None if bias is None else _bits16(bias)[0]
+    r, nr = _rows(rows)
+    R = M if r is None else nr
+    Y64 = np.zeros((R, N), np.float64)
+    Y = np.zeros((R, N), np.uint16)
+    lib().orc_fp_linear_forward(_p(xb), dt, M, K, _p(wb), N, _p(bb), _p(r), nr, _p(Y64), _p(Y))
+    return dict(Y64=Y64, Y=Y, dt=dt)

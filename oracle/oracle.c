@@ -604,6 +604,30 @@ void orc_fp8_weight_only_forward(const uint16_t *X, int dt, int64_t M, int64_t K
 }
 
 /* ------------------------------------------------------------------ */
+/* Unquantised 16-bit linear: the layers kept in fp16 because they write */
+/* or cancel massive activations (Image21-Turbo-OrbitQuant-W4A4,        */
+/* section "What 4-bit breaks here and what stays in fp16").            */
+/* ------------------------------------------------------------------ */
+
+/* Y64[i,j] = sum_k X[i,k] * W[j,k] + bias[j] in double (each product of two
+ * 16-bit values is exact); Y = Y64 rounded once to the dtype of X and W. */
+void orc_fp_linear_forward(const uint16_t *X, int dt, int64_t M, int64_t K, const uint16_t *W, int64_t N,
+                           const uint16_t *bias, const int64_t *rows, int64_t nrows, double *Y64, uint16_t *Y) {
+    if (!rows) nrows = M;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < nrows; ++r) {
+        int64_t i = rows ? rows[r] : r;
+        for (int64_t j = 0; j < N; ++j) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k) acc += widen(X[i * K + k], dt) * widen(W[j * K + k], dt);
+            if (bias) acc += widen(bias[j], dt);
+            if (Y64) Y64[r * N + j] = acc;
+            if (Y) Y[r * N + j] = narrow(acc, dt);
+        }
+    }
+}
+
+/* ------------------------------------------------------------------ */
 /* W4A8: int4 per-group weights, int8 per-token activations.           */
 /* ------------------------------------------------------------------ */
 

@@ -492,3 +492,53 @@ def test_int8_block_forward_within_rounding_bound():
     s_bad[:, 0] *= 3.0
     bad = oracle.int8_block_forward(X, q, s_bad, block=B, bias=bias)
     assert np.any(np.abs(bad["Y64"] - exact) > bound)
+
+
+# ---------------------------------------------------------------------------
+# Unquantised 16-bit linear (the layers kept in fp16)
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+def test_fp_linear_identity_returns_the_weight(dtype):
+    K, N = 48, 20
+    W = rand_w(N, K, 31, dtype)
+    r = oracle.fp_linear_forward(torch.eye(K, dtype=dtype), W)
+    assert np.array_equal(r["Y"], W.T.contiguous().view(torch.int16).numpy().view(np.uint16))
+
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+def test_fp_linear_small_integers_are_exact(dtype):
+    """Integer inputs small enough that every sum is an integer the dtype
+    holds exactly: the result is the integer matmul, brute force."""
+    g = torch.Generator().manual_seed(32)
+    M, K, N = 9, 40, 11
+    xi = torch.randint(-3, 4, (M, K), generator=g)
+    wi = torch.randint(-3, 4, (N, K), generator=g)
+    bi = torch.randint(-5, 6, (N,), generator=g)
+    r = oracle.fp_linear_forward(xi.to(dtype), wi.to(dtype), bias=bi.to(dtype))
+    ref = np.zeros((M, N), np.int64)
+    for i in range(M):
+        for j in range(N):
+            ref[i, j] = sum(int(xi[i, k]) * int(wi[j, k]) for k in range(K)) + int(bi[j])
+    assert np.array_equal(r["Y64"], ref.astype(np.float64))
+    assert np.abs(ref).max() <= 256                      # exact in bf16's 8-bit significand
+    assert np.array_equal(oracle.bits_to_torch(r["Y"], r["dt"]).double().numpy(), ref.astype(np.float64))
+
+
+@pytest.mark.parametrize("dtype", [torch.float16, torch.bfloat16])
+def test_fp_linear_rounds_once_to_the_dtype(dtype):
+    """Y is Y64 rounded to nearest even in the dtype (torch's own cast of the
+    fp64 value), and Y64 is within fp64 summation error of X W^T + b."""
+    X = rand_x(6, 128, 33, dtype)
+    W = rand_w(14, 128, 34, dtype)
+    bias = (torch.randn(14, generator=torch.Generator().manual_seed(35)) * 0.1).to(dtype)
+    r = oracle.fp_linear_forward(X, W, bias=bias)
+    cast = torch.from_numpy(r["Y64"]).to(dtype).contiguous().view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(r["Y"], cast)
+    x, w = X.double().numpy(), W.double().numpy()
+    exact = x @ w.T + bias.double().numpy()[None, :]
+    scale = np.abs(x) @ np.abs(w).T + np.abs(bias.double().numpy())[None, :]
+    assert np.all(np.abs(r["Y64"] - exact) <= 1e-13 * scale)
+    # rows= selects rows of the same result
+    sub = oracle.fp_linear_forward(X, W, bias=bias, rows=[5, 0])
+    assert np.array_equal(sub["Y"], r["Y"][[5, 0]])
