@@ -56,7 +56,9 @@ qlin_status check_cuda(cudaError_t e, const char* what) {
 struct DeviceInfo {
   int sms = 0;
   bool sm100 = false;
-  bool gemm_attr_set[64] = {};
+  // set once per kernel instantiation; host threads may race to set it, and
+  // setting a function attribute twice is harmless
+  std::atomic<bool> gemm_attr_set[64] = {};
 };
 std::mutex g_dev_mu;
 DeviceInfo g_dev[16];
@@ -170,7 +172,7 @@ qlin_status launch_gemm_bn(const CUtensorMap& ta, const void* B, EpiParams ep, c
   auto kern = k_gemm<KIND, EPI, TOut, BN, STAGES>;
   constexpr int smem = GemmSmem<BN, STAGES>::TOTAL;
   static_assert(smem <= 227 * 1024, "k_gemm shared memory");
-  if (!d->gemm_attr_set[attr_slot]) {
+  if (!d->gemm_attr_set[attr_slot].load(std::memory_order_acquire)) {
     // the kernel's warpgroups trade registers with setmaxnreg: the launch
     // register count must leave enough in the block's pool for the split
     cudaFuncAttributes fa{};
@@ -182,7 +184,7 @@ qlin_status launch_gemm_bn(const CUtensorMap& ta, const void* B, EpiParams ep, c
     s = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem),
                    "cudaFuncSetAttribute");
     if (s != QLIN_OK) return s;
-    d->gemm_attr_set[attr_slot] = true;
+    d->gemm_attr_set[attr_slot].store(true, std::memory_order_release);
   }
   const int64_t tiles = ((ep.M + GEMM_BM - 1) / GEMM_BM) * ((ep.N + BN - 1) / BN);
   const int grid = grid_ctas > 0 ? grid_ctas : static_cast<int>(tiles < d->sms ? tiles : d->sms);
@@ -278,14 +280,14 @@ qlin_status launch_prep_v(const void* X, const PrepArgs& a, int sms, cudaStream_
   const int NW = static_cast<int>((a.K + 31) / 32);
   const size_t smem = ((OUTL ? static_cast<size_t>(8 * NW) : 0) + 15) / 16 * 16 +
                       static_cast<size_t>(PF_DEPTH) * V * RQ_THREADS * 16;
-  static bool attr_set[16] = {};
+  static std::atomic<bool> attr_set[16] = {};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 16 && !attr_set[dev]) {
+  if (dev >= 0 && dev < 16 && !attr_set[dev].load(std::memory_order_acquire)) {
     qlin_status s0 = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024),
                                 "cudaFuncSetAttribute");
     if (s0 != QLIN_OK) return s0;
-    attr_set[dev] = true;
+    attr_set[dev].store(true, std::memory_order_release);
   }
   int per_sm = 0;
   qlin_status s = check_cuda(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, RQ_THREADS, smem),
@@ -893,10 +895,10 @@ qlin_status launch_w4a8(const int8_t* Xq, const uint8_t* Wq4, const W4Params& wp
   if ((s = make_tmap_bytes(&tb, Wq4, wp.N, wp.K / 2, W4_G / 2, W4_BN, CU_TENSOR_MAP_SWIZZLE_NONE)) != QLIN_OK)
     return s;
   auto kern = k_gemm_w4a8<TOut>;
-  static bool attr_set[16] = {};
+  static std::atomic<bool> attr_set[16] = {};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 16 && !attr_set[dev]) {
+  if (dev >= 0 && dev < 16 && !attr_set[dev].load(std::memory_order_acquire)) {
     // the warpgroups trade registers with setmaxnreg: the launch register
     // count must leave enough in the block's pool for the split
     cudaFuncAttributes fa{};
@@ -908,7 +910,7 @@ qlin_status launch_w4a8(const int8_t* Xq, const uint8_t* Wq4, const W4Params& wp
     s = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, W4Smem::TOTAL),
                    "cudaFuncSetAttribute");
     if (s != QLIN_OK) return s;
-    attr_set[dev] = true;
+    attr_set[dev].store(true, std::memory_order_release);
   }
   const int64_t tiles = ((wp.M + W4_BM - 1) / W4_BM) * ((wp.N + W4_BN - 1) / W4_BN);
   const int grid = static_cast<int>(tiles < d->sms ? tiles : d->sms);
