@@ -542,3 +542,19 @@ def test_fp_linear_rounds_once_to_the_dtype(dtype):
     # rows= selects rows of the same result
     sub = oracle.fp_linear_forward(X, W, bias=bias, rows=[5, 0])
     assert np.array_equal(sub["Y"], r["Y"][[5, 0]])
+
+
+def test_weight_only_fp8_at_unit_scale_is_the_16bit_linear():
+    """With s_w = 1 the dequantised weight is the decoded e4m3 value itself,
+    which bf16 holds exactly: the weight-only forward is then the plain
+    16-bit linear of that weight."""
+    N, K, M = 10, 64, 5
+    codes = _finite_e4m3_codes((N, K), 36)
+    one = np.full(N, 0x3F80, np.uint16)                     # bf16 1.0
+    Wd = torch.from_numpy(oracle.fp8_weight_only_dequant(codes, one).view(np.int16)).view(torch.bfloat16)
+    assert np.array_equal(Wd.double().numpy(), decode_e4m3_torch(codes))
+    X = rand_x(M, K, 37)
+    bias = (torch.randn(N, generator=torch.Generator().manual_seed(38)) * 0.1).to(torch.bfloat16)
+    a = oracle.fp8_weight_only_forward(X, codes, one, bias=bias)
+    b = oracle.fp_linear_forward(X, Wd, bias=bias)
+    assert np.array_equal(a["Y"], b["Y"]) and np.array_equal(a["Y64"], b["Y64"])
