@@ -392,6 +392,47 @@ def test_w4a8_equal_group_scales_reduce_to_per_channel():
     assert np.array_equal(p["Xq"], r["Xq"]) and np.array_equal(p["s_x"], r["s_x"])
 
 
+def test_w4a8_unequal_group_scales_within_rounding_bound():
+    """Groups whose scales differ by up to 50x: the output stays within the
+    half-step bound of X W^T + b (every int4 code is its weight rounded to the
+    nearest step of its own group's scale, every int8 code its activation to
+    the nearest step of the row scale), per-group int32 sums equal numpy's
+    integer matmul of the unpacked codes, and a swapped pair of group scales
+    breaks the bound. A wrong group index in the scale combination fails here."""
+    M, K, N, G = 6, 512, 9, 128
+    X = rand_x(M, K, 31)
+    g = torch.Generator().manual_seed(32)
+    W = torch.randn((N, K), generator=g) * 0.02
+    for gi, f in enumerate((1.0, 50.0, 0.2, 7.0)):   # a different magnitude in every group
+        W[:, gi * G:(gi + 1) * G] *= f
+    W = W.to(torch.bfloat16)
+    bias = (torch.randn(N, generator=torch.Generator().manual_seed(33)) * 0.1).to(torch.bfloat16)
+    q, s = oracle.quantize_weight(W, "int4_g128")
+    assert np.all(s.max(axis=1) > 40 * s.min(axis=1))
+    r = oracle.w4a8_forward(X, q, s, group=G, bias=bias, want_cg=True)
+    u = unpack_int4(q, K).astype(np.int64)
+    for gi in range(K // G):
+        sl = slice(gi * G, (gi + 1) * G)
+        assert np.array_equal(r["Cg"][:, :, gi].astype(np.int64), r["Xq"][:, sl].astype(np.int64) @ u[:, sl].T)
+    x = X.double().numpy()
+    w = W.double().numpy()
+    exact = x @ w.T + bias.double().numpy()[None, :]
+    sx = r["s_x"].astype(np.float64)[:, None, None]
+    sw = np.repeat(s.astype(np.float64), G, axis=1)[None, :, :]
+    bound = ((np.abs(x)[:, None, :] + sx / 2) * sw / 2 + np.abs(w)[None, :, :] * sx / 2).sum(axis=2)
+    err = np.abs(r["Y64"] - exact)
+    assert np.all(err <= bound * (1 + 1e-6) + 1e-12)
+    assert np.linalg.norm(err) < 0.25 * np.linalg.norm(exact)   # int4 steps: about 11% noise here
+    # the scale-weighted group sum the page's format defines, from the oracle's own partials
+    y = r["s_x"].astype(np.float64)[:, None] * (r["Cg"].astype(np.float64) * s.astype(np.float64)[None]).sum(axis=2)
+    np.testing.assert_allclose(r["Y64"], y + bias.double().numpy()[None, :], rtol=1e-12, atol=1e-12)
+    # the scales of groups 0 and 1 exchanged: far outside the bound
+    s_bad = s.copy()
+    s_bad[:, [0, 1]] = s_bad[:, [1, 0]]
+    bad = oracle.w4a8_forward(X, q, s_bad, group=G, bias=bias)
+    assert np.any(np.abs(bad["Y64"] - exact) > bound)
+
+
 def test_rows_subset_matches_full():
     wl = workloads.get_workload("tiny_int8")
     X, W, bias = workloads.make_linear(wl, wl.linears[0])
@@ -542,6 +583,31 @@ def test_fp_linear_rounds_once_to_the_dtype(dtype):
     # rows= selects rows of the same result
     sub = oracle.fp_linear_forward(X, W, bias=bias, rows=[5, 0])
     assert np.array_equal(sub["Y"], r["Y"][[5, 0]])
+
+
+def test_fp_linear_mixed_magnitudes_within_fp64_summation_bound():
+    """Products spread over 2^-40 .. 2^40 with cancellation: the oracle adds
+    the exact products one by one in fp64, so Y64 is within the recursive
+    summation bound (K - 1) * 2^-53 * sum |x w| of the exact rational sum
+    (Python fractions), and Y is Y64 rounded once to the dtype."""
+    from fractions import Fraction
+    g = torch.Generator().manual_seed(39)
+    M, K, N = 4, 64, 6
+    ex = torch.randint(-20, 21, (M, K), generator=g).double()
+    ew = torch.randint(-20, 21, (N, K), generator=g).double()
+    X = (torch.randn((M, K), generator=g).double() * torch.pow(2.0, ex)).to(torch.bfloat16)
+    W = (torch.randn((N, K), generator=g).double() * torch.pow(2.0, ew)).to(torch.bfloat16)
+    X[:, 1] = -X[:, 0]                                     # exact cancellation of large pairs
+    W[:, 1] = W[:, 0]
+    r = oracle.fp_linear_forward(X, W)
+    x, w = X.double().numpy(), W.double().numpy()
+    for i in range(M):
+        for j in range(N):
+            exact = sum(Fraction(float(x[i, k])) * Fraction(float(w[j, k])) for k in range(K))
+            mag = sum(abs(Fraction(float(x[i, k])) * Fraction(float(w[j, k]))) for k in range(K))
+            assert abs(Fraction(float(r["Y64"][i, j])) - exact) <= Fraction(K - 1, 2 ** 53) * mag
+    cast = torch.from_numpy(r["Y64"]).to(torch.bfloat16).contiguous().view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(r["Y"], cast)
 
 
 def test_weight_only_fp8_at_unit_scale_is_the_16bit_linear():
