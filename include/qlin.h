@@ -257,10 +257,14 @@ QLIN_API qlin_status qlin_e4m3_encode_f32(const float *t, uint8_t *codes, int64_
  * array of QLIN_NOALLOC_SCRATCH_BYTES inside the library, which every GPU
  * that loads the library holds until the process exits. The model-card pages
  * have no counterpart of this entry point.
- *   - Shapes whose qlin_workspace_bytes(QLIN_OP_INT8_OUTLIER, M, N, K) exceeds
- *     QLIN_NOALLOC_SCRATCH_BYTES are rejected with QLIN_ERR_UNSUPPORTED and a
- *     message; nothing is enqueued. Arguments are otherwise validated as in
- *     qlin_int8_outlier_forward.
+ *   - Its scratch holds the workspace layout of qlin_int8_outlier_forward
+ *     without the stream-K partial slots (the GEMM then takes whole tiles;
+ *     the results are the same). That is about M*K bytes of codes plus
+ *     2*(M+N)*round_up(K,8) bytes for the worst-case outlier columns X_O and
+ *     W_O: M = 2048, K = N = 4096 needs 56.3 MiB and fits; the 1024^2 DiT
+ *     linears (M = 4352, K or N = 12288) do not. Larger shapes are rejected
+ *     with QLIN_ERR_UNSUPPORTED and a message; nothing is enqueued. Arguments
+ *     are otherwise validated as in qlin_int8_outlier_forward.
  *   - It calls no cudaMalloc, cudaFree or other allocating routine.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress); make that first call before any stream capture.

@@ -388,7 +388,9 @@ int sk_capacity(int64_t M, int64_t N, int64_t K) {
   return static_cast<int>(T < GEMM_SK_MAX_CTAS ? T : GEMM_SK_MAX_CTAS);
 }
 
-Int8Ws int8_layout(void* base, int64_t M, int64_t N, int64_t K, bool with_gemm_parts) {
+// with_sk: room for the stream-K arrival counters and partial slots (the
+// GEMM then may run stream-K); without it the GEMM takes whole tiles only.
+Int8Ws int8_layout(void* base, int64_t M, int64_t N, int64_t K, bool with_gemm_parts, bool with_sk = true) {
   Int8Ws w{};
   uint8_t* p = static_cast<uint8_t*>(base);
   size_t off = 0;
@@ -398,7 +400,7 @@ Int8Ws int8_layout(void* base, int64_t M, int64_t N, int64_t K, bool with_gemm_p
     return r;
   };
   const int64_t NW = (K + 31) / 32;
-  const int64_t nctr = with_gemm_parts ? GEMM_EPI_GROUPS * sk_tiles(M, N) : 0;
+  const int64_t nctr = with_gemm_parts && with_sk ? GEMM_EPI_GROUPS * sk_tiles(M, N) : 0;
   uint8_t* hdr = take(16 + 4 * NW + 4 * nctr);
   w.sync = reinterpret_cast<uint32_t*>(hdr);
   w.count = reinterpret_cast<int32_t*>(hdr ? hdr + 4 : nullptr);
@@ -416,9 +418,10 @@ Int8Ws int8_layout(void* base, int64_t M, int64_t N, int64_t K, bool with_gemm_p
     w.W_O = reinterpret_cast<uint16_t*>(take(static_cast<size_t>(2 * N * w.ostride)));
     w.XqO = reinterpret_cast<int8_t*>(take(static_cast<size_t>(M * OUTL_CODES)));
     w.WqO = reinterpret_cast<int8_t*>(take(static_cast<size_t>(N * OUTL_CODES)));
-    w.sk_ctas = sk_capacity(M, N, K);
-    w.sk_part = reinterpret_cast<int32_t*>(
-        take(static_cast<size_t>(2 * w.sk_ctas) * GEMM_BM * GEMM_SK_BN * sizeof(int32_t)));
+    w.sk_ctas = with_sk ? sk_capacity(M, N, K) : 0;
+    w.sk_part = with_sk ? reinterpret_cast<int32_t*>(
+                              take(static_cast<size_t>(2 * w.sk_ctas) * GEMM_BM * GEMM_SK_BN * sizeof(int32_t)))
+                        : nullptr;
   }
   w.total = off;
   return w;
@@ -455,6 +458,29 @@ qlin_status check_common(const void* X, qlin_dtype dt, int64_t M, int64_t K, int
   if (X == nullptr && M > 0) return fail(QLIN_ERR_INVALID_ARG, "X is NULL");
   if (!aligned16(X)) return fail(QLIN_ERR_ALIGNMENT, "X is not 16-byte aligned");
   return QLIN_OK;
+}
+
+// The two stages of the LLM.int8 forward on a workspace already carved
+// (arguments validated by the caller).
+qlin_status int8_outlier_prepare_ws(const void* X, qlin_dtype xdt, int64_t M, int64_t K, const int8_t* Wq,
+                                    const float* w_scale, int64_t N, float threshold, const Int8Ws& w,
+                                    cudaStream_t st) {
+  const WoGather wo{Wq, w_scale, N, w.O, w.W_O, w.WqO};
+  return xdt == QLIN_BF16
+             ? int8_prep_impl<__nv_bfloat16>(X, M, K, threshold, w, w.Xq, w.s_x, w.X_O, w.ostride, st, wo)
+             : int8_prep_impl<__half>(X, M, K, threshold, w, w.Xq, w.s_x, w.X_O, w.ostride, st, wo);
+}
+
+qlin_status int8_outlier_gemm_ws(qlin_dtype xdt, int64_t M, int64_t K, const int8_t* Wq, const float* w_scale,
+                                 int64_t N, const void* bias, void* Y, const Int8Ws& w, cudaStream_t st) {
+  EpiParams ep{};
+  ep.M = M; ep.N = N; ep.K = K; ep.Y = Y;
+  ep.s_x = w.s_x; ep.s_w = w_scale; ep.bias = static_cast<const uint16_t*>(bias);
+  ep.count = w.count; ep.X_O = w.X_O; ep.W_O = w.W_O; ep.ostride = w.ostride;
+  ep.Xq = w.Xq; ep.Wq = Wq; ep.O = w.O; ep.XqO = w.XqO; ep.WqO = w.WqO;
+  ep.sk_count = w.sk_count; ep.sk_part = w.sk_part;
+  if (xdt == QLIN_BF16) return launch_gemm<0, EPI_INT8_OUTLIER, __nv_bfloat16>(w.Xq, Wq, ep, st, 1, w.sk_ctas);
+  return launch_gemm<0, EPI_INT8_OUTLIER, __half>(w.Xq, Wq, ep, st, 2, w.sk_ctas);
 }
 
 #define QLIN_TRY(...)                  \
@@ -697,13 +723,8 @@ qlin_status qlin_int8_outlier_prepare(const void* X, qlin_dtype xdt, int64_t M, 
   QLIN_REQ_PTR(workspace, "workspace");
   DeviceInfo* d;
   QLIN_TRY(device_info(&d));
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  Int8Ws w = int8_layout(workspace, M, N, K, true);
-  const bool bf = (xdt == QLIN_BF16);
-  const WoGather wo{Wq, w_scale, N, w.O, w.W_O, w.WqO};
-  QLIN_TRY(bf ? int8_prep_impl<__nv_bfloat16>(X, M, K, threshold, w, w.Xq, w.s_x, w.X_O, w.ostride, st, wo)
-              : int8_prep_impl<__half>(X, M, K, threshold, w, w.Xq, w.s_x, w.X_O, w.ostride, st, wo));
-  (void)d;
+  QLIN_TRY(int8_outlier_prepare_ws(X, xdt, M, K, Wq, w_scale, N, threshold, int8_layout(workspace, M, N, K, true),
+                                   static_cast<cudaStream_t>(stream)));
   return ok();
 }
 
@@ -722,16 +743,8 @@ qlin_status qlin_int8_outlier_gemm(qlin_dtype xdt, int64_t M, int64_t K, const i
   if (workspace == nullptr || ws_bytes < qlin_workspace_bytes(QLIN_OP_INT8_OUTLIER, M, N, K))
     return fail(QLIN_ERR_WORKSPACE, "workspace too small");
   QLIN_REQ_PTR(workspace, "workspace");
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  Int8Ws w = int8_layout(workspace, M, N, K, true);
-  EpiParams ep{};
-  ep.M = M; ep.N = N; ep.K = K; ep.Y = Y;
-  ep.s_x = w.s_x; ep.s_w = w_scale; ep.bias = static_cast<const uint16_t*>(bias);
-  ep.count = w.count; ep.X_O = w.X_O; ep.W_O = w.W_O; ep.ostride = w.ostride;
-  ep.Xq = w.Xq; ep.Wq = Wq; ep.O = w.O; ep.XqO = w.XqO; ep.WqO = w.WqO;
-  ep.sk_count = w.sk_count; ep.sk_part = w.sk_part;
-  if (xdt == QLIN_BF16) QLIN_TRY((launch_gemm<0, EPI_INT8_OUTLIER, __nv_bfloat16>(w.Xq, Wq, ep, st, 1, w.sk_ctas)));
-  else QLIN_TRY((launch_gemm<0, EPI_INT8_OUTLIER, __half>(w.Xq, Wq, ep, st, 2, w.sk_ctas)));
+  QLIN_TRY(int8_outlier_gemm_ws(xdt, M, K, Wq, w_scale, N, bias, Y, int8_layout(workspace, M, N, K, true),
+                                static_cast<cudaStream_t>(stream)));
   return ok();
 }
 
@@ -1035,6 +1048,12 @@ qlin_status noalloc_scratch(void** out) {
   *out = g_noalloc_ptr[dev];
   return QLIN_OK;
 }
+
+// Bytes of built-in scratch the forward needs: the LLM.int8 workspace layout
+// without the stream-K arrival counters and partial slots.
+size_t noalloc_scratch_needed(int64_t M, int64_t N, int64_t K) {
+  return int8_layout(nullptr, M, N, K, true, false).total;
+}
 }  // namespace
 
 extern "C" qlin_status qlin_int8_outlier_forward_noalloc(const void* X, qlin_dtype xdt, int64_t M, int64_t K,
@@ -1042,17 +1061,29 @@ extern "C" qlin_status qlin_int8_outlier_forward_noalloc(const void* X, qlin_dty
                                                          float threshold, const void* bias, void* Y, void* stream) {
   QLIN_TRY(check_common(X, xdt, M, K, N));
   if (M == 0 || N == 0) return ok();
-  const size_t need = qlin_workspace_bytes(QLIN_OP_INT8_OUTLIER, M, N, K);
+  // the built-in scratch holds the forward's layout without the stream-K
+  // partial slots (the GEMM then takes whole tiles, the same results)
+  const size_t need = noalloc_scratch_needed(M, N, K);
   if (need > static_cast<size_t>(QLIN_NOALLOC_SCRATCH_BYTES))
     return fail(QLIN_ERR_UNSUPPORTED,
                 "qlin_int8_outlier_forward_noalloc: M=%lld N=%lld K=%lld needs %zu bytes of scratch, more than the "
                 "%lld bytes of its built-in array; use qlin_int8_outlier_forward with a workspace",
                 static_cast<long long>(M), static_cast<long long>(N), static_cast<long long>(K), need,
                 static_cast<long long>(QLIN_NOALLOC_SCRATCH_BYTES));
+  QLIN_REQ_PTR(Y, "Y");
+  QLIN_REQ_PTR(Wq, "Wq");
+  QLIN_REQ_PTR(w_scale, "w_scale");
+  if (bias != nullptr && !aligned16(bias)) return fail(QLIN_ERR_ALIGNMENT, "bias is not 16-byte aligned");
+  DeviceInfo* d;
+  QLIN_TRY(device_info(&d));
   void* ws = nullptr;
   QLIN_TRY(noalloc_scratch(&ws));
-  return qlin_int8_outlier_forward(X, xdt, M, K, Wq, w_scale, N, threshold, bias, Y, ws,
-                                   static_cast<size_t>(QLIN_NOALLOC_SCRATCH_BYTES), stream);
+  const Int8Ws w = int8_layout(ws, M, N, K, true, false);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  QLIN_TRY(int8_outlier_prepare_ws(X, xdt, M, K, Wq, w_scale, N, threshold, w, st));
+  QLIN_TRY(int8_outlier_gemm_ws(xdt, M, K, Wq, w_scale, N, bias, Y, w, st));
+  return ok();
 }
+
 
 

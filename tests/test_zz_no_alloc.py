@@ -17,8 +17,9 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import workloads
-from tests._parity import ROW_REL_TOL
+from tests._parity import ROW_REL_TOL, assert_rows_close
 
 pytestmark = pytest.mark.gpu
 
@@ -70,6 +71,30 @@ def test_noalloc_matches_regular_forward_twice():
         torch.cuda.synchronize()
         assert torch.isfinite(got.float()).all()
         assert _row_rel(got, ref) <= ROW_REL_TOL
+        # and directly against the CPU oracle, as the other parity tests do
+        r = oracle.int8_outlier_forward(X, Wq.cpu().numpy(), s_w.cpu().numpy(), 6.0, bias=bias)
+        assert_rows_close(got, r, what="no-alloc forward")
+    assert q.qlin_get_device_status() == 0
+
+
+def test_noalloc_accepts_the_documented_example_shape():
+    """M = 2048, K = N = 4096 needs about 56 MiB of the 64 MiB array (the
+    workspace layout without stream-K slots): accepted, and equal to the
+    regular forward within the parity tolerance."""
+    import quantized_w8a8_linear_b200 as q
+    g = torch.Generator().manual_seed(12)
+    M, K, N = 2048, 4096, 4096
+    X = torch.randn((M, K), generator=g)
+    X[5, 100] = 20.0
+    X[1000, 4000] = -7.5
+    X = X.to(torch.bfloat16).cuda()
+    W = (torch.randn((N, K), generator=g) * 0.02).to(torch.bfloat16).cuda()
+    Wq, s_w = q.qlin_quantize_weight(W, q.QLIN_W_INT8_ROW)
+    ref = q.qlin_int8_outlier_forward(X, Wq, s_w, 6.0)
+    got = _noalloc(q, X, Wq, s_w, 6.0)
+    torch.cuda.synchronize()
+    assert torch.isfinite(got.float()).all()
+    assert _row_rel(got, ref) <= ROW_REL_TOL
     assert q.qlin_get_device_status() == 0
 
 
