@@ -1,9 +1,12 @@
 // prep.cuh -- HBM-bound kernels around the GEMM:
 //   * k_prep_rows: per-row absmax, scale and int8 or E4M3 codes (activations
-//     and weights); for LLM.int8 activations the same cooperative launch also
-//     detects the outlier columns (any |x| > threshold in the column, over
-//     every token of the call), excludes them from the row absmax, copies
-//     them exactly into X_O and writes the outlier weight columns W_O;
+//     and weights); for LLM.int8 activations it also flags the outlier columns
+//     (any |x| > threshold in the column, over every token of the call) and
+//     leaves entries above the threshold out of the row absmax;
+//   * k_ws_reset / k_outlier_finish: the rest of the LLM.int8 prepare stage
+//     around that pass (zeroed header before it; after it the outlier list,
+//     exact copies X_O of the outlier columns, the rows whose absmax sat in
+//     an outlier column requantised, and the outlier weight columns W_O);
 //   * k_gather_wo: dequantised outlier weight columns (standalone)
 //   * k_zero_outlier_cols: zero codes of the outlier columns (standalone)
 //     W_O[j,o] = dtype(fp32(Wq[j,O[o]]) * s_w[j]) (the weight.to(dtype) *
@@ -91,6 +94,7 @@ struct WoGather {
 constexpr int OUTL_CODES = 32;
 constexpr int OUTL_FP_MMA_K = 16;
 constexpr int OUTL_LIST = 64;   // outlier counts up to this keep the column list in shared memory
+constexpr int OUTL_MAX_K = 32768; // the largest K the library takes
 
 // Round-half-even of an fp32 value in (-2^22, 2^22) to an integer, read from
 // the low byte of t + 1.5 * 2^23: the add rounds to nearest even, and within
@@ -143,26 +147,16 @@ __device__ __forceinline__ uint32_t keep_mask(uint32_t om, int i) {
 // scale is bf16(absmax / QMAX) and the codes use that rounded value (the
 // [out,1] bf16 weight scales of the Text-Encoder-FP8 page).
 //
-// OUTL (LLM.int8 activations) reads X from HBM once, in one cooperative
-// launch:
-//   pass 1   every row is quantised with the absmax over its entries with
-//            |x| <= thr (entries above the threshold get code 0 and set their
-//            column's bit in the outlier bitmap). Because a column outside
-//            the outlier set O holds no entry above the threshold, this absmax
-//            equals the exact one (over k not in O) unless the maximum sits in
-//            a column of O; the raw absmax pattern is kept per row;
-//   barrier  bounded grid-wide barrier (flags and the counter are zeroed by
-//            the host before the launch; all CTAs are co-resident);
-//   compact  every CTA scans the bitmap into shared memory (per-word prefix
-//            counts); CTA 0 writes the ascending list O and the count;
-//   fix-up   per row, one warp reads the row's values in the O columns and
-//            copies them to X_O (zero-padded to a multiple of 8, or to 16) and, for up
-//            to OUTL_CODES columns, minus the codes pass 1 left there to XqO
-//            (the GEMM takes those codes' products back out, so Xq keeps them); if
-//            the largest of the values that is <= thr reaches the kept
-//            absmax, the row is requantised with the exact absmax (by the
-//            whole CTA, from shared memory), its outlier codes then 0;
-//   W_O      the dequantised outlier weight columns (wo.N > 0).
+// OUTL (LLM.int8 activations): the streaming pass of the prepare stage. Every
+// row is quantised with the absmax over its entries with |x| <= thr; entries
+// above the threshold get code 0 and set their column's bit in the outlier
+// bitmap. Because a column outside the outlier set O holds no entry above the
+// threshold, this absmax equals the exact one (over k not in O) unless the
+// maximum sits in a column of O; the raw absmax pattern is kept per row so
+// that k_outlier_finish can tell. The bitmap is zeroed by k_ws_reset, the
+// kernel launched just before this one: this kernel is its programmatic
+// dependent, so it runs while k_ws_reset finishes, and waits for it
+// (griddepcontrol.wait) only before OR-ing its columns into the bitmap.
 // ---------------------------------------------------------------------------
 constexpr int RQ_THREADS = 256;
 constexpr int RQ_WARPS = RQ_THREADS / 32;
@@ -178,26 +172,7 @@ struct PrepArgs {
   uint16_t* s_bf16;
   uint16_t* amax_bits; // [M] pass-1 absmax pattern (OUTL)
   uint32_t* flags;     // [NW] outlier bitmap (zero on entry for OUTL)
-  int32_t* O;          // [K]  ascending outlier columns (written by CTA 0)
-  int32_t* count;      // [1]
-  uint32_t* sync;      // grid barrier counter (zero on entry for OUTL)
-  uint32_t* rowctr;    // next-row counter (zero on entry), or nullptr for a static row split
-  uint16_t* X_O;
-  int64_t ostride;
-  int8_t* XqO;         // [M, OUTL_CODES] minus the codes in the outlier columns (count <= OUTL_CODES), or nullptr
-  WoGather wo;
 };
-
-// The (o+1)-th outlier column, from the shared bitmap and its word prefixes.
-__device__ __forceinline__ int outlier_col(const uint32_t* sflags, const int32_t* swpre, int NW, int o) {
-  int lo = 0, hi = NW - 1;   // largest w with swpre[w] <= o
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (swpre[mid] <= o) lo = mid;
-    else hi = mid - 1;
-  }
-  return lo * 32 + static_cast<int>(__fns(sflags[lo], 0, o - swpre[lo] + 1));
-}
 
 template <typename T, int CODE>
 __device__ __forceinline__ uint2 quant_vec(const uint4& v, uint32_t om, float inv, bool fast, bool zero) {
@@ -233,14 +208,17 @@ __device__ __forceinline__ uint2 quant_vec(const uint4& v, uint32_t om, float in
   }
 }
 
-// 8 flags: bit e set iff the 16-bit |x| pattern of element e exceeds tb.
-__device__ __forceinline__ uint32_t above_bits(const uint4& v, uint32_t tb) {
-  uint16_t h[8];
-  unpack8(v, h);
-  uint32_t m = 0;
-#pragma unroll
-  for (int e = 0; e < 8; ++e) m |= ((h[e] & 0x7FFFu) > tb ? 1u : 0u) << e;
-  return m;
+// Lanes of a packed 16-bit pair whose |x| pattern exceeds tb: with a = |x|
+// (<= 0x7FFF) and c = 0x7FFF - tb, a > tb exactly when a + c >= 0x8000, and
+// a + c <= 0xFFFE never carries into the other lane, so bit 15 of each lane
+// of (a + c) flags it. c2 = c * 0x10001 (both lanes).
+__device__ __forceinline__ uint32_t above2(uint32_t w, uint32_t c2) { return ((w & 0x7FFF7FFFu) + c2) & 0x80008000u; }
+// All-ones in the flagged lanes of above2's result.
+__device__ __forceinline__ uint32_t lanes_of(uint32_t flagged) { return (flagged >> 15) * 0xFFFFu; }
+// The 8 flags of a vector (bit e: element e; element 2i is the low lane of word i).
+__device__ __forceinline__ uint32_t flag_byte(uint32_t f0, uint32_t f1, uint32_t f2, uint32_t f3) {
+  return ((f0 >> 15) & 1u) | ((f0 >> 30) & 2u) | ((f1 >> 13) & 4u) | ((f1 >> 28) & 8u) | ((f2 >> 11) & 16u) |
+         ((f2 >> 26) & 32u) | ((f3 >> 9) & 64u) | ((f3 >> 24) & 128u);
 }
 
 // Running packed |x| max of one vector into m2 (16-bit pairs).
@@ -256,22 +234,23 @@ __device__ __forceinline__ uint32_t pair_max_bits(uint32_t m2) {
 
 template <typename T, int V, int CODE, bool SCALE_BF16, bool OUTL>
 __global__ void __launch_bounds__(RQ_THREADS, 3) k_prep_rows(const T* __restrict__ X, const PrepArgs a) {
-  // the GEMM that follows may be scheduled now (it waits for this grid's
+  // the kernel that follows may be scheduled now (it waits for this grid's
   // completion before it reads anything this kernel writes)
   griddep_launch_dependents();
-  extern __shared__ uint32_t psm[];   // OUTL: sflags[NW], swpre[NW]
+  extern __shared__ uint4 stage[];   // [PF_DEPTH][V][RQ_THREADS] 16-byte vectors
   __shared__ uint32_t red[2][RQ_WARPS];
+  // OUTL: the CTA's outlier columns, OR-ed into the global bitmap once at the
+  // end (per-row global atomics on the few words of the outlier columns
+  // contend with every other CTA's and were measured to stall the rows)
+  __shared__ uint32_t sbits[OUTL ? (OUTL_MAX_K / 32) : 1];
   const int64_t M = a.M, K = a.K;
   const int KV = static_cast<int>(K / 8);
-  const int NW = static_cast<int>((K + 31) / 32);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int rw = a.rw;
   const int units = RQ_WARPS / rw;
   const int unit = warp / rw;
   const int ut = tid - unit * rw * 32;   // thread index inside the unit
   const int UT = rw * 32;
-  uint32_t* sflags = psm;
-  int32_t* swpre = reinterpret_cast<int32_t*>(psm + NW);
   constexpr float QMAX = CODE == 0 ? 127.0f : 448.0f;
 
   // max over the unit (warp redux, then the unit's warps through shared
@@ -288,21 +267,21 @@ __global__ void __launch_bounds__(RQ_THREADS, 3) k_prep_rows(const T* __restrict
     return m;
   };
 
-  // ---------------- pass 1: rows of this unit, PF_DEPTH - 1 rows in flight ----------------
-  // staging: [PF_DEPTH][V][RQ_THREADS] 16-byte vectors, each thread only
-  // touches its own column, so cp.async.wait_group alone orders it
-  uint4* stage = reinterpret_cast<uint4*>(psm + ((OUTL ? 2 * NW : 0) + 3) / 4 * 4);
-  // rows: taken one at a time from a global counter (balances the units when
-  // rows cost different amounts), or split statically. The unit's leader keeps
-  // a ring of the unit's next row indices in shared memory, PF_DEPTH ahead.
+  // staging: each thread only touches its own column of `stage`, so
+  // cp.async.wait_group alone orders it.
+  // Rows: unit u of CTA b takes rows (d * G + b) * units + u, d = 0, 1, ...
+  // (a static split: a global row counter was measured to cost 2-3 us in
+  // contended atomics). The unit's leader keeps a ring of the unit's next row
+  // indices in shared memory.
   const int64_t first = static_cast<int64_t>(blockIdx.x) * units + unit;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * units;
   __shared__ long long rowq[RQ_WARPS][8];
   long long* myq = rowq[unit];
-  auto grab = [&](int k) -> long long {
-    return a.rowctr != nullptr ? static_cast<long long>(atomicAdd(a.rowctr, 1u))
-                               : static_cast<long long>(first + static_cast<int64_t>(k) * stride);
-  };
+  auto grab = [&](int k) -> long long { return static_cast<long long>(first + static_cast<int64_t>(k) * stride); };
+  if constexpr (OUTL) {
+    for (int i = tid; i < (K + 31) / 32; i += RQ_THREADS) sbits[i] = 0u;
+    __syncthreads();
+  }
   auto issue = [&](int64_t r, int slot) {
     const uint4* xr = reinterpret_cast<const uint4*>(X + (r < M ? r : 0) * K);
 #pragma unroll
@@ -341,25 +320,24 @@ __global__ void __launch_bounds__(RQ_THREADS, 3) k_prep_rows(const T* __restrict
 #pragma unroll
     for (int u = 0; u < V; ++u) m2 = vec_absmax2<T>(m2, cur[u]);
     uint32_t mb = unit_max(pair_max_bits(m2));
-    uint32_t om[V];
-#pragma unroll
-    for (int u = 0; u < V; ++u) om[u] = 0u;
     if (OUTL && mb > a.thr_bits) {
-      // some entry of this row exceeds the threshold: flag its column and
-      // leave it out of the absmax
+      // some entry of this row exceeds the threshold: flag its column, and
+      // zero it, which leaves it out of the absmax and gives it code 0
+      const uint32_t c2 = (0x7FFFu - a.thr_bits) * 0x10001u;
       uint32_t mm = 0;
 #pragma unroll
       for (int u = 0; u < V; ++u) {
-        const int idx = ut + u * UT;
-        if (idx < KV) {
-          om[u] = above_bits(cur[u], a.thr_bits);
-          if (om[u]) atomicOr(a.flags + (idx >> 2), om[u] << ((idx & 3) * 8));
-        }
+        const int idx = ut + u * UT;   // vectors past the row are zero: never flagged
         uint4 x = cur[u];
-        x.x &= keep_mask(om[u], 0);
-        x.y &= keep_mask(om[u], 1);
-        x.z &= keep_mask(om[u], 2);
-        x.w &= keep_mask(om[u], 3);
+        const uint32_t f0 = above2(x.x, c2), f1 = above2(x.y, c2), f2 = above2(x.z, c2), f3 = above2(x.w, c2);
+        if ((f0 | f1 | f2 | f3) != 0u) {
+          atomicOr(&sbits[idx >> 2], flag_byte(f0, f1, f2, f3) << ((idx & 3) * 8));
+          x.x &= ~lanes_of(f0);
+          x.y &= ~lanes_of(f1);
+          x.z &= ~lanes_of(f2);
+          x.w &= ~lanes_of(f3);
+          cur[u] = x;
+        }
         mm = vec_absmax2<T>(mm, x);
       }
       mb = unit_max(pair_max_bits(mm));
@@ -383,36 +361,100 @@ __global__ void __launch_bounds__(RQ_THREADS, 3) k_prep_rows(const T* __restrict
 #pragma unroll
     for (int u = 0; u < V; ++u) {
       const int idx = ut + u * UT;
-      if (idx < KV) qr[idx] = quant_vec<T, CODE>(cur[u], om[u], inv, fast, zero);
+      if (idx < KV) qr[idx] = quant_vec<T, CODE>(cur[u], 0u, inv, fast, zero);
     }
   }
   cp_async_wait<0>();
-  if constexpr (!OUTL) return;
-
-  // ---------------- grid barrier (bounded) ----------------
-  __shared__ int bar_ok;
-  __syncthreads();
-  if (tid == 0) {
-    __threadfence();
-    atomicAdd(a.sync, 1u);
-    int ok = 1;
-    const uint64_t t0 = globaltimer();
-    while (*reinterpret_cast<volatile uint32_t*>(a.sync) < gridDim.x) {
-      if (globaltimer() - t0 > g_wait_timeout_ns) {
-        atomicExch(&g_status, 6 /* QLIN_ERR_TIMEOUT */);
-        ok = 0;
-        break;
-      }
-    }
-    __threadfence();
-    bar_ok = ok;
+  if constexpr (OUTL) {
+    // the global bitmap was zeroed by the kernel before this one (this grid is
+    // its programmatic dependent; a no-op without a programmatic launch)
+    griddep_wait();
+    __syncthreads();
+    for (int i = tid; i < (K + 31) / 32; i += RQ_THREADS)
+      if (sbits[i] != 0u) atomicOr(a.flags + i, sbits[i]);
   }
-  __syncthreads();
-  if (!bar_ok) return;
+}
+
+// Zeroes the per-call header of the LLM.int8 workspace (row counter, outlier
+// count and bitmap, stream-K arrival counters) at the start of a prepare
+// stage. The streaming pass is launched as its programmatic dependent.
+__global__ void __launch_bounds__(256) k_ws_reset(uint32_t* __restrict__ hdr, int64_t words) {
+  griddep_launch_dependents();
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < words;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    hdr[i] = 0u;
+}
+
+// ---------------------------------------------------------------------------
+// The rest of the LLM.int8 prepare stage, once the streaming pass has seen
+// every row (a programmatic dependent of it: scheduled as its CTAs leave,
+// then griddepcontrol.wait until it has completed):
+//   compact  every CTA scans the bitmap into shared memory (per-word prefix
+//            counts; the ascending list itself for up to OUTL_LIST columns);
+//            CTA 0 writes the list O and the count;
+//   W_O      one thread per weight row: its codes in the O columns, then
+//            W_O[j, 0..pad) = dtype(fp32(code) * s_w[j]) and, for up to
+//            OUTL_CODES columns, WqO[j, 0..32) = the codes (zero-padded), as
+//            16-byte stores;
+//   fix-up   one lane segment (8, 16 or 32 lanes) per activation row: the
+//            row's values in the O columns go to X_O (zero-padded to `pad`)
+//            and, for up to OUTL_CODES columns, minus the codes the streaming
+//            pass left there to XqO (the GEMM takes those codes' products back
+//            out, so Xq keeps them); if the largest of those values that is
+//            <= thr reaches the pass-1 absmax, the absmax may sit in an
+//            outlier column: the row is requantised with the exact absmax by
+//            the whole CTA (its outlier codes then 0, its XqO row 0).
+// ---------------------------------------------------------------------------
+// The (o+1)-th outlier column, from the shared bitmap and its word prefixes.
+__device__ __forceinline__ int outlier_col(const uint32_t* sflags, const int32_t* swpre, int NW, int o) {
+  int lo = 0, hi = NW - 1;   // largest w with swpre[w] <= o
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (swpre[mid] <= o) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo * 32 + static_cast<int>(__fns(sflags[lo], 0, o - swpre[lo] + 1));
+}
+
+constexpr int FIN_THREADS = 256;
+constexpr int FIN_WARPS = FIN_THREADS / 32;
+constexpr int FIN_RQ_LIST = 64;   // rows a CTA queues for requantisation by the whole CTA
+
+struct FinishArgs {
+  int64_t M, K;
+  uint32_t thr_bits;
+  const uint32_t* flags;     // [NW]
+  int32_t* O;                // [K]
+  int32_t* count;            // [1]
+  const uint16_t* amax_bits; // [M]
+  float* s_x;                // [M]
+  uint8_t* Q;                // [M,K]
+  uint16_t* X_O;             // [M, ostride]
+  int64_t ostride;
+  int8_t* XqO;               // [M, OUTL_CODES] or nullptr
+  WoGather wo;
+};
+
+template <typename T>
+__global__ void __launch_bounds__(FIN_THREADS) k_outlier_finish(const T* __restrict__ X, const FinishArgs a) {
+  griddep_launch_dependents();   // the GEMM may be scheduled now; it waits for this grid to complete
+  griddep_wait();                // the streaming pass has completed and its writes are visible
+  extern __shared__ uint32_t fsm[];   // sflags[NW], swpre[NW]
+  __shared__ int warp_tot[FIN_WARPS];
+  __shared__ int o_list[OUTL_LIST];
+  __shared__ long long rq_rows[FIN_RQ_LIST];
+  __shared__ int rq_n;
+  __shared__ uint32_t red[FIN_WARPS];
+  const int64_t M = a.M, K = a.K;
+  const int KV = static_cast<int>(K / 8);
+  const int NW = static_cast<int>((K + 31) / 32);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  uint32_t* sflags = fsm;
+  int32_t* swpre = reinterpret_cast<int32_t*>(fsm + NW);
+  constexpr float QMAX = 127.0f;
 
   // ---------------- compaction of the bitmap into shared memory ----------------
-  __shared__ int warp_tot[RQ_WARPS];
-  const int per = (NW + RQ_THREADS - 1) / RQ_THREADS;   // <= 4 (K <= 32768)
+  const int per = (NW + FIN_THREADS - 1) / FIN_THREADS;   // <= 4 (K <= 32768)
   int local = 0;
   for (int u = 0; u < per; ++u) {
     const int w = tid * per + u;
@@ -429,16 +471,13 @@ __global__ void __launch_bounds__(RQ_THREADS, 3) k_prep_rows(const T* __restrict
     if (lane >= o) incl += n;
   }
   if (lane == 31) warp_tot[warp] = incl;
+  if (tid == 0) rq_n = 0;
   __syncthreads();
   int base = 0, cnt = 0;
-  for (int i = 0; i < RQ_WARPS; ++i) {
+  for (int i = 0; i < FIN_WARPS; ++i) {
     if (i < warp) base += warp_tot[i];
     cnt += warp_tot[i];
   }
-  // the ascending list O: in global memory (CTA 0) and, for up to OUTL_LIST
-  // columns, in every CTA's shared memory (lookups then take one load, not
-  // a search over the bitmap)
-  __shared__ int o_list[OUTL_LIST];
   int run = base + incl - local;
   for (int u = 0; u < per; ++u) {
     const int w = tid * per + u;
@@ -463,14 +502,9 @@ __global__ void __launch_bounds__(RQ_THREADS, 3) k_prep_rows(const T* __restrict
   // X_O and W_O are zero-padded to a multiple of 8 columns, and to 16 for up
   // to 16 outlier columns (one K = 16 tensor-core step of the fp part)
   const int pad = cnt <= OUTL_FP_MMA_K ? OUTL_FP_MMA_K : (cnt + 7) & ~7;
+  const bool codes = a.XqO != nullptr && cnt <= OUTL_CODES;
 
-  // ---------------- fix-up: one warp per row ----------------
-  constexpr int RQ_LIST = 32;
-  __shared__ long long rq_rows[RQ_LIST];
-  __shared__ int rq_n;
-  if (tid == 0) rq_n = 0;
-  __syncthreads();
-  // a vector of the row with its outlier columns' entries zeroed
+  // a vector of row xr with its outlier columns' entries zeroed
   auto masked_vec = [&](const T* xr, int64_t idx) -> uint4 {
     uint4 x = ld_nc_v4(reinterpret_cast<const uint4*>(xr) + idx);
     const uint32_t omv = (sflags[idx >> 2] >> ((idx & 3) * 8)) & 0xFFu;
@@ -480,151 +514,209 @@ __global__ void __launch_bounds__(RQ_THREADS, 3) k_prep_rows(const T* __restrict
     x.w &= keep_mask(omv, 3);
     return x;
   };
-  for (int64_t row = static_cast<int64_t>(blockIdx.x) * RQ_WARPS + warp; row < M;
-       row += static_cast<int64_t>(gridDim.x) * RQ_WARPS) {
+  // the CTA requantises a row below (or this thread alone, if its list is full)
+  auto queue_requant = [&](int64_t row) {
+    const int slot = atomicAdd(&rq_n, 1);
+    if (slot < FIN_RQ_LIST) {
+      rq_rows[slot] = row;
+      return;
+    }
     const T* xr = X + row * K;
-    uint32_t mo = 0;   // largest |x| pattern <= threshold among the outlier columns
-    for (int o = lane; o < pad; o += 32) {
-      uint16_t h = 0;
-      if (o < cnt) {
-        const int k = ocol(o);
-        h = reinterpret_cast<const uint16_t*>(xr)[k];
-        const uint32_t ah = h & 0x7FFFu;
-        if (ah <= a.thr_bits) mo = max(mo, ah);
+    uint32_t m = 0;
+    for (int64_t idx = 0; idx < KV; ++idx) m = vec_absmax2<T>(m, masked_vec(xr, idx));
+    const float sc = to_f<T>(static_cast<uint16_t>(pair_max_bits(m))) / QMAX;
+    a.s_x[row] = sc;
+    const float inv = 1.0f / sc;
+    const bool zero = (sc == 0.0f), fast = sc >= 1.17549435e-38f;
+    for (int64_t idx = 0; idx < KV; ++idx) {
+      const uint4 x = ld_nc_v4(reinterpret_cast<const uint4*>(xr) + idx);
+      const uint32_t omv = (sflags[idx >> 2] >> ((idx & 3) * 8)) & 0xFFu;
+      *reinterpret_cast<uint2*>(a.Q + row * K + idx * 8) = quant_vec<T, 0>(x, omv, inv, fast, zero);
+    }
+  };
+
+  // Work of this thread: (1) at most one weight row j of the compact gather
+  // (counts up to OUTL_CODES; rows go to warp w of every CTA before warp w+1
+  // of any, so that the gather spreads over all CTAs); (2) per pass, one
+  // outlier column o of one activation row in a segment of L lanes (counts up
+  // to 32; larger counts loop over the columns). Every independent load is
+  // issued before any of them is used: the kernel is latency-bound.
+  const int64_t wg = static_cast<int64_t>(warp) * gridDim.x + blockIdx.x;
+  const int64_t wstride = static_cast<int64_t>(gridDim.x) * FIN_WARPS;
+  const bool wcompact = a.wo.N > 0 && a.wo.WqO != nullptr && cnt <= OUTL_CODES;
+  const int64_t j = wg * 32 + lane;
+  const bool has_j = wcompact && j < a.wo.N;
+  int8_t wc[OUTL_CODES];   // the weight row's codes in the O columns
+  float sw = 0.0f;
+  if (has_j) {
+    const int8_t* wr = a.wo.Wq + j * K;
+    sw = __ldg(a.wo.s_w + j);
+#pragma unroll
+    for (int o = 0; o < OUTL_CODES; ++o) wc[o] = o < cnt ? __ldg(wr + o_list[o]) : int8_t{0};
+  }
+  // the weight row's stores: WqO[j, 0..32) and W_O[j, 0..pad), 16 bytes at a time
+  auto store_w = [&]() {
+    if (!has_j) return;
+    uint32_t cw[OUTL_CODES / 4];
+#pragma unroll
+    for (int i = 0; i < OUTL_CODES / 4; ++i)
+      cw[i] = static_cast<uint32_t>(static_cast<uint8_t>(wc[4 * i])) |
+              (static_cast<uint32_t>(static_cast<uint8_t>(wc[4 * i + 1])) << 8) |
+              (static_cast<uint32_t>(static_cast<uint8_t>(wc[4 * i + 2])) << 16) |
+              (static_cast<uint32_t>(static_cast<uint8_t>(wc[4 * i + 3])) << 24);
+    uint4* q4 = reinterpret_cast<uint4*>(a.wo.WqO + j * OUTL_CODES);
+    q4[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
+    q4[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
+    uint4* w4 = reinterpret_cast<uint4*>(a.wo.W_O + j * a.ostride);
+#pragma unroll
+    for (int v = 0; v < OUTL_CODES / 8; ++v) {
+      if (v * 8 >= pad) break;
+      uint32_t hw[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int oo = v * 8 + 2 * e;
+        hw[e] = static_cast<uint32_t>(from_f<T>(__fmul_rn(static_cast<float>(wc[oo]), sw))) |
+                (static_cast<uint32_t>(from_f<T>(__fmul_rn(static_cast<float>(wc[oo + 1]), sw))) << 16);
       }
-      a.X_O[row * a.ostride + o] = h;
+      w4[v] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
     }
-    mo = __reduce_max_sync(0xffffffffu, mo);
-    const uint32_t mb = __ldcg(a.amax_bits + row);
-    if (a.XqO != nullptr && cnt <= OUTL_CODES && lane < OUTL_CODES) {
-      // minus the codes pass 1 left in the outlier columns (a requantised row has 0 there)
+  };
+
+  if (a.wo.N > 0 && !wcompact) {   // the element-wise gather (counts above OUTL_CODES)
+    const int64_t total = a.wo.N * pad;
+    for (int64_t t = static_cast<int64_t>(blockIdx.x) * FIN_THREADS + tid; t < total;
+         t += static_cast<int64_t>(gridDim.x) * FIN_THREADS) {
+      const int64_t jj = t / pad;
+      const int oo = static_cast<int>(t - jj * pad);
+      float val = 0.0f;
+      if (oo < cnt) val = __fmul_rn(static_cast<float>(a.wo.Wq[jj * K + ocol(oo)]), __ldg(a.wo.s_w + jj));
+      a.wo.W_O[jj * a.ostride + oo] = from_f<T>(val);
+    }
+  }
+
+  const int L = pad <= 8 ? 8 : pad <= 16 ? 16 : 32;
+  const int rpw = 32 / L;                 // rows per warp and pass
+  const int seg = lane / L, sl = lane - seg * L;
+  if (pad <= 32) {
+    // one column per lane: o = sl (pad <= L)
+    const int o = sl;
+    const int k = o < cnt ? o_list[o] : 0;   // cnt <= 32 <= OUTL_LIST
+    bool first = true;
+    for (int64_t rb = wg * rpw; rb < M; rb += wstride * rpw) {   // warp-uniform
+      const int64_t row = rb + seg;
+      const bool ok = row < M;
+      // loads: the value and the pass-1 code in column O[o], the pass-1 absmax
+      uint16_t h = 0;
       int8_t c = 0;
-      if (lane < cnt && mo < mb) c = static_cast<int8_t>(__ldcg(a.Q + row * K + ocol(lane)));
-      a.XqO[row * OUTL_CODES + lane] = static_cast<int8_t>(-c);   // codes lie in [-127, 127]
-    }
-    if (mo >= mb) {
-      // the pass-1 absmax may sit in an outlier column: requantise exactly,
-      // by the whole CTA below (a row is up to 64 KB: one warp alone would
-      // take tens of microseconds), or by this warp if the list is full
-      int slot = 0;
-      if (lane == 0) slot = atomicAdd(&rq_n, 1);
-      slot = __shfl_sync(0xffffffffu, slot, 0);
-      if (slot < RQ_LIST) {
-        if (lane == 0) rq_rows[slot] = row;
-      } else {
-        uint32_t m = 0;
-        for (int64_t idx = lane; idx < KV; idx += 32) m = vec_absmax2<T>(m, masked_vec(xr, idx));
-        m = __reduce_max_sync(0xffffffffu, pair_max_bits(m));
-        const float s = to_f<T>(static_cast<uint16_t>(m)) / QMAX;
-        if (lane == 0) a.s_f32[row] = s;
-        const float inv = 1.0f / s;
-        const bool zero = (s == 0.0f), fast = s >= 1.17549435e-38f;
-        for (int64_t idx = lane; idx < KV; idx += 32) {
-          const uint4 x = ld_nc_v4(reinterpret_cast<const uint4*>(xr) + idx);
-          const uint32_t omv = (sflags[idx >> 2] >> ((idx & 3) * 8)) & 0xFFu;
-          *reinterpret_cast<uint2*>(a.Q + row * K + idx * 8) = quant_vec<T, CODE>(x, omv, inv, fast, zero);
+      uint32_t mb = 0xFFFFu;
+      if (ok) {
+        mb = __ldcg(a.amax_bits + row);
+        if (o < cnt) {
+          h = __ldg(reinterpret_cast<const uint16_t*>(X + row * K) + k);
+          if (codes) c = static_cast<int8_t>(__ldcg(a.Q + row * K + k));
         }
       }
+      if (first) {   // the weight row's stores, once these loads are in flight
+        first = false;
+        store_w();
+      }
+      const uint32_t ah = h & 0x7FFFu;
+      uint32_t mo = (o < cnt && ah <= a.thr_bits) ? ah : 0u;   // largest |x| <= thr among the O columns
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1)
+        if (off < L) mo = max(mo, __shfl_xor_sync(0xffffffffu, mo, off));
+      const bool requant = ok && mo >= mb;
+      if (ok) {
+        if (o < pad) a.X_O[row * a.ostride + o] = h;
+        if (codes)   // minus the pass-1 codes of the O columns (a requantised row has 0 there)
+          for (int oo = o; oo < OUTL_CODES; oo += L)
+            a.XqO[row * OUTL_CODES + oo] = static_cast<int8_t>(oo == o && !requant ? -c : 0);
+      }
+      if (requant && sl == 0) queue_requant(row);
+    }
+    if (first) store_w();   // this warp had no activation row
+  } else {
+    // more than 32 columns: each lane loops over its columns
+    for (int64_t rb = wg; rb < M; rb += wstride) {   // one row per warp
+      const int64_t row = rb;
+      const T* xr = X + row * K;
+      uint32_t mo = 0;
+      for (int o = lane; o < pad; o += 32) {
+        uint16_t h = 0;
+        if (o < cnt) {
+          h = reinterpret_cast<const uint16_t*>(xr)[ocol(o)];
+          const uint32_t ah = h & 0x7FFFu;
+          if (ah <= a.thr_bits) mo = max(mo, ah);
+        }
+        a.X_O[row * a.ostride + o] = h;
+      }
+      mo = __reduce_max_sync(0xffffffffu, mo);
+      const uint32_t mb = __ldcg(a.amax_bits + row);
+      if (mo >= mb && lane == 0) queue_requant(row);
     }
   }
   __syncthreads();
-  // the CTA's listed rows, each read once into the pass-1 staging area (which
-  // holds at least one row), then reduced and quantised from there
-  const int nrq = min(rq_n, RQ_LIST);
-  for (int i = 0; i < nrq; ++i) {
-    const int64_t row = rq_rows[i];
-    const uint4* xr = reinterpret_cast<const uint4*>(X + row * K);
-    for (int idx = tid; idx < KV; idx += RQ_THREADS) cp_async16(&stage[idx], xr + idx, true);
-    cp_async_commit();
-    cp_async_wait<0>();
-    __syncthreads();
-    uint32_t m = 0;
-    for (int idx = tid; idx < KV; idx += RQ_THREADS) {
-      uint4 x = stage[idx];
-      const uint32_t omv = (sflags[idx >> 2] >> ((idx & 3) * 8)) & 0xFFu;
-      x.x &= keep_mask(omv, 0);
-      x.y &= keep_mask(omv, 1);
-      x.z &= keep_mask(omv, 2);
-      x.w &= keep_mask(omv, 3);
-      m = vec_absmax2<T>(m, x);
-    }
+  // the CTA's listed rows: absmax over the non-outlier columns, then the codes;
+  // rows of up to FIN_THREADS * 8 vectors (K <= 16384) are held in registers
+  // (one read), longer ones are read twice (the second read hits L2)
+  const int nrq = min(rq_n, FIN_RQ_LIST);
+  constexpr int RV = 8;
+  auto block_max = [&](uint32_t m) -> uint32_t {
     m = __reduce_max_sync(0xffffffffu, pair_max_bits(m));
-    if (lane == 0) red[0][warp] = m;
+    if (lane == 0) red[warp] = m;
     __syncthreads();
     m = 0;
 #pragma unroll
-    for (int w = 0; w < RQ_WARPS; ++w) m = max(m, red[0][w]);
-    const float s = to_f<T>(static_cast<uint16_t>(m)) / QMAX;
-    if (tid == 0) a.s_f32[row] = s;
-    const float inv = 1.0f / s;
-    const bool zero = (s == 0.0f), fast = s >= 1.17549435e-38f;
-    for (int idx = tid; idx < KV; idx += RQ_THREADS) {
-      const uint32_t omv = (sflags[idx >> 2] >> ((idx & 3) * 8)) & 0xFFu;
-      *reinterpret_cast<uint2*>(a.Q + row * K + static_cast<int64_t>(idx) * 8) =
-          quant_vec<T, CODE>(stage[idx], omv, inv, fast, zero);
-    }
-    __syncthreads();   // stage and red are reused by the next row
-  }
-
-  // ---------------- outlier weight columns ----------------
-  if (a.wo.N > 0 && a.wo.WqO != nullptr && cnt <= OUTL_CODES) {
-    // one thread per weight row: its codes in the O columns (independent
-    // loads, one round trip), then W_O[j, 0..pad) and WqO[j, 0..32) as
-    // 16-byte stores
-    // rows go to warp w of every CTA before warp w+1 of any, so that the
-    // gather spreads over all CTAs (each finishes its own fix-up first)
-    const int64_t wg = static_cast<int64_t>(warp) * gridDim.x + blockIdx.x;
-    for (int64_t j = wg * 32 + lane; j < a.wo.N; j += static_cast<int64_t>(gridDim.x) * RQ_THREADS) {
-      const int8_t* wr = a.wo.Wq + j * K;
-      const float sw = __ldg(a.wo.s_w + j);
-      int8_t c[OUTL_CODES];
+    for (int w = 0; w < FIN_WARPS; ++w) m = max(m, red[w]);
+    return m;
+  };
+  auto vec_mask = [&](int idx) -> uint32_t { return (sflags[idx >> 2] >> ((idx & 3) * 8)) & 0xFFu; };
+  for (int i = 0; i < nrq; ++i) {
+    const int64_t row = rq_rows[i];
+    const uint4* xr = reinterpret_cast<const uint4*>(X + row * K);
+    uint2* qr = reinterpret_cast<uint2*>(a.Q + row * K);
+    if (KV <= FIN_THREADS * RV) {
+      uint4 v[RV];
+      uint32_t m = 0;
 #pragma unroll
-      for (int o = 0; o < OUTL_CODES; ++o) c[o] = o < cnt ? wr[o_list[o]] : int8_t{0};
-      uint32_t cw[OUTL_CODES / 4];
+      for (int r = 0; r < RV; ++r) {
+        const int idx = tid + r * FIN_THREADS;
+        v[r] = idx < KV ? ld_nc_v4(xr + idx) : make_uint4(0u, 0u, 0u, 0u);
+      }
 #pragma unroll
-      for (int i = 0; i < OUTL_CODES / 4; ++i)
-        cw[i] = static_cast<uint32_t>(static_cast<uint8_t>(c[4 * i])) |
-                (static_cast<uint32_t>(static_cast<uint8_t>(c[4 * i + 1])) << 8) |
-                (static_cast<uint32_t>(static_cast<uint8_t>(c[4 * i + 2])) << 16) |
-                (static_cast<uint32_t>(static_cast<uint8_t>(c[4 * i + 3])) << 24);
-      uint4* q4 = reinterpret_cast<uint4*>(a.wo.WqO + j * OUTL_CODES);
-      q4[0] = make_uint4(cw[0], cw[1], cw[2], cw[3]);
-      q4[1] = make_uint4(cw[4], cw[5], cw[6], cw[7]);
-      uint4* w4 = reinterpret_cast<uint4*>(a.wo.W_O + j * a.ostride);
-#pragma unroll
-      for (int v = 0; v < OUTL_CODES / 8; ++v) {
-        if (v * 8 >= pad) break;
-        uint32_t h[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int o = v * 8 + 2 * e;
-          const uint32_t lo = from_f<T>(__fmul_rn(static_cast<float>(c[o]), sw));
-          const uint32_t hi = from_f<T>(__fmul_rn(static_cast<float>(c[o + 1]), sw));
-          h[e] = lo | (hi << 16);
+      for (int r = 0; r < RV; ++r) {
+        const int idx = tid + r * FIN_THREADS;
+        if (idx < KV) {
+          const uint32_t omv = vec_mask(idx);
+          uint4 x = v[r];
+          x.x &= keep_mask(omv, 0);
+          x.y &= keep_mask(omv, 1);
+          x.z &= keep_mask(omv, 2);
+          x.w &= keep_mask(omv, 3);
+          m = vec_absmax2<T>(m, x);
         }
-        w4[v] = make_uint4(h[0], h[1], h[2], h[3]);
       }
-    }
-  } else if (a.wo.N > 0) {
-    const int64_t total = a.wo.N * pad;
-    for (int64_t t = static_cast<int64_t>(blockIdx.x) * RQ_THREADS + tid; t < total;
-         t += static_cast<int64_t>(gridDim.x) * RQ_THREADS) {
-      const int64_t j = t / pad;
-      const int o = static_cast<int>(t - j * pad);
-      float val = 0.0f;
-      if (o < cnt)
-        val = __fmul_rn(static_cast<float>(a.wo.Wq[j * K + ocol(o)]), __ldg(a.wo.s_w + j));
-      a.wo.W_O[j * a.ostride + o] = from_f<T>(val);
-    }
-    if (a.wo.WqO != nullptr && cnt <= OUTL_CODES) {
-      const int64_t tq = a.wo.N * OUTL_CODES;
-      for (int64_t t = static_cast<int64_t>(blockIdx.x) * RQ_THREADS + tid; t < tq;
-           t += static_cast<int64_t>(gridDim.x) * RQ_THREADS) {
-        const int64_t j = t / OUTL_CODES;
-        const int o = static_cast<int>(t - j * OUTL_CODES);
-        a.wo.WqO[t] = o < cnt ? a.wo.Wq[j * K + ocol(o)] : int8_t{0};
+      m = block_max(m);
+      const float sc = to_f<T>(static_cast<uint16_t>(m)) / QMAX;
+      if (tid == 0) a.s_x[row] = sc;
+      const float inv = 1.0f / sc;
+      const bool zero = (sc == 0.0f), fast = sc >= 1.17549435e-38f;
+#pragma unroll
+      for (int r = 0; r < RV; ++r) {
+        const int idx = tid + r * FIN_THREADS;
+        if (idx < KV) qr[idx] = quant_vec<T, 0>(v[r], vec_mask(idx), inv, fast, zero);
       }
+    } else {
+      uint32_t m = 0;
+      for (int idx = tid; idx < KV; idx += FIN_THREADS) m = vec_absmax2<T>(m, masked_vec(X + row * K, idx));
+      m = block_max(m);
+      const float sc = to_f<T>(static_cast<uint16_t>(m)) / QMAX;
+      if (tid == 0) a.s_x[row] = sc;
+      const float inv = 1.0f / sc;
+      const bool zero = (sc == 0.0f), fast = sc >= 1.17549435e-38f;
+      for (int idx = tid; idx < KV; idx += FIN_THREADS) qr[idx] = quant_vec<T, 0>(ld_nc_v4(xr + idx), vec_mask(idx), inv, fast, zero);
     }
+    __syncthreads();   // red is reused by the next row
   }
 }
 

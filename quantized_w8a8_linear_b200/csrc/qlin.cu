@@ -140,6 +140,7 @@ qlin_status make_tmap_y16(CUtensorMap* m, void* Y, int64_t M, int64_t N) {
 // would leave many SMs idle.
 qlin_status make_tmap_bytes(CUtensorMap* m, const void* base, int64_t rows, int64_t row_bytes, int box_inner,
                             int box_rows, CUtensorMapSwizzle sw, int64_t stride_bytes = 0);
+static_assert(kMaxK == OUTL_MAX_K, "the streaming pass keeps a bitmap of up to kMaxK columns in shared memory");
 static_assert(OUTL_CODES == GEMM_CORR_K, "the prep's compact outlier codes feed the GEMM's correction MMA");
 
 template <int KIND, int EPI, typename TOut, int BN, int STAGES>
@@ -277,9 +278,7 @@ qlin_status launch_gemm(const void* A, const void* B, EpiParams ep, cudaStream_t
 template <typename T, int V, int CODE, bool SBF16, bool OUTL>
 qlin_status launch_prep_v(const void* X, const PrepArgs& a, int sms, cudaStream_t st) {
   auto kern = k_prep_rows<T, V, CODE, SBF16, OUTL>;
-  const int NW = static_cast<int>((a.K + 31) / 32);
-  const size_t smem = ((OUTL ? static_cast<size_t>(8 * NW) : 0) + 15) / 16 * 16 +
-                      static_cast<size_t>(PF_DEPTH) * V * RQ_THREADS * 16;
+  const size_t smem = static_cast<size_t>(PF_DEPTH) * V * RQ_THREADS * 16;
   static std::atomic<bool> attr_set[16] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -303,9 +302,11 @@ qlin_status launch_prep_v(const void* X, const PrepArgs& a, int sms, cudaStream_
   cfg.blockDim = dim3(RQ_THREADS);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
+  // LLM.int8: a programmatic dependent of k_ws_reset, which zeroes the row
+  // counter and the bitmap this pass uses (it waits for it before using them)
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;   // the grid barrier needs every CTA resident
-  attr[0].val.cooperative = OUTL ? 1 : 0;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = OUTL ? 1 : 0;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return check_cuda(cudaLaunchKernelEx(&cfg, kern, static_cast<const T*>(X), a), "k_prep_rows launch");
@@ -360,9 +361,8 @@ qlin_status launch_rowquant(const void* X, int64_t rows, int64_t K, uint8_t* Q, 
 
 // ---- LLM.int8 workspace layout -----------------------------------------------
 struct Int8Ws {
-  uint32_t* sync;     // [1]  grid barrier counter of the prep kernel
+  uint32_t* hdr;      // the per-call header, zeroed by k_ws_reset: count, flags, sk_count
   int32_t* count;     // [1]
-  uint32_t* rowctr;   // [1]  next-row counter of the prep kernel
   uint32_t* flags;    // [NW]
   int32_t* O;         // [K]
   float* s_x;         // [M]
@@ -376,7 +376,7 @@ struct Int8Ws {
   int32_t* sk_part;   // [sk_ctas * 2][128 * 256] stream-K partial accumulators
   int sk_ctas;        // CTAs the partial slots serve
   int64_t ostride;
-  size_t memset_bytes;  // zeroed each call: sync, count, rowctr, flags, sk_count
+  int64_t hdr_words;  // 32-bit words of the header
   size_t total;
 };
 
@@ -401,13 +401,13 @@ Int8Ws int8_layout(void* base, int64_t M, int64_t N, int64_t K, bool with_gemm_p
   };
   const int64_t NW = (K + 31) / 32;
   const int64_t nctr = with_gemm_parts && with_sk ? GEMM_EPI_GROUPS * sk_tiles(M, N) : 0;
+  // header: [reserved, count, reserved, reserved], flags [NW], sk_count [nctr]
   uint8_t* hdr = take(16 + 4 * NW + 4 * nctr);
-  w.sync = reinterpret_cast<uint32_t*>(hdr);
+  w.hdr = reinterpret_cast<uint32_t*>(hdr);
   w.count = reinterpret_cast<int32_t*>(hdr ? hdr + 4 : nullptr);
-  w.rowctr = reinterpret_cast<uint32_t*>(hdr ? hdr + 8 : nullptr);
   w.flags = reinterpret_cast<uint32_t*>(hdr ? hdr + 16 : nullptr);
   w.sk_count = reinterpret_cast<int32_t*>(hdr && nctr > 0 ? hdr + 16 + 4 * NW : nullptr);
-  w.memset_bytes = static_cast<size_t>(16 + 4 * NW + 4 * nctr);
+  w.hdr_words = 4 + NW + nctr;
   w.O = reinterpret_cast<int32_t*>(take(4 * K));
   w.ostride = round_up(K, 8);
   w.amax = reinterpret_cast<uint16_t*>(take(2 * M));
@@ -429,21 +429,54 @@ Int8Ws int8_layout(void* base, int64_t M, int64_t N, int64_t K, bool with_gemm_p
 
 bool decomposition_on(float thr) { return thr > 0.0f && !std::isinf(thr); }
 
+// The finishing kernel of the LLM.int8 prepare stage (a programmatic
+// dependent of the streaming pass).
+template <typename T>
+qlin_status launch_finish(const void* X, const FinishArgs& f, int sms, cudaStream_t st) {
+  const int64_t NW = (f.K + 31) / 32;
+  cudaLaunchConfig_t cfg{};
+  // one wave (two CTAs per SM): the kernel is a few dependent round trips long
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * sms));
+  cfg.blockDim = dim3(FIN_THREADS);
+  cfg.dynamicSmemBytes = static_cast<size_t>(8 * NW);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return check_cuda(cudaLaunchKernelEx(&cfg, k_outlier_finish<T>, static_cast<const T*>(X), f),
+                    "k_outlier_finish launch");
+}
+
+// The LLM.int8 prepare stage: k_ws_reset (zeroed header), the streaming pass
+// (codes, scales, outlier bitmap) and, with the decomposition on,
+// k_outlier_finish (outlier list, X_O, XqO, requantised rows, W_O, WqO); each
+// a programmatic dependent of the one before.
 template <typename T>
 qlin_status int8_prep_impl(const void* X, int64_t M, int64_t K, float thr, const Int8Ws& w, int8_t* Xq, float* s_x,
                            uint16_t* X_O, int64_t ostride, cudaStream_t st,
                            WoGather wo = WoGather{nullptr, nullptr, 0, nullptr, nullptr, nullptr}) {
-  qlin_status s = check_cuda(cudaMemsetAsync(w.sync, 0, w.memset_bytes, st), "cudaMemsetAsync");
+  DeviceInfo* d;
+  qlin_status s = device_info(&d);
+  if (s != QLIN_OK) return s;
+  const int64_t rgrid = std::min<int64_t>(16, (w.hdr_words + 255) / 256);
+  k_ws_reset<<<static_cast<unsigned>(rgrid), 256, 0, st>>>(w.hdr, w.hdr_words);
+  s = check_cuda(cudaGetLastError(), "k_ws_reset launch");
   if (s != QLIN_OK) return s;
   if (M == 0) return QLIN_OK;
   if (decomposition_on(thr)) {
     PrepArgs a{};
     a.M = M; a.K = K; a.thr = thr; a.thr_bits = threshold_bits<T>(thr);
     a.Q = reinterpret_cast<uint8_t*>(Xq); a.s_f32 = s_x; a.amax_bits = w.amax;
-    a.flags = w.flags; a.O = w.O; a.count = w.count; a.sync = w.sync; a.X_O = X_O;
-    a.rowctr = M < (int64_t{1} << 31) ? w.rowctr : nullptr;
-    a.XqO = w.XqO; a.ostride = ostride; a.wo = wo;
-    return launch_prep<T, 0, false, true>(X, a, st);
+    a.flags = w.flags;
+    s = launch_prep<T, 0, false, true>(X, a, st);
+    if (s != QLIN_OK) return s;
+    FinishArgs f{};
+    f.M = M; f.K = K; f.thr_bits = a.thr_bits; f.flags = w.flags; f.O = w.O; f.count = w.count;
+    f.amax_bits = w.amax; f.s_x = s_x; f.Q = reinterpret_cast<uint8_t*>(Xq); f.X_O = X_O; f.ostride = ostride;
+    f.XqO = w.XqO; f.wo = wo;
+    return launch_finish<T>(X, f, d->sms, st);
   }
   return launch_rowquant<T, 0, false>(X, M, K, reinterpret_cast<uint8_t*>(Xq), s_x, nullptr, st);
 }
