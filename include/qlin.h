@@ -193,6 +193,32 @@ QLIN_API qlin_status qlin_w4a8_gemm(qlin_dtype xdt, int64_t M, int64_t K, const 
                            const float *s_x, const uint8_t *Wq4, const float *w_scale,
                            int64_t N, const void *bias, void *Y, void *stream);
 
+/* Unquantised 16-bit linear, for the layers a model keeps in floating point
+ * (Image21-Turbo-OrbitQuant-W4A4 page, "What 4-bit breaks here and what stays
+ * in fp16": the projections that write or cancel the massive activations stay
+ * in fp16 while the rest are quantised):
+ *   Y = dtype(X W^T + bias), X [M,K], W [N,K], bias [N] and Y [M,N] all in
+ *   xdt (QLIN_F16 or QLIN_BF16); products exact, fp32 accumulation in the
+ *   tensor cores (tcgen05 kind::f16), one rounding to xdt at the end.
+ * No workspace. Same shape and alignment rules as the other forwards. */
+QLIN_API qlin_status qlin_fp_linear_forward(const void *X, qlin_dtype xdt, int64_t M, int64_t K, const void *W,
+                                   int64_t N, const void *bias, void *Y, void *stream);
+
+/* Weight-only FP8 linear (Qwen-Image-2.1-Text-Encoder-FP8 page, "Format": the
+ * E4M3 weights and their bf16 [out,1] scales are consumed as
+ * weight.to(bf16) * weight_scale, the activations are not quantised):
+ *   W_deq[j,k] = bf16(decode(Wq[j,k]) * w_scale[j])  (one rounding: the fp32
+ *                product of the 4-bit and 8-bit significands is exact)
+ *   Y = bf16(X W_deq^T + bias), fp32 accumulation (tcgen05 kind::f16).
+ * W_deq is formed tile by tile in shared memory and never written out.
+ * X, bias and Y are bf16 (xdt must be QLIN_BF16: the tensor core multiplies
+ * operands of one type, and the rule dequantises to bf16; QLIN_ERR_UNSUPPORTED
+ * otherwise). Wq e4m3 [N,K] and w_scale bf16 [N] as qlin_quantize_weight
+ * (QLIN_W_FP8_CHANNEL) writes them. No workspace. */
+QLIN_API qlin_status qlin_fp8_weight_only_forward(const void *X, qlin_dtype xdt, int64_t M, int64_t K,
+                                         const uint8_t *Wq, const void *w_scale, int64_t N,
+                                         const void *bias, void *Y, void *stream);
+
 /* ---------------- parity exports: the same kernels, intermediates written out ------ */
 
 /* LLM.int8 activation prep alone. Outputs: Xq int8 [M,K]; s_x fp32 [M];

@@ -58,6 +58,8 @@ def _load() -> ctypes.CDLL:
         "qlin_int8_outlier_gemm_i32": (st, [i64, i64, P, i64, P, P, sz, P]),
         "qlin_fp8_gemm": (st, [i32, i64, i64, P, P, P, P, i32, i64, P, P, P, P]),
         "qlin_w4a8_forward": (st, [P, i32, i64, i64, P, P, i64, P, P, P, sz, P]),
+        "qlin_fp_linear_forward": (st, [P, i32, i64, i64, P, i64, P, P, P]),
+        "qlin_fp8_weight_only_forward": (st, [P, i32, i64, i64, P, P, i64, P, P, P]),
         "qlin_w4a8_gemm": (st, [i32, i64, i64, P, P, P, P, i64, P, P, P]),
         "qlin_w4a8_prep": (st, [P, i32, i64, i64, P, P, P]),
         "qlin_w4a8_group_i32": (st, [P, P, i64, i64, i64, i32, P, P]),
@@ -276,6 +278,32 @@ def qlin_w4a8_forward(X: torch.Tensor, Wq4: torch.Tensor, w_scale: torch.Tensor,
         ws = workspace(QLIN_OP_W4A8, M, N, K, X.device)
     _check(lib.qlin_w4a8_forward(_ptr(X), _dt(X), M, K, _ptr(Wq4), _ptr(w_scale), N, _ptr(bias), _ptr(Y),
                                  _ptr(ws), ws.numel(), _stream(X.device)))
+    return Y
+
+
+def qlin_fp_linear_forward(X: torch.Tensor, W: torch.Tensor, bias: Optional[torch.Tensor] = None,
+                           Y: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Unquantised 16-bit linear Y = X W^T + bias (X, W, bias in one dtype), tcgen05 kind::f16."""
+    M, K = X.shape
+    N = W.shape[0]
+    if W.dtype != X.dtype or (bias is not None and bias.dtype != X.dtype):
+        raise TypeError("X, W and bias must share one 16-bit dtype")
+    if Y is None:
+        Y = torch.empty((M, N), dtype=X.dtype, device=X.device)
+    _check(lib.qlin_fp_linear_forward(_ptr(X), _dt(X), M, K, _ptr(W), N, _ptr(bias), _ptr(Y), _stream(X.device)))
+    return Y
+
+
+def qlin_fp8_weight_only_forward(X: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tensor,
+                                 bias: Optional[torch.Tensor] = None,
+                                 Y: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Weight-only FP8 linear: Y = X (bf16(decode(Wq) * w_scale))^T + bias, bf16 activations."""
+    M, K = X.shape
+    N = Wq.shape[0]
+    if Y is None:
+        Y = torch.empty((M, N), dtype=X.dtype, device=X.device)
+    _check(lib.qlin_fp8_weight_only_forward(_ptr(X), _dt(X), M, K, _ptr(Wq), _ptr(w_scale), N, _ptr(bias), _ptr(Y),
+                                            _stream(X.device)))
     return Y
 
 

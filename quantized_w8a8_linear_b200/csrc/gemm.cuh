@@ -1,7 +1,10 @@
 // gemm.cuh -- persistent, warp-specialised tcgen05 GEMM for sm_100a.
 //
 //   C[M,N] = A[M,K] B[N,K]^T, A and B 8-bit (int8 -> int32 with kind::i8, or
-//   E4M3 -> fp32 with kind::f8f6f4), both K-major in global memory.
+//   E4M3 -> fp32 with kind::f8f6f4) or 16-bit (bf16 or fp16 -> fp32 with
+//   kind::f16), both K-major in global memory. Tiles are addressed in bytes:
+//   a stage holds 128 bytes of K (128 8-bit or 64 16-bit elements), and every
+//   MMA takes 32 bytes of K, so the pipeline is the same for all three kinds.
 //
 // Roles (one CTA per SM, 20 warps = 5 warpgroups; the last gives most of its
 // registers to the first four with setmaxnreg):
@@ -37,7 +40,9 @@ namespace qlin {
 
 // EPI_INT8_OUTLIER_I32: the int32 accumulator of the LLM.int8 path after the
 // outlier-column correction, written out (parity export of the same kernel).
-enum EpiKind { EPI_I32 = 0, EPI_INT8_OUTLIER = 1, EPI_FP8_TENSOR = 2, EPI_FP8_ROWCOL = 3, EPI_INT8_OUTLIER_I32 = 4 };
+// EPI_F16: Y = dtype(acc + bias), the unquantised 16-bit linear (kind::f16).
+enum EpiKind { EPI_I32 = 0, EPI_INT8_OUTLIER = 1, EPI_FP8_TENSOR = 2, EPI_FP8_ROWCOL = 3, EPI_INT8_OUTLIER_I32 = 4,
+               EPI_F16 = 5 };
 
 constexpr int GEMM_BM = 128;
 constexpr int GEMM_BK = 128;                 // bytes (= elements) per stage along K
@@ -80,7 +85,7 @@ constexpr int GEMM_EPI_KB = 26;
 constexpr int GEMM_GROUP_M = 16;
 
 struct EpiParams {
-  int64_t M, N, K;
+  int64_t M, N, K;            // K: bytes of a row of A and of B (elements for 8-bit operands)
   void* Y;                    // [M,N]: int32 (EPI_I32, EPI_INT8_OUTLIER_I32) or 16-bit output dtype
   const float* s_x;           // [M] per-token scale
   const float* s_w;           // [N] fp32 per-channel weight scale
@@ -327,7 +332,7 @@ __device__ __forceinline__ void epi_stage(const EpiParams& p, EpiStage<BN>& es, 
     if (mine && n < p.N) {
       if constexpr (EPI == EPI_INT8_OUTLIER) sw[i] = __ldg(p.s_w + n);
       if constexpr (EPI == EPI_FP8_ROWCOL) sw[i] = to_f<__nv_bfloat16>(__ldg(p.s_w_bf16 + n));
-      if constexpr (EPI == EPI_INT8_OUTLIER || EPI == EPI_FP8_TENSOR || EPI == EPI_FP8_ROWCOL)
+      if constexpr (EPI == EPI_INT8_OUTLIER || EPI == EPI_FP8_TENSOR || EPI == EPI_FP8_ROWCOL || EPI == EPI_F16)
         if (p.bias != nullptr) b[i] = to_f<TOut>(__ldg(p.bias + n));
       if constexpr (OUTL) {
         if (cn > 0) {
@@ -434,7 +439,7 @@ __device__ __forceinline__ void epi_chunk(const EpiParams& p, const EpiStage<BN>
       const float4 sbv = es.sb[(c * GEMM_CW + j) >> 1];   // {scale j, scale j+1, bias j, bias j+1}
       const unsigned long long b2 = f32x2_of(__float_as_uint(sbv.z), __float_as_uint(sbv.w));
       unsigned long long v;
-      if constexpr (EPI == EPI_FP8_TENSOR) {
+      if constexpr (EPI == EPI_FP8_TENSOR || EPI == EPI_F16) {   // alpha = 1 for EPI_F16: fma(acc, 1, b) = acc + b
         v = fma_f32x2(f32x2_of(r[j], r[j + 1]), f32x2_of(__float_as_uint(alpha), __float_as_uint(alpha)), b2);
       } else {
         // acc * (s_x * s_w) + bias, as fmaf(acc, s_x * s_w, bias) per column
@@ -726,7 +731,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   } else if (warp == GEMM_WARP_MMA) {
     if (lane == 0) {
       // ---------------- MMA issuer ----------------
-      constexpr uint32_t idesc = KIND == 0 ? idesc_i8(GEMM_BM, BN) : idesc_e4m3(GEMM_BM, BN);
+      constexpr uint32_t idesc = KIND == 0   ? idesc_i8(GEMM_BM, BN)
+                                 : KIND == 1 ? idesc_e4m3(GEMM_BM, BN)
+                                             : idesc_f16(GEMM_BM, BN, std::is_same<TOut, __nv_bfloat16>::value);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -789,6 +796,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
     float alpha = 0.0f;
     if constexpr (EPI == EPI_INT8_OUTLIER || EPI == EPI_INT8_OUTLIER_I32) cnt = *p.count;
     if constexpr (EPI == EPI_FP8_TENSOR) alpha = __ldg(p.x_scale) * __ldg(p.w_scale);
+    if constexpr (EPI == EPI_F16) alpha = 1.0f;
     const int cn = cnt == 0 ? 0 : cnt <= 2 ? 2 : cnt <= 4 ? 4 : cnt <= 8 ? 8 : cnt <= GEMM_OUTL_STAGED ? 16 : -1;
     int acc = 0;
     uint32_t acc_phase = 0;

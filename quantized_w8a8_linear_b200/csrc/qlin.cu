@@ -20,6 +20,7 @@
 #include "common.cuh"
 #include "gemm.cuh"
 #include "gemm_w4a8.cuh"
+#include "gemm_wo8.cuh"
 #include "prep.cuh"
 
 using namespace qlin;
@@ -907,6 +908,24 @@ qlin_status qlin_fp8_forward(const void* X, qlin_dtype xdt, int64_t M, int64_t K
   return qlin_fp8_gemm(xdt, M, K, Xq, s_x, Wq, w_scale, wmode, N, x_scale, bias, Y, stream);
 }
 
+// Unquantised 16-bit linear: the tcgen05 GEMM with kind::f16 operands (the
+// tiles hold 64 elements of K, 128 bytes, per stage) and a bias epilogue.
+qlin_status qlin_fp_linear_forward(const void* X, qlin_dtype xdt, int64_t M, int64_t K, const void* W, int64_t N,
+                                   const void* bias, void* Y, void* stream) {
+  QLIN_TRY(check_common(X, xdt, M, K, N));
+  if (M == 0 || N == 0) return ok();
+  QLIN_REQ_PTR(W, "W");
+  QLIN_REQ_PTR(Y, "Y");
+  if (bias != nullptr && !aligned16(bias)) return fail(QLIN_ERR_ALIGNMENT, "bias is not 16-byte aligned");
+  EpiParams ep{};
+  ep.M = M; ep.N = N; ep.K = 2 * K; ep.Y = Y;
+  ep.bias = static_cast<const uint16_t*>(bias);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (xdt == QLIN_BF16) QLIN_TRY((launch_gemm<2, EPI_F16, __nv_bfloat16>(X, W, ep, st, 8)));
+  else QLIN_TRY((launch_gemm<2, EPI_F16, __half>(X, W, ep, st, 9)));
+  return ok();
+}
+
 }  // extern "C"
 
 // ---------------------------------------------------------------------------
@@ -1042,6 +1061,54 @@ qlin_status qlin_w4a8_forward(const void* X, qlin_dtype xdt, int64_t M, int64_t 
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Weight-only FP8
+// ---------------------------------------------------------------------------
+namespace {
+
+qlin_status launch_wo8(const void* X, const uint8_t* Wq, const Wo8Params& wp, cudaStream_t st) {
+  DeviceInfo* d;
+  qlin_status s = device_info(&d);
+  if (s != QLIN_OK) return s;
+  CUtensorMap ta, tb;
+  if ((s = make_tmap_k128(&ta, X, wp.M, 2 * wp.K, WO8_BM)) != QLIN_OK) return s;
+  if ((s = make_tmap_bytes(&tb, Wq, wp.N, wp.K, WO8_BK, WO8_BN, CU_TENSOR_MAP_SWIZZLE_NONE)) != QLIN_OK) return s;
+  static std::atomic<bool> attr_set[16] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 16 && !attr_set[dev].load(std::memory_order_acquire)) {
+    s = check_cuda(cudaFuncSetAttribute(k_gemm_wo8, cudaFuncAttributeMaxDynamicSharedMemorySize, Wo8Smem::TOTAL),
+                   "cudaFuncSetAttribute");
+    if (s != QLIN_OK) return s;
+    attr_set[dev].store(true, std::memory_order_release);
+  }
+  const int64_t tiles = ((wp.M + WO8_BM - 1) / WO8_BM) * ((wp.N + WO8_BN - 1) / WO8_BN);
+  const int grid = static_cast<int>(tiles < d->sms ? tiles : d->sms);
+  k_gemm_wo8<<<grid, WO8_THREADS, Wo8Smem::TOTAL, st>>>(ta, tb, wp);
+  return check_cuda(cudaGetLastError(), "k_gemm_wo8 launch");
+}
+
+}  // namespace
+
+extern "C" qlin_status qlin_fp8_weight_only_forward(const void* X, qlin_dtype xdt, int64_t M, int64_t K,
+                                                    const uint8_t* Wq, const void* w_scale, int64_t N,
+                                                    const void* bias, void* Y, void* stream) {
+  QLIN_TRY(check_common(X, xdt, M, K, N));
+  if (xdt != QLIN_BF16)
+    return fail(QLIN_ERR_UNSUPPORTED, "weight-only FP8 takes bf16 activations (the weight dequantises to bf16)");
+  if (M == 0 || N == 0) return ok();
+  QLIN_REQ_PTR(Wq, "Wq");
+  QLIN_REQ_PTR(w_scale, "w_scale");
+  QLIN_REQ_PTR(Y, "Y");
+  if (bias != nullptr && !aligned16(bias)) return fail(QLIN_ERR_ALIGNMENT, "bias is not 16-byte aligned");
+  Wo8Params wp{};
+  wp.M = M; wp.N = N; wp.K = K; wp.Y = Y;
+  wp.s_w = static_cast<const uint16_t*>(w_scale);
+  wp.bias = static_cast<const uint16_t*>(bias);
+  QLIN_TRY(launch_wo8(X, Wq, wp, static_cast<cudaStream_t>(stream)));
+  return ok();
+}
 
 
 // ---------------------------------------------------------------------------
