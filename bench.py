@@ -185,6 +185,12 @@ class LinearRun:
             self.Xq = torch.empty((M, K), dtype=torch.int8, device=device)
             self.s_x = torch.empty((M,), dtype=torch.float32, device=device)
             self.prep_bytes = 3.0 * M * K
+        elif self.mode == "fp8_weight_only":
+            self.Wq, self.s_w = q.qlin_quantize_weight(Wd, q.QLIN_W_FP8_CHANNEL)
+            self.prep_bytes = 0.0
+        elif self.mode == "fp_linear":
+            self.Wq, self.s_w = Wd.clone(), None
+            self.prep_bytes = 0.0
         else:
             wmode = q.QLIN_W_FP8_TENSOR if self.mode == "fp8_static" else q.QLIN_W_FP8_CHANNEL
             self.wmode = wmode
@@ -199,6 +205,8 @@ class LinearRun:
 
     def prepare(self):
         q = self.q
+        if self.mode in ("fp8_weight_only", "fp_linear"):
+            return   # one kernel: the activations are not quantised
         if self.mode == "int8_outlier":
             q.qlin_int8_outlier_prepare(self.X, self.Wq, self.s_w, 6.0, self.ws)
         elif self.mode == "w4a8":
@@ -209,6 +217,12 @@ class LinearRun:
 
     def gemm(self):
         q = self.q
+        if self.mode == "fp8_weight_only":
+            q.qlin_fp8_weight_only_forward(self.X, self.Wq, self.s_w, Y=self.Y)
+            return
+        if self.mode == "fp_linear":
+            q.qlin_fp_linear_forward(self.X, self.Wq, Y=self.Y)
+            return
         if self.mode == "int8_outlier":
             q.qlin_int8_outlier_gemm(self.dtype, self.M, self.K, self.Wq, self.s_w, self.Y, self.ws)
         elif self.mode == "w4a8":
@@ -229,11 +243,19 @@ class LinearRun:
             q.qlin_int8_outlier_forward(self.X, self.Wq, self.s_w, 6.0, Y=self.Y, ws=self.ws)
         elif self.mode == "w4a8":
             q.qlin_w4a8_forward(self.X, self.Wq, self.s_w, Y=self.Y)
+        elif self.mode in ("fp8_weight_only", "fp_linear"):
+            self.gemm()
         else:
             q.qlin_fp8_forward(self.X, self.Wq, self.s_w, self.wmode, x_scale=self.x_scale, Y=self.Y)
 
-    # kernels of ours launched per forward: the prep kernel and the GEMM
+    # kernels of ours launched per forward: LLM.int8 reset, streaming pass,
+    # finishing kernel and GEMM; the FP8 and W4A8 forwards a prep kernel and
+    # the GEMM; the weight-only FP8 and 16-bit linears one GEMM
     def launches(self):
+        if self.mode == "int8_outlier":
+            return 4
+        if self.mode in ("fp8_weight_only", "fp_linear"):
+            return 1
         return 2
 
 
@@ -545,18 +567,23 @@ def main():
     # -------- secondary workloads (FP8, 2048^2 DiT block), rank-local, reported beside --------
     secondary = {}
     if not args.no_secondary:
-        for name in ("dit1024_fp8_static_qkv", "te_fp8_dynamic_mlp", "dit2048_block_int8", "dit2048_block_w4a8"):
+        for name in ("dit1024_fp8_static_qkv", "te_fp8_dynamic_mlp", "dit2048_block_int8", "dit2048_block_w4a8",
+                     "te_fp8_weight_only_mlp", "dit1024_bf16_mlp"):
             w2 = workloads.get_workload(name)
             r2 = [LinearRun(q, w2, lin, i, device) for i, lin in enumerate(w2.linears)]
             steps2 = max(20, args.steps // 5)
             p2, g2 = time_steps(r2, steps2, 3, flush)
             ops2 = sum(r.ops for r in r2)
             tot2 = sum(p2) + sum(g2)
+            # the 16-bit contractions (kind::f16) against the bf16 peak, the rest against int8/fp8
+            pk = float(peaks["bf16_tflops"]) if w2.mode in ("fp8_weight_only", "fp_linear") else peak_tops
             secondary[name] = {"TOPS": steps2 * ops2 / (tot2 * 1e-3) / 1e12,
                                "gemm_TOPS": steps2 * ops2 / (sum(g2) * 1e-3) / 1e12,
-                               "gemm_frac_of_peak": steps2 * ops2 / (sum(g2) * 1e-3) / 1e12 / peak_tops,
+                               "gemm_frac_of_peak": steps2 * ops2 / (sum(g2) * 1e-3) / 1e12 / pk,
+                               "peak_TOPS": pk,
                                "ms_per_step": tot2 / steps2,
-                               "prep_GBps": steps2 * sum(r.prep_bytes for r in r2) / (sum(p2) * 1e-3) / 1e9,
+                               "prep_GBps": (steps2 * sum(r.prep_bytes for r in r2) / (sum(p2) * 1e-3) / 1e9
+                                             if sum(p2) > 0 else None),
                                "gemm_TOPS_per_linear": {r.lin.name: steps2 * r.ops / (g * 1e-3) / 1e12
                                                         for r, g in zip(r2, g2)}}
             blocks = w2.extra.get("blocks") if w2.extra else None

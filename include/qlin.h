@@ -314,6 +314,17 @@ QLIN_API qlin_status qlin_get_device_status(int32_t *status, int reset);
  * 2e9). Synchronous; call it outside stream capture. */
 QLIN_API qlin_status qlin_set_wait_timeout_ns(uint64_t ns);
 
+/* Test switch of the failure path (the model-card pages have no counterpart):
+ * with on != 0, every later launch of the int8 / FP8 / 16-bit GEMM first waits
+ * on a barrier that nothing arrives on, so that its bounded wait runs out
+ * after the wait limit (qlin_set_wait_timeout_ns). The kernel then records
+ * QLIN_ERR_TIMEOUT in the device status word, stops its other roles, waits
+ * (up to max(limit, 1 s)) for its own copies and MMAs in flight, frees its
+ * TMEM and returns, leaving Y unwritten; later launches work normally once the
+ * switch is off again. Off by default. Synchronous; call it outside stream
+ * capture. */
+QLIN_API qlin_status qlin_debug_inject_wait_timeout(int on);
+
 /* Work schedule of the LLM.int8 GEMMs (qlin_int8_outlier_forward / _gemm /
  * _gemm_i32), process-wide, read at each launch:
  *   0  automatic (default): whole output tiles handed out round-robin, or

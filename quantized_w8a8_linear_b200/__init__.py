@@ -71,6 +71,7 @@ def _load() -> ctypes.CDLL:
         "qlin_get_device_status": (st, [P, i32]),
         "qlin_set_wait_timeout_ns": (st, [ctypes.c_uint64]),
         "qlin_set_gemm_schedule": (st, [ctypes.c_int]),
+        "qlin_debug_inject_wait_timeout": (st, [ctypes.c_int]),
         "qlin_last_error_string": (ctypes.c_char_p, []),
         "qlin_version": (i32, []),
     }
@@ -405,6 +406,11 @@ def qlin_get_device_status(reset: bool = False) -> int:
 
 def qlin_set_wait_timeout_ns(ns: int) -> None:
     _check(lib.qlin_set_wait_timeout_ns(int(ns)))
+
+
+def qlin_debug_inject_wait_timeout(on: bool) -> None:
+    """Test switch: later GEMM launches wait once on a barrier nothing arrives on (bounded)."""
+    _check(lib.qlin_debug_inject_wait_timeout(1 if on else 0))
 
 
 def qlin_set_gemm_schedule(mode: int) -> None:

@@ -20,11 +20,24 @@ namespace qlin {
 // ---------------------------------------------------------------------------
 __device__ int g_status = 0;
 __device__ unsigned long long g_wait_timeout_ns = 2000000000ull;
+// Test switch of the abort path (off unless qlin_debug_inject_wait_timeout
+// sets it): the GEMM's MMA warp first waits on a barrier that nothing
+// arrives on, so that its bounded wait runs out.
+__device__ int g_inject_wait_timeout = 0;
 
 __device__ __forceinline__ uint64_t globaltimer() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
+}
+
+// Limit of the waits an aborting CTA makes for its own hardware operations
+// in flight (TMA copies into its shared memory, MMAs into its TMEM) before it
+// frees TMEM and exits: those complete on their own, so the limit is the
+// larger of the wait limit and one second, however short the wait limit is.
+__device__ __forceinline__ uint64_t drain_limit_ns() {
+  const uint64_t l = g_wait_timeout_ns;
+  return l > 1000000000ull ? l : 1000000000ull;
 }
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

@@ -723,7 +723,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
           if (issued & (1u << stage)) {
             const uint32_t a = smem_u32(&full_bar[stage]);
             const uint64_t t0 = globaltimer();
-            while (!mbar_try_wait(a, phase) && globaltimer() - t0 < g_wait_timeout_ns) {}
+            while (!mbar_try_wait(a, phase) && globaltimer() - t0 < drain_limit_ns()) {}
           }
         }
       }
@@ -739,6 +739,9 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       int acc = 0;
       uint32_t acc_phase = 0;
       bool ok = true;
+      // test of the abort path (qlin_debug_inject_wait_timeout): nothing has
+      // committed to the drain barrier yet, so this bounded wait runs out
+      if (g_inject_wait_timeout != 0) ok = mbar_wait(drain_bar, 0u, abort_flag);
       SegIter its(sk, num_tiles, p.sk_dp_tiles, num_kb);
       Seg sg;
       while (ok && its.next(sg)) {
@@ -781,7 +784,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
       umma_commit(drain_bar);
       const uint32_t a = smem_u32(drain_bar);
       const uint64_t t0 = globaltimer();
-      while (!mbar_try_wait(a, 0) && globaltimer() - t0 < g_wait_timeout_ns) {}
+      while (!mbar_try_wait(a, 0) && globaltimer() - t0 < drain_limit_ns()) {}
     }
   }
   } else {

@@ -167,7 +167,7 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
           if (issued & (1u << stage)) {
             const uint32_t a = smem_u32(&full_bar[stage]);
             const uint64_t t0 = globaltimer();
-            while (!mbar_try_wait(a, phase) && globaltimer() - t0 < g_wait_timeout_ns) {}
+            while (!mbar_try_wait(a, phase) && globaltimer() - t0 < drain_limit_ns()) {}
           }
         }
       }
@@ -200,7 +200,7 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
       umma_commit(drain_bar);
       const uint32_t a = smem_u32(drain_bar);
       const uint64_t t0 = globaltimer();
-      while (!mbar_try_wait(a, 0) && globaltimer() - t0 < g_wait_timeout_ns) {}
+      while (!mbar_try_wait(a, 0) && globaltimer() - t0 < drain_limit_ns()) {}
     }
   } else if (warp == 2 || warp == 3 || warp == 12 || warp == 13) {
     // ---------------- converters: packed int4 -> swizzled int8 ----------------

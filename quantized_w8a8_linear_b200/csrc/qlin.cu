@@ -570,6 +570,12 @@ qlin_status qlin_get_device_status(int32_t* status, int reset) {
   return ok();
 }
 
+qlin_status qlin_debug_inject_wait_timeout(int on) {
+  const int v = on ? 1 : 0;
+  QLIN_TRY(check_cuda(cudaMemcpyToSymbol(qlin::g_inject_wait_timeout, &v, sizeof(v)), "cudaMemcpyToSymbol"));
+  return ok();
+}
+
 qlin_status qlin_set_gemm_schedule(int mode) {
   if (mode < 0 || mode > 2) return fail(QLIN_ERR_INVALID_ARG, "schedule mode must be 0, 1 or 2 (got %d)", mode);
   g_gemm_schedule.store(mode, std::memory_order_relaxed);

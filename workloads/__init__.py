@@ -45,7 +45,7 @@ class Linear:
 class Workload:
     """A named synthetic workload: its linears, dtype, mode and outlier recipe."""
     name: str
-    mode: str                 # "int8_outlier" | "fp8_static" | "fp8_dynamic" | "w4a8"
+    mode: str                 # "int8_outlier" | "fp8_static" | "fp8_dynamic" | "w4a8" | "fp8_weight_only" | "fp_linear"
     dtype: torch.dtype
     linears: List[Linear]
     seed: int
@@ -176,6 +176,21 @@ WORKLOADS: Dict[str, Workload] = {
                  Linear("mlp_up", _TOK_2048, _H, 4 * _H), Linear("mlp_down", _TOK_2048, 4 * _H, _H)],
         fixed_channels=[17, 200], fixed_tokens=10, fixed_range=(8.0, 12.0),
         extra={"blocks": 32, "group": 128}),
+    # Weight-only FP8 (E4M3 weights, bf16 per-channel scales, bf16 activations)
+    # at the text-encoder MLP shapes.
+    "te_fp8_weight_only_mlp": Workload(
+        name="te_fp8_weight_only_mlp", mode="fp8_weight_only", dtype=torch.bfloat16, seed=6,
+        linears=[Linear("gate", 512, 4096, 12288), Linear("up", 512, 4096, 12288),
+                 Linear("down", 512, 12288, 4096)],
+        massive_pairs=[(5, 2276, 9000.0), (0, 2276, 13000.0)]),
+    # The unquantised 16-bit linear (a layer kept in floating point) at the
+    # DiT MLP shapes of 1024^2, bf16.
+    "dit1024_bf16_mlp": Workload(
+        name="dit1024_bf16_mlp", mode="fp_linear", dtype=torch.bfloat16, seed=7,
+        linears=[Linear("mlp_up", _TOK_1024, _H, 4 * _H),
+                 Linear("mlp_down", _TOK_1024, 4 * _H, _H)],
+        random_channels=4, random_token_frac=0.05, random_range=(8.0, 40.0),
+        massive_text_tokens=4, massive_value=9000.0),
 }
 
 
