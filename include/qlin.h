@@ -75,8 +75,10 @@ typedef enum qlin_wmode {
     QLIN_W_INT8_ROW = 0,     /* Wq int8 [N,K];  w_scale fp32 [N]   = absmax_k|W[j,k]| / 127          */
     QLIN_W_FP8_TENSOR = 1,   /* Wq e4m3 [N,K];  w_scale fp32 [1]   = absmax|W| / 448                 */
     QLIN_W_FP8_CHANNEL = 2,  /* Wq e4m3 [N,K];  w_scale bf16 [N,1] = bf16(absmax_k|W[j,k]| / 448)    */
-    QLIN_W_INT4_G128 = 3     /* Wq uint8 [N,K/2] (k even: low nibble, k odd: high nibble, two's
+    QLIN_W_INT4_G128 = 3,    /* Wq uint8 [N,K/2] (k even: low nibble, k odd: high nibble, two's
                                 complement, codes in [-7,7]); w_scale fp32 [N,K/128] = absmax/7      */
+    QLIN_W_INT8_BLOCK32 = 4  /* Wq int8 [N,K]; w_scale fp32 [N,K/32] = absmax of each run of 32
+                                weights of a row / 127 (K % 32 == 0)                               */
 } qlin_wmode;
 
 /* Operations whose scratch size qlin_workspace_bytes() reports. */
@@ -85,7 +87,8 @@ typedef enum qlin_op {
     QLIN_OP_FP8 = 1,            /* qlin_fp8_forward                                 */
     QLIN_OP_W4A8 = 2,           /* qlin_w4a8_forward                                */
     QLIN_OP_QUANTIZE_WEIGHT = 3,/* qlin_quantize_weight and qlin_calibrate_input_scale */
-    QLIN_OP_INT8_PREP = 4       /* qlin_int8_prep                                   */
+    QLIN_OP_INT8_PREP = 4,      /* qlin_int8_prep                                   */
+    QLIN_OP_INT8_BLOCK = 5      /* qlin_int8_block_forward                          */
 } qlin_op;
 
 /* Bytes of device scratch `op` needs for an [M,K] x [N,K]^T problem (0 when
@@ -219,7 +222,31 @@ QLIN_API qlin_status qlin_fp8_weight_only_forward(const void *X, qlin_dtype xdt,
                                          const uint8_t *Wq, const void *w_scale, int64_t N,
                                          const void *bias, void *Y, void *stream);
 
+/* Block-scaled int8 linear (Qwen-Image-2.1-Text-Encoder-FP8 page, "How it was
+ * tested": GGUF Q8_0 stores int8 weight codes with one scale per run of 32
+ * weights of a row and was measured closest to bf16):
+ *   activations: per-token int8, s_x[i] = absmax_i / 127, as in W4A8 mode;
+ *   weights: Wq int8 [N,K], w_scale fp32 [N,K/32] from
+ *            qlin_quantize_weight(QLIN_W_INT8_BLOCK32);
+ *   Y = dtype(s_x[i] * sum_b w_scale[j,b] * C_b[i,j] + bias[j]),
+ *   C_b = sum over the 32 columns of block b of Xq * Wq.
+ * The kernel applies each weight's block scale before the sum: the weight
+ * tile is dequantised on chip to fp16 (q * s rounded to 11 significant bits),
+ * the activation codes enter as exact fp16 values, and tcgen05 kind::f16
+ * accumulates in fp32, so the result is within 2^-11 relative per weight of
+ * the exact int32 block sums (the per-block int32 partials are not formed).
+ * K % 32 == 0. workspace: qlin_workspace_bytes(QLIN_OP_INT8_BLOCK, M, N, K). */
+QLIN_API qlin_status qlin_int8_block_forward(const void *X, qlin_dtype xdt, int64_t M, int64_t K,
+                                    const int8_t *Wq, const float *w_scale, int64_t N, const void *bias,
+                                    void *Y, void *workspace, size_t ws_bytes, void *stream);
+
 /* ---------------- parity exports: the same kernels, intermediates written out ------ */
+
+/* The activation stage of qlin_int8_block_forward: per-token int8 codes
+ * (round-half-even of X * (1/s_x), IEEE fp32) written as fp16 values Xq16
+ * [M,K] (exact), and s_x fp32 [M] = absmax_i / 127. */
+QLIN_API qlin_status qlin_int8_block_prep(const void *X, qlin_dtype xdt, int64_t M, int64_t K, void *Xq16,
+                                 float *s_x, void *stream);
 
 /* LLM.int8 activation prep alone. Outputs: Xq int8 [M,K]; s_x fp32 [M];
  * flags uint32 [ceil(K/32)] (bit k%32 of word k/32 set iff column k is an

@@ -27,8 +27,9 @@ LIB_PATH = os.path.join(_HERE, "libqlin.so")
 QLIN_OK, QLIN_ERR_INVALID_ARG, QLIN_ERR_UNSUPPORTED, QLIN_ERR_ALIGNMENT = 0, 1, 2, 3
 QLIN_ERR_WORKSPACE, QLIN_ERR_CUDA, QLIN_ERR_TIMEOUT = 4, 5, 6
 QLIN_F16, QLIN_BF16 = 0, 1
-QLIN_W_INT8_ROW, QLIN_W_FP8_TENSOR, QLIN_W_FP8_CHANNEL, QLIN_W_INT4_G128 = 0, 1, 2, 3
+QLIN_W_INT8_ROW, QLIN_W_FP8_TENSOR, QLIN_W_FP8_CHANNEL, QLIN_W_INT4_G128, QLIN_W_INT8_BLOCK32 = 0, 1, 2, 3, 4
 QLIN_OP_INT8_OUTLIER, QLIN_OP_FP8, QLIN_OP_W4A8, QLIN_OP_QUANTIZE_WEIGHT, QLIN_OP_INT8_PREP = 0, 1, 2, 3, 4
+QLIN_OP_INT8_BLOCK = 5
 
 _STATUS_NAMES = {0: "QLIN_OK", 1: "QLIN_ERR_INVALID_ARG", 2: "QLIN_ERR_UNSUPPORTED", 3: "QLIN_ERR_ALIGNMENT",
                  4: "QLIN_ERR_WORKSPACE", 5: "QLIN_ERR_CUDA", 6: "QLIN_ERR_TIMEOUT"}
@@ -60,6 +61,8 @@ def _load() -> ctypes.CDLL:
         "qlin_w4a8_forward": (st, [P, i32, i64, i64, P, P, i64, P, P, P, sz, P]),
         "qlin_fp_linear_forward": (st, [P, i32, i64, i64, P, i64, P, P, P]),
         "qlin_fp8_weight_only_forward": (st, [P, i32, i64, i64, P, P, i64, P, P, P]),
+        "qlin_int8_block_forward": (st, [P, i32, i64, i64, P, P, i64, P, P, P, sz, P]),
+        "qlin_int8_block_prep": (st, [P, i32, i64, i64, P, P, P]),
         "qlin_w4a8_gemm": (st, [i32, i64, i64, P, P, P, P, i64, P, P, P]),
         "qlin_w4a8_prep": (st, [P, i32, i64, i64, P, P, P]),
         "qlin_w4a8_group_i32": (st, [P, P, i64, i64, i64, i32, P, P]),
@@ -164,6 +167,9 @@ def qlin_quantize_weight(W: torch.Tensor, mode: int):
     elif mode == QLIN_W_INT4_G128:
         Wq = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
         s = torch.empty((N, K // 128), dtype=torch.float32, device=dev)
+    elif mode == QLIN_W_INT8_BLOCK32:
+        Wq = torch.empty((N, K), dtype=torch.int8, device=dev)
+        s = torch.empty((N, K // 32), dtype=torch.float32, device=dev)
     else:
         raise ValueError(mode)
     ws = workspace(QLIN_OP_QUANTIZE_WEIGHT, 0, N, K, dev)
@@ -306,6 +312,30 @@ def qlin_fp8_weight_only_forward(X: torch.Tensor, Wq: torch.Tensor, w_scale: tor
     _check(lib.qlin_fp8_weight_only_forward(_ptr(X), _dt(X), M, K, _ptr(Wq), _ptr(w_scale), N, _ptr(bias), _ptr(Y),
                                             _stream(X.device)))
     return Y
+
+
+def qlin_int8_block_forward(X: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tensor,
+                            bias: Optional[torch.Tensor] = None, Y: Optional[torch.Tensor] = None,
+                            ws: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Block-scaled int8 linear: one fp32 weight scale per 32 weights of a row, per-token int8 activations."""
+    M, K = X.shape
+    N = Wq.shape[0]
+    if Y is None:
+        Y = torch.empty((M, N), dtype=X.dtype, device=X.device)
+    if ws is None:
+        ws = workspace(QLIN_OP_INT8_BLOCK, M, N, K, X.device)
+    _check(lib.qlin_int8_block_forward(_ptr(X), _dt(X), M, K, _ptr(Wq), _ptr(w_scale), N, _ptr(bias), _ptr(Y),
+                                       _ptr(ws), ws.numel(), _stream(X.device)))
+    return Y
+
+
+def qlin_int8_block_prep(X: torch.Tensor):
+    """Activation stage of the block-scaled int8 forward: int8 codes as fp16 values [M,K] and s_x [M]."""
+    M, K = X.shape
+    Xq16 = torch.empty((M, K), dtype=torch.float16, device=X.device)
+    s_x = torch.empty((M,), dtype=torch.float32, device=X.device)
+    _check(lib.qlin_int8_block_prep(_ptr(X), _dt(X), M, K, _ptr(Xq16), _ptr(s_x), _stream(X.device)))
+    return Xq16, s_x
 
 
 def qlin_w4a8_prep(X: torch.Tensor, Xq: Optional[torch.Tensor] = None, s_x: Optional[torch.Tensor] = None):

@@ -1,30 +1,39 @@
-// gemm_wo8.cuh -- weight-only FP8 linear for sm_100a (Qwen-Image-2.1-Text-
-// Encoder-FP8 page, "Format": E4M3 weights with one bf16 scale per output
-// channel, consumed as weight.to(bf16) * weight_scale; the activations stay
-// in bf16):
+// gemm_cvt.cuh -- GEMMs whose 8-bit weights are dequantised to 16 bits in
+// shared memory, tile by tile, and contracted with tcgen05 kind::f16 (fp32
+// accumulation); the dequantised weight never reaches global memory.
 //
+// FMT 0, weight-only FP8 (Qwen-Image-2.1-Text-Encoder-FP8 page, "Format": E4M3
+// weights with one bf16 scale per output channel, consumed as
+// weight.to(bf16) * weight_scale; the activations stay in bf16):
 //   W_deq[j,k] = bf16( decode(Wq[j,k]) * s_w[j] )   (one rounding: the e4m3 value
 //                has 4 significant bits and s_w 8, so the fp32 product is exact)
-//   Y[i,j]     = bf16( sum_k X[i,k] * W_deq[j,k] + bias[j] )   (fp32 accumulation)
-//
-// The dequantised weight never reaches global memory: each stage's e4m3 tile
-// is converted in shared memory into the 128B-swizzled K-major bf16 layout
-// the tensor core reads, and contracted with tcgen05 kind::f16.
+//   Y[i,j]     = bf16( sum_k X[i,k] * W_deq[j,k] + bias[j] )
+// FMT 1, block-scaled int8 weights (Qwen-Image-2.1-Text-Encoder-FP8 page, "How
+// it was tested": GGUF Q8_0, int8 codes with one scale per 32 weights of a
+// row) with per-token int8 activations, whose codes arrive as exact fp16:
+//   W_deq[j,k] = fp16( float(Wq[j,k]) * s_w[j, k/32] )   (11 significant bits)
+//   Y[i,j]     = dtype( s_x[i] * sum_k Xq[i,k] * W_deq[j,k] + bias[j] )
+//   i.e. s_x[i] * sum_b s_w[j,b] * C_b[i,j] with the weight's scale applied
+//   per element before the sum instead of per block after it (relative error
+//   at most 2^-11 per weight, against the exact int32 block sums).
 //
 // Roles (one CTA per SM, 16 warps, persistent over 128x256 output tiles, two
 // 256-column TMEM accumulators so the epilogue of one tile overlaps the main
 // loop of the next):
-//   warp 0       TMA producer: the bf16 A tile (128 rows x 64 elements, 128B
-//                swizzle) and the raw e4m3 B tile (256 rows x 64 bytes) of one
-//                stage of K;
+//   warp 0       TMA producer: the 16-bit A tile (128 rows x 64 elements,
+//                128B swizzle) and the raw 8-bit B tile (256 rows x 64 bytes)
+//                of one stage of K;
 //   warp 1       MMA issuer: 4 x kind::f16 (K = 16) per stage;
 //   warps 4-11   converters: one 16-byte chunk of raw codes at a time (16
-//                weights of one row) -> 16 bf16 values into two 16-byte chunks
-//                of the swizzled row, then hand the stage to the MMA;
-//   warps 12-15  epilogue, one per TMEM lane quarter: Y = acc + bias;
+//                weights of one row) -> 16 16-bit values into two 16-byte
+//                chunks of the swizzled row, then hand the stage to the MMA;
+//   warps 12-15  epilogue, one per TMEM lane quarter: Y = acc + bias (FMT 0)
+//                or s_x * acc + bias (FMT 1);
 //   warps 2-3    idle.
 // All waits are bounded (common.cuh).
 #pragma once
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace qlin {
@@ -38,15 +47,17 @@ constexpr int WO8_WARP_CONV0 = 4, WO8_WARP_EPI0 = 12;
 
 struct Wo8Params {
   int64_t M, N, K;
-  void* Y;                    // [M,N] bf16
-  const uint16_t* s_w;        // [N] bf16 per-channel weight scale
-  const uint16_t* bias;       // [N] bf16, nullable
+  void* Y;                    // [M,N] 16-bit (bf16 for FMT 0)
+  const uint16_t* s_w;        // FMT 0: [N] bf16 per-channel weight scale
+  const float* s_wb;          // FMT 1: [N, K/32] fp32 block weight scales
+  const float* s_x;           // FMT 1: [M] fp32 per-token activation scale
+  const uint16_t* bias;       // [N] output dtype, nullable
 };
 
 struct Wo8Smem {
-  static constexpr int A_BYTES = WO8_BM * WO8_BK * 2;      // 16 KB bf16, swizzled
-  static constexpr int B_BYTES = WO8_BN * WO8_BK * 2;      // 32 KB bf16, swizzled (converted)
-  static constexpr int R_BYTES = WO8_BN * WO8_BK;          // 16 KB e4m3 (raw)
+  static constexpr int A_BYTES = WO8_BM * WO8_BK * 2;      // 16 KB 16-bit, swizzled
+  static constexpr int B_BYTES = WO8_BN * WO8_BK * 2;      // 32 KB 16-bit, swizzled (converted)
+  static constexpr int R_BYTES = WO8_BN * WO8_BK;          // 16 KB 8-bit codes (raw)
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES + R_BYTES;
   static constexpr int BIAS_BYTES = 2 * WO8_BN * 4;        // two tiles' biases (fp32)
   static constexpr int BAR_BYTES = 8 * (3 * WO8_STAGES + 4 + 2) + 16;
@@ -77,8 +88,36 @@ __device__ __forceinline__ void e4m3x16_to_bf16(const uint4& raw, float s, uint4
   hi8 = make_uint4(out[4], out[5], out[6], out[7]);
 }
 
+// 16 int8 codes (element e in byte e) times the scale s, each product
+// rounded to fp16 (the fp32 product rounds first when s has more than 16
+// significant bits): 16 fp16 values as two 16-byte chunks. A code q reads as
+// float from the bits 0x4B000000 | (q ^ 0x80), i.e. 2^23 + 128 + q.
+__device__ __forceinline__ void int8x16_to_f16(const uint4& raw, float s, uint4& lo8, uint4& hi8) {
+  const uint32_t w[4] = {raw.x ^ 0x80808080u, raw.y ^ 0x80808080u, raw.z ^ 0x80808080u, raw.w ^ 0x80808080u};
+  const unsigned long long off2 = f32x2_of(__float_as_uint(-8388736.0f), __float_as_uint(-8388736.0f));
+  const unsigned long long s2 = f32x2_of(__float_as_uint(s), __float_as_uint(s));
+  uint32_t out[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const uint32_t a = __byte_perm(w[i], 0x4B000000u, 0x7650u + 2 * h);       // code 4i+2h
+      const uint32_t b = __byte_perm(w[i], 0x4B000000u, 0x7650u + 2 * h + 1);   // code 4i+2h+1
+      const unsigned long long v = mul_f32x2(add_f32x2(f32x2_of(a, b), off2), s2);
+      uint32_t hv;
+      // cvt.rn.f16x2.f32 d, x, y puts x in the upper half
+      asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(hv) : "f"(hi_f(v)), "f"(lo_f(v)));
+      out[2 * i + h] = hv;
+    }
+  }
+  lo8 = make_uint4(out[0], out[1], out[2], out[3]);
+  hi8 = make_uint4(out[4], out[5], out[6], out[7]);
+}
+
+template <int FMT, typename TOut>
 __global__ void __launch_bounds__(WO8_THREADS, 1)
-    k_gemm_wo8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const Wo8Params p) {
+    k_gemm_cvt(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const Wo8Params p) {
+  static_assert(FMT == 1 || std::is_same<TOut, __nv_bfloat16>::value, "weight-only FP8 writes bf16");
   using L = Wo8Smem;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -164,7 +203,7 @@ __global__ void __launch_bounds__(WO8_THREADS, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------- MMA issuer ----------------
-      constexpr uint32_t idesc = idesc_f16(WO8_BM, WO8_BN, true);
+      constexpr uint32_t idesc = idesc_f16(WO8_BM, WO8_BN, FMT == 0);   // bf16 (FMT 0) or fp16 operands
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
@@ -197,19 +236,35 @@ __global__ void __launch_bounds__(WO8_THREADS, 1)
   } else if (warp >= WO8_WARP_CONV0 && warp < WO8_WARP_CONV0 + WO8_CONV_WARPS) {
     // ---------------- converters: e4m3 * s_w -> bf16, swizzled ----------------
     const int ct = threadIdx.x - 32 * WO8_WARP_CONV0;   // 0..255
+    const int64_t nblk = K / 32;                        // FMT 1: weight-scale blocks per row
+    const int cb = (ct & 3) >> 1;                       // FMT 1: this thread's block within a stage
     int stage = 0;
     uint32_t phase = 0;
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
       const int nb = tile / num_m;
       // this thread's rows of the tile: ct/4 + 64q, q = 0..3
-      float sc[4];
+      float sc[4];       // FMT 0: the rows' scales; FMT 1: their block scales for stage kb
+      float sn[4];       // FMT 1: the same for stage kb + 1 (loaded one stage ahead)
+      auto block_scales = [&](int kb, float (&d)[4]) {
 #pragma unroll
-      for (int qd = 0; qd < 4; ++qd) {
-        const int64_t n = static_cast<int64_t>(nb) * WO8_BN + (ct >> 2) + 64 * qd;
-        sc[qd] = n < N ? to_f<__nv_bfloat16>(__ldg(p.s_w + n)) : 0.0f;
+        for (int qd = 0; qd < 4; ++qd) {
+          const int64_t n = static_cast<int64_t>(nb) * WO8_BN + (ct >> 2) + 64 * qd;
+          const int64_t b = 2 * static_cast<int64_t>(kb) + cb;
+          d[qd] = (n < N && b < nblk) ? __ldg(p.s_wb + n * nblk + b) : 0.0f;
+        }
+      };
+      if constexpr (FMT == 0) {
+#pragma unroll
+        for (int qd = 0; qd < 4; ++qd) {
+          const int64_t n = static_cast<int64_t>(nb) * WO8_BN + (ct >> 2) + 64 * qd;
+          sc[qd] = n < N ? to_f<__nv_bfloat16>(__ldg(p.s_w + n)) : 0.0f;
+        }
+      } else {
+        block_scales(0, sc);
       }
       for (int kb = 0; kb < num_kb; ++kb) {
+        if constexpr (FMT == 1) block_scales(kb + 1, sn);
         if (!mbar_wait(&full_bar[stage], phase, abort_flag)) { ok = false; break; }
         const uint8_t* raw = sR(stage);
         uint8_t* dst = sB(stage);
@@ -219,7 +274,8 @@ __global__ void __launch_bounds__(WO8_THREADS, 1)
           const int r = id >> 2, c = id & 3;
           const uint4 v = *reinterpret_cast<const uint4*>(raw + r * WO8_BK + c * 16);
           uint4 lo, hi;
-          e4m3x16_to_bf16(v, sc[qd], lo, hi);
+          if constexpr (FMT == 0) e4m3x16_to_bf16(v, sc[qd], lo, hi);
+          else int8x16_to_f16(v, sc[qd], lo, hi);
           // row r's 128 bf16 bytes: 16-byte chunk ch sits at chunk (ch ^ (r & 7))
           *reinterpret_cast<uint4*>(dst + r * 128 + (((2 * c) ^ (r & 7)) << 4)) = lo;
           *reinterpret_cast<uint4*>(dst + r * 128 + (((2 * c + 1) ^ (r & 7)) << 4)) = hi;
@@ -228,10 +284,14 @@ __global__ void __launch_bounds__(WO8_THREADS, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&conv_bar[stage]);
         if (++stage == WO8_STAGES) { stage = 0; phase ^= 1u; }
+        if constexpr (FMT == 1) {
+#pragma unroll
+          for (int qd = 0; qd < 4; ++qd) sc[qd] = sn[qd];
+        }
       }
     }
   } else if (warp >= WO8_WARP_EPI0) {
-    // ---------------- epilogue: Y = acc + bias ----------------
+    // ---------------- epilogue: Y = acc + bias (FMT 0) or s_x * acc + bias (FMT 1) ----------------
     const int q = warp & 3;                      // TMEM lane quarter
     const int et = threadIdx.x - 32 * WO8_WARP_EPI0;   // 0..127
     int acc = 0;
@@ -246,13 +306,15 @@ __global__ void __launch_bounds__(WO8_THREADS, 1)
       float* bt = sbias + acc * WO8_BN;
       for (int j = et; j < WO8_BN; j += 32 * WO8_EPI_WARPS) {
         const int64_t n = n_base + j;
-        bt[j] = (p.bias != nullptr && n < N) ? to_f<__nv_bfloat16>(__ldg(p.bias + n)) : 0.0f;
+        bt[j] = (p.bias != nullptr && n < N) ? to_f<TOut>(__ldg(p.bias + n)) : 0.0f;
       }
       if (!epi_bar(epi_mbar, bar_phase, abort_flag)) break;
       if (!mbar_wait(&tfull_bar[acc], acc_phase, abort_flag)) break;
       tc_fence_after();
       const uint32_t t_row = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(acc * WO8_BN);
       uint32_t r[32];
+      float sx = 1.0f;
+      if constexpr (FMT == 1) sx = row < M ? __ldg(p.s_x + row) : 0.0f;
       for (int c = 0; c < WO8_BN; c += 32) {
         __syncwarp();
         tmem_ld32(t_row + static_cast<uint32_t>(c), r);
@@ -263,7 +325,10 @@ __global__ void __launch_bounds__(WO8_THREADS, 1)
 #pragma unroll
           for (int j = 0; j < 16; ++j) {
             const float2 b2 = *reinterpret_cast<const float2*>(bt + c + 2 * j);
-            out[j] = pack2<__nv_bfloat16>(__uint_as_float(r[2 * j]) + b2.x, __uint_as_float(r[2 * j + 1]) + b2.y);
+            if constexpr (FMT == 0)
+              out[j] = pack2<TOut>(__uint_as_float(r[2 * j]) + b2.x, __uint_as_float(r[2 * j + 1]) + b2.y);
+            else
+              out[j] = pack2<TOut>(fmaf(__uint_as_float(r[2 * j]), sx, b2.x), fmaf(__uint_as_float(r[2 * j + 1]), sx, b2.y));
           }
           uint16_t* y = reinterpret_cast<uint16_t*>(p.Y) + row * N + n0;
           if (vec && n0 + 32 <= N) {

@@ -143,7 +143,9 @@ __device__ __forceinline__ uint32_t keep_mask(uint32_t om, int i) {
 // PF_DEPTH - 1 rows into private shared-memory slots with cp.async, so those
 // rows are in flight while the current one is quantised).
 //
-// CODE 0: int8 (QMAX 127), CODE 1: E4M3 (QMAX 448). SCALE_BF16: the stored
+// CODE 0: int8 (QMAX 127), CODE 1: E4M3 (QMAX 448), CODE 2: the int8 codes
+// stored as fp16 values (exact; the A operand of a kind::f16 contraction, 2
+// bytes per code: Q is then [rows, K] fp16). SCALE_BF16: the stored
 // scale is bf16(absmax / QMAX) and the codes use that rounded value (the
 // [out,1] bf16 weight scales of the Text-Encoder-FP8 page).
 //
@@ -208,6 +210,20 @@ __device__ __forceinline__ uint2 quant_vec(const uint4& v, uint32_t om, float in
   }
 }
 
+// 8 int8 codes (element e in byte e) as 8 fp16 values (exact: |code| <= 127).
+__device__ __forceinline__ uint4 codes_as_f16x8(const uint2& c) {
+  const uint32_t w[2] = {c.x, c.y};
+  uint32_t h[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int lo = static_cast<int8_t>((w[i >> 1] >> (16 * (i & 1))) & 0xFFu);
+    const int hi = static_cast<int8_t>((w[i >> 1] >> (16 * (i & 1) + 8)) & 0xFFu);
+    h[i] = static_cast<uint32_t>(__half_as_ushort(__int2half_rn(lo))) |
+           (static_cast<uint32_t>(__half_as_ushort(__int2half_rn(hi))) << 16);
+  }
+  return make_uint4(h[0], h[1], h[2], h[3]);
+}
+
 // Lanes of a packed 16-bit pair whose |x| pattern exceeds tb: with a = |x|
 // (<= 0x7FFF) and c = 0x7FFF - tb, a > tb exactly when a + c >= 0x8000, and
 // a + c <= 0xFFFE never carries into the other lane, so bit 15 of each lane
@@ -251,7 +267,7 @@ __global__ void __launch_bounds__(RQ_THREADS, 3) k_prep_rows(const T* __restrict
   const int unit = warp / rw;
   const int ut = tid - unit * rw * 32;   // thread index inside the unit
   const int UT = rw * 32;
-  constexpr float QMAX = CODE == 0 ? 127.0f : 448.0f;
+  constexpr float QMAX = CODE == 1 ? 448.0f : 127.0f;
 
   // max over the unit (warp redux, then the unit's warps through shared
   // memory, double-buffered so one named barrier per reduction suffices)
@@ -357,11 +373,20 @@ __global__ void __launch_bounds__(RQ_THREADS, 3) k_prep_rows(const T* __restrict
     const bool zero = (s == 0.0f);
     // a normal scale keeps |x * inv| below QMAX + 1/2 for every entry in the absmax
     const bool fast = s >= 1.17549435e-38f;
-    uint2* qr = reinterpret_cast<uint2*>(a.Q + row * K);
+    if constexpr (CODE == 2) {
+      uint4* qr = reinterpret_cast<uint4*>(a.Q + row * K * 2);
 #pragma unroll
-    for (int u = 0; u < V; ++u) {
-      const int idx = ut + u * UT;
-      if (idx < KV) qr[idx] = quant_vec<T, CODE>(cur[u], 0u, inv, fast, zero);
+      for (int u = 0; u < V; ++u) {
+        const int idx = ut + u * UT;
+        if (idx < KV) qr[idx] = codes_as_f16x8(quant_vec<T, 0>(cur[u], 0u, inv, fast, zero));
+      }
+    } else {
+      uint2* qr = reinterpret_cast<uint2*>(a.Q + row * K);
+#pragma unroll
+      for (int u = 0; u < V; ++u) {
+        const int idx = ut + u * UT;
+        if (idx < KV) qr[idx] = quant_vec<T, CODE>(cur[u], 0u, inv, fast, zero);
+      }
     }
   }
   cp_async_wait<0>();
@@ -863,6 +888,48 @@ __global__ void __launch_bounds__(256) k_int4_group_quant(const T* __restrict__ 
   }
   *reinterpret_cast<uint16_t*>(Q4 + j * (K / 2) + g * (G / 2) + lane * 2) = static_cast<uint16_t>(packed);
   if (lane == 0) s_w[j * ng + g] = s;
+}
+
+// Block-scaled int8 weights: one thread per (row j, block b of 32 weights
+// along K): s_w[j,b] = absmax / 127, codes rne(w * (1/s)) clamped to +-127
+// (the row format's quantiser on each block), 0 for an all-zero block.
+template <typename T>
+__global__ void __launch_bounds__(256) k_int8_block_quant(const T* __restrict__ W, int64_t N, int64_t K,
+                                                        int8_t* __restrict__ Q, float* __restrict__ s_w) {
+  const int64_t nb = K / 32;
+  for (int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; t < N * nb;
+       t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t j = t / nb, b = t - j * nb;
+    const uint4* src = reinterpret_cast<const uint4*>(W + j * K + b * 32);
+    uint16_t h[32];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint16_t e[8];
+      unpack8(ld_nc_v4(src + i), e);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) h[8 * i + k] = e[k];
+    }
+    float m = 0.0f;
+#pragma unroll
+    for (int k = 0; k < 32; ++k) m = fmaxf(m, fabsf(to_f<T>(h[k])));
+    const float s = m / 127.0f;
+    const float inv = 1.0f / s;
+    uint32_t w[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      uint32_t v = 0;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const int q = s == 0.0f ? 0 : q_int(to_f<T>(h[4 * i + k]), inv, 127);
+        v |= (static_cast<uint32_t>(q) & 0xFFu) << (8 * k);
+      }
+      w[i] = v;
+    }
+    uint4* dst = reinterpret_cast<uint4*>(Q + j * K + b * 32);
+    dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+    dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    s_w[t] = s;
+  }
 }
 
 }  // namespace qlin

@@ -20,7 +20,7 @@
 #include "common.cuh"
 #include "gemm.cuh"
 #include "gemm_w4a8.cuh"
-#include "gemm_wo8.cuh"
+#include "gemm_cvt.cuh"
 #include "prep.cuh"
 
 using namespace qlin;
@@ -552,6 +552,8 @@ size_t qlin_workspace_bytes(qlin_op op, int64_t M, int64_t N, int64_t K) {
       return static_cast<size_t>(round_up(M * K, 256) + round_up(4 * M, 256));
     case QLIN_OP_QUANTIZE_WEIGHT:
       return 256;
+    case QLIN_OP_INT8_BLOCK:
+      return static_cast<size_t>(round_up(2 * M * K, 256) + round_up(4 * M, 256));
     default:
       return 0;
   }
@@ -592,6 +594,8 @@ qlin_status qlin_quantize_weight(const void* W, qlin_dtype wdt, int64_t N, int64
                                  void* w_scale, void* workspace, size_t ws_bytes, void* stream) {
   QLIN_TRY(check_common(W, wdt, N, K, 0));
   if (mode == QLIN_W_INT4_G128 && K % 128 != 0) return fail(QLIN_ERR_ALIGNMENT, "int4 format needs K % 128 == 0");
+  if (mode == QLIN_W_INT8_BLOCK32 && K % 32 != 0)
+    return fail(QLIN_ERR_ALIGNMENT, "block-scaled int8 needs K % 32 == 0");
   if (N == 0) return ok();
   QLIN_REQ_PTR(Wq, "Wq");
   QLIN_REQ_PTR(w_scale, "w_scale");
@@ -643,6 +647,19 @@ qlin_status qlin_quantize_weight(const void* W, qlin_dtype wdt, int64_t N, int64
         k_int4_group_quant<__half><<<static_cast<unsigned>(blocks), 256, 0, st>>>(
             static_cast<const __half*>(W), N, K, static_cast<uint8_t*>(Wq), static_cast<float*>(w_scale));
       QLIN_TRY(check_cuda(cudaGetLastError(), "int4 quant launch"));
+      return ok();
+    }
+    case QLIN_W_INT8_BLOCK32: {
+      const int64_t blocks = N * (K / 32);
+      const int64_t want = (blocks + 255) / 256, cap = static_cast<int64_t>(d->sms) * 16;
+      const unsigned grid = static_cast<unsigned>(want < cap ? want : cap);
+      if (bf)
+        k_int8_block_quant<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(W), N, K,
+                                                                static_cast<int8_t*>(Wq), static_cast<float*>(w_scale));
+      else
+        k_int8_block_quant<__half><<<grid, 256, 0, st>>>(static_cast<const __half*>(W), N, K, static_cast<int8_t*>(Wq),
+                                                         static_cast<float*>(w_scale));
+      QLIN_TRY(check_cuda(cudaGetLastError(), "int8 block quant launch"));
       return ok();
     }
     default:
@@ -1073,26 +1090,28 @@ qlin_status qlin_w4a8_forward(const void* X, qlin_dtype xdt, int64_t M, int64_t 
 // ---------------------------------------------------------------------------
 namespace {
 
-qlin_status launch_wo8(const void* X, const uint8_t* Wq, const Wo8Params& wp, cudaStream_t st) {
+template <int FMT, typename TOut>
+qlin_status launch_cvt(const void* A, const void* Wq, const Wo8Params& wp, cudaStream_t st) {
   DeviceInfo* d;
   qlin_status s = device_info(&d);
   if (s != QLIN_OK) return s;
   CUtensorMap ta, tb;
-  if ((s = make_tmap_k128(&ta, X, wp.M, 2 * wp.K, WO8_BM)) != QLIN_OK) return s;
+  if ((s = make_tmap_k128(&ta, A, wp.M, 2 * wp.K, WO8_BM)) != QLIN_OK) return s;
   if ((s = make_tmap_bytes(&tb, Wq, wp.N, wp.K, WO8_BK, WO8_BN, CU_TENSOR_MAP_SWIZZLE_NONE)) != QLIN_OK) return s;
+  auto kern = k_gemm_cvt<FMT, TOut>;
   static std::atomic<bool> attr_set[16] = {};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 16 && !attr_set[dev].load(std::memory_order_acquire)) {
-    s = check_cuda(cudaFuncSetAttribute(k_gemm_wo8, cudaFuncAttributeMaxDynamicSharedMemorySize, Wo8Smem::TOTAL),
+    s = check_cuda(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, Wo8Smem::TOTAL),
                    "cudaFuncSetAttribute");
     if (s != QLIN_OK) return s;
     attr_set[dev].store(true, std::memory_order_release);
   }
   const int64_t tiles = ((wp.M + WO8_BM - 1) / WO8_BM) * ((wp.N + WO8_BN - 1) / WO8_BN);
   const int grid = static_cast<int>(tiles < d->sms ? tiles : d->sms);
-  k_gemm_wo8<<<grid, WO8_THREADS, Wo8Smem::TOTAL, st>>>(ta, tb, wp);
-  return check_cuda(cudaGetLastError(), "k_gemm_wo8 launch");
+  kern<<<grid, WO8_THREADS, Wo8Smem::TOTAL, st>>>(ta, tb, wp);
+  return check_cuda(cudaGetLastError(), "k_gemm_cvt launch");
 }
 
 }  // namespace
@@ -1112,7 +1131,45 @@ extern "C" qlin_status qlin_fp8_weight_only_forward(const void* X, qlin_dtype xd
   wp.M = M; wp.N = N; wp.K = K; wp.Y = Y;
   wp.s_w = static_cast<const uint16_t*>(w_scale);
   wp.bias = static_cast<const uint16_t*>(bias);
-  QLIN_TRY(launch_wo8(X, Wq, wp, static_cast<cudaStream_t>(stream)));
+  QLIN_TRY((launch_cvt<0, __nv_bfloat16>(X, Wq, wp, static_cast<cudaStream_t>(stream))));
+  return ok();
+}
+
+extern "C" qlin_status qlin_int8_block_prep(const void* X, qlin_dtype xdt, int64_t M, int64_t K, void* Xq16,
+                                            float* s_x, void* stream) {
+  QLIN_TRY(check_common(X, xdt, M, K, 0));
+  if (M == 0) return ok();
+  QLIN_REQ_PTR(Xq16, "Xq16");
+  QLIN_REQ_PTR(s_x, "s_x");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (xdt == QLIN_BF16)
+    return launch_rowquant<__nv_bfloat16, 2, false>(X, M, K, static_cast<uint8_t*>(Xq16), s_x, nullptr, st);
+  return launch_rowquant<__half, 2, false>(X, M, K, static_cast<uint8_t*>(Xq16), s_x, nullptr, st);
+}
+
+extern "C" qlin_status qlin_int8_block_forward(const void* X, qlin_dtype xdt, int64_t M, int64_t K, const int8_t* Wq,
+                                               const float* w_scale, int64_t N, const void* bias, void* Y,
+                                               void* workspace, size_t ws_bytes, void* stream) {
+  QLIN_TRY(check_common(X, xdt, M, K, N));
+  if (K % 32 != 0) return fail(QLIN_ERR_ALIGNMENT, "block-scaled int8 needs K a multiple of 32");
+  if (M == 0 || N == 0) return ok();
+  QLIN_REQ_PTR(Wq, "Wq");
+  QLIN_REQ_PTR(w_scale, "w_scale");
+  QLIN_REQ_PTR(Y, "Y");
+  if (bias != nullptr && !aligned16(bias)) return fail(QLIN_ERR_ALIGNMENT, "bias is not 16-byte aligned");
+  if (workspace == nullptr || ws_bytes < qlin_workspace_bytes(QLIN_OP_INT8_BLOCK, M, N, K))
+    return fail(QLIN_ERR_WORKSPACE, "workspace too small");
+  QLIN_REQ_PTR(workspace, "workspace");
+  uint8_t* Xq16 = static_cast<uint8_t*>(workspace);
+  float* s_x = reinterpret_cast<float*>(Xq16 + round_up(2 * M * K, 256));
+  QLIN_TRY(qlin_int8_block_prep(X, xdt, M, K, Xq16, s_x, stream));
+  Wo8Params wp{};
+  wp.M = M; wp.N = N; wp.K = K; wp.Y = Y;
+  wp.s_wb = w_scale; wp.s_x = s_x;
+  wp.bias = static_cast<const uint16_t*>(bias);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (xdt == QLIN_BF16) QLIN_TRY((launch_cvt<1, __nv_bfloat16>(Xq16, Wq, wp, st)));
+  else QLIN_TRY((launch_cvt<1, __half>(Xq16, Wq, wp, st)));
   return ok();
 }
 
