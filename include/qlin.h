@@ -75,8 +75,9 @@ typedef enum qlin_wmode {
     QLIN_W_INT8_ROW = 0,     /* Wq int8 [N,K];  w_scale fp32 [N]   = absmax_k|W[j,k]| / 127          */
     QLIN_W_FP8_TENSOR = 1,   /* Wq e4m3 [N,K];  w_scale fp32 [1]   = absmax|W| / 448                 */
     QLIN_W_FP8_CHANNEL = 2,  /* Wq e4m3 [N,K];  w_scale bf16 [N,1] = bf16(absmax_k|W[j,k]| / 448)    */
-    QLIN_W_INT4_G128 = 3,    /* Wq uint8 [N,K/2] (k even: low nibble, k odd: high nibble, two's
-                                complement, codes in [-7,7]); w_scale fp32 [N,K/128] = absmax/7      */
+    QLIN_W_INT4_G128 = 3,    /* Wq uint8 [N,K/2]: each block of 32 consecutive k in 16 bytes, byte b
+                                holding element b (low nibble) and element b+16 (high nibble), two's
+                                complement, codes in [-7,7]; w_scale fp32 [N,K/128] = absmax/7      */
     QLIN_W_INT8_BLOCK32 = 4  /* Wq int8 [N,K]; w_scale fp32 [N,K/32] = absmax of each run of 32
                                 weights of a row / 127 (K % 32 == 0)                               */
 } qlin_wmode;
@@ -172,8 +173,9 @@ QLIN_API qlin_status qlin_fp8_gemm(qlin_dtype xdt, int64_t M, int64_t K, const u
  * int8 activations, fp32 scales; group 128 along K):
  *   activations: per-token int8, s_x[i] = absmax_i / 127 (no outlier split);
  *   C_g = sum over the 128 columns of group g of Xq * Wq4 (int32, exact; the
- *         int4 weights are unpacked to int8 in shared memory and contracted
- *         with tcgen05 kind::i8, one TMEM accumulator per group);
+ *         int4 weights are unpacked to int8 (as 16 * code) in shared memory
+ *         and contracted with tcgen05 kind::i8, one TMEM accumulator per
+ *         group);
  *   Y   = dtype(s_x[i] * sum_g w_scale[j,g] * C_g + bias[j]), the group sum in
  *         fp32 in ascending g.
  * Wq4 uint8 [N, K/2] and w_scale fp32 [N, K/128] from

@@ -343,8 +343,10 @@ void orc_quantize_weight_fp8_channel(const uint16_t *W, int dt, int64_t N, int64
 }
 
 /* int4, symmetric, one fp32 scale per (output channel, group of G along K):
- * s = absmax_group / 7, codes in [-7, 7]. Packing: byte k/2 of row j holds
- * k even in its low nibble and k odd in its high nibble, two's complement. */
+ * s = absmax_group / 7, codes in [-7, 7]. Packing (the page fixes no byte
+ * layout): each row is cut into blocks of 32 consecutive k stored in 16
+ * bytes; byte b of a block holds its element b in the low nibble and its
+ * element b + 16 in the high nibble, two's complement. K % 32 == 0. */
 void orc_quantize_weight_int4(const uint16_t *W, int dt, int64_t N, int64_t K, int64_t G,
                               uint8_t *Wq4, float *s_w) {
     float *w = widen_all(W, dt, N * K);
@@ -358,8 +360,9 @@ void orc_quantize_weight_int4(const uint16_t *W, int dt, int64_t N, int64_t K, i
             for (int64_t k = 0; k < G; ++k) {
                 int q = s == 0.0f ? 0 : q_int(wg[k], inv, 7);
                 int64_t kk = g * G + k;
-                uint8_t *b = Wq4 + j * (K / 2) + kk / 2;
-                if ((kk & 1) == 0) *b = (uint8_t)((*b & 0xf0) | (q & 0xf));
+                int64_t e = kk % 32;   /* position in its block of 32 */
+                uint8_t *b = Wq4 + j * (K / 2) + (kk / 32) * 16 + e % 16;
+                if (e < 16) *b = (uint8_t)((*b & 0xf0) | (q & 0xf));
                 else *b = (uint8_t)((*b & 0x0f) | ((q & 0xf) << 4));
             }
         }
@@ -368,8 +371,9 @@ void orc_quantize_weight_int4(const uint16_t *W, int dt, int64_t N, int64_t K, i
 }
 
 static int int4_at(const uint8_t *Wq4, int64_t K, int64_t j, int64_t k) {
-    uint8_t b = Wq4[j * (K / 2) + k / 2];
-    int nib = (k & 1) ? (b >> 4) : (b & 0xf);
+    int64_t e = k % 32;
+    uint8_t b = Wq4[j * (K / 2) + (k / 32) * 16 + e % 16];
+    int nib = e >= 16 ? (b >> 4) : (b & 0xf);
     return nib >= 8 ? nib - 16 : nib;
 }
 

@@ -5,23 +5,37 @@
 //   C_g[i,j] = sum_{k in group g} Xq[i,k] * Wq4[j,k]          (int32, exact)
 //   Y[i,j]   = dtype( s_x[i] * sum_g s_w[j,g] * C_g[i,j] + bias[j] )
 //
-// Roles (one CTA per SM, 16 warps, persistent over 128x128 output tiles):
+// Roles (one CTA per SM, 24 warps, persistent over 128x128 output tiles):
 //   warp 0       TMA producer: the int8 A tile (128 x 128 B) and the packed
 //                int4 B tile (128 rows x 64 B) of one group per stage;
 //   warp 1       MMA issuer: TMEM holds four 128-column int32 group
 //                accumulators; each group is 4 x tcgen05.mma kind::i8 (K=32)
-//                into a fresh accumulator;
-//   warps 2-3,   converters: unpack the int4 B tile to int8 in the 128-byte
-//   12-13        swizzled K-major layout the MMA reads (the same layout TMA
+//                accumulating onto the seed 0x4B400000 (below). The MMA
+//                computes the transposed tile C_g^T = Wq4 Xq^T (the unpacked
+//                weight tile is the A operand): TMEM lane = output column j,
+//                TMEM column = token i, so a thread of the promotion holds one
+//                output column and needs one weight scale per group;
+//   warps 2-7    converters: unpack the int4 B tile to int8 in the 128-byte
+//                swizzled K-major layout the MMA reads (the same layout TMA
 //                writes), then hand the stage to the MMA;
-//   warps 14-15  idle;
-//   warps 4-11   promotion + epilogue, two warps per 32-lane TMEM quarter,
-//                each with 64 columns: per group, int32 -> fp32 (exact: |C_g|
-//                <= 128*127*7 < 2^22) and sum += s_w[j,g] * C_g in registers
-//                (packed f32x2 arithmetic); the next group's accumulator is
-//                read from TMEM while this one is promoted, and an accumulator
-//                is handed back to the MMA as soon as it has been read;
-//                after the last group, y = s_x[i] * sum + bias -> Y.
+//   warps 8-23   promotion + epilogue, four warps per 32-lane TMEM quarter
+//                (32 output columns), each with 32 tokens: per group, int32 ->
+//                fp32 and sum += s_w[j,g] * C_g in registers (packed f32x2
+//                arithmetic, one scale per thread); after the last group,
+//                y = s_x[i] * sum + bias[j] -> Y. The promotion is a chain of
+//                TMEM loads, waits and barrier hand-offs per group, so it
+//                gets four warps per scheduler to overlap them.
+//
+// The weights reach the MMA as 16 t (unpacking is two masks and a shift per
+// word, see unpack_int4x32), so the MMA computes 16 C_g, exactly.
+// The int32 -> fp32 step costs no integer instruction: an accumulator is
+// seeded with the bits 0x4B400000 (1.5 * 2^23 as an fp32) by the promotion
+// warps (tcgen05.st) once they have read it, and the MMA adds the group's
+// products to that seed in int32. |16 C_g| <= 16*128*127*7 < 2^21, so the
+// seeded word never overflows and, read as an fp32 f, is exactly
+// 1.5 * 2^23 + 16 C_g; one packed fma f * 2^-4 - 1.5 * 2^19 then gives C_g
+// exactly (the product is exact and so is the integer difference). The
+// int32 partial sums stay exact: C_g is (accumulator word - seed) / 16.
 // All waits are bounded (common.cuh).
 #pragma once
 #include "common.cuh"
@@ -30,18 +44,19 @@ namespace qlin {
 
 constexpr int W4_BM = 128, W4_BN = 128, W4_G = 128;   // tile rows, tile columns, group (= K per stage)
 constexpr int W4_STAGES = 4;
-constexpr int W4_CONV_WARPS = 4, W4_PROMO_WARPS = 8;
-constexpr int W4_THREADS = 512;   // 16 warps: 4 warpgroups (see the role list above)
+constexpr int W4_CONV_WARPS = 6, W4_PROMO_WARPS = 16;
+constexpr int W4_THREADS = 768;   // 24 warps: 6 warpgroups (see the role list above)
 constexpr int W4_ACC = 4;                             // TMEM group accumulators (4 x 128 columns)
 constexpr int W4_SWIN = 32;                           // groups per staged window of weight scales
-// Register split (setmaxnreg): warpgroups 0 and 3 (producer, MMA, converters)
-// drop to W4_REGS_LOW, the promotion warpgroups 1 and 2 rise to W4_REGS_HIGH.
-// It fits the block's pool when 2 * 128 (R - LOW) >= 256 (HIGH - R) for the
+constexpr uint32_t W4_SEED = 0x4B400000u;             // fp32 bits of 1.5 * 2^23, the accumulators' start value
+// Register split (setmaxnreg): warpgroups 0 and 1 (producer, MMA, converters)
+// drop to W4_REGS_LOW, the promotion warpgroups 2-5 rise to W4_REGS_HIGH.
+// It fits the block's pool when 256 (R - LOW) >= 512 (HIGH - R) for the
 // launch count R.
-constexpr int W4_REGS_LOW = 40;
-constexpr int W4_REGS_HIGH = 216;
-constexpr int W4_REGS_MIN_LAUNCH = 128;
-static_assert(2 * 128 * (W4_REGS_MIN_LAUNCH - W4_REGS_LOW) >= 256 * (W4_REGS_HIGH - W4_REGS_MIN_LAUNCH),
+constexpr int W4_REGS_LOW = 32;
+constexpr int W4_REGS_HIGH = 104;
+constexpr int W4_REGS_MIN_LAUNCH = 80;
+static_assert(256 * (W4_REGS_MIN_LAUNCH - W4_REGS_LOW) >= 512 * (W4_REGS_HIGH - W4_REGS_MIN_LAUNCH),
               "register split must fit the launch pool");
 
 struct W4Params {
@@ -60,32 +75,49 @@ struct W4Smem {
   static constexpr int BU_BYTES = W4_BN * W4_G;           // 16 KB unpacked int8 (swizzled)
   static constexpr int STAGE_BYTES = A_BYTES + BP_BYTES + BU_BYTES;
   static constexpr int SW_BYTES = 4 * W4_SWIN * W4_BN;    // 16 KB weight-scale window
+  static constexpr int SX_BYTES = 4 * W4_BM;              // the tile's token scales
   static constexpr int BAR_BYTES = 8 * (3 * W4_STAGES + 2 * W4_ACC + 2) + 16;
-  static constexpr int TOTAL = 1024 + W4_STAGES * STAGE_BYTES + SW_BYTES + BAR_BYTES;
+  static constexpr int TOTAL = 1024 + W4_STAGES * STAGE_BYTES + SW_BYTES + SX_BYTES + BAR_BYTES;
 };
 
-// 32 signed int4 (16 packed bytes, even k in the low nibble) -> 32 int8.
-// Per byte: 0x80 | (nibble ^ 8) is 0x80 + (t + 8) for the nibble's value t,
-// so subtracting 8 borrows from no neighbour and leaves 0x80 + t, and
-// flipping bit 7 gives t in two's complement.
-__device__ __forceinline__ uint32_t sext_nibbles(uint32_t nib4) {   // four nibbles in the low halves of 4 bytes
-  return ((((nib4 & 0x0F0F0F0Fu) ^ 0x88888888u) - 0x08080808u) ^ 0x80808080u);
-}
+// 32 int4 codes t (16 packed bytes; byte b holds element b of the block in
+// its low nibble and element b + 16 in its high nibble) -> 32 int8 bytes
+// holding 16 t: a nibble moved to the top half of a byte, with the low half
+// cleared, is the int8 16 t (its sign bit is the byte's). Elements 0..15 go to
+// lo16, 16..31 to hi16.
 __device__ __forceinline__ void unpack_int4x32(const uint4& p, uint4& lo16, uint4& hi16) {
-  const uint32_t w[4] = {p.x, p.y, p.z, p.w};
-  uint32_t o[8];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const uint32_t l = sext_nibbles(w[i]);        // even k
-    const uint32_t h = sext_nibbles(w[i] >> 4);   // odd k
-    o[2 * i] = __byte_perm(l, h, 0x5140);
-    o[2 * i + 1] = __byte_perm(l, h, 0x7362);
-  }
-  lo16 = make_uint4(o[0], o[1], o[2], o[3]);
-  hi16 = make_uint4(o[4], o[5], o[6], o[7]);
+  lo16 = make_uint4((p.x << 4) & 0xF0F0F0F0u, (p.y << 4) & 0xF0F0F0F0u, (p.z << 4) & 0xF0F0F0F0u,
+                    (p.w << 4) & 0xF0F0F0F0u);
+  hi16 = make_uint4(p.x & 0xF0F0F0F0u, p.y & 0xF0F0F0F0u, p.z & 0xF0F0F0F0u, p.w & 0xF0F0F0F0u);
 }
 
-template <typename TOut>
+// 32 lanes x 8 consecutive 32-bit columns from registers
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
+               "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+
+// fma.rn.f32x2 on the pair {lo, hi} built inside the instruction's own asm
+// block (a register-pair move), and the two halves of a pair read back the
+// same way.
+__device__ __forceinline__ unsigned long long fma2_pk(uint32_t lo, uint32_t hi, unsigned long long b,
+                                                      unsigned long long c) {
+  unsigned long long d;
+  asm("{\n\t.reg .b64 t;\n\tmov.b64 t, {%1, %2};\n\tfma.rn.f32x2 %0, t, %3, %4;\n\t}"
+      : "=l"(d)
+      : "r"(lo), "r"(hi), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ void split2(unsigned long long v, float& lo, float& hi) {
+  uint32_t a, b;
+  asm("mov.b64 {%0, %1}, %2;" : "=r"(a), "=r"(b) : "l"(v));
+  lo = __uint_as_float(a);
+  hi = __uint_as_float(b);
+}
+
+// DBG: parity export (int32 partials of group p.dbg_group into p.dbg, no Y)
+template <typename TOut, bool DBG>
 __global__ void __launch_bounds__(W4_THREADS, 1)
     k_gemm_w4a8(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const W4Params p) {
   using L = W4Smem;
@@ -96,7 +128,9 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
   auto sBu = [&](int s) { return smem + s * L::STAGE_BYTES + L::A_BYTES; };
   auto sBp = [&](int s) { return smem + s * L::STAGE_BYTES + L::A_BYTES + L::BU_BYTES; };
   float* s_win = reinterpret_cast<float*>(smem + W4_STAGES * L::STAGE_BYTES);   // [W4_SWIN][W4_BN]
-  uint64_t* full_bar = reinterpret_cast<uint64_t*>(smem + W4_STAGES * L::STAGE_BYTES + L::SW_BYTES);
+  float* s_xt = s_win + W4_SWIN * W4_BN;                                          // [W4_BM]
+  uint64_t* full_bar =
+      reinterpret_cast<uint64_t*>(smem + W4_STAGES * L::STAGE_BYTES + L::SW_BYTES + L::SX_BYTES);
   uint64_t* conv_bar = full_bar + W4_STAGES;
   uint64_t* empty_bar = conv_bar + W4_STAGES;
   uint64_t* gfull_bar = empty_bar + W4_STAGES;
@@ -141,7 +175,7 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp < 4 || warp >= 12) {
+  if (warp < 8) {
   setmaxnreg_dec<W4_REGS_LOW>();
   if (warp == 0) {
     if (lane == 0) {
@@ -183,14 +217,16 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
         for (int g = 0; g < G; ++g) {
-          if (!mbar_wait(&gempty_bar[buf], buf_phase ^ 1u, abort_flag)) { ok = false; break; }
+          // the u-th use of an accumulator waits for its u-th seeding
+          if (!mbar_wait(&gempty_bar[buf], buf_phase, abort_flag)) { ok = false; break; }
           if (!mbar_wait(&conv_bar[stage], phase, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * W4_BN);
-          const uint64_t adesc = sdesc_k128(smem_u32(sA(stage)));
-          const uint64_t bdesc = sdesc_k128(smem_u32(sBu(stage)));
+          // A = the unpacked weight tile (rows j), B = the activation tile (rows i)
+          const uint64_t adesc = sdesc_k128(smem_u32(sBu(stage)));
+          const uint64_t bdesc = sdesc_k128(smem_u32(sA(stage)));
 #pragma unroll
-          for (int k = 0; k < W4_G / 32; ++k) umma<0>(d_tmem, adesc + 2u * k, bdesc + 2u * k, idesc, k != 0 ? 1u : 0u);
+          for (int k = 0; k < W4_G / 32; ++k) umma<0>(d_tmem, adesc + 2u * k, bdesc + 2u * k, idesc, 1u);
           umma_commit(&empty_bar[stage]);
           umma_commit(&gfull_bar[buf]);
           if (++stage == W4_STAGES) { stage = 0; phase ^= 1u; }
@@ -202,9 +238,9 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
       const uint64_t t0 = globaltimer();
       while (!mbar_try_wait(a, 0) && globaltimer() - t0 < drain_limit_ns()) {}
     }
-  } else if (warp == 2 || warp == 3 || warp == 12 || warp == 13) {
+  } else {
     // ---------------- converters: packed int4 -> swizzled int8 ----------------
-    const int ct = warp < 4 ? threadIdx.x - 64 : threadIdx.x - 384 + 64;   // 0..127
+    const int ct = threadIdx.x - 64;   // 0..191
     int stage = 0;
     uint32_t phase = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
@@ -213,9 +249,8 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
         if (!mbar_wait(&full_bar[stage], phase, abort_flag)) { ok = false; break; }
         const uint4* src = reinterpret_cast<const uint4*>(sBp(stage));
         uint8_t* dst = sBu(stage);
-#pragma unroll
-        for (int i = 0; i < (L::BP_BYTES / 16) / (32 * W4_CONV_WARPS); ++i) {
-          const int c = ct + i * 32 * W4_CONV_WARPS;   // 16-byte chunk of the packed tile
+#pragma unroll 1
+        for (int c = ct; c < L::BP_BYTES / 16; c += 32 * W4_CONV_WARPS) {   // 16-byte chunk c of the packed tile
           const int r = c >> 2, part = c & 3;          // row, quarter of the row's 64 packed bytes
           uint4 lo, hi;
           unpack_int4x32(src[c], lo, hi);
@@ -234,125 +269,129 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
   } else {
     setmaxnreg_inc<W4_REGS_HIGH>();
     // ---------------- promotion + epilogue ----------------
-    const int pw = warp - 4;                     // 0..7
-    const int q = warp & 3;                      // TMEM lane quarter
-    const int c0 = (pw >> 2) * 64;               // this warp's first column of the tile
-    const int pt = threadIdx.x - 128;            // 0..255
+    const int pw = warp - 8;                     // 0..15
+    const int q = warp & 3;                      // TMEM lane quarter: output columns 32q..32q+31 of the tile
+    const int c0 = (pw >> 2) * 32;               // this warp's first token (TMEM column) of the tile
+    const int pt = threadIdx.x - 256;            // 0..511
+    const int jl = q * 32 + lane;                // this thread's output column within the tile
     int buf = 0;
     uint32_t buf_phase = 0, bar_phase = 0;
     bool ok = true;
-    // TMEM address of this warp's lane quarter, columns c0 + 32h of accumulator buffer b
+    // TMEM address of this warp's lane quarter, tokens c0 + 16h of accumulator buffer b
     auto taddr = [&](int b, int h) {
-      return tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * W4_BN + c0 + 32 * h);
+      return tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * W4_BN + c0 + 16 * h);
     };
-    uint32_t ra0[32], ra1[32], rb0[32], rb1[32];   // two groups' 64 columns (halves 0 and 1)
+    uint32_t ra[16], rb[16];   // the two 16-token halves of the warp's share of one group
+    // this warp's 32 columns of accumulator b back to the seed, from a block
+    // of 8 registers that stays live (each value is made opaque so that the
+    // compiler keeps the block instead of rebuilding it for every store)
+    uint32_t seedv[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) asm volatile("mov.b32 %0, %1;" : "=r"(seedv[k]) : "n"(W4_SEED));
+    auto seed = [&](int b) {
+#pragma unroll
+      for (int k = 0; k < 32; k += 8) tmem_st8(taddr(b, 0) + k, seedv);
+    };
+    // the seed stores of accumulator b have landed: hand it to the MMA
+    auto release = [&](int b) {
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&gempty_bar[b]);
+    };
+    for (int b = 0; b < W4_ACC; ++b) seed(b);
+    for (int b = 0; b < W4_ACC; ++b) release(b);
     for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
       const int mb = tile % num_m, nb = tile / num_m;
-      const int64_t n_base = static_cast<int64_t>(nb) * W4_BN;
-      const int64_t row = static_cast<int64_t>(mb) * W4_BM + q * 32 + lane;
-      const bool row_ok = row < M;
-      unsigned long long acc[32];   // 64 fp32 sums as pairs
+      const int64_t m_base = static_cast<int64_t>(mb) * W4_BM;
+      const int64_t n = static_cast<int64_t>(nb) * W4_BN + jl;   // this thread's output column
+      const bool n_ok = n < N;
+      unsigned long long acc[16];   // 32 fp32 sums (tokens c0..c0+31) as pairs
 #pragma unroll
-      for (int j = 0; j < 32; ++j) acc[j] = 0ull;
-      // acc[16h..16h+15] += s_w[., g] * float(C_g) for half h of the warp's columns
-      auto promote = [&](int g, int h, const uint32_t (&r)[32]) {
-        const float2* sw = reinterpret_cast<const float2*>(s_win + (g % W4_SWIN) * W4_BN + c0 + 32 * h);
-        // int32 -> fp32: |C| < 2^22, so C + 1.5*2^23 is exact as a float and subtracting gives C
-        const unsigned long long magic = f32x2_of(__float_as_uint(-12582912.0f), __float_as_uint(-12582912.0f));
+      for (int j = 0; j < 16; ++j) acc[j] = 0ull;
+      // acc[8h..8h+7] += s * C_g for half h of the warp's tokens, s = s_w[n, g];
+      // r holds the seeded words 0x4B400000 + 16 C_g
+      auto promote = [&](int g, int h, const uint32_t (&r)[16], unsigned long long s2) {
+        const unsigned long long sixteenth = f32x2_of(0x3D800000u, 0x3D800000u);   // 2^-4
+        const unsigned long long neg_base = f32x2_of(0xC9400000u, 0xC9400000u);    // -1.5 * 2^19
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const unsigned long long c =
-              add_f32x2(f32x2_of(static_cast<uint32_t>(static_cast<int32_t>(r[2 * j]) + 0x4B400000),
-                                 static_cast<uint32_t>(static_cast<int32_t>(r[2 * j + 1]) + 0x4B400000)),
-                        magic);
-          const float2 s2 = sw[j];
-          acc[16 * h + j] = fma_f32x2(f32x2_of(__float_as_uint(s2.x), __float_as_uint(s2.y)), c, acc[16 * h + j]);
-        }
-        if (p.dbg != nullptr && g == p.dbg_group && row_ok) {
-          for (int j = 0; j < 32; ++j) {
-            const int64_t n = n_base + c0 + 32 * h + j;
-            if (n < N) p.dbg[row * N + n] = static_cast<int32_t>(r[j]);
+        for (int j = 0; j < 8; ++j)
+          acc[8 * h + j] = fma_f32x2(s2, fma2_pk(r[2 * j], r[2 * j + 1], sixteenth, neg_base), acc[8 * h + j]);
+        if constexpr (DBG) {
+          if (g == p.dbg_group && n_ok) {
+            for (int j = 0; j < 16; ++j) {
+              const int64_t i = m_base + c0 + 16 * h + j;
+              if (i < M) p.dbg[i * N + n] = static_cast<int32_t>(r[j] - W4_SEED) >> 4;
+            }
           }
         }
       };
-      // Groups alternate between register sets a and b: group g+1's loads are
-      // issued right after group g's have landed and fly while g is promoted
-      // (tcgen05.wait::ld waits for all of a thread's loads, so the overlap is
-      // one group deep). An accumulator goes back to the MMA once it is read.
-      auto fetch = [&](uint32_t (&r0)[32], uint32_t (&r1)[32]) -> bool {
+      // wait until the MMA has finished accumulator `buf`, then start reading half 0 of it
+      auto fetch = [&](uint32_t (&r)[16]) -> bool {
         if (!mbar_wait(&gfull_bar[buf], buf_phase, abort_flag)) return false;
         tc_fence_after();
         __syncwarp();
-        tmem_ld32(taddr(buf, 0), r0);
-        tmem_ld32(taddr(buf, 1), r1);
+        tmem_ld16(taddr(buf, 0), r);
         return true;
       };
-      auto landed = [&](uint32_t (&r0)[32], uint32_t (&r1)[32]) {
-        __syncwarp();
-        tmem_wait_regs32(r0);
-        tmem_wait_regs32(r1);
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&gempty_bar[buf]);
-        if (++buf == W4_ACC) { buf = 0; buf_phase ^= 1u; }
-      };
-      static_assert(W4_SWIN % 2 == 0, "scale windows start on even groups (register set a)");
-      if (!fetch(ra0, ra1)) { ok = false; break; }
-      for (int g = 0; g < G; g += 2) {
+      // One TMEM load is always in flight while the other half is promoted
+      // (tcgen05.wait::ld waits for all of a thread's loads): half 1 of group
+      // g loads during half 0, half 0 of group g+1 during half 1. An
+      // accumulator is re-seeded and goes back to the MMA once both halves
+      // are promoted.
+      if (!fetch(ra)) { ok = false; break; }
+      for (int g = 0; g < G; ++g) {
         if (g % W4_SWIN == 0) {
-          // stage the weight scales of groups [g, g + W4_SWIN) for the tile's columns
+          // stage the weight scales of groups [g, g + W4_SWIN) for the tile's
+          // columns (and, with the first window, the tile's token scales)
           if (!epi_bar(promo_bar, bar_phase, abort_flag)) { ok = false; break; }
           for (int idx = pt; idx < W4_SWIN * W4_BN; idx += 32 * W4_PROMO_WARPS) {
             const int gg = idx / W4_BN, j = idx - gg * W4_BN;
-            const int64_t n = n_base + j;
-            s_win[idx] = (p.s_w != nullptr && n < N && g + gg < G) ? __ldg(p.s_w + n * G + g + gg) : 0.0f;
+            const int64_t nn = static_cast<int64_t>(nb) * W4_BN + j;
+            s_win[idx] = (p.s_w != nullptr && nn < N && g + gg < G) ? __ldg(p.s_w + nn * G + g + gg) : 0.0f;
           }
+          if (g == 0 && pt < W4_BM)
+            s_xt[pt] = (p.s_x != nullptr && m_base + pt < M) ? __ldg(p.s_x + m_base + pt) : 0.0f;
           if (!epi_bar(promo_bar, bar_phase, abort_flag)) { ok = false; break; }
         }
-        landed(ra0, ra1);
-        if (g + 1 < G && !fetch(rb0, rb1)) { ok = false; break; }
-        promote(g, 0, ra0);
-        promote(g, 1, ra1);
-        if (g + 1 >= G) break;
-        landed(rb0, rb1);
-        if (g + 2 < G && !fetch(ra0, ra1)) { ok = false; break; }
-        promote(g + 1, 0, rb0);
-        promote(g + 1, 1, rb1);
+        const float sw = s_win[(g % W4_SWIN) * W4_BN + jl];
+        const unsigned long long s2 = f32x2_of(__float_as_uint(sw), __float_as_uint(sw));
+        tmem_wait16(ra);
+        tmem_ld16(taddr(buf, 1), rb);
+        promote(g, 0, ra, s2);
+        tmem_wait16(rb);
+        const int b = buf;
+        if (++buf == W4_ACC) { buf = 0; buf_phase ^= 1u; }
+        if (g + 1 < G && !fetch(ra)) { ok = false; break; }
+        promote(g, 1, rb, s2);
+        seed(b);
+        release(b);
       }
       if (!ok) {
-        tmem_ld_wait();   // no TMEM load of this warp is left in flight when the CTA winds down
+        // no TMEM access of this warp is left in flight when the CTA winds down
+        tmem_ld_wait();
+        tmem_st_wait();
         break;
       }
-      if (row_ok && p.dbg == nullptr) {
-        const float sx = __ldg(p.s_x + row);
+      if (!DBG && n_ok) {
+        const float bn = p.bias != nullptr ? to_f<TOut>(__ldg(p.bias + n)) : 0.0f;
+        uint16_t* yp = reinterpret_cast<uint16_t*>(p.Y) + n;
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
-          const int64_t n0 = n_base + c0 + 32 * h;
-          if (n0 >= N) continue;
-          float y[32];
+          const float4* sx4 = reinterpret_cast<const float4*>(s_xt + c0 + 16 * h);
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int64_t n = n0 + j;
-            const float b = (p.bias != nullptr && n < N) ? to_f<TOut>(__ldg(p.bias + n)) : 0.0f;
-            const unsigned long long a2 = acc[16 * h + j / 2];
-            const float a = __uint_as_float(static_cast<uint32_t>((j & 1) ? (a2 >> 32) : a2));
-            y[j] = sx * a + b;
-          }
-          uint16_t* yp = reinterpret_cast<uint16_t*>(p.Y) + row * N + n0;
-          if (n0 + 32 <= N && (N & 7) == 0) {
+          for (int j4 = 0; j4 < 4; ++j4) {
+            const float4 sx = sx4[j4];
+            const float xs[4] = {sx.x, sx.y, sx.z, sx.w};
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              uint4 v;
-              v.x = pack2<TOut>(y[8 * i + 0], y[8 * i + 1]);
-              v.y = pack2<TOut>(y[8 * i + 2], y[8 * i + 3]);
-              v.z = pack2<TOut>(y[8 * i + 4], y[8 * i + 5]);
-              v.w = pack2<TOut>(y[8 * i + 6], y[8 * i + 7]);
-              reinterpret_cast<uint4*>(yp)[i] = v;
+            for (int e = 0; e < 4; ++e) {
+              const int jj = 4 * j4 + e;
+              const int64_t i = m_base + c0 + 16 * h + jj;
+              float alo, ahi;
+              split2(acc[8 * h + jj / 2], alo, ahi);
+              const float a = (jj & 1) ? ahi : alo;
+              if (i < M) yp[i * N] = from_f<TOut>(xs[e] * a + bn);
             }
-          } else {
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (n0 + j < N) yp[j] = from_f<TOut>(y[j]);
           }
         }
       }

@@ -860,8 +860,11 @@ __global__ void __launch_bounds__(256) k_fp8_tensor_quant(const T* __restrict__ 
 }
 
 // int4 per-group weights: one warp per (row, group of 128). Lane l holds
-// columns [4l, 4l+4) of the group; s = absmax / 7; codes in [-7, 7]; byte
-// k/2 holds column k even in the low nibble, k odd in the high nibble.
+// columns [4l, 4l+4) of the group; s = absmax / 7; codes in [-7, 7]. Each
+// block of 32 columns is stored in 16 bytes, byte b holding column b of the
+// block in its low nibble and column b + 16 in its high nibble: lanes
+// 8m..8m+3 own the low nibbles of block m and take the high nibbles from
+// lanes 8m+4..8m+7.
 template <typename T>
 __global__ void __launch_bounds__(256) k_int4_group_quant(const T* __restrict__ W, int64_t N, int64_t K,
                                                         uint8_t* __restrict__ Q4, float* __restrict__ s_w) {
@@ -880,13 +883,16 @@ __global__ void __launch_bounds__(256) k_int4_group_quant(const T* __restrict__ 
   m = warp_max(m);
   const float s = m / 7.0f;
   const float inv = 1.0f / s;
-  uint32_t packed = 0;
+  uint32_t nib = 0;   // code e in the low nibble of byte e
 #pragma unroll
   for (int e = 0; e < 4; ++e) {
     const int q = (s == 0.0f) ? 0 : q_int(to_f<T>(h[e]), inv, 7);
-    packed |= (static_cast<uint32_t>(q) & 0xFu) << (4 * e);
+    nib |= (static_cast<uint32_t>(q) & 0xFu) << (8 * e);
   }
-  *reinterpret_cast<uint16_t*>(Q4 + j * (K / 2) + g * (G / 2) + lane * 2) = static_cast<uint16_t>(packed);
+  const uint32_t upper = __shfl_down_sync(0xFFFFFFFFu, nib, 4);
+  if ((lane & 4) == 0)
+    *reinterpret_cast<uint32_t*>(Q4 + j * (K / 2) + g * (G / 2) + (lane >> 3) * 16 + (lane & 3) * 4) =
+        nib | (upper << 4);
   if (lane == 0) s_w[j * ng + g] = s;
 }
 

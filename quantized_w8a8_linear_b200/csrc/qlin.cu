@@ -973,7 +973,7 @@ qlin_status make_tmap_bytes(CUtensorMap* m, const void* base, int64_t rows, int6
   return QLIN_OK;
 }
 
-template <typename TOut>
+template <typename TOut, bool DBG = false>
 qlin_status launch_w4a8(const int8_t* Xq, const uint8_t* Wq4, const W4Params& wp, cudaStream_t st) {
   DeviceInfo* d;
   qlin_status s = device_info(&d);
@@ -982,7 +982,7 @@ qlin_status launch_w4a8(const int8_t* Xq, const uint8_t* Wq4, const W4Params& wp
   if ((s = make_tmap_bytes(&ta, Xq, wp.M, wp.K, W4_G, W4_BM, CU_TENSOR_MAP_SWIZZLE_128B)) != QLIN_OK) return s;
   if ((s = make_tmap_bytes(&tb, Wq4, wp.N, wp.K / 2, W4_G / 2, W4_BN, CU_TENSOR_MAP_SWIZZLE_NONE)) != QLIN_OK)
     return s;
-  auto kern = k_gemm_w4a8<TOut>;
+  auto kern = k_gemm_w4a8<TOut, DBG>;
   static std::atomic<bool> attr_set[16] = {};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -1052,7 +1052,7 @@ qlin_status qlin_w4a8_group_i32(const int8_t* Xq, const uint8_t* Wq4, int64_t M,
   W4Params wp{};
   wp.M = M; wp.N = N; wp.K = K; wp.Y = nullptr; wp.s_x = nullptr; wp.s_w = nullptr; wp.bias = nullptr;
   wp.dbg = C; wp.dbg_group = group;
-  QLIN_TRY(launch_w4a8<__nv_bfloat16>(Xq, Wq4, wp, static_cast<cudaStream_t>(stream)));
+  QLIN_TRY((launch_w4a8<__nv_bfloat16, true>(Xq, Wq4, wp, static_cast<cudaStream_t>(stream))));
   return ok();
 }
 

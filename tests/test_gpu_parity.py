@@ -509,13 +509,13 @@ def test_fp8_dynamic_text_encoder_full_size(q, li):
 # W4A8: int4 per-group-128 weights, per-token int8 activations
 # ---------------------------------------------------------------------------
 
-def _unpack_int4(packed: np.ndarray, K: int) -> np.ndarray:
-    lo = (packed & 0x0F).astype(np.int16)
-    hi = (packed >> 4).astype(np.int16)
-    q = np.empty((packed.shape[0], K), np.int64)
-    q[:, 0::2] = np.where(lo >= 8, lo - 16, lo)
-    q[:, 1::2] = np.where(hi >= 8, hi - 16, hi)
-    return q
+def _unpack_int4(packed, K):
+    """int4 codes [N,K] from the packed [N,K/2] bytes: byte b of each 16-byte
+    block holds element b of the block's 32 in its low nibble, b + 16 in its
+    high nibble, two's complement."""
+    b = packed.reshape(packed.shape[0], K // 32, 16)
+    nib = np.concatenate([b & 0x0F, b >> 4], axis=2).reshape(packed.shape[0], K).astype(np.int64)
+    return np.where(nib >= 8, nib - 16, nib)
 
 
 @pytest.mark.parametrize("M,K", [(64, 128), (129, 1024), (333, 3072), (7, 12288)])

@@ -287,12 +287,12 @@ def test_fp8_dynamic_scales_and_channel_dequant():
 # ---------------------------------------------------------------- W4A8 ---
 
 def unpack_int4(packed, K):
-    lo = (packed & 0x0F).astype(np.int16)
-    hi = (packed >> 4).astype(np.int16)
-    q = np.empty((packed.shape[0], K), np.int16)
-    q[:, 0::2] = np.where(lo >= 8, lo - 16, lo)
-    q[:, 1::2] = np.where(hi >= 8, hi - 16, hi)
-    return q
+    """int4 codes [N,K] from the packed [N,K/2] bytes: byte b of each 16-byte
+    block holds element b of the block's 32 in its low nibble, b + 16 in its
+    high nibble, two's complement."""
+    b = packed.reshape(packed.shape[0], K // 32, 16)
+    nib = np.concatenate([b & 0x0F, b >> 4], axis=2).reshape(packed.shape[0], K).astype(np.int16)
+    return np.where(nib >= 8, nib - 16, nib)
 
 
 # ---------------------------------------------------------------------------
@@ -366,6 +366,26 @@ def test_int4_pack_layout_and_range():
     # scale = group absmax / 7
     wf = W.float().numpy().reshape(8, 2, 128)
     assert np.array_equal(s, np.abs(wf).max(axis=2).astype(np.float32) / np.float32(7.0))
+
+
+def test_int4_pack_bytes_by_hand():
+    """The packed bytes of known codes, written out by hand: weights that are
+    exact multiples of their group's step 0.5 (each group holds a +-3.5, so
+    s = 3.5 / 7 = 0.5 and the code of w is 2w). Byte b of the 16-byte block m
+    must hold code 32m + b in its low nibble and code 32m + b + 16 in its high
+    nibble, two's complement; swapping the nibbles, packing even/odd pairs or
+    dropping the sign would each change a byte here."""
+    K = 256
+    codes = np.array([[((5 * k + 3 * j) % 15) - 7 for k in range(K)] for j in range(3)], np.int64)
+    codes[:, ::128] = 7   # a full-scale code in every group
+    W = torch.tensor(codes * 0.5, dtype=torch.float32).to(torch.bfloat16)
+    q, s = oracle.quantize_weight(W, "int4_g128")
+    assert np.all(s == np.float32(0.5))
+    for j in range(3):
+        for m in range(K // 32):
+            for b in range(16):
+                lo, hi = codes[j, 32 * m + b] & 0xF, codes[j, 32 * m + b + 16] & 0xF
+                assert int(q[j, 16 * m + b]) == (lo | (hi << 4)), (j, m, b)
 
 
 def test_w4a8_equal_group_scales_reduce_to_per_channel():
