@@ -5,26 +5,28 @@
 //   C_g[i,j] = sum_{k in group g} Xq[i,k] * Wq4[j,k]          (int32, exact)
 //   Y[i,j]   = dtype( s_x[i] * sum_g s_w[j,g] * C_g[i,j] + bias[j] )
 //
-// Roles (one CTA per SM, 24 warps, persistent over 128x128 output tiles):
-//   warp 0       TMA producer: the int8 A tile (128 x 128 B) and the packed
-//                int4 B tile (128 rows x 64 B) of one group per stage;
-//   warp 1       MMA issuer: TMEM holds four 128-column int32 group
-//                accumulators; each group is 4 x tcgen05.mma kind::i8 (K=32)
-//                accumulating onto the seed 0x4B400000 (below). The MMA
-//                computes the transposed tile C_g^T = Wq4 Xq^T (the unpacked
-//                weight tile is the A operand): TMEM lane = output column j,
-//                TMEM column = token i, so a thread of the promotion holds one
-//                output column and needs one weight scale per group;
-//   warps 2-7    converters: unpack the int4 B tile to int8 in the 128-byte
-//                swizzled K-major layout the MMA reads (the same layout TMA
-//                writes), then hand the stage to the MMA;
-//   warps 8-23   promotion + epilogue, four warps per 32-lane TMEM quarter
-//                (32 output columns), each with 32 tokens: per group, int32 ->
+// Roles (one CTA per SM, 20 warps, persistent over tiles of 256 tokens x 128
+// output columns):
+//   warp 0       TMA producer: the int8 activation tile (256 x 128 B) and the
+//                packed int4 weight tile (128 rows x 64 B) of one group per
+//                stage;
+//   warp 1       MMA issuer: TMEM holds two 256-column int32 group
+//                accumulators; each group is 4 x tcgen05.mma kind::i8
+//                (M = 128, N = 256, K = 32) accumulating onto the seed
+//                0x4B400000 (below). The MMA computes the transposed tile
+//                C_g^T = Wq4 Xq^T (the unpacked weight tile is the A operand):
+//                TMEM lane = output column j, TMEM column = token i, so a
+//                thread of the promotion holds one output column and needs one
+//                weight scale per group;
+//   warps 2-3    converters: unpack the int4 weight tile to int8 in the
+//                128-byte swizzled K-major layout the MMA reads (the same
+//                layout TMA writes), then hand the stage to the MMA; one
+//                unpacked tile serves 256 tokens;
+//   warps 4-19   promotion + epilogue, four warps per 32-lane TMEM quarter
+//                (32 output columns), each with 64 tokens: per group, int32 ->
 //                fp32 and sum += s_w[j,g] * C_g in registers (packed f32x2
 //                arithmetic, one scale per thread); after the last group,
-//                y = s_x[i] * sum + bias[j] -> Y. The promotion is a chain of
-//                TMEM loads, waits and barrier hand-offs per group, so it
-//                gets four warps per scheduler to overlap them.
+//                y = s_x[i] * sum + bias[j] -> Y.
 //
 // The weights reach the MMA as 16 t (unpacking is two masks and a shift per
 // word, see unpack_int4x32), so the MMA computes 16 C_g, exactly.
@@ -42,21 +44,22 @@
 
 namespace qlin {
 
-constexpr int W4_BM = 128, W4_BN = 128, W4_G = 128;   // tile rows, tile columns, group (= K per stage)
-constexpr int W4_STAGES = 4;
-constexpr int W4_CONV_WARPS = 6, W4_PROMO_WARPS = 16;
-constexpr int W4_THREADS = 768;   // 24 warps: 6 warpgroups (see the role list above)
-constexpr int W4_ACC = 4;                             // TMEM group accumulators (4 x 128 columns)
+constexpr int W4_BM = 256, W4_BN = 128, W4_G = 128;   // tokens per tile, output columns per tile, group (= K per stage)
+constexpr int W4_STAGES = 4;                          // TMA stages: activations + packed weights
+constexpr int W4_URING = 3;                           // unpacked weight tiles (converter -> MMA)
+constexpr int W4_CONV_WARPS = 2, W4_PROMO_WARPS = 16;
+constexpr int W4_PT = W4_BM / 4;                      // tokens per promotion warp
+constexpr int W4_THREADS = 640;   // 20 warps: 5 warpgroups (see the role list above)
+constexpr int W4_ACC = 2;                             // TMEM group accumulators (2 x 256 columns)
 constexpr int W4_SWIN = 32;                           // groups per staged window of weight scales
 constexpr uint32_t W4_SEED = 0x4B400000u;             // fp32 bits of 1.5 * 2^23, the accumulators' start value
-// Register split (setmaxnreg): warpgroups 0 and 1 (producer, MMA, converters)
-// drop to W4_REGS_LOW, the promotion warpgroups 2-5 rise to W4_REGS_HIGH.
-// It fits the block's pool when 256 (R - LOW) >= 512 (HIGH - R) for the
-// launch count R.
+// Register split (setmaxnreg): warpgroup 0 (producer, MMA, converters) drops
+// to W4_REGS_LOW, the promotion warpgroups 1-4 rise to W4_REGS_HIGH. It fits
+// the block's pool when 128 (R - LOW) >= 512 (HIGH - R) for the launch count R.
 constexpr int W4_REGS_LOW = 32;
-constexpr int W4_REGS_HIGH = 104;
-constexpr int W4_REGS_MIN_LAUNCH = 80;
-static_assert(256 * (W4_REGS_MIN_LAUNCH - W4_REGS_LOW) >= 512 * (W4_REGS_HIGH - W4_REGS_MIN_LAUNCH),
+constexpr int W4_REGS_HIGH = 112;
+constexpr int W4_REGS_MIN_LAUNCH = 96;
+static_assert(128 * (W4_REGS_MIN_LAUNCH - W4_REGS_LOW) >= 512 * (W4_REGS_HIGH - W4_REGS_MIN_LAUNCH),
               "register split must fit the launch pool");
 
 struct W4Params {
@@ -70,14 +73,15 @@ struct W4Params {
 };
 
 struct W4Smem {
-  static constexpr int A_BYTES = W4_BM * W4_G;            // 16 KB int8
+  static constexpr int A_BYTES = W4_BM * W4_G;            // 32 KB int8
   static constexpr int BP_BYTES = W4_BN * W4_G / 2;       // 8 KB packed int4
   static constexpr int BU_BYTES = W4_BN * W4_G;           // 16 KB unpacked int8 (swizzled)
-  static constexpr int STAGE_BYTES = A_BYTES + BP_BYTES + BU_BYTES;
+  static constexpr int STAGE_BYTES = A_BYTES + BP_BYTES;   // one TMA stage
   static constexpr int SW_BYTES = 4 * W4_SWIN * W4_BN;    // 16 KB weight-scale window
   static constexpr int SX_BYTES = 4 * W4_BM;              // the tile's token scales
-  static constexpr int BAR_BYTES = 8 * (3 * W4_STAGES + 2 * W4_ACC + 2) + 16;
-  static constexpr int TOTAL = 1024 + W4_STAGES * STAGE_BYTES + SW_BYTES + SX_BYTES + BAR_BYTES;
+  static constexpr int BAR_BYTES = 8 * (2 * W4_STAGES + 2 * W4_URING + 2 * W4_ACC + 2) + 16;
+  static constexpr int TOTAL =
+      1024 + W4_STAGES * STAGE_BYTES + W4_URING * BU_BYTES + SW_BYTES + SX_BYTES + BAR_BYTES;
 };
 
 // 32 int4 codes t (16 packed bytes; byte b holds element b of the block in
@@ -95,6 +99,19 @@ __device__ __forceinline__ void unpack_int4x32(const uint4& p, uint4& lo16, uint
 __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
   asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
                "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+
+// 32 lanes x 8 consecutive 32-bit columns into registers, and the wait naming them
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait8(uint32_t (&r)[8]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7])
+               :
                : "memory");
 }
 
@@ -123,17 +140,19 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
   using L = W4Smem;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  // per stage: [A 16 KB | unpacked B 16 KB | packed B 8 KB] (A and unpacked B 1024-aligned)
+  // TMA stage s: [activations 32 KB | packed weights 8 KB]; then the ring of
+  // unpacked weight tiles, 16 KB each (all 1024-aligned)
   auto sA = [&](int s) { return smem + s * L::STAGE_BYTES; };
-  auto sBu = [&](int s) { return smem + s * L::STAGE_BYTES + L::A_BYTES; };
-  auto sBp = [&](int s) { return smem + s * L::STAGE_BYTES + L::A_BYTES + L::BU_BYTES; };
-  float* s_win = reinterpret_cast<float*>(smem + W4_STAGES * L::STAGE_BYTES);   // [W4_SWIN][W4_BN]
-  float* s_xt = s_win + W4_SWIN * W4_BN;                                          // [W4_BM]
-  uint64_t* full_bar =
-      reinterpret_cast<uint64_t*>(smem + W4_STAGES * L::STAGE_BYTES + L::SW_BYTES + L::SX_BYTES);
-  uint64_t* conv_bar = full_bar + W4_STAGES;
-  uint64_t* empty_bar = conv_bar + W4_STAGES;
-  uint64_t* gfull_bar = empty_bar + W4_STAGES;
+  auto sBp = [&](int s) { return smem + s * L::STAGE_BYTES + L::A_BYTES; };
+  auto sBu = [&](int u) { return smem + W4_STAGES * L::STAGE_BYTES + u * L::BU_BYTES; };
+  uint8_t* tail = smem + W4_STAGES * L::STAGE_BYTES + W4_URING * L::BU_BYTES;
+  float* s_win = reinterpret_cast<float*>(tail);   // [W4_SWIN][W4_BN]
+  float* s_xt = s_win + W4_SWIN * W4_BN;           // [W4_BM]
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(tail + L::SW_BYTES + L::SX_BYTES);
+  uint64_t* empty_bar = full_bar + W4_STAGES;
+  uint64_t* ufull_bar = empty_bar + W4_STAGES;     // unpacked tile u written (converters)
+  uint64_t* uempty_bar = ufull_bar + W4_URING;     // unpacked tile u read (MMA commit)
+  uint64_t* gfull_bar = uempty_bar + W4_URING;
   uint64_t* gempty_bar = gfull_bar + W4_ACC;
   uint64_t* drain_bar = gempty_bar + W4_ACC;
   uint64_t* promo_bar = drain_bar + 1;
@@ -150,8 +169,11 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < W4_STAGES; ++s) {
       mbar_init(&full_bar[s], 1);
-      mbar_init(&conv_bar[s], W4_CONV_WARPS);
       mbar_init(&empty_bar[s], 1);
+    }
+    for (int u = 0; u < W4_URING; ++u) {
+      mbar_init(&ufull_bar[u], W4_CONV_WARPS);
+      mbar_init(&uempty_bar[u], 1);
     }
     for (int b = 0; b < W4_ACC; ++b) {
       mbar_init(&gfull_bar[b], 1);
@@ -175,7 +197,7 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp < 8) {
+  if (warp < 4) {
   setmaxnreg_dec<W4_REGS_LOW>();
   if (warp == 0) {
     if (lane == 0) {
@@ -209,9 +231,9 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------- MMA issuer ----------------
-      constexpr uint32_t idesc = idesc_i8(W4_BM, W4_BN);
-      int stage = 0;
-      uint32_t phase = 0;
+      constexpr uint32_t idesc = idesc_i8(W4_BN, W4_BM);   // M = output columns, N = tokens
+      int stage = 0, u = 0;
+      uint32_t phase = 0, uphase = 0;
       int buf = 0;
       uint32_t buf_phase = 0;
       bool ok = true;
@@ -219,17 +241,20 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
         for (int g = 0; g < G; ++g) {
           // the u-th use of an accumulator waits for its u-th seeding
           if (!mbar_wait(&gempty_bar[buf], buf_phase, abort_flag)) { ok = false; break; }
-          if (!mbar_wait(&conv_bar[stage], phase, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(&full_bar[stage], phase, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(&ufull_bar[u], uphase, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * W4_BN);
+          const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * W4_BM);
           // A = the unpacked weight tile (rows j), B = the activation tile (rows i)
-          const uint64_t adesc = sdesc_k128(smem_u32(sBu(stage)));
+          const uint64_t adesc = sdesc_k128(smem_u32(sBu(u)));
           const uint64_t bdesc = sdesc_k128(smem_u32(sA(stage)));
 #pragma unroll
           for (int k = 0; k < W4_G / 32; ++k) umma<0>(d_tmem, adesc + 2u * k, bdesc + 2u * k, idesc, 1u);
           umma_commit(&empty_bar[stage]);
+          umma_commit(&uempty_bar[u]);
           umma_commit(&gfull_bar[buf]);
           if (++stage == W4_STAGES) { stage = 0; phase ^= 1u; }
+          if (++u == W4_URING) { u = 0; uphase ^= 1u; }
           if (++buf == W4_ACC) { buf = 0; buf_phase ^= 1u; }
         }
       }
@@ -240,16 +265,17 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
     }
   } else {
     // ---------------- converters: packed int4 -> swizzled int8 ----------------
-    const int ct = threadIdx.x - 64;   // 0..191
-    int stage = 0;
-    uint32_t phase = 0;
+    const int ct = threadIdx.x - 64;   // 0..63
+    int stage = 0, u = 0;
+    uint32_t phase = 0, uphase = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
       bool ok = true;
       for (int g = 0; g < G; ++g) {
         if (!mbar_wait(&full_bar[stage], phase, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(&uempty_bar[u], uphase ^ 1u, abort_flag)) { ok = false; break; }
         const uint4* src = reinterpret_cast<const uint4*>(sBp(stage));
-        uint8_t* dst = sBu(stage);
-#pragma unroll 1
+        uint8_t* dst = sBu(u);
+#pragma unroll 2
         for (int c = ct; c < L::BP_BYTES / 16; c += 32 * W4_CONV_WARPS) {   // 16-byte chunk c of the packed tile
           const int r = c >> 2, part = c & 3;          // row, quarter of the row's 64 packed bytes
           uint4 lo, hi;
@@ -260,8 +286,9 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
         }
         fence_proxy_async_smem();   // generic writes -> read by the tensor core (async proxy)
         __syncwarp();
-        if (lane == 0) mbar_arrive(&conv_bar[stage]);
+        if (lane == 0) mbar_arrive(&ufull_bar[u]);
         if (++stage == W4_STAGES) { stage = 0; phase ^= 1u; }
+        if (++u == W4_URING) { u = 0; uphase ^= 1u; }
       }
       if (!ok) break;
     }
@@ -269,28 +296,26 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
   } else {
     setmaxnreg_inc<W4_REGS_HIGH>();
     // ---------------- promotion + epilogue ----------------
-    const int pw = warp - 8;                     // 0..15
+    const int pw = warp - 4;                     // 0..15
     const int q = warp & 3;                      // TMEM lane quarter: output columns 32q..32q+31 of the tile
-    const int c0 = (pw >> 2) * 32;               // this warp's first token (TMEM column) of the tile
-    const int pt = threadIdx.x - 256;            // 0..511
+    const int c0 = (pw >> 2) * W4_PT;            // this warp's first token (TMEM column) of the tile
+    const int pt = threadIdx.x - 128;            // 0..511
     const int jl = q * 32 + lane;                // this thread's output column within the tile
     int buf = 0;
     uint32_t buf_phase = 0, bar_phase = 0;
     bool ok = true;
-    // TMEM address of this warp's lane quarter, tokens c0 + 16h of accumulator buffer b
-    auto taddr = [&](int b, int h) {
-      return tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(b * W4_BN + c0 + 16 * h);
-    };
-    uint32_t ra[16], rb[16];   // the two 16-token halves of the warp's share of one group
-    // this warp's 32 columns of accumulator b back to the seed, from a block
-    // of 8 registers that stays live (each value is made opaque so that the
-    // compiler keeps the block instead of rebuilding it for every store)
-    uint32_t seedv[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) asm volatile("mov.b32 %0, %1;" : "=r"(seedv[k]) : "n"(W4_SEED));
+    // TMEM address of this warp's lane quarter, tokens c0 + 8k of accumulator buffer b
+    const uint32_t tq = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + static_cast<uint32_t>(c0);
+    auto taddr = [&](int b, int k) { return tq + static_cast<uint32_t>(b * W4_BM + 8 * k); };
+    constexpr int NCH = W4_PT / 8;   // 8-token chunks per warp and group
+    uint32_t ra[8], rb[8];           // chunks of the warp's share of one group, alternating
+    // this warp's 64 columns of accumulator b back to the seed
     auto seed = [&](int b) {
 #pragma unroll
-      for (int k = 0; k < 32; k += 8) tmem_st8(taddr(b, 0) + k, seedv);
+      for (int k = 0; k < W4_PT; k += 8)
+        asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(taddr(b, 0) + k),
+                     "r"(W4_SEED)
+                     : "memory");
     };
     // the seed stores of accumulator b have landed: hand it to the MMA
     auto release = [&](int b) {
@@ -306,39 +331,38 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
       const int64_t m_base = static_cast<int64_t>(mb) * W4_BM;
       const int64_t n = static_cast<int64_t>(nb) * W4_BN + jl;   // this thread's output column
       const bool n_ok = n < N;
-      unsigned long long acc[16];   // 32 fp32 sums (tokens c0..c0+31) as pairs
+      unsigned long long acc[W4_PT / 2];   // 64 fp32 sums (tokens c0..c0+63) as pairs
 #pragma unroll
-      for (int j = 0; j < 16; ++j) acc[j] = 0ull;
-      // acc[8h..8h+7] += s * C_g for half h of the warp's tokens, s = s_w[n, g];
+      for (int j = 0; j < W4_PT / 2; ++j) acc[j] = 0ull;
+      // acc[4k..4k+3] += s * C_g for the warp's 8-token chunk k, s = s_w[n, g];
       // r holds the seeded words 0x4B400000 + 16 C_g
-      auto promote = [&](int g, int h, const uint32_t (&r)[16], unsigned long long s2) {
+      auto promote = [&](int g, int k, const uint32_t (&r)[8], unsigned long long s2) {
         const unsigned long long sixteenth = f32x2_of(0x3D800000u, 0x3D800000u);   // 2^-4
         const unsigned long long neg_base = f32x2_of(0xC9400000u, 0xC9400000u);    // -1.5 * 2^19
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          acc[8 * h + j] = fma_f32x2(s2, fma2_pk(r[2 * j], r[2 * j + 1], sixteenth, neg_base), acc[8 * h + j]);
+        for (int j = 0; j < 4; ++j)
+          acc[4 * k + j] = fma_f32x2(s2, fma2_pk(r[2 * j], r[2 * j + 1], sixteenth, neg_base), acc[4 * k + j]);
         if constexpr (DBG) {
           if (g == p.dbg_group && n_ok) {
-            for (int j = 0; j < 16; ++j) {
-              const int64_t i = m_base + c0 + 16 * h + j;
+            for (int j = 0; j < 8; ++j) {
+              const int64_t i = m_base + c0 + 8 * k + j;
               if (i < M) p.dbg[i * N + n] = static_cast<int32_t>(r[j] - W4_SEED) >> 4;
             }
           }
         }
       };
-      // wait until the MMA has finished accumulator `buf`, then start reading half 0 of it
-      auto fetch = [&](uint32_t (&r)[16]) -> bool {
+      // wait until the MMA has finished accumulator `buf`, then start reading chunk 0 of it
+      auto fetch = [&](uint32_t (&r)[8]) -> bool {
         if (!mbar_wait(&gfull_bar[buf], buf_phase, abort_flag)) return false;
         tc_fence_after();
         __syncwarp();
-        tmem_ld16(taddr(buf, 0), r);
+        tmem_ld8(taddr(buf, 0), r);
         return true;
       };
-      // One TMEM load is always in flight while the other half is promoted
-      // (tcgen05.wait::ld waits for all of a thread's loads): half 1 of group
-      // g loads during half 0, half 0 of group g+1 during half 1. An
-      // accumulator is re-seeded and goes back to the MMA once both halves
-      // are promoted.
+      // One TMEM load is always in flight while the previous chunk is promoted
+      // (tcgen05.wait::ld waits for all of a thread's loads); the last chunk
+      // of group g overlaps the first load of group g+1. An accumulator is
+      // re-seeded and goes back to the MMA once its four chunks are promoted.
       if (!fetch(ra)) { ok = false; break; }
       for (int g = 0; g < G; ++g) {
         if (g % W4_SWIN == 0) {
@@ -356,14 +380,23 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
         }
         const float sw = s_win[(g % W4_SWIN) * W4_BN + jl];
         const unsigned long long s2 = f32x2_of(__float_as_uint(sw), __float_as_uint(sw));
-        tmem_wait16(ra);
-        tmem_ld16(taddr(buf, 1), rb);
-        promote(g, 0, ra, s2);
-        tmem_wait16(rb);
+#pragma unroll
+        for (int k = 0; k < NCH - 2; k += 2) {
+          tmem_wait8(ra);
+          tmem_ld8(taddr(buf, k + 1), rb);
+          promote(g, k, ra, s2);
+          tmem_wait8(rb);
+          tmem_ld8(taddr(buf, k + 2), ra);
+          promote(g, k + 1, rb, s2);
+        }
+        tmem_wait8(ra);
+        tmem_ld8(taddr(buf, NCH - 1), rb);
+        promote(g, NCH - 2, ra, s2);
+        tmem_wait8(rb);
         const int b = buf;
         if (++buf == W4_ACC) { buf = 0; buf_phase ^= 1u; }
         if (g + 1 < G && !fetch(ra)) { ok = false; break; }
-        promote(g, 1, rb, s2);
+        promote(g, NCH - 1, rb, s2);
         seed(b);
         release(b);
       }
@@ -377,18 +410,18 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
         const float bn = p.bias != nullptr ? to_f<TOut>(__ldg(p.bias + n)) : 0.0f;
         uint16_t* yp = reinterpret_cast<uint16_t*>(p.Y) + n;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const float4* sx4 = reinterpret_cast<const float4*>(s_xt + c0 + 16 * h);
+        for (int k = 0; k < W4_PT / 16; ++k) {
+          const float4* sx4 = reinterpret_cast<const float4*>(s_xt + c0 + 16 * k);
 #pragma unroll
           for (int j4 = 0; j4 < 4; ++j4) {
             const float4 sx = sx4[j4];
             const float xs[4] = {sx.x, sx.y, sx.z, sx.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const int jj = 4 * j4 + e;
-              const int64_t i = m_base + c0 + 16 * h + jj;
+              const int jj = 4 * j4 + e;   // token c0 + 16k + jj is pair (16k + jj) / 2 of acc
+              const int64_t i = m_base + c0 + 16 * k + jj;
               float alo, ahi;
-              split2(acc[8 * h + jj / 2], alo, ahi);
+              split2(acc[8 * k + jj / 2], alo, ahi);
               const float a = (jj & 1) ? ahi : alo;
               if (i < M) yp[i * N] = from_f<TOut>(xs[e] * a + bn);
             }
