@@ -200,6 +200,8 @@ class LinearRun:
                 self.x_scale = q.qlin_calibrate_input_scale(workloads.make_calibration(wl, lin, index=index).to(device))
             self.Xq = torch.empty((M, K), dtype=torch.uint8, device=device)
             self.s_x = torch.empty((M,), dtype=torch.float32, device=device)
+            self.gws = torch.empty(max(256, q.qlin_workspace_bytes(q.QLIN_OP_FP8_GEMM, M, N, K)), dtype=torch.uint8,
+                                   device=device)
             self.prep_bytes = 3.0 * M * K
         del Wd
 
@@ -229,7 +231,7 @@ class LinearRun:
             q.qlin_w4a8_gemm(self.Xq, self.s_x, self.Wq, self.s_w, self.dtype, Y=self.Y)
         else:
             q.qlin_fp8_gemm(self.Xq, self.s_x, self.Wq, self.s_w, self.wmode, self.dtype, x_scale=self.x_scale,
-                            Y=self.Y)
+                            Y=self.Y, ws=self.gws)
 
     def forward(self):
         self.prepare()

@@ -89,7 +89,8 @@ typedef enum qlin_op {
     QLIN_OP_W4A8 = 2,           /* qlin_w4a8_forward                                */
     QLIN_OP_QUANTIZE_WEIGHT = 3,/* qlin_quantize_weight and qlin_calibrate_input_scale */
     QLIN_OP_INT8_PREP = 4,      /* qlin_int8_prep                                   */
-    QLIN_OP_INT8_BLOCK = 5      /* qlin_int8_block_forward                          */
+    QLIN_OP_INT8_BLOCK = 5,     /* qlin_int8_block_forward                          */
+    QLIN_OP_FP8_GEMM = 6        /* qlin_fp8_gemm's optional scratch                 */
 } qlin_op;
 
 /* Bytes of device scratch `op` needs for an [M,K] x [N,K]^T problem (0 when
@@ -163,11 +164,17 @@ QLIN_API qlin_status qlin_fp8_forward(const void *X, qlin_dtype xdt, int64_t M, 
                              void *workspace, size_t ws_bytes, void *stream);
 
 /* The GEMM stage of qlin_fp8_forward: Xq e4m3 [M,K] and (dynamic mode) s_x
- * fp32 [M] as qlin_fp8_prep wrote them. Same wmode / x_scale rules. */
+ * fp32 [M] as qlin_fp8_prep wrote them. Same wmode / x_scale rules.
+ * workspace: NULL (whole output tiles per CTA), or a 16-byte aligned buffer of
+ * qlin_workspace_bytes(QLIN_OP_FP8_GEMM, M, N, K) bytes, owned by the caller
+ * and not shared with a concurrent call: the GEMM may then split tiles along K
+ * across CTAs (stream-K), with fp32 partial sums added in a fixed order, so
+ * the output does not depend on timing. The call clears the buffer's arrival
+ * counters itself (an extra memset on `stream`); no other initialisation. */
 QLIN_API qlin_status qlin_fp8_gemm(qlin_dtype xdt, int64_t M, int64_t K, const uint8_t *Xq,
                           const float *s_x, const uint8_t *Wq, const void *w_scale,
                           qlin_wmode wmode, int64_t N, const float *x_scale, const void *bias,
-                          void *Y, void *stream);
+                          void *Y, void *workspace, size_t ws_bytes, void *stream);
 
 /* W4A8 forward (Qwen-Image-fni8 page, "Format": int4 per-group weights,
  * int8 activations, fp32 scales; group 128 along K):

@@ -29,7 +29,7 @@ QLIN_ERR_WORKSPACE, QLIN_ERR_CUDA, QLIN_ERR_TIMEOUT = 4, 5, 6
 QLIN_F16, QLIN_BF16 = 0, 1
 QLIN_W_INT8_ROW, QLIN_W_FP8_TENSOR, QLIN_W_FP8_CHANNEL, QLIN_W_INT4_G128, QLIN_W_INT8_BLOCK32 = 0, 1, 2, 3, 4
 QLIN_OP_INT8_OUTLIER, QLIN_OP_FP8, QLIN_OP_W4A8, QLIN_OP_QUANTIZE_WEIGHT, QLIN_OP_INT8_PREP = 0, 1, 2, 3, 4
-QLIN_OP_INT8_BLOCK = 5
+QLIN_OP_INT8_BLOCK, QLIN_OP_FP8_GEMM = 5, 6
 
 _STATUS_NAMES = {0: "QLIN_OK", 1: "QLIN_ERR_INVALID_ARG", 2: "QLIN_ERR_UNSUPPORTED", 3: "QLIN_ERR_ALIGNMENT",
                  4: "QLIN_ERR_WORKSPACE", 5: "QLIN_ERR_CUDA", 6: "QLIN_ERR_TIMEOUT"}
@@ -57,7 +57,7 @@ def _load() -> ctypes.CDLL:
         "qlin_int8_outlier_forward_noalloc": (st, [P, i32, i64, i64, P, P, i64, f32, P, P, P]),
         "qlin_int8_outlier_gemm": (st, [i32, i64, i64, P, P, i64, P, P, P, sz, P]),
         "qlin_int8_outlier_gemm_i32": (st, [i64, i64, P, i64, P, P, sz, P]),
-        "qlin_fp8_gemm": (st, [i32, i64, i64, P, P, P, P, i32, i64, P, P, P, P]),
+        "qlin_fp8_gemm": (st, [i32, i64, i64, P, P, P, P, i32, i64, P, P, P, P, sz, P]),
         "qlin_w4a8_forward": (st, [P, i32, i64, i64, P, P, i64, P, P, P, sz, P]),
         "qlin_fp_linear_forward": (st, [P, i32, i64, i64, P, i64, P, P, P]),
         "qlin_fp8_weight_only_forward": (st, [P, i32, i64, i64, P, P, i64, P, P, P]),
@@ -246,15 +246,18 @@ def qlin_int8_outlier_gemm_i32(M: int, K: int, Wq: torch.Tensor, ws: torch.Tenso
 
 def qlin_fp8_gemm(Xq: torch.Tensor, s_x: Optional[torch.Tensor], Wq: torch.Tensor, w_scale: torch.Tensor,
                   wmode: int, dtype: torch.dtype, x_scale: Optional[torch.Tensor] = None,
-                  bias: Optional[torch.Tensor] = None, Y: Optional[torch.Tensor] = None) -> torch.Tensor:
-    """GEMM stage of the FP8 forward on codes from qlin_fp8_prep."""
+                  bias: Optional[torch.Tensor] = None, Y: Optional[torch.Tensor] = None,
+                  ws: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """GEMM stage of the FP8 forward on codes from qlin_fp8_prep. ws: optional
+    scratch of workspace(QLIN_OP_FP8_GEMM, ...) bytes (lets the GEMM split
+    tiles along K across CTAs); None: whole tiles only."""
     M, K = Xq.shape
     N = Wq.shape[0]
     if Y is None:
         Y = torch.empty((M, N), dtype=dtype, device=Xq.device)
     dt = QLIN_BF16 if dtype == torch.bfloat16 else QLIN_F16
     _check(lib.qlin_fp8_gemm(dt, M, K, _ptr(Xq), _ptr(s_x), _ptr(Wq), _ptr(w_scale), wmode, N, _ptr(x_scale),
-                             _ptr(bias), _ptr(Y), _stream(Xq.device)))
+                             _ptr(bias), _ptr(Y), _ptr(ws), 0 if ws is None else ws.numel(), _stream(Xq.device)))
     return Y
 
 

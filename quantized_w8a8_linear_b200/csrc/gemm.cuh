@@ -67,7 +67,7 @@ static_assert(128 * (GEMM_REGS_MIN_LAUNCH - GEMM_REGS_LOW) >=
 constexpr int GEMM_CW = 16;                  // accumulator columns per tcgen05.ld in the epilogue
 constexpr int GEMM_OUTL_STAGED = 16;         // outlier counts up to this take the staged fp part in the epilogue
 constexpr int GEMM_CORR_K = 32;              // outlier counts up to this take their int8 products out with one MMA
-// Stream-K (kind::i8, 128 x 256 tiles): at most this many CTAs (partial slots
+// Stream-K (kind::i8 and kind::f8f6f4, 128 x 256 tiles): at most this many CTAs (partial slots
 // in the workspace: two per CTA), each with at least GEMM_SK_MIN_ITERS k-blocks
 // unless forced. A cut tile costs its parties about GEMM_SK_COST_KB k-blocks of
 // main loop (measured: 4 us to write a partial and fence it, 3 us to add one),
@@ -236,15 +236,54 @@ __device__ __forceinline__ void sk_store_partial(int32_t* slot, uint32_t t_row, 
   }
 }
 // Adds the other parties' partial slots to the group's columns of the TMEM
-// accumulator (int32: exact in any order). Parties q = 0..nc: the owner ob
-// (q = 0, slot 2ob+1) and the contributors ob+q (slot 2(ob+q)); self_q is
-// this CTA's own party, whose part is already in TMEM.
-template <int BN, int BNG>
+// accumulator. Parties q = 0..nc: the owner ob (q = 0, slot 2ob+1) and the
+// contributors ob+q (slot 2(ob+q)); self_q is this CTA's own party, whose
+// part is already in TMEM. int32 (FP false) is exact in any order. fp32 (FP
+// true) is summed in party order, p_0 + p_1 + ... + p_nc with this CTA's own
+// part taken from TMEM at its place, so the result does not depend on which
+// party finishes the tile.
+template <int BN, int BNG, bool FP>
 __device__ __forceinline__ void sk_add_partials(const int32_t* part, int ob, int nc, int self_q, uint32_t t_row,
                                                 int g, int row_in_tile) {
   constexpr int NCH = BNG / GEMM_CW;
   constexpr int64_t SLOT_V4 = static_cast<int64_t>(GEMM_BM) * BN / 4;
   const int4* src0 = reinterpret_cast<const int4*>(part) + static_cast<int64_t>(g * NCH) * 4 * GEMM_BM + row_in_tile;
+  if constexpr (FP) {
+#pragma unroll 1
+    for (int c = 0; c < NCH; ++c) {   // one 16-column chunk at a time
+      uint32_t own[GEMM_CW];
+      float sum[GEMM_CW];
+      tmem_ld16(t_row + static_cast<uint32_t>(c * GEMM_CW), own);
+      tmem_wait16(own);
+#pragma unroll 1
+      for (int q = 0; q <= nc; ++q) {
+        float v[GEMM_CW];
+        if (q == self_q) {
+#pragma unroll
+          for (int e = 0; e < GEMM_CW; ++e) v[e] = __uint_as_float(own[e]);
+        } else {
+          const int slot = q == 0 ? 2 * ob + 1 : 2 * (ob + q);
+          const int4* src = src0 + slot * SLOT_V4 + static_cast<int64_t>(c) * 4 * GEMM_BM;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int4 w = __ldcg(src + static_cast<int64_t>(j) * GEMM_BM);
+            v[4 * j] = __int_as_float(w.x);
+            v[4 * j + 1] = __int_as_float(w.y);
+            v[4 * j + 2] = __int_as_float(w.z);
+            v[4 * j + 3] = __int_as_float(w.w);
+          }
+        }
+#pragma unroll
+        for (int e = 0; e < GEMM_CW; ++e) sum[e] = q == 0 ? v[e] : __fadd_rn(sum[e], v[e]);
+      }
+      uint32_t out[GEMM_CW];
+#pragma unroll
+      for (int e = 0; e < GEMM_CW; ++e) out[e] = __float_as_uint(sum[e]);
+      tmem_st16(t_row + static_cast<uint32_t>(c * GEMM_CW), out);
+    }
+    tmem_st_wait();
+    return;
+  }
 #pragma unroll 1
   for (int c0 = 0; c0 < NCH; c0 += 4) {
     uint32_t r[4][GEMM_CW];
@@ -633,9 +672,10 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
   // (K = 16) computes X_O W_O^T there, so the epilogue only adds it.
   constexpr bool FT = EPI == EPI_INT8_OUTLIER && BN == 128;
   constexpr int TMEM_COLS = FT ? 4 * BN : 2 * BN;
-  // stream-K: int32 partials only (exact), and not with the FT accumulators,
-  // which only the tile's owner segment computes
-  constexpr bool SK_OK = KIND == 0 && BN == GEMM_SK_BN;
+  // stream-K: int32 partials (exact) for kind::i8, fp32 ones summed in party
+  // order for kind::f8f6f4; 128 x 256 tiles only, so never with the FT
+  // accumulators, which only the tile's owner segment would compute
+  constexpr bool SK_OK = (KIND == 0 || KIND == 1) && BN == GEMM_SK_BN;
   const bool sk = SK_OK && p.sk != 0;
 
   if (threadIdx.x == 0) {
@@ -827,8 +867,8 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         if (!mbar_wait(&tfull_bar[acc], acc_phase, abort_flag)) break;
         tc_fence_after();
       } else if constexpr (SK_OK) {
-        // A cut tile (stream-K). Every party but one leaves its int32 partial
-        // in its slot and counts itself in; the one that finishes the tile is
+        // A cut tile (stream-K). Every party but one leaves its partial (int32,
+        // or fp32 for kind::f8f6f4) in its slot and counts itself in; the one that finishes the tile is
         // the owner if all contributors have arrived when its own part is
         // done (then it writes no partial), else the last to arrive. Nobody
         // waits for another CTA.
@@ -857,7 +897,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
         if (doer) {
           __threadfence();
           if (et == 0) *ctr = 0;   // every other party has counted itself in: ready for the next launch
-          sk_add_partials<BN, BNG>(p.sk_part, ob, nc, self_q, t_row, g, row_in_tile);
+          sk_add_partials<BN, BNG, KIND == 1>(p.sk_part, ob, nc, self_q, t_row, g, row_in_tile);
           if constexpr (EPI != EPI_I32) {
             if (!epi_bar(&epi_mbar[g], bar_phase, abort_flag)) break;
             epi_stage<TOut, EPI, BNG>(p, es, n_base, et, cn);

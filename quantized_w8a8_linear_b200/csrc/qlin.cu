@@ -247,7 +247,7 @@ qlin_status launch_gemm(const void* A, const void* B, EpiParams ep, cudaStream_t
   // projection, 51 MB, and the FP8 QKV, 41 MB, lost 1-2% to them)
   ep.group_m = (ep.M + ep.N) * ep.K > (int64_t{56} << 20) ? GEMM_GROUP_M : 0;
   const int mode = g_gemm_schedule.load(std::memory_order_relaxed);
-  if constexpr (KIND == 0) {
+  if constexpr (KIND == 0 || KIND == 1) {
     const int64_t G0 = std::min<int64_t>(sms, sk_cap);
     if (G0 >= 2 && mode != 1 && ep.sk_count != nullptr && ep.sk_part != nullptr) {
       const int64_t W = t256 / G0;                      // whole waves
@@ -387,6 +387,27 @@ int64_t sk_tiles(int64_t M, int64_t N) { return ((M + GEMM_BM - 1) / GEMM_BM) * 
 int sk_capacity(int64_t M, int64_t N, int64_t K) {
   const int64_t T = sk_tiles(M, N) * ((K + GEMM_BK - 1) / GEMM_BK);
   return static_cast<int>(T < GEMM_SK_MAX_CTAS ? T : GEMM_SK_MAX_CTAS);
+}
+
+// Scratch of the FP8 GEMM: the stream-K arrival counters (zeroed by every
+// call, left zero by the kernel) and the fp32 partial slots, two per CTA.
+struct Fp8GemmWs {
+  int32_t* sk_count;
+  int32_t* sk_part;
+  int sk_ctas;
+  int64_t nctr;
+  size_t total;
+};
+Fp8GemmWs fp8_gemm_layout(void* base, int64_t M, int64_t N, int64_t K) {
+  Fp8GemmWs w{};
+  uint8_t* p = static_cast<uint8_t*>(base);
+  w.nctr = GEMM_EPI_GROUPS * sk_tiles(M, N);
+  w.sk_ctas = sk_capacity(M, N, K);
+  const size_t ctr_bytes = static_cast<size_t>(round_up(4 * w.nctr, 256));
+  w.sk_count = p ? reinterpret_cast<int32_t*>(p) : nullptr;
+  w.sk_part = p ? reinterpret_cast<int32_t*>(p + ctr_bytes) : nullptr;
+  w.total = ctr_bytes + static_cast<size_t>(2 * w.sk_ctas) * GEMM_BM * GEMM_SK_BN * sizeof(int32_t);
+  return w;
 }
 
 // with_sk: room for the stream-K arrival counters and partial slots (the
@@ -548,6 +569,10 @@ size_t qlin_workspace_bytes(qlin_op op, int64_t M, int64_t N, int64_t K) {
     case QLIN_OP_INT8_PREP:
       return int8_layout(nullptr, M, N, K, false).total;
     case QLIN_OP_FP8:
+      return static_cast<size_t>(round_up(M * K, 256) + round_up(4 * M, 256)) +
+             fp8_gemm_layout(nullptr, M, N, K).total;
+    case QLIN_OP_FP8_GEMM:
+      return fp8_gemm_layout(nullptr, M, N, K).total;
     case QLIN_OP_W4A8:
       return static_cast<size_t>(round_up(M * K, 256) + round_up(4 * M, 256));
     case QLIN_OP_QUANTIZE_WEIGHT:
@@ -874,7 +899,7 @@ qlin_status qlin_fp8_prep(const void* X, qlin_dtype xdt, int64_t M, int64_t K, c
 
 qlin_status qlin_fp8_gemm(qlin_dtype xdt, int64_t M, int64_t K, const uint8_t* Xq, const float* s_x,
                           const uint8_t* Wq, const void* w_scale, qlin_wmode wmode, int64_t N, const float* x_scale,
-                          const void* bias, void* Y, void* stream) {
+                          const void* bias, void* Y, void* workspace, size_t ws_bytes, void* stream) {
   if (xdt != QLIN_F16 && xdt != QLIN_BF16) return fail(QLIN_ERR_INVALID_ARG, "bad dtype");
   if (wmode != QLIN_W_FP8_TENSOR && wmode != QLIN_W_FP8_CHANNEL)
     return fail(QLIN_ERR_INVALID_ARG, "wmode must be QLIN_W_FP8_TENSOR or QLIN_W_FP8_CHANNEL");
@@ -895,18 +920,33 @@ qlin_status qlin_fp8_gemm(qlin_dtype xdt, int64_t M, int64_t K, const uint8_t* X
   if (wmode == QLIN_W_FP8_TENSOR) {
     if (x_scale == nullptr) return fail(QLIN_ERR_UNSUPPORTED, "per-tensor weight scales need a static x_scale");
     QLIN_REQ_PTR(x_scale, "x_scale");
-    ep.x_scale = x_scale;
-    ep.w_scale = static_cast<const float*>(w_scale);
-    if (bf) QLIN_TRY((launch_gemm<1, EPI_FP8_TENSOR, __nv_bfloat16>(Xq, Wq, ep, st, 3)));
-    else QLIN_TRY((launch_gemm<1, EPI_FP8_TENSOR, __half>(Xq, Wq, ep, st, 4)));
   } else {
     if (x_scale != nullptr)
       return fail(QLIN_ERR_UNSUPPORTED, "per-channel weight scales go with dynamic per-token activations");
     QLIN_REQ_PTR(s_x, "s_x");
+  }
+  // with scratch: stream-K may cut tiles across CTAs (fp32 partials, summed
+  // in a fixed order); the arrival counters start from zero on every call
+  int sk_cap = 0;
+  if (workspace != nullptr) {
+    const Fp8GemmWs w = fp8_gemm_layout(workspace, M, N, K);
+    if (ws_bytes < w.total) return fail(QLIN_ERR_WORKSPACE, "workspace too small");
+    if (!aligned16(workspace)) return fail(QLIN_ERR_ALIGNMENT, "workspace is not 16-byte aligned");
+    QLIN_TRY(check_cuda(cudaMemsetAsync(w.sk_count, 0, static_cast<size_t>(4 * w.nctr), st), "cudaMemsetAsync"));
+    ep.sk_count = w.sk_count;
+    ep.sk_part = w.sk_part;
+    sk_cap = w.sk_ctas;
+  }
+  if (wmode == QLIN_W_FP8_TENSOR) {
+    ep.x_scale = x_scale;
+    ep.w_scale = static_cast<const float*>(w_scale);
+    if (bf) QLIN_TRY((launch_gemm<1, EPI_FP8_TENSOR, __nv_bfloat16>(Xq, Wq, ep, st, 3, sk_cap)));
+    else QLIN_TRY((launch_gemm<1, EPI_FP8_TENSOR, __half>(Xq, Wq, ep, st, 4, sk_cap)));
+  } else {
     ep.s_x = s_x;
     ep.s_w_bf16 = static_cast<const uint16_t*>(w_scale);
-    if (bf) QLIN_TRY((launch_gemm<1, EPI_FP8_ROWCOL, __nv_bfloat16>(Xq, Wq, ep, st, 5)));
-    else QLIN_TRY((launch_gemm<1, EPI_FP8_ROWCOL, __half>(Xq, Wq, ep, st, 6)));
+    if (bf) QLIN_TRY((launch_gemm<1, EPI_FP8_ROWCOL, __nv_bfloat16>(Xq, Wq, ep, st, 5, sk_cap)));
+    else QLIN_TRY((launch_gemm<1, EPI_FP8_ROWCOL, __half>(Xq, Wq, ep, st, 6, sk_cap)));
   }
   return ok();
 }
@@ -927,8 +967,10 @@ qlin_status qlin_fp8_forward(const void* X, qlin_dtype xdt, int64_t M, int64_t K
   QLIN_REQ_PTR(workspace, "workspace");
   uint8_t* Xq = static_cast<uint8_t*>(workspace);
   float* s_x = reinterpret_cast<float*>(Xq + round_up(M * K, 256));
+  uint8_t* scratch = Xq + round_up(M * K, 256) + round_up(4 * M, 256);
   QLIN_TRY(qlin_fp8_prep(X, xdt, M, K, x_scale, Xq, s_x, stream));
-  return qlin_fp8_gemm(xdt, M, K, Xq, s_x, Wq, w_scale, wmode, N, x_scale, bias, Y, stream);
+  return qlin_fp8_gemm(xdt, M, K, Xq, s_x, Wq, w_scale, wmode, N, x_scale, bias, Y, scratch,
+                       fp8_gemm_layout(nullptr, M, N, K).total, stream);
 }
 
 // Unquantised 16-bit linear: the tcgen05 GEMM with kind::f16 operands (the
