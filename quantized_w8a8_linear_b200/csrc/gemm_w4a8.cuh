@@ -12,8 +12,8 @@
 //                stage;
 //   warp 1       MMA issuer: TMEM holds two 256-column int32 group
 //                accumulators; each group is 4 x tcgen05.mma kind::i8
-//                (M = 128, N = 256, K = 32) accumulating onto the seed
-//                0x4B400000 (below). The MMA computes the transposed tile
+//                (M = 128, N = 256, K = 32) into a fresh accumulator. The MMA
+//                computes the transposed tile
 //                C_g^T = Wq4 Xq^T (the unpacked weight tile is the A operand):
 //                TMEM lane = output column j, TMEM column = token i, so a
 //                thread of the promotion holds one output column and needs one
@@ -30,14 +30,12 @@
 //
 // The weights reach the MMA as 16 t (unpacking is two masks and a shift per
 // word, see unpack_int4x32), so the MMA computes 16 C_g, exactly.
-// The int32 -> fp32 step costs no integer instruction: an accumulator is
-// seeded with the bits 0x4B400000 (1.5 * 2^23 as an fp32) by the promotion
-// warps (tcgen05.st) once they have read it, and the MMA adds the group's
-// products to that seed in int32. |16 C_g| <= 16*128*127*7 < 2^21, so the
-// seeded word never overflows and, read as an fp32 f, is exactly
-// 1.5 * 2^23 + 16 C_g; one packed fma f * 2^-4 - 1.5 * 2^19 then gives C_g
-// exactly (the product is exact and so is the integer difference). The
-// int32 partial sums stay exact: C_g is (accumulator word - seed) / 16.
+// int32 -> fp32: the promotion adds the bits 0x4B400000 (1.5 * 2^23 as an
+// fp32) to each accumulator word. |16 C_g| <= 16*128*127*7 < 2^21, so the sum
+// read as an fp32 f is exactly 1.5 * 2^23 + 16 C_g, and one packed fma
+// f * 2^-4 - 1.5 * 2^19 gives C_g exactly (the product is exact and so is the
+// integer difference). An accumulator goes back to the MMA as soon as its
+// last chunk is in registers, before that chunk is promoted.
 // All waits are bounded (common.cuh).
 #pragma once
 #include "common.cuh"
@@ -52,7 +50,7 @@ constexpr int W4_PT = W4_BM / 4;                      // tokens per promotion wa
 constexpr int W4_THREADS = 640;   // 20 warps: 5 warpgroups (see the role list above)
 constexpr int W4_ACC = 2;                             // TMEM group accumulators (2 x 256 columns)
 constexpr int W4_SWIN = 32;                           // groups per staged window of weight scales
-constexpr uint32_t W4_SEED = 0x4B400000u;             // fp32 bits of 1.5 * 2^23, the accumulators' start value
+constexpr uint32_t W4_SEED = 0x4B400000u;             // fp32 bits of 1.5 * 2^23, added to each accumulator word
 // Register split (setmaxnreg): warpgroup 0 (producer, MMA, converters) drops
 // to W4_REGS_LOW, the promotion warpgroups 1-4 rise to W4_REGS_HIGH. It fits
 // the block's pool when 128 (R - LOW) >= 512 (HIGH - R) for the launch count R.
@@ -93,13 +91,6 @@ __device__ __forceinline__ void unpack_int4x32(const uint4& p, uint4& lo16, uint
   lo16 = make_uint4((p.x << 4) & 0xF0F0F0F0u, (p.y << 4) & 0xF0F0F0F0u, (p.z << 4) & 0xF0F0F0F0u,
                     (p.w << 4) & 0xF0F0F0F0u);
   hi16 = make_uint4(p.x & 0xF0F0F0F0u, p.y & 0xF0F0F0F0u, p.z & 0xF0F0F0F0u, p.w & 0xF0F0F0F0u);
-}
-
-// 32 lanes x 8 consecutive 32-bit columns from registers
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
-               "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
-               : "memory");
 }
 
 // 32 lanes x 8 consecutive 32-bit columns into registers, and the wait naming them
@@ -239,7 +230,7 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
         for (int g = 0; g < G; ++g) {
-          // the u-th use of an accumulator waits for its u-th seeding
+          // the u-th use of an accumulator waits for its u-th release (the first is at start-up)
           if (!mbar_wait(&gempty_bar[buf], buf_phase, abort_flag)) { ok = false; break; }
           if (!mbar_wait(&full_bar[stage], phase, abort_flag)) { ok = false; break; }
           if (!mbar_wait(&ufull_bar[u], uphase, abort_flag)) { ok = false; break; }
@@ -249,7 +240,7 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
           const uint64_t adesc = sdesc_k128(smem_u32(sBu(u)));
           const uint64_t bdesc = sdesc_k128(smem_u32(sA(stage)));
 #pragma unroll
-          for (int k = 0; k < W4_G / 32; ++k) umma<0>(d_tmem, adesc + 2u * k, bdesc + 2u * k, idesc, 1u);
+          for (int k = 0; k < W4_G / 32; ++k) umma<0>(d_tmem, adesc + 2u * k, bdesc + 2u * k, idesc, k != 0 ? 1u : 0u);
           umma_commit(&empty_bar[stage]);
           umma_commit(&uempty_bar[u]);
           umma_commit(&gfull_bar[buf]);
@@ -309,22 +300,12 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
     auto taddr = [&](int b, int k) { return tq + static_cast<uint32_t>(b * W4_BM + 8 * k); };
     constexpr int NCH = W4_PT / 8;   // 8-token chunks per warp and group
     uint32_t ra[8], rb[8];           // chunks of the warp's share of one group, alternating
-    // this warp's 64 columns of accumulator b back to the seed
-    auto seed = [&](int b) {
-#pragma unroll
-      for (int k = 0; k < W4_PT; k += 8)
-        asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%1,%1,%1,%1,%1,%1,%1};" ::"r"(taddr(b, 0) + k),
-                     "r"(W4_SEED)
-                     : "memory");
-    };
-    // the seed stores of accumulator b have landed: hand it to the MMA
+    // hand accumulator b to the MMA: this warp's reads of it have completed
     auto release = [&](int b) {
-      tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&gempty_bar[b]);
     };
-    for (int b = 0; b < W4_ACC; ++b) seed(b);
     for (int b = 0; b < W4_ACC; ++b) release(b);
     for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
       const int mb = tile % num_m, nb = tile / num_m;
@@ -335,18 +316,19 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
 #pragma unroll
       for (int j = 0; j < W4_PT / 2; ++j) acc[j] = 0ull;
       // acc[4k..4k+3] += s * C_g for the warp's 8-token chunk k, s = s_w[n, g];
-      // r holds the seeded words 0x4B400000 + 16 C_g
+      // r holds the int32 words 16 C_g
       auto promote = [&](int g, int k, const uint32_t (&r)[8], unsigned long long s2) {
         const unsigned long long sixteenth = f32x2_of(0x3D800000u, 0x3D800000u);   // 2^-4
         const unsigned long long neg_base = f32x2_of(0xC9400000u, 0xC9400000u);    // -1.5 * 2^19
 #pragma unroll
         for (int j = 0; j < 4; ++j)
-          acc[4 * k + j] = fma_f32x2(s2, fma2_pk(r[2 * j], r[2 * j + 1], sixteenth, neg_base), acc[4 * k + j]);
+          acc[4 * k + j] =
+              fma_f32x2(s2, fma2_pk(r[2 * j] + W4_SEED, r[2 * j + 1] + W4_SEED, sixteenth, neg_base), acc[4 * k + j]);
         if constexpr (DBG) {
           if (g == p.dbg_group && n_ok) {
             for (int j = 0; j < 8; ++j) {
               const int64_t i = m_base + c0 + 8 * k + j;
-              if (i < M) p.dbg[i * N + n] = static_cast<int32_t>(r[j] - W4_SEED) >> 4;
+              if (i < M) p.dbg[i * N + n] = static_cast<int32_t>(r[j]) >> 4;
             }
           }
         }
@@ -361,8 +343,8 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
       };
       // One TMEM load is always in flight while the previous chunk is promoted
       // (tcgen05.wait::ld waits for all of a thread's loads); the last chunk
-      // of group g overlaps the first load of group g+1. An accumulator is
-      // re-seeded and goes back to the MMA once its four chunks are promoted.
+      // of group g overlaps the first load of group g+1. An accumulator goes
+      // back to the MMA once its last chunk is in registers.
       if (!fetch(ra)) { ok = false; break; }
       for (int g = 0; g < G; ++g) {
         if (g % W4_SWIN == 0) {
@@ -393,17 +375,14 @@ __global__ void __launch_bounds__(W4_THREADS, 1)
         tmem_ld8(taddr(buf, NCH - 1), rb);
         promote(g, NCH - 2, ra, s2);
         tmem_wait8(rb);
-        const int b = buf;
+        release(buf);
         if (++buf == W4_ACC) { buf = 0; buf_phase ^= 1u; }
         if (g + 1 < G && !fetch(ra)) { ok = false; break; }
         promote(g, NCH - 1, rb, s2);
-        seed(b);
-        release(b);
       }
       if (!ok) {
-        // no TMEM access of this warp is left in flight when the CTA winds down
+        // no TMEM load of this warp is left in flight when the CTA winds down
         tmem_ld_wait();
-        tmem_st_wait();
         break;
       }
       if (!DBG && n_ok) {
