@@ -90,6 +90,11 @@ def lib() -> ctypes.CDLL:
             "orc_fp_linear_forward": (None, [P, i32, i64, i64, P, i64, P, P, i64, P, P]),
             "orc_fp8_weight_only_dequant": (None, [P, P, i64, i64, P]),
             "orc_fp8_weight_only_forward": (None, [P, i32, i64, i64, P, P, i64, P, P, i64, P, P]),
+            "orc_e2m1_decode": (ctypes.c_double, [ctypes.c_uint8]),
+            "orc_e2m1_encode": (ctypes.c_uint8, [f32]),
+            "orc_quantize_weight_nvfp4": (None, [P, i32, i64, i64, P, P, P]),
+            "orc_nvfp4_code": (ctypes.c_uint8, [P, i64, i64, i64]),
+            "orc_nvfp4_weight_only_forward": (None, [P, i32, i64, i64, P, P, f32, i64, P, P, i64, P, P]),
             "orc_num_threads": (i32, []),
         }
         for name, (res, args) in sig.items():
@@ -369,6 +374,52 @@ def fp8_weight_only_forward(X, Wq, s_w_bits, bias=None, rows: Optional[Sequence[
     Y64 = np.zeros((R, N), np.float64)
     Y = np.zeros((R, N), np.uint16)
     lib().orc_fp8_weight_only_forward(_p(xb), dt, M, K, _p(Wq), _p(sw), N, _p(bb), _p(r), nr, _p(Y64), _p(Y))
+    return dict(Y64=Y64, Y=Y, dt=dt)
+
+
+# ---------------------------------------------------------------------------
+# NVFP4 weights (E2M1 codes, E4M3 per-16 scales, fp32 tensor scale)
+# ---------------------------------------------------------------------------
+
+def e2m1_decode(c: int) -> float:
+    return float(lib().orc_e2m1_decode(int(c)))
+
+
+def e2m1_encode(t: float) -> int:
+    return int(lib().orc_e2m1_encode(float(t)))
+
+
+def quantize_weight_nvfp4(W):
+    """(codes uint8 [N,K/2] packed in blocks of 32, block scales uint8 e4m3 [N,K/16], tensor scale float)."""
+    wb, dt = _bits16(W)
+    N, K = W.shape
+    assert K % 32 == 0
+    q = np.zeros((N, K // 2), np.uint8)
+    sb = np.zeros((N, K // 16), np.uint8)
+    st = np.zeros((1,), np.float32)
+    lib().orc_quantize_weight_nvfp4(_p(wb), dt, N, K, _p(q), _p(sb), _p(st))
+    return q, sb, float(st[0])
+
+
+def nvfp4_code(Wq, K: int, j: int, k: int) -> int:
+    Wq = _np(Wq, np.uint8)
+    return int(lib().orc_nvfp4_code(_p(Wq), K, j, k))
+
+
+def nvfp4_weight_only_forward(X, Wq, s_b, s_t: float, bias=None, rows: Optional[Sequence[int]] = None):
+    """NVFP4 weight-only linear: Y = s_t * X (code * s_b)^T + bias, activations unquantised."""
+    xb, dt = _bits16(X)
+    M, K = X.shape
+    Wq = _np(Wq, np.uint8)
+    sb = _np(s_b, np.uint8)
+    N = Wq.shape[0]
+    bb = None if bias is None else _bits16(bias)[0]
+    r, nr = _rows(rows)
+    R = M if r is None else nr
+    Y64 = np.zeros((R, N), np.float64)
+    Y = np.zeros((R, N), np.uint16)
+    lib().orc_nvfp4_weight_only_forward(_p(xb), dt, M, K, _p(Wq), _p(sb), float(s_t), N, _p(bb), _p(r), nr,
+                                        _p(Y64), _p(Y))
     return dict(Y64=Y64, Y=Y, dt=dt)
 
 

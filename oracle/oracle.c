@@ -735,6 +735,106 @@ void orc_int8_block_forward(const uint16_t *X, int dt, int64_t M, int64_t K, con
     free(s_x);
 }
 
+/* ------------------------------------------------------------------ */
+/* NVFP4 weights, 16-bit activations. The Darkstar pages name NVFP4 as */
+/* the family's primary release format and give no layout; this is the */
+/* plainest reading of the name: E2M1 codes, one E4M3 scale per 16     */
+/* consecutive weights of a row, one fp32 scale per tensor.            */
+/* ------------------------------------------------------------------ */
+
+/* E2M1: sign bit 3, 2 exponent bits (bias 1), 1 mantissa bit, no inf or
+ * NaN. Exponent 0 is subnormal: magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6. */
+double orc_e2m1_decode(uint8_t c) {
+    int e = (c >> 1) & 3, m = c & 1;
+    double mag = e == 0 ? 0.5 * m : ldexp(1.0 + 0.5 * m, e - 1);
+    return (c & 8) ? -mag : mag;
+}
+
+/* Nearest E2M1 value, ties to the even mantissa bit, saturating at 6; the
+ * sign of t (also of -0) goes to bit 3. Found by searching the 8
+ * magnitudes. */
+uint8_t orc_e2m1_encode(float t) {
+    uint8_t sign = signbit(t) ? 8 : 0;
+    double a = fabs((double)t);
+    if (a >= 6.0) return sign | 7;   /* saturation (far above 6 the distances to 4 and 6 round equal) */
+    uint8_t best = 0;
+    double bd = INFINITY;
+    for (uint8_t c = 0; c < 8; ++c) {
+        double d = fabs(orc_e2m1_decode(c) - a);
+        if (d < bd || (d == bd && (c & 1) == 0)) {
+            best = c;
+            bd = d;
+        }
+    }
+    return sign | best;
+}
+
+/* W [N,K] (K % 32 == 0) -> codes Wq [N,K/2] packed like the int4 format
+ * (each block of 32 k in 16 bytes, byte b holding element b in its low
+ * nibble and element b + 16 in its high nibble), block scales s_b e4m3
+ * [N,K/16], tensor scale s_t:
+ *   s_t  = absmax(W) / 2688                  (2688 = 6 * 448)
+ *   s_b  = e4m3(absmax(block) / (6 * s_t))   (rne, saturating at 448; 0 if s_t == 0)
+ *   code = e2m1(w / (decode(s_b) * s_t))     (0 where that divisor is 0)
+ * each division and product one IEEE fp32 operation. */
+void orc_quantize_weight_nvfp4(const uint16_t *W, int dt, int64_t N, int64_t K, uint8_t *Wq, uint8_t *s_b,
+                               float *s_t) {
+    float *w = widen_all(W, dt, N * K);
+    const float st = absmax_range(w, N * K) / 2688.0f;
+    const float six_st = 6.0f * st;
+    *s_t = st;
+    memset(Wq, 0, (size_t)(N * K / 2));
+    for (int64_t j = 0; j < N; ++j) {
+        for (int64_t b = 0; b < K / 16; ++b) {
+            const float *wb = w + j * K + b * 16;
+            const uint8_t sc = six_st == 0.0f ? 0 : orc_e4m3_encode(absmax_range(wb, 16) / six_st);
+            s_b[j * (K / 16) + b] = sc;
+            const float d = (float)orc_e4m3_decode(sc) * st;
+            for (int64_t e = 0; e < 16; ++e) {
+                const int64_t k = b * 16 + e;
+                const uint8_t c = d == 0.0f ? 0 : orc_e2m1_encode(wb[e] / d);
+                const int64_t pos = k % 32;
+                uint8_t *byte = Wq + j * (K / 2) + (k / 32) * 16 + pos % 16;
+                if (pos < 16) *byte = (uint8_t)((*byte & 0xf0) | (c & 0xf));
+                else *byte = (uint8_t)((*byte & 0x0f) | ((c & 0xf) << 4));
+            }
+        }
+    }
+    free(w);
+}
+
+/* The E2M1 code of weight (j, k) in the packed layout above. */
+uint8_t orc_nvfp4_code(const uint8_t *Wq, int64_t K, int64_t j, int64_t k) {
+    const int64_t pos = k % 32;
+    const uint8_t byte = Wq[j * (K / 2) + (k / 32) * 16 + pos % 16];
+    return pos < 16 ? (byte & 0xf) : (byte >> 4);
+}
+
+/* Y64[i,j] = s_t * sum_k X[i,k] * decode(code[j,k]) * decode(s_b[j,k/16]) + bias[j]
+ * in double (each product exact); Y = Y64 rounded once to the dtype of X. */
+void orc_nvfp4_weight_only_forward(const uint16_t *X, int dt, int64_t M, int64_t K, const uint8_t *Wq,
+                                   const uint8_t *s_b, float s_t, int64_t N, const uint16_t *bias,
+                                   const int64_t *rows, int64_t nrows, double *Y64, uint16_t *Y) {
+    double *Wd = (double *)malloc(sizeof(double) * (size_t)(N * K > 0 ? N * K : 1));
+    for (int64_t j = 0; j < N; ++j)
+        for (int64_t k = 0; k < K; ++k)
+            Wd[j * K + k] = orc_e2m1_decode(orc_nvfp4_code(Wq, K, j, k)) * orc_e4m3_decode(s_b[j * (K / 16) + k / 16]);
+    if (!rows) nrows = M;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < nrows; ++r) {
+        int64_t i = rows ? rows[r] : r;
+        for (int64_t j = 0; j < N; ++j) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k) acc += widen(X[i * K + k], dt) * Wd[j * K + k];
+            acc *= (double)s_t;
+            if (bias) acc += widen(bias[j], dt);
+            if (Y64) Y64[r * N + j] = acc;
+            if (Y) Y[r * N + j] = narrow(acc, dt);
+        }
+    }
+    free(Wd);
+}
+
 int orc_num_threads(void) {
 #ifdef _OPENMP
     return omp_get_max_threads();
