@@ -188,6 +188,9 @@ class LinearRun:
         elif self.mode == "fp8_weight_only":
             self.Wq, self.s_w = q.qlin_quantize_weight(Wd, q.QLIN_W_FP8_CHANNEL)
             self.prep_bytes = 0.0
+        elif self.mode == "nvfp4_weight_only":
+            self.Wq, self.s_w = q.qlin_quantize_weight(Wd, q.QLIN_W_NVFP4)
+            self.prep_bytes = 0.0
         elif self.mode == "fp_linear":
             self.Wq, self.s_w = Wd.clone(), None
             self.prep_bytes = 0.0
@@ -207,7 +210,7 @@ class LinearRun:
 
     def prepare(self):
         q = self.q
-        if self.mode in ("fp8_weight_only", "fp_linear"):
+        if self.mode in ("fp8_weight_only", "fp_linear", "nvfp4_weight_only"):
             return   # one kernel: the activations are not quantised
         if self.mode == "int8_outlier":
             q.qlin_int8_outlier_prepare(self.X, self.Wq, self.s_w, 6.0, self.ws)
@@ -221,6 +224,9 @@ class LinearRun:
         q = self.q
         if self.mode == "fp8_weight_only":
             q.qlin_fp8_weight_only_forward(self.X, self.Wq, self.s_w, Y=self.Y)
+            return
+        if self.mode == "nvfp4_weight_only":
+            q.qlin_nvfp4_weight_only_forward(self.X, self.Wq, self.s_w, Y=self.Y)
             return
         if self.mode == "fp_linear":
             q.qlin_fp_linear_forward(self.X, self.Wq, Y=self.Y)
@@ -245,7 +251,7 @@ class LinearRun:
             q.qlin_int8_outlier_forward(self.X, self.Wq, self.s_w, 6.0, Y=self.Y, ws=self.ws)
         elif self.mode == "w4a8":
             q.qlin_w4a8_forward(self.X, self.Wq, self.s_w, Y=self.Y)
-        elif self.mode in ("fp8_weight_only", "fp_linear"):
+        elif self.mode in ("fp8_weight_only", "fp_linear", "nvfp4_weight_only"):
             self.gemm()
         else:
             q.qlin_fp8_forward(self.X, self.Wq, self.s_w, self.wmode, x_scale=self.x_scale, Y=self.Y)
@@ -256,7 +262,7 @@ class LinearRun:
     def launches(self):
         if self.mode == "int8_outlier":
             return 4
-        if self.mode in ("fp8_weight_only", "fp_linear"):
+        if self.mode in ("fp8_weight_only", "fp_linear", "nvfp4_weight_only"):
             return 1
         return 2
 
@@ -570,7 +576,7 @@ def main():
     secondary = {}
     if not args.no_secondary:
         for name in ("dit1024_fp8_static_qkv", "te_fp8_dynamic_mlp", "dit2048_block_int8", "dit2048_block_w4a8",
-                     "te_fp8_weight_only_mlp", "dit1024_bf16_mlp"):
+                     "te_fp8_weight_only_mlp", "te_nvfp4_weight_only_mlp", "dit1024_bf16_mlp"):
             w2 = workloads.get_workload(name)
             r2 = [LinearRun(q, w2, lin, i, device) for i, lin in enumerate(w2.linears)]
             steps2 = max(20, args.steps // 5)
@@ -578,7 +584,8 @@ def main():
             ops2 = sum(r.ops for r in r2)
             tot2 = sum(p2) + sum(g2)
             # the 16-bit contractions (kind::f16) against the bf16 peak, the rest against int8/fp8
-            pk = float(peaks["bf16_tflops"]) if w2.mode in ("fp8_weight_only", "fp_linear") else peak_tops
+            pk = (float(peaks["bf16_tflops"]) if w2.mode in ("fp8_weight_only", "fp_linear", "nvfp4_weight_only")
+                  else peak_tops)
             secondary[name] = {"TOPS": steps2 * ops2 / (tot2 * 1e-3) / 1e12,
                                "gemm_TOPS": steps2 * ops2 / (sum(g2) * 1e-3) / 1e12,
                                "gemm_frac_of_peak": steps2 * ops2 / (sum(g2) * 1e-3) / 1e12 / pk,

@@ -78,8 +78,16 @@ typedef enum qlin_wmode {
     QLIN_W_INT4_G128 = 3,    /* Wq uint8 [N,K/2]: each block of 32 consecutive k in 16 bytes, byte b
                                 holding element b (low nibble) and element b+16 (high nibble), two's
                                 complement, codes in [-7,7]; w_scale fp32 [N,K/128] = absmax/7      */
-    QLIN_W_INT8_BLOCK32 = 4  /* Wq int8 [N,K]; w_scale fp32 [N,K/32] = absmax of each run of 32
+    QLIN_W_INT8_BLOCK32 = 4, /* Wq int8 [N,K]; w_scale fp32 [N,K/32] = absmax of each run of 32
                                 weights of a row / 127 (K % 32 == 0)                               */
+    QLIN_W_NVFP4 = 5         /* Wq uint8 [N,K/2]: E2M1 codes packed like QLIN_W_INT4_G128 (blocks
+                                of 32 k in 16 bytes, byte b: element b low nibble, b+16 high);
+                                w_scale: E4M3 block scales uint8 [N,K/16] (one per 16 weights of
+                                a row), then at byte offset round_up(N*K/16, 16) the fp32 tensor
+                                scale s_t: 16-byte aligned, round_up(N*K/16,16) + 4 bytes.
+                                s_t = absmax(W)/2688, s_b = e4m3(absmax(block)/(6 s_t)),
+                                code = e2m1_rne(w/(s_b s_t)), saturating at 6. K % 64 == 0.
+                                Workspace: QLIN_OP_QUANTIZE_WEIGHT.                               */
 } qlin_wmode;
 
 /* Operations whose scratch size qlin_workspace_bytes() reports. */
@@ -175,6 +183,17 @@ QLIN_API qlin_status qlin_fp8_gemm(qlin_dtype xdt, int64_t M, int64_t K, const u
                           const float *s_x, const uint8_t *Wq, const void *w_scale,
                           qlin_wmode wmode, int64_t N, const float *x_scale, const void *bias,
                           void *Y, void *workspace, size_t ws_bytes, void *stream);
+
+/* NVFP4 weight-only linear (a reading of the release format the Darkstar
+ * ModelOpt-FP8 page names; the page gives no layout): weights from
+ * qlin_quantize_weight(QLIN_W_NVFP4), bf16 activations as they are:
+ *   W_deq[j,k] = e2m1(code[j,k]) * e4m3(s_b[j,k/16])   (exact in bf16)
+ *   Y = bf16( s_t * sum_k X[i,k] * W_deq[j,k] + bias[j] ), fp32 accumulation.
+ * The weight is dequantised tile by tile in shared memory and contracted with
+ * tcgen05 kind::f16 (bf16). X bf16 [M,K], K % 64 == 0; Y bf16 [M,N]. */
+QLIN_API qlin_status qlin_nvfp4_weight_only_forward(const void *X, qlin_dtype xdt, int64_t M, int64_t K,
+                                           const uint8_t *Wq, const void *w_scale, int64_t N,
+                                           const void *bias, void *Y, void *stream);
 
 /* W4A8 forward (Qwen-Image-fni8 page, "Format": int4 per-group weights,
  * int8 activations, fp32 scales; group 128 along K):

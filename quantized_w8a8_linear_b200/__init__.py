@@ -28,6 +28,7 @@ QLIN_OK, QLIN_ERR_INVALID_ARG, QLIN_ERR_UNSUPPORTED, QLIN_ERR_ALIGNMENT = 0, 1, 
 QLIN_ERR_WORKSPACE, QLIN_ERR_CUDA, QLIN_ERR_TIMEOUT = 4, 5, 6
 QLIN_F16, QLIN_BF16 = 0, 1
 QLIN_W_INT8_ROW, QLIN_W_FP8_TENSOR, QLIN_W_FP8_CHANNEL, QLIN_W_INT4_G128, QLIN_W_INT8_BLOCK32 = 0, 1, 2, 3, 4
+QLIN_W_NVFP4 = 5
 QLIN_OP_INT8_OUTLIER, QLIN_OP_FP8, QLIN_OP_W4A8, QLIN_OP_QUANTIZE_WEIGHT, QLIN_OP_INT8_PREP = 0, 1, 2, 3, 4
 QLIN_OP_INT8_BLOCK, QLIN_OP_FP8_GEMM = 5, 6
 
@@ -61,6 +62,7 @@ def _load() -> ctypes.CDLL:
         "qlin_w4a8_forward": (st, [P, i32, i64, i64, P, P, i64, P, P, P, sz, P]),
         "qlin_fp_linear_forward": (st, [P, i32, i64, i64, P, i64, P, P, P]),
         "qlin_fp8_weight_only_forward": (st, [P, i32, i64, i64, P, P, i64, P, P, P]),
+        "qlin_nvfp4_weight_only_forward": (st, [P, i32, i64, i64, P, P, i64, P, P, P]),
         "qlin_int8_block_forward": (st, [P, i32, i64, i64, P, P, i64, P, P, P, sz, P]),
         "qlin_int8_block_prep": (st, [P, i32, i64, i64, P, P, P]),
         "qlin_w4a8_gemm": (st, [i32, i64, i64, P, P, P, P, i64, P, P, P]),
@@ -170,12 +172,27 @@ def qlin_quantize_weight(W: torch.Tensor, mode: int):
     elif mode == QLIN_W_INT8_BLOCK32:
         Wq = torch.empty((N, K), dtype=torch.int8, device=dev)
         s = torch.empty((N, K // 32), dtype=torch.float32, device=dev)
+    elif mode == QLIN_W_NVFP4:
+        Wq = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+        s = torch.empty((nvfp4_scale_offset(N, K) + 4,), dtype=torch.uint8, device=dev)
     else:
         raise ValueError(mode)
     ws = workspace(QLIN_OP_QUANTIZE_WEIGHT, 0, N, K, dev)
     _check(lib.qlin_quantize_weight(_ptr(W), _dt(W), N, K, mode, _ptr(Wq), _ptr(s), _ptr(ws), ws.numel(),
                                     _stream(dev)))
     return Wq, s
+
+
+def nvfp4_scale_offset(N: int, K: int) -> int:
+    """Byte offset of the fp32 tensor scale in a QLIN_W_NVFP4 w_scale buffer
+    (after the E4M3 block scales [N, K/16], rounded up to 16 bytes)."""
+    return (N * K // 16 + 15) // 16 * 16
+
+
+def nvfp4_scales(w_scale: torch.Tensor, N: int, K: int):
+    """(E4M3 block scales uint8 [N, K/16], fp32 tensor scale [1]) views of a QLIN_W_NVFP4 w_scale buffer."""
+    off = nvfp4_scale_offset(N, K)
+    return w_scale[: N * K // 16].view(N, K // 16), w_scale[off:off + 4].view(torch.float32)
 
 
 def qlin_calibrate_input_scale(X: torch.Tensor) -> torch.Tensor:
@@ -314,6 +331,19 @@ def qlin_fp8_weight_only_forward(X: torch.Tensor, Wq: torch.Tensor, w_scale: tor
         Y = torch.empty((M, N), dtype=X.dtype, device=X.device)
     _check(lib.qlin_fp8_weight_only_forward(_ptr(X), _dt(X), M, K, _ptr(Wq), _ptr(w_scale), N, _ptr(bias), _ptr(Y),
                                             _stream(X.device)))
+    return Y
+
+
+def qlin_nvfp4_weight_only_forward(X: torch.Tensor, Wq: torch.Tensor, w_scale: torch.Tensor,
+                                   bias: Optional[torch.Tensor] = None,
+                                   Y: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """NVFP4 weight-only linear: Y = s_t * X (e2m1(code) * e4m3(s_b))^T + bias, bf16 activations."""
+    M, K = X.shape
+    N = Wq.shape[0]
+    if Y is None:
+        Y = torch.empty((M, N), dtype=X.dtype, device=X.device)
+    _check(lib.qlin_nvfp4_weight_only_forward(_ptr(X), _dt(X), M, K, _ptr(Wq), _ptr(w_scale), N, _ptr(bias),
+                                              _ptr(Y), _stream(X.device)))
     return Y
 
 

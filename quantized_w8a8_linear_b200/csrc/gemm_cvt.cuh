@@ -16,6 +16,13 @@
 //   i.e. s_x[i] * sum_b s_w[j,b] * C_b[i,j] with the weight's scale applied
 //   per element before the sum instead of per block after it (relative error
 //   at most 2^-11 per weight, against the exact int32 block sums).
+// FMT 2, NVFP4 weights (a reading of the release format the Darkstar
+// ModelOpt-FP8 page names: E2M1 codes, one E4M3 scale per 16 weights of a
+// row, one fp32 scale per tensor) with bf16 activations:
+//   W_deq[j,k] = bf16( e2m1(code[j,k]) * e4m3(s_b[j,k/16]) )   (exact: at most
+//                6 significant bits)
+//   Y[i,j]     = bf16( s_t * sum_k X[i,k] * W_deq[j,k] + bias[j] )
+//   The raw tile is 256 rows x 32 bytes (64 codes) per stage.
 //
 // Roles (one CTA per SM, 16 warps, persistent over 128x256 output tiles, two
 // 256-column TMEM accumulators so the epilogue of one tile overlaps the main
@@ -51,6 +58,8 @@ struct Wo8Params {
   const uint16_t* s_w;        // FMT 0: [N] bf16 per-channel weight scale
   const float* s_wb;          // FMT 1: [N, K/32] fp32 block weight scales
   const float* s_x;           // FMT 1: [M] fp32 per-token activation scale
+  const uint8_t* s_b4;        // FMT 2: [N, K/16] e4m3 block scales
+  const float* s_t;           // FMT 2: [1] fp32 tensor scale
   const uint16_t* bias;       // [N] output dtype, nullable
 };
 
@@ -88,6 +97,61 @@ __device__ __forceinline__ void e4m3x16_to_bf16(const uint4& raw, float s, uint4
   hi8 = make_uint4(out[4], out[5], out[6], out[7]);
 }
 
+// 32 NVFP4 codes (16 packed bytes, byte b holding element b in its low nibble
+// and element b + 16 in its high nibble) -> 32 bf16 values code * scale, exact
+// (an E2M1 value times an E4M3 scale has at most 6 significant bits).
+// sp0 / sp1: the block scales of elements 0..15 / 16..31 as bf16 pairs.
+// out[0], out[1]: elements 0-7, 8-15; out[2], out[3]: elements 16-23, 24-31.
+// A nibble's magnitude (its low 3 bits) selects the two bytes of its bf16
+// value from byte tables (__byte_perm); its bit 3 becomes bit 15 (the sign).
+__device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+__device__ __forceinline__ void nvfp4x32_to_bf16(const uint4& raw, uint32_t sp0, uint32_t sp1, uint4 (&out)[4]) {
+  // bf16 of the magnitudes 0, 0.5, 1, 1.5 | 2, 3, 4, 6: high bytes, low bytes
+  constexpr uint32_t HI_A = 0x3F3F3F00u, HI_B = 0x40404040u;
+  constexpr uint32_t LO_A = 0xC0800000u, LO_B = 0xC0804000u;
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+  uint32_t lo[8], hi[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      // h = 0: the low nibbles (elements 4i..4i+3), h = 1: the high ones (16+4i..)
+      const uint32_t v = h ? (w[i] >> 4) : w[i];
+      const uint32_t m = v & 0x07070707u;             // magnitudes m0..m3, one per byte
+      const uint32_t sel = m | (m >> 12);              // selector nibbles m0, m2, m1, m3
+      const uint32_t hb = __byte_perm(HI_A, HI_B, sel);
+      const uint32_t lb = __byte_perm(LO_A, LO_B, sel);   // bytes of elements 0, 2, 1, 3
+      uint32_t p01 = __byte_perm(lb, hb, 0x6240);      // bf16 pair (element 0, element 1)
+      uint32_t p23 = __byte_perm(lb, hb, 0x7351);      // bf16 pair (element 2, element 3)
+      const uint32_t sg = v & 0x08080808u;             // signs at bits 3, 11, 19, 27
+      p01 |= ((sg << 12) & 0x00008000u) | ((sg << 20) & 0x80000000u);
+      p23 |= ((sg >> 4) & 0x00008000u) | ((sg << 4) & 0x80000000u);
+      uint32_t* d = h ? hi : lo;
+      const uint32_t sp = h ? sp1 : sp0;
+      d[2 * i] = bf16x2_mul(p01, sp);
+      d[2 * i + 1] = bf16x2_mul(p23, sp);
+    }
+  }
+  out[0] = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+  out[1] = make_uint4(lo[4], lo[5], lo[6], lo[7]);
+  out[2] = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+  out[3] = make_uint4(hi[4], hi[5], hi[6], hi[7]);
+}
+
+// Two e4m3 block scales (low byte first) -> bf16 pairs (s0, s0) and (s1, s1), exact.
+__device__ __forceinline__ void e4m3x2_scale_pairs(uint16_t two, uint32_t& sp0, uint32_t& sp1) {
+  uint32_t f16x2;
+  asm("{\n\t.reg .b16 t;\n\tmov.b16 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}" : "=r"(f16x2) : "h"(two));
+  const float a = __half2float(__ushort_as_half(static_cast<uint16_t>(f16x2 & 0xFFFFu)));
+  const float b = __half2float(__ushort_as_half(static_cast<uint16_t>(f16x2 >> 16)));
+  asm("cvt.rn.bf16x2.f32 %0, %1, %1;" : "=r"(sp0) : "f"(a));
+  asm("cvt.rn.bf16x2.f32 %0, %1, %1;" : "=r"(sp1) : "f"(b));
+}
+
 // 16 int8 codes (element e in byte e) times the scale s, each product
 // rounded to fp16 (the fp32 product rounds first when s has more than 16
 // significant bits): 16 fp16 values as two 16-byte chunks. A code q reads as
@@ -117,7 +181,9 @@ __device__ __forceinline__ void int8x16_to_f16(const uint4& raw, float s, uint4&
 template <int FMT, typename TOut>
 __global__ void __launch_bounds__(WO8_THREADS, 1)
     k_gemm_cvt(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, const Wo8Params p) {
-  static_assert(FMT == 1 || std::is_same<TOut, __nv_bfloat16>::value, "weight-only FP8 writes bf16");
+  static_assert(FMT == 1 || std::is_same<TOut, __nv_bfloat16>::value, "weight-only FP8 and NVFP4 write bf16");
+  // raw weight bytes per row and stage: 64 8-bit codes (FMT 0, 1) or 64 packed 4-bit codes (FMT 2)
+  constexpr int RAW_ROW = FMT == 2 ? WO8_BK / 2 : WO8_BK;
   using L = Wo8Smem;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -181,9 +247,9 @@ __global__ void __launch_bounds__(WO8_THREADS, 1)
         const int mb = tile % num_m, nb = tile / num_m;
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
-          mbar_arrive_expect_tx(&full_bar[stage], L::A_BYTES + L::R_BYTES);
+          mbar_arrive_expect_tx(&full_bar[stage], L::A_BYTES + WO8_BN * RAW_ROW);
           tma_load_2d(sA(stage), &tmA, &full_bar[stage], kb * WO8_BK * 2, mb * WO8_BM);
-          tma_load_2d(sR(stage), &tmB, &full_bar[stage], kb * WO8_BK, nb * WO8_BN);
+          tma_load_2d(sR(stage), &tmB, &full_bar[stage], kb * RAW_ROW, nb * WO8_BN);
           issued |= 1u << stage;
           if (++stage == WO8_STAGES) { stage = 0; phase ^= 1u; }
         }
@@ -203,7 +269,7 @@ __global__ void __launch_bounds__(WO8_THREADS, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------- MMA issuer ----------------
-      constexpr uint32_t idesc = idesc_f16(WO8_BM, WO8_BN, FMT == 0);   // bf16 (FMT 0) or fp16 operands
+      constexpr uint32_t idesc = idesc_f16(WO8_BM, WO8_BN, FMT != 1);   // bf16 (FMT 0, 2) or fp16 operands
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
@@ -234,8 +300,57 @@ __global__ void __launch_bounds__(WO8_THREADS, 1)
       while (!mbar_try_wait(a, 0) && globaltimer() - t0 < drain_limit_ns()) {}
     }
   } else if (warp >= WO8_WARP_CONV0 && warp < WO8_WARP_CONV0 + WO8_CONV_WARPS) {
-    // ---------------- converters: e4m3 * s_w -> bf16, swizzled ----------------
+    // ---------------- converters: codes * scale -> 16 bits, swizzled ----------------
     const int ct = threadIdx.x - 32 * WO8_WARP_CONV0;   // 0..255
+    if constexpr (FMT == 2) {
+      // two 16-byte raw chunks per thread and stage: rows ct/2 and ct/2 + 128,
+      // chunk ct%2 (codes 32c..32c+31 of the stage, block scales 2c and 2c+1)
+      const int c = ct & 1;
+      const int64_t nsb = K / 16;
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+        const int nb = tile / num_m;
+        uint16_t sc[2], sn[2];   // the two rows' scale pairs for stage kb, and kb + 1
+        auto scale_pairs = [&](int kb, uint16_t (&d)[2]) {
+#pragma unroll
+          for (int qd = 0; qd < 2; ++qd) {
+            const int64_t n = static_cast<int64_t>(nb) * WO8_BN + (ct >> 1) + 128 * qd;
+            const int64_t b = 4 * static_cast<int64_t>(kb) + 2 * c;
+            d[qd] = (n < N && kb < num_kb)   // K % 64 == 0: b + 1 < K/16
+                        ? __ldg(reinterpret_cast<const unsigned short*>(p.s_b4 + n * nsb + b))
+                        : static_cast<uint16_t>(0);
+          }
+        };
+        scale_pairs(0, sc);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          scale_pairs(kb + 1, sn);
+          if (!mbar_wait(&full_bar[stage], phase, abort_flag)) { ok = false; break; }
+          const uint8_t* raw = sR(stage);
+          uint8_t* dst = sB(stage);
+#pragma unroll
+          for (int qd = 0; qd < 2; ++qd) {
+            const int r = (ct >> 1) + 128 * qd;
+            const uint4 v = *reinterpret_cast<const uint4*>(raw + r * RAW_ROW + c * 16);
+            uint32_t sp0, sp1;
+            e4m3x2_scale_pairs(sc[qd], sp0, sp1);
+            uint4 o[4];
+            nvfp4x32_to_bf16(v, sp0, sp1, o);
+            // row r's 128 bf16 bytes: 16-byte chunk ch sits at chunk (ch ^ (r & 7))
+#pragma unroll
+            for (int x = 0; x < 4; ++x)
+              *reinterpret_cast<uint4*>(dst + r * 128 + (((4 * c + x) ^ (r & 7)) << 4)) = o[x];
+          }
+          fence_proxy_async_smem();   // generic writes -> read by the tensor core (async proxy)
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&conv_bar[stage]);
+          if (++stage == WO8_STAGES) { stage = 0; phase ^= 1u; }
+          sc[0] = sn[0];
+          sc[1] = sn[1];
+        }
+      }
+    } else {
     const int64_t nblk = K / 32;                        // FMT 1: weight-scale blocks per row
     const int cb = (ct & 3) >> 1;                       // FMT 1: this thread's block within a stage
     int stage = 0;
@@ -290,8 +405,9 @@ __global__ void __launch_bounds__(WO8_THREADS, 1)
         }
       }
     }
+    }
   } else if (warp >= WO8_WARP_EPI0) {
-    // ---------------- epilogue: Y = acc + bias (FMT 0) or s_x * acc + bias (FMT 1) ----------------
+    // ---------------- epilogue: Y = acc + bias (FMT 0), s_x * acc + bias (FMT 1), s_t * acc + bias (FMT 2) ----------------
     const int q = warp & 3;                      // TMEM lane quarter
     const int et = threadIdx.x - 32 * WO8_WARP_EPI0;   // 0..127
     int acc = 0;
@@ -315,6 +431,7 @@ __global__ void __launch_bounds__(WO8_THREADS, 1)
       uint32_t r[32];
       float sx = 1.0f;
       if constexpr (FMT == 1) sx = row < M ? __ldg(p.s_x + row) : 0.0f;
+      if constexpr (FMT == 2) sx = __ldg(p.s_t);
       for (int c = 0; c < WO8_BN; c += 32) {
         __syncwarp();
         tmem_ld32(t_row + static_cast<uint32_t>(c), r);

@@ -896,6 +896,78 @@ __global__ void __launch_bounds__(256) k_int4_group_quant(const T* __restrict__ 
   if (lane == 0) s_w[j * ng + g] = s;
 }
 
+// NVFP4 weights (a reading of the release format the Darkstar ModelOpt-FP8
+// page names): one thread per (row j, block of 32 columns), each step one
+// IEEE fp32 operation:
+//   s_t  = absmax(W) / 2688                 (2688 = 6 * 448)
+//   s_b  = e4m3(absmax(16 weights) / (6 * s_t))   (rne, saturating; 0 if s_t == 0)
+//   code = e2m1(w / (decode(s_b) * s_t))    (0 where that divisor is 0)
+// packed like the int4 format: byte b of the block's 16 holds element b in
+// its low nibble and element b + 16 in its high nibble.
+// E2M1 rounding: the magnitude's code is the number of rounding boundaries
+// below it (0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5 between 0, 0.5, 1, 1.5, 2, 3,
+// 4, 6); at a boundary it goes to the even mantissa (> or >=), and anything
+// above 5 saturates to 6.
+__device__ __forceinline__ uint32_t e2m1_rne(float t) {
+  const float a = fabsf(t);
+  const uint32_t c = static_cast<uint32_t>(a > 0.25f) + static_cast<uint32_t>(a >= 0.75f) +
+                     static_cast<uint32_t>(a > 1.25f) + static_cast<uint32_t>(a >= 1.75f) +
+                     static_cast<uint32_t>(a > 2.5f) + static_cast<uint32_t>(a >= 3.5f) + static_cast<uint32_t>(a > 5.0f);
+  return c | (signbit(t) ? 8u : 0u);
+}
+__device__ __forceinline__ float e4m3_value(uint32_t code) {
+  uint32_t f16x2;
+  const uint16_t pair = static_cast<uint16_t>(code & 0xFFu);
+  asm("{\n\t.reg .b16 t;\n\tmov.b16 t, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, t;\n\t}" : "=r"(f16x2) : "h"(pair));
+  return __half2float(__ushort_as_half(static_cast<uint16_t>(f16x2 & 0xFFFFu)));
+}
+template <typename T>
+__global__ void __launch_bounds__(256) k_nvfp4_quant(const T* __restrict__ W, int64_t N, int64_t K,
+                                                     const uint32_t* __restrict__ amax_bits, uint8_t* __restrict__ Q,
+                                                     uint8_t* __restrict__ s_b, float* __restrict__ s_t) {
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t nb = K / 32;
+  if (t >= N * nb) return;
+  const int64_t j = t / nb, m = t - j * nb;
+  const float st = __fdiv_rn(__uint_as_float(*amax_bits), 2688.0f);
+  const float six_st = __fmul_rn(6.0f, st);
+  if (t == 0) *s_t = st;
+  float w[32];
+  const uint4* src = reinterpret_cast<const uint4*>(W + j * K + m * 32);
+#pragma unroll
+  for (int v = 0; v < 4; ++v) {
+    uint16_t h[8];
+    unpack8(__ldg(src + v), h);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) w[8 * v + e] = to_f<T>(h[e]);
+  }
+  uint32_t sc[2];
+  float d[2];
+#pragma unroll
+  for (int hb = 0; hb < 2; ++hb) {
+    float bm = 0.0f;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) bm = fmaxf(bm, fabsf(w[16 * hb + e]));
+    sc[hb] = six_st == 0.0f ? 0u : (e4m3x2(__fdiv_rn(bm, six_st), 0.0f) & 0xFFu);
+    d[hb] = __fmul_rn(e4m3_value(sc[hb]), st);
+  }
+  uint32_t out[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint32_t word = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int b = 4 * i + e;
+      const uint32_t lo = d[0] == 0.0f ? 0u : e2m1_rne(__fdiv_rn(w[b], d[0]));
+      const uint32_t hi = d[1] == 0.0f ? 0u : e2m1_rne(__fdiv_rn(w[16 + b], d[1]));
+      word |= (lo | (hi << 4)) << (8 * e);
+    }
+    out[i] = word;
+  }
+  *reinterpret_cast<uint4*>(Q + j * (K / 2) + m * 16) = make_uint4(out[0], out[1], out[2], out[3]);
+  *reinterpret_cast<uint16_t*>(s_b + j * (K / 16) + 2 * m) = static_cast<uint16_t>(sc[0] | (sc[1] << 8));
+}
+
 // Block-scaled int8 weights: one thread per (row j, block b of 32 weights
 // along K): s_w[j,b] = absmax / 127, codes rne(w * (1/s)) clamped to +-127
 // (the row format's quantiser on each block), 0 for an all-zero block.

@@ -621,6 +621,7 @@ qlin_status qlin_quantize_weight(const void* W, qlin_dtype wdt, int64_t N, int64
   if (mode == QLIN_W_INT4_G128 && K % 128 != 0) return fail(QLIN_ERR_ALIGNMENT, "int4 format needs K % 128 == 0");
   if (mode == QLIN_W_INT8_BLOCK32 && K % 32 != 0)
     return fail(QLIN_ERR_ALIGNMENT, "block-scaled int8 needs K % 32 == 0");
+  if (mode == QLIN_W_NVFP4 && K % 64 != 0) return fail(QLIN_ERR_ALIGNMENT, "NVFP4 format needs K % 64 == 0");
   if (N == 0) return ok();
   QLIN_REQ_PTR(Wq, "Wq");
   QLIN_REQ_PTR(w_scale, "w_scale");
@@ -685,6 +686,30 @@ qlin_status qlin_quantize_weight(const void* W, qlin_dtype wdt, int64_t N, int64
         k_int8_block_quant<__half><<<grid, 256, 0, st>>>(static_cast<const __half*>(W), N, K, static_cast<int8_t*>(Wq),
                                                          static_cast<float*>(w_scale));
       QLIN_TRY(check_cuda(cudaGetLastError(), "int8 block quant launch"));
+      return ok();
+    }
+    case QLIN_W_NVFP4: {
+      if (workspace == nullptr || ws_bytes < qlin_workspace_bytes(QLIN_OP_QUANTIZE_WEIGHT, 0, N, K))
+        return fail(QLIN_ERR_WORKSPACE, "workspace too small");
+      QLIN_REQ_PTR(workspace, "workspace");
+      if (!aligned16(w_scale)) return fail(QLIN_ERR_ALIGNMENT, "w_scale is not 16-byte aligned");
+      uint32_t* amax = static_cast<uint32_t*>(workspace);
+      uint8_t* sb = static_cast<uint8_t*>(w_scale);
+      float* s_t = reinterpret_cast<float*>(sb + round_up(N * K / 16, 16));
+      QLIN_TRY(check_cuda(cudaMemsetAsync(amax, 0, 4, st), "cudaMemsetAsync"));
+      const int grid = d->sms * 4;
+      const int64_t threads = N * (K / 32);
+      const unsigned blocks = static_cast<unsigned>((threads + 255) / 256);
+      if (bf) {
+        k_absmax<__nv_bfloat16><<<grid, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(W), nvec, amax);
+        k_nvfp4_quant<__nv_bfloat16><<<blocks, 256, 0, st>>>(static_cast<const __nv_bfloat16*>(W), N, K, amax,
+                                                            static_cast<uint8_t*>(Wq), sb, s_t);
+      } else {
+        k_absmax<__half><<<grid, 256, 0, st>>>(static_cast<const __half*>(W), nvec, amax);
+        k_nvfp4_quant<__half><<<blocks, 256, 0, st>>>(static_cast<const __half*>(W), N, K, amax,
+                                                     static_cast<uint8_t*>(Wq), sb, s_t);
+      }
+      QLIN_TRY(check_cuda(cudaGetLastError(), "nvfp4 quant launch"));
       return ok();
     }
     default:
@@ -1139,7 +1164,9 @@ qlin_status launch_cvt(const void* A, const void* Wq, const Wo8Params& wp, cudaS
   if (s != QLIN_OK) return s;
   CUtensorMap ta, tb;
   if ((s = make_tmap_k128(&ta, A, wp.M, 2 * wp.K, WO8_BM)) != QLIN_OK) return s;
-  if ((s = make_tmap_bytes(&tb, Wq, wp.N, wp.K, WO8_BK, WO8_BN, CU_TENSOR_MAP_SWIZZLE_NONE)) != QLIN_OK) return s;
+  if ((s = make_tmap_bytes(&tb, Wq, wp.N, FMT == 2 ? wp.K / 2 : wp.K, FMT == 2 ? WO8_BK / 2 : WO8_BK, WO8_BN,
+                           CU_TENSOR_MAP_SWIZZLE_NONE)) != QLIN_OK)
+    return s;
   auto kern = k_gemm_cvt<FMT, TOut>;
   static std::atomic<bool> attr_set[16] = {};
   int dev = 0;
@@ -1174,6 +1201,28 @@ extern "C" qlin_status qlin_fp8_weight_only_forward(const void* X, qlin_dtype xd
   wp.s_w = static_cast<const uint16_t*>(w_scale);
   wp.bias = static_cast<const uint16_t*>(bias);
   QLIN_TRY((launch_cvt<0, __nv_bfloat16>(X, Wq, wp, static_cast<cudaStream_t>(stream))));
+  return ok();
+}
+
+extern "C" qlin_status qlin_nvfp4_weight_only_forward(const void* X, qlin_dtype xdt, int64_t M, int64_t K,
+                                                      const uint8_t* Wq, const void* w_scale, int64_t N,
+                                                      const void* bias, void* Y, void* stream) {
+  QLIN_TRY(check_common(X, xdt, M, K, N));
+  if (xdt != QLIN_BF16)
+    return fail(QLIN_ERR_UNSUPPORTED, "NVFP4 weight-only takes bf16 activations (the weight dequantises to bf16)");
+  if (K % 64 != 0) return fail(QLIN_ERR_ALIGNMENT, "NVFP4 format needs K % 64 == 0");
+  if (M == 0 || N == 0) return ok();
+  QLIN_REQ_PTR(Wq, "Wq");
+  QLIN_REQ_PTR(w_scale, "w_scale");
+  QLIN_REQ_PTR(Y, "Y");
+  if (!aligned16(w_scale)) return fail(QLIN_ERR_ALIGNMENT, "w_scale is not 16-byte aligned");
+  if (bias != nullptr && !aligned16(bias)) return fail(QLIN_ERR_ALIGNMENT, "bias is not 16-byte aligned");
+  Wo8Params wp{};
+  wp.M = M; wp.N = N; wp.K = K; wp.Y = Y;
+  wp.s_b4 = static_cast<const uint8_t*>(w_scale);
+  wp.s_t = reinterpret_cast<const float*>(static_cast<const uint8_t*>(w_scale) + round_up(N * K / 16, 16));
+  wp.bias = static_cast<const uint16_t*>(bias);
+  QLIN_TRY((launch_cvt<2, __nv_bfloat16>(X, Wq, wp, static_cast<cudaStream_t>(stream))));
   return ok();
 }
 

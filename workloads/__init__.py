@@ -45,7 +45,7 @@ class Linear:
 class Workload:
     """A named synthetic workload: its linears, dtype, mode and outlier recipe."""
     name: str
-    mode: str                 # "int8_outlier" | "fp8_static" | "fp8_dynamic" | "w4a8" | "fp8_weight_only" | "fp_linear"
+    mode: str                 # "int8_outlier" | "fp8_static" | "fp8_dynamic" | "w4a8" | "fp8_weight_only" | "fp_linear" | "nvfp4_weight_only"
     dtype: torch.dtype
     linears: List[Linear]
     seed: int
@@ -180,6 +180,13 @@ WORKLOADS: Dict[str, Workload] = {
     # at the text-encoder MLP shapes.
     "te_fp8_weight_only_mlp": Workload(
         name="te_fp8_weight_only_mlp", mode="fp8_weight_only", dtype=torch.bfloat16, seed=6,
+        linears=[Linear("gate", 512, 4096, 12288), Linear("up", 512, 4096, 12288),
+                 Linear("down", 512, 12288, 4096)],
+        massive_pairs=[(5, 2276, 9000.0), (0, 2276, 13000.0)]),
+    # NVFP4 weights (E2M1 codes, E4M3 per-16 and fp32 per-tensor scales) with
+    # bf16 activations at the same text-encoder MLP shapes and inputs.
+    "te_nvfp4_weight_only_mlp": Workload(
+        name="te_nvfp4_weight_only_mlp", mode="nvfp4_weight_only", dtype=torch.bfloat16, seed=6,
         linears=[Linear("gate", 512, 4096, 12288), Linear("up", 512, 4096, 12288),
                  Linear("down", 512, 12288, 4096)],
         massive_pairs=[(5, 2276, 9000.0), (0, 2276, 13000.0)]),
