@@ -20,8 +20,9 @@
 //                weight scale per group;
 //   warps 2-3    converters: unpack the int4 weight tile to int8 in the
 //                128-byte swizzled K-major layout the MMA reads (the same
-//                layout TMA writes), then hand the stage to the MMA; one
-//                unpacked tile serves 256 tokens;
+//                layout TMA writes), into one of three unpacked tiles (a ring
+//                of its own, so a TMA stage holds only what TMA writes), then
+//                hand it to the MMA; one unpacked tile serves 256 tokens;
 //   warps 4-19   promotion + epilogue, four warps per 32-lane TMEM quarter
 //                (32 output columns), each with 64 tokens: per group, int32 ->
 //                fp32 and sum += s_w[j,g] * C_g in registers (packed f32x2
