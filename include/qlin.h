@@ -177,8 +177,9 @@ QLIN_API qlin_status qlin_fp8_forward(const void *X, qlin_dtype xdt, int64_t M, 
  * qlin_workspace_bytes(QLIN_OP_FP8_GEMM, M, N, K) bytes, owned by the caller
  * and not shared with a concurrent call: the GEMM may then split tiles along K
  * across CTAs (stream-K), with fp32 partial sums added in a fixed order, so
- * the output does not depend on timing. The call clears the buffer's arrival
- * counters itself (an extra memset on `stream`); no other initialisation. */
+ * the output does not depend on timing. When it cuts tiles, the call clears
+ * the buffer's arrival counters itself (a memset on `stream`); no other
+ * initialisation. */
 QLIN_API qlin_status qlin_fp8_gemm(qlin_dtype xdt, int64_t M, int64_t K, const uint8_t *Xq,
                           const float *s_x, const uint8_t *Wq, const void *w_scale,
                           qlin_wmode wmode, int64_t N, const float *x_scale, const void *bias,

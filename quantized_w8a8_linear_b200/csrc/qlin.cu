@@ -265,6 +265,15 @@ qlin_status launch_gemm(const void* A, const void* B, EpiParams ep, cudaStream_t
         if (mode == 2 || std::max(main, epi) < 0.95 * std::min(dpc256, dpc128)) {
           ep.sk = 1;
           ep.sk_dp_tiles = static_cast<int>(dp_tiles);
+          // kind::f8f6f4 takes its counters from the caller's scratch: clear
+          // them here, only when tiles are cut (the int8 prepare stage clears
+          // its own); the kernel leaves them zero
+          if constexpr (KIND == 1) {
+            const qlin_status z = check_cuda(
+                cudaMemsetAsync(ep.sk_count, 0, sizeof(int32_t) * GEMM_EPI_GROUPS * static_cast<size_t>(t256), st),
+                "cudaMemsetAsync");
+            if (z != QLIN_OK) return z;
+          }
           return launch_gemm_bn<KIND, EPI, TOut, 256, 4>(ta, B, ep, ty, d, st, 2 * attr_slot, static_cast<int>(G));
         }
       }
@@ -951,13 +960,12 @@ qlin_status qlin_fp8_gemm(qlin_dtype xdt, int64_t M, int64_t K, const uint8_t* X
     QLIN_REQ_PTR(s_x, "s_x");
   }
   // with scratch: stream-K may cut tiles across CTAs (fp32 partials, summed
-  // in a fixed order); the arrival counters start from zero on every call
+  // in a fixed order); launch_gemm clears the arrival counters when it does
   int sk_cap = 0;
   if (workspace != nullptr) {
     const Fp8GemmWs w = fp8_gemm_layout(workspace, M, N, K);
     if (ws_bytes < w.total) return fail(QLIN_ERR_WORKSPACE, "workspace too small");
     if (!aligned16(workspace)) return fail(QLIN_ERR_ALIGNMENT, "workspace is not 16-byte aligned");
-    QLIN_TRY(check_cuda(cudaMemsetAsync(w.sk_count, 0, static_cast<size_t>(4 * w.nctr), st), "cudaMemsetAsync"));
     ep.sk_count = w.sk_count;
     ep.sk_part = w.sk_part;
     sk_cap = w.sk_ctas;
