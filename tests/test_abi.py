@@ -67,6 +67,35 @@ def test_workspace_holds_stream_k_slots(q):
     assert base + 2 * 2 * 128 * 256 * 4 <= small < base + 2 * 2 * 128 * 256 * 4 + (1 << 16)
 
 
+def test_fp8_workspace_holds_its_gemm_scratch(q):
+    # FP8 forward: e4m3 codes + s_x + the GEMM scratch; the scratch: arrival
+    # counters for the 128 x 256 tiles' 4 column groups + two fp32 128 x 256
+    # partial slots per stream-K CTA (at most 160, at most one per k-block)
+    M, N, K = 512, 12288, 4096
+    scratch = q.qlin_workspace_bytes(q.QLIN_OP_FP8_GEMM, M, N, K)
+    tiles = (M // 128) * (N // 256)
+    assert 2 * 160 * 128 * 256 * 4 + 4 * 4 * tiles <= scratch < 2 * 160 * 128 * 256 * 4 + 4 * 4 * tiles + 512
+    assert q.qlin_workspace_bytes(q.QLIN_OP_FP8, M, N, K) >= M * K + 4 * M + scratch
+    M, N, K = 128, 256, 256   # one tile of 2 k-blocks: 2 stream-K CTAs at most
+    assert q.qlin_workspace_bytes(q.QLIN_OP_FP8_GEMM, M, N, K) >= 2 * 2 * 128 * 256 * 4
+
+
+def test_nvfp4_scale_buffer_layout(q):
+    # E4M3 block scales [N, K/16], then the fp32 tensor scale at a 16-byte boundary
+    for N, K in [(8, 64), (257, 128), (12288, 4096)]:
+        off = q.nvfp4_scale_offset(N, K)
+        assert off >= N * K // 16 and off % 16 == 0 and off - N * K // 16 < 16
+
+
+def test_nvfp4_rejects_k_not_multiple_of_64(q):
+    st = q.lib.qlin_nvfp4_weight_only_forward(ctypes.c_void_p(4096), q.QLIN_BF16, 8, 96, ctypes.c_void_p(4096),
+                                              ctypes.c_void_p(4096), 8, None, ctypes.c_void_p(4096), None)
+    assert st == q.QLIN_ERR_ALIGNMENT
+    st = q.lib.qlin_nvfp4_weight_only_forward(ctypes.c_void_p(4096), q.QLIN_F16, 8, 128, ctypes.c_void_p(4096),
+                                              ctypes.c_void_p(4096), 8, None, ctypes.c_void_p(4096), None)
+    assert st == q.QLIN_ERR_UNSUPPORTED   # bf16 activations only
+
+
 def test_gemm_schedule_modes(q):
     for mode in (0, 1, 2):
         assert q.lib.qlin_set_gemm_schedule(mode) == q.QLIN_OK
