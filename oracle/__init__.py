@@ -95,6 +95,7 @@ def lib() -> ctypes.CDLL:
             "orc_quantize_weight_nvfp4": (None, [P, i32, i64, i64, P, P, P]),
             "orc_nvfp4_code": (ctypes.c_uint8, [P, i64, i64, i64]),
             "orc_nvfp4_weight_only_forward": (None, [P, i32, i64, i64, P, P, f32, i64, P, P, i64, P, P]),
+            "orc_nvfp4_forward": (None, [P, i32, i64, i64, P, P, f32, i64, P, P, i64, P, P, P, P, P]),
             "orc_num_threads": (i32, []),
         }
         for name, (res, args) in sig.items():
@@ -421,6 +422,28 @@ def nvfp4_weight_only_forward(X, Wq, s_b, s_t: float, bias=None, rows: Optional[
     lib().orc_nvfp4_weight_only_forward(_p(xb), dt, M, K, _p(Wq), _p(sb), float(s_t), N, _p(bb), _p(r), nr,
                                         _p(Y64), _p(Y))
     return dict(Y64=Y64, Y=Y, dt=dt)
+
+
+def nvfp4_forward(X, Wq, s_bw, s_tw: float, bias=None, rows: Optional[Sequence[int]] = None):
+    """NVFP4 activations and weights (W4A4): X quantised per call like a weight,
+    Y = s_tx * s_tw * (cx * sbx)(cw * sbw)^T + bias. Returns Y64, Y, Xq, s_bx, s_tx."""
+    xb, dt = _bits16(X)
+    M, K = X.shape
+    assert K % 32 == 0
+    Wq = _np(Wq, np.uint8)
+    sbw = _np(s_bw, np.uint8)
+    N = Wq.shape[0]
+    bb = None if bias is None else _bits16(bias)[0]
+    r, nr = _rows(rows)
+    R = M if r is None else nr
+    Xq = np.zeros((M, K // 2), np.uint8)
+    sbx = np.zeros((M, K // 16), np.uint8)
+    stx = np.zeros((1,), np.float32)
+    Y64 = np.zeros((R, N), np.float64)
+    Y = np.zeros((R, N), np.uint16)
+    lib().orc_nvfp4_forward(_p(xb), dt, M, K, _p(Wq), _p(sbw), float(s_tw), N, _p(bb), _p(r), nr, _p(Xq), _p(sbx),
+                            _p(stx), _p(Y64), _p(Y))
+    return dict(Y64=Y64, Y=Y, Xq=Xq, s_bx=sbx, s_tx=float(stx[0]), dt=dt)
 
 
 # ---------------------------------------------------------------------------

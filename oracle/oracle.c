@@ -835,6 +835,43 @@ void orc_nvfp4_weight_only_forward(const uint16_t *X, int dt, int64_t M, int64_t
     free(Wd);
 }
 
+/* NVFP4 activations and weights (W4A4; the next step of the NVFP4 reading):
+ * X [M,K] is quantised per call exactly like a weight (orc_quantize_weight_nvfp4
+ * applied to X: its tensor scale from this call's absmax, one E4M3 scale per
+ * 16 values of a row), then
+ *   Y64[i,j] = s_tx * s_tw * sum_k (e2m1(cx[i,k]) * e4m3(sbx[i,k/16]))
+ *                                * (e2m1(cw[j,k]) * e4m3(sbw[j,k/16])) + bias[j]
+ * in double (each product exact). Xq [M,K/2], s_bx [M,K/16], s_tx [1] are
+ * written out (codes for every row; Y64/Y only for `rows`). */
+void orc_nvfp4_forward(const uint16_t *X, int dt, int64_t M, int64_t K, const uint8_t *Wq, const uint8_t *s_bw,
+                       float s_tw, int64_t N, const uint16_t *bias, const int64_t *rows, int64_t nrows,
+                       uint8_t *Xq, uint8_t *s_bx, float *s_tx, double *Y64, uint16_t *Y) {
+    orc_quantize_weight_nvfp4(X, dt, M, K, Xq, s_bx, s_tx);
+    double *Wd = (double *)malloc(sizeof(double) * (size_t)(N * K > 0 ? N * K : 1));
+    for (int64_t j = 0; j < N; ++j)
+        for (int64_t k = 0; k < K; ++k)
+            Wd[j * K + k] = orc_e2m1_decode(orc_nvfp4_code(Wq, K, j, k)) * orc_e4m3_decode(s_bw[j * (K / 16) + k / 16]);
+    const double st = (double)*s_tx * (double)s_tw;
+    if (!rows) nrows = M;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < nrows; ++r) {
+        int64_t i = rows ? rows[r] : r;
+        double *xd = (double *)malloc(sizeof(double) * (size_t)(K > 0 ? K : 1));
+        for (int64_t k = 0; k < K; ++k)
+            xd[k] = orc_e2m1_decode(orc_nvfp4_code(Xq, K, i, k)) * orc_e4m3_decode(s_bx[i * (K / 16) + k / 16]);
+        for (int64_t j = 0; j < N; ++j) {
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k) acc += xd[k] * Wd[j * K + k];
+            acc *= st;
+            if (bias) acc += widen(bias[j], dt);
+            if (Y64) Y64[r * N + j] = acc;
+            if (Y) Y[r * N + j] = narrow(acc, dt);
+        }
+        free(xd);
+    }
+    free(Wd);
+}
+
 int orc_num_threads(void) {
 #ifdef _OPENMP
     return omp_get_max_threads();

@@ -112,3 +112,42 @@ def test_nvfp4_within_half_step_and_swapped_scales_break_it():
     a2 = np.abs(wd2 / np.where(d2 == 0, 1, d2))
     half2 = np.where(a2 < 2, 0.25, np.where(a2 < 4, 0.5, 1.0))
     assert not np.all(np.abs(w - wd2) <= half2 * d2 * (1 + 1e-6) + 1e-30)
+
+
+def test_nvfp4_w4a4_forward_matches_matmul_of_both_decoded_operands():
+    """W4A4: the activations quantised per call by the same rule as a weight
+    (their tensor scale from the call's absmax); the forward against a
+    matmul of both operands decoded here."""
+    g = torch.Generator().manual_seed(13)
+    M, N, K = 6, 20, 192
+    X = torch.randn((M, K), generator=g).to(torch.bfloat16)
+    X[2, 5] = 90.0                      # a large entry: that row's block scale and the tensor scale follow it
+    W = (torch.randn((N, K), generator=g) * 0.02).to(torch.bfloat16)
+    bias = (torch.randn(N, generator=g) * 0.1).to(torch.bfloat16)
+    q, sb, st = oracle.quantize_weight_nvfp4(W)
+    r = oracle.nvfp4_forward(X, q, sb, st, bias=bias)
+    qx, sbx, stx = oracle.quantize_weight_nvfp4(X)
+    assert np.array_equal(r["Xq"], qx) and np.array_equal(r["s_bx"], sbx) and r["s_tx"] == stx
+    assert stx == np.float32(90.0) / np.float32(2688.0)
+    ref = _decode_np(qx, sbx, stx, K) @ _decode_np(q, sb, st, K).T + bias.double().numpy()
+    assert np.allclose(r["Y64"], ref, rtol=1e-12, atol=1e-12)
+    # only the listed rows are computed, in the listed order
+    rr = oracle.nvfp4_forward(X, q, sb, st, bias=bias, rows=[4, 0])
+    assert np.array_equal(rr["Y64"], r["Y64"][[4, 0]])
+
+
+def test_nvfp4_w4a4_close_to_the_unquantised_product():
+    """The W4A4 output is the unquantised product up to 4-bit noise (a few
+    percent normwise here), and leaving out the activations' tensor scale,
+    a plausible slip, moves it far outside that."""
+    g = torch.Generator().manual_seed(17)
+    M, N, K = 4, 12, 512
+    X = torch.randn((M, K), generator=g).to(torch.bfloat16)
+    W = (torch.randn((N, K), generator=g) * 0.02).to(torch.bfloat16)
+    q, sb, st = oracle.quantize_weight_nvfp4(W)
+    r = oracle.nvfp4_forward(X, q, sb, st)
+    exact = X.double().numpy() @ W.double().numpy().T
+    rel = np.linalg.norm(r["Y64"] - exact) / np.linalg.norm(exact)
+    assert 1e-3 < rel < 0.15, rel
+    wrong = r["Y64"] / r["s_tx"]      # the same sum without the activations' tensor scale
+    assert np.linalg.norm(wrong - exact) / np.linalg.norm(exact) > 1.0
